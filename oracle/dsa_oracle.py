@@ -1,0 +1,233 @@
+"""Plain fp64 CPU oracle for the DeepSeek Sparse Attention (DSA) forward path.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. The CUDA library
+shares no code, table or constant with it, and it never reads a value the
+CUDA path produced.
+
+What it follows ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language
+Models", bud-325 paper digest):
+  * "Key claims", §2.1 Eq. 1: the lightning-indexer score
+        I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])
+    over H_I indexer heads, in FP8;
+  * same passage, §2.1 Eq. 2 / Fig. 2: attention runs only on the top-k key-value
+    entries selected by I[t,:], in MLA's MQA mode (one latent row shared by all
+    query heads);
+  * "Method": k = 2048, one latent vector per token shared by all heads.
+The eu.36kr.com article (section 02) adds that candidates are the query's
+preceding tokens and that top-k index scores pick the entries that are read.
+
+Readings where the pages are silent (each one is listed in the design notes):
+  * candidates for query row t at absolute position p = q_pos0 + t are keys s <= p;
+  * FP8 values carry positive fp32 scales: one per key row of k^I, one per
+    (token, head) row of q^I. A positive scale commutes with ReLU, so
+    I[t,s] = s^k[s] * sum_j w[t,j] * s^q[t,j] * max(0, qhat[t,j] . khat[s]);
+  * ties at the k-th score go to the lowest key index; the selected set is
+    returned in ascending key order, padded with -1 when fewer than k exist;
+  * attention is exact softmax(sm_scale * q . c_s) over the selected rows with
+    values c_s[:Dv]; lse is the natural-log log-sum-exp of the scaled logits;
+    a row with no valid key gives zeros and lse = -inf.
+
+Every function here is a direct transcription of those definitions in numpy
+float64 with library primitives (matmul, argsort, exp) as single steps.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# ---------------------------------------------------------------------------
+# Storage formats
+# ---------------------------------------------------------------------------
+
+
+def e4m3_table() -> np.ndarray:
+    """Value of every FP8 E4M3 (OCP "fn" variant) byte, built from the bit layout.
+
+    Layout S.EEEE.MMM, exponent bias 7, no infinities; S.1111.111 is NaN.
+    Exponent field 0 is subnormal: value = (-1)^S * 2^(1-7) * M/8.
+    """
+    out = np.empty(256, dtype=np.float64)
+    for b in range(256):
+        sign = -1.0 if (b >> 7) & 1 else 1.0
+        e = (b >> 3) & 0xF
+        m = b & 0x7
+        if e == 0xF and m == 0x7:
+            out[b] = np.nan
+        elif e == 0:
+            out[b] = sign * (m / 8.0) * 2.0 ** (1 - 7)
+        else:
+            out[b] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return out
+
+
+_E4M3 = e4m3_table()
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    return _E4M3[np.asarray(codes, dtype=np.uint8)]
+
+
+def decode_bf16(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns (uint16) -> float64 (exact: bf16 is the top half of fp32)."""
+    u32 = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u32.view(np.float32).astype(np.float64)
+
+
+def to_f64(x: np.ndarray) -> np.ndarray:
+    """Decode a stored array: uint16 means bf16 bits, floats are widened."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return decode_bf16(x)
+    return x.astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Lightning indexer (Eq. 1)
+# ---------------------------------------------------------------------------
+
+
+def index_scores(qI: np.ndarray, qI_scale: np.ndarray, w: np.ndarray,
+                 kI: np.ndarray, kI_scale: np.ndarray) -> np.ndarray:
+    """I[s] for one query row against keys kI[0..n).
+
+    qI: uint8 e4m3 codes [H_I, d_I]; qI_scale: [H_I]; w: [H_I] (f32 or bf16 bits)
+    kI: uint8 e4m3 codes [n, d_I];   kI_scale: [n]
+    Returns float64 [n]:  I[s] = sum_j w_j * ReLU(q^I_j . k^I_s), where the
+    dequantised vectors are q^I_j = qhat_j * s^q_j and k^I_s = khat_s * s^k_s.
+    """
+    q = decode_e4m3(qI) * to_f64(qI_scale)[:, None]          # [H_I, d_I]
+    kk = decode_e4m3(kI) * to_f64(kI_scale)[:, None]         # [n, d_I]
+    dots = q @ kk.T                                          # [H_I, n]
+    return to_f64(w) @ np.maximum(dots, 0.0)                 # [n]
+
+
+# ---------------------------------------------------------------------------
+# Fine-grained token selection
+# ---------------------------------------------------------------------------
+
+
+def topk_select(scores: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest scores, ties to the lowest index.
+
+    scores: float64 [n], the candidates 0..n-1 of one query row. Returns int64
+    [k]: the selected indices in ascending order, padded with -1 if n < k.
+    """
+    n = scores.shape[0]
+    out = np.full(k, -1, dtype=np.int64)
+    if n <= k:
+        out[:n] = np.arange(n)
+        return out
+    order = np.argsort(-scores, kind="stable")   # stable: equal scores keep index order
+    out[:] = np.sort(order[:k])
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Sparse MLA in MQA mode
+# ---------------------------------------------------------------------------
+
+
+def sparse_mla(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, sm_scale: float, Dv: int):
+    """Exact softmax attention of one query token over its selected latent rows.
+
+    q: [H, Dqk] (bf16 bits or float); kv: [n_keys, Dqk] latent rows of the
+    sequence (bf16 bits or float); idx: selected key indices, entries < 0 or
+    >= n_keys are skipped. Every head attends to the same rows (MQA mode):
+        z[h,s] = sm_scale * q[h] . c_s,  out[h] = sum_s softmax(z[h])_s * c_s[:Dv]
+    Returns (out float64 [H, Dv], lse float64 [H]).
+    """
+    qf = to_f64(q)
+    H = qf.shape[0]
+    idx = np.asarray(idx)
+    valid = idx[(idx >= 0) & (idx < kv.shape[0])]
+    if valid.size == 0:
+        return np.zeros((H, Dv)), np.full(H, -np.inf)
+    c = to_f64(kv[valid])                                    # [n_sel, Dqk]
+    z = sm_scale * (qf @ c.T)                                # [H, n_sel]
+    m = z.max(axis=1, keepdims=True)
+    p = np.exp(z - m)
+    denom = p.sum(axis=1, keepdims=True)
+    out = (p @ c[:, :Dv]) / denom
+    lse = m[:, 0] + np.log(denom[:, 0])
+    return out, lse
+
+
+def dense_causal_mqa(q: np.ndarray, kv: np.ndarray, sm_scale: float, Dv: int, q_pos0: int = 0):
+    """Dense causal MQA attention, written independently of ``sparse_mla``.
+
+    q: [Lq, H, Dqk]; kv: [Lk, Dqk]. Row t attends to keys 0..q_pos0+t with a
+    per-key loop and a running (max, sum) pair. Used only to pin the sparse path:
+    when k covers every causal key the two must agree.
+    """
+    qf = to_f64(q)
+    cf = to_f64(kv)
+    Lq, H, _ = qf.shape
+    out = np.zeros((Lq, H, Dv))
+    lse = np.zeros((Lq, H))
+    for t in range(Lq):
+        last = q_pos0 + t
+        for h in range(H):
+            mx = -np.inf
+            tot = 0.0
+            acc = np.zeros(Dv)
+            for s in range(last + 1):
+                zz = sm_scale * float(np.dot(qf[t, h], cf[s]))
+                if zz > mx:
+                    r = np.exp(mx - zz) if np.isfinite(mx) else 0.0
+                    tot *= r
+                    acc *= r
+                    mx = zz
+                e = np.exp(zz - mx)
+                tot += e
+                acc += e * cf[s, :Dv]
+            out[t, h] = acc / tot
+            lse[t, h] = mx + np.log(tot)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Whole forward on chosen rows
+# ---------------------------------------------------------------------------
+
+
+def forward_rows(inp: dict, cfg, b: int, rows, with_scores: bool = True) -> dict:
+    """DSA forward for query rows ``rows`` of sequence ``b``.
+
+    inp: dict of numpy arrays in storage format (see ``numpy_inputs``).
+    Returns per-row lists: 'scores' (float64 [p+1]), 'idx' (int64 [k]),
+    'out' (float64 [H, Dv]), 'lse' (float64 [H]).
+    """
+    res = {"scores": [], "idx": [], "out": [], "lse": []}
+    for t in rows:
+        p = cfg.q_pos0 + t
+        n = p + 1
+        if with_scores or n > cfg.k:
+            sc = index_scores(inp["qI"][b, t], inp["qI_scale"][b, t], inp["w"][b, t],
+                              inp["kI"][b, :n], inp["kI_scale"][b, :n])
+        else:
+            sc = None
+        idx = topk_select(sc, cfg.k) if n > cfg.k else topk_select(np.zeros(n), cfg.k)
+        out, lse = sparse_mla(inp["q"][b, t], inp["kv"][b], idx, cfg.sm_scale, cfg.Dv)
+        res["scores"].append(sc)
+        res["idx"].append(idx)
+        res["out"].append(out)
+        res["lse"].append(lse)
+    return res
+
+
+def numpy_inputs(tensors: dict) -> dict:
+    """Torch tensors from the input generator -> numpy storage arrays.
+
+    bf16 tensors become uint16 bit patterns, e4m3 stays uint8, fp32 stays fp32.
+    Accepts tensors on any device (copies to host).
+    """
+    import torch
+
+    out = {}
+    for name, t in tensors.items():
+        t = t.detach().to("cpu")
+        if t.dtype == torch.bfloat16:
+            out[name] = t.view(torch.int16).numpy().view(np.uint16)
+        else:
+            out[name] = t.numpy()
+    return out
