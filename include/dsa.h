@@ -1,0 +1,214 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) DeepSeek Sparse Attention forward path.
+ *
+ * The method ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language
+ * Models", bud-325 paper digest, "Key claims", section 2.1 Eq. 1-2, Fig. 2, and
+ * "Method"):
+ *   1. a lightning indexer scores every causal key s of query token t as
+ *        I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])   over H_I heads, in FP8;
+ *   2. the top-k keys by I[t,:] are selected (k = 2048 in the paper);
+ *   3. MLA attention in MQA mode runs over only those k latent rows, one latent
+ *      row shared by all query heads of the token.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except in
+ *     dsa_forward_host. The library never allocates device memory; scratch
+ *     space comes from the caller's workspace. Pointers must be 16-byte aligned.
+ *   - All tensors are dense, row-major, contiguous, with the shapes given below.
+ *     FP8 e4m3 (OCP "fn" encoding) is passed as uint8_t, bf16 as uint16_t bits.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued asynchronously; a call returns once it is enqueued.
+ *   - Query row t of a sequence sits at absolute position p = q_pos0 + t and its
+ *     candidate keys are s = 0..p (requires q_pos0 + Lq <= Lk). Prefill uses
+ *     q_pos0 = 0, Lq = Lk; decode uses q_pos0 = Lk - Lq.
+ *   - Every call validates all arguments before launching anything. On failure
+ *     it returns a negative DSA_ERR_* code, launches nothing, and records a
+ *     message readable with dsa_last_error() from the same thread.
+ *   - Supported shapes: indexer (H_I, d_I) in {(4, 32), (64, 128)};
+ *     attention (H, Dqk, Dv) in {(8, 80, 64), (128, 576, 512)}; k a multiple of 32,
+ *     1 <= k <= 4096 for selection (k <= 2048 when selection and attention are
+ *     fused in dsa_forward).
+ *   - Device-side waits are bounded. A wait that runs out sets a device status
+ *     word that dsa_check_status() reads; the kernel then returns early, leaving
+ *     its outputs undefined. It never traps.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define DSA_OK 0
+#define DSA_ERR_INVALID_ARG (-1)       /* null pointer, bad size, misalignment */
+#define DSA_ERR_UNSUPPORTED_SHAPE (-2) /* valid but not one of the supported shapes */
+#define DSA_ERR_WORKSPACE_TOO_SMALL (-3)
+#define DSA_ERR_CUDA (-4)              /* a CUDA runtime/driver call failed */
+#define DSA_ERR_TIMEOUT (-5)           /* a bounded device wait ran out */
+
+/* Element type of the index weights w. */
+#define DSA_DTYPE_F32 0
+#define DSA_DTYPE_BF16 1
+
+#define DSA_MODE_PREFILL 0
+#define DSA_MODE_DECODE 1
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* dsa_last_error(void);
+
+/* Library version string. */
+const char* dsa_version(void);
+
+/*
+ * dsa_indexer_scores - lightning-indexer scores, materialised (Eq. 1).
+ *   qI        [B, Lq, H_I, d_I] e4m3 codes of the indexer queries
+ *   qI_scale  [B, Lq, H_I] fp32, > 0: dequantised q^I[t,j] = code * qI_scale[t,j]
+ *   kI        [B, Lk, d_I] e4m3 codes of the indexer keys
+ *   kI_scale  [B, Lk] fp32, > 0: dequantised k^I[s] = code * kI_scale[s]
+ *   w         [B, Lq, H_I], fp32 or bf16 (w_dtype); any sign
+ *   scores    [B, Lq, Lk] fp32 output:
+ *               scores[b,t,s] = kI_scale[s] * sum_j w[t,j] * qI_scale[t,j]
+ *                               * max(0, qhat[t,j] . khat[s])     for s <= q_pos0+t
+ *               scores[b,t,s] = -INFINITY                          for s >  q_pos0+t
+ * The whole [Lq, Lk] matrix is written; dsa_forward never materialises it.
+ */
+int dsa_indexer_scores(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
+                       const float* kI_scale, const void* w, int w_dtype, float* scores,
+                       int B, int Lq, int Lk, int q_pos0, int H_I, int d_I, void* stream);
+
+/*
+ * dsa_topk_select - fine-grained token selection ("Key claims", section 2.1;
+ * "Method": k = 2048).
+ *   scores [B, Lq, Lk] fp32 (row (b,t) reads only s <= q_pos0 + t; NaN not allowed)
+ *   idx    [B, Lq, k] int32 output: the k keys with the largest score, ties to the
+ *          lowest key index, written in ascending key order; when a row has
+ *          fewer than k candidates it selects all of them and pads with -1.
+ *          -0.0 and +0.0 compare equal.
+ */
+int dsa_topk_select(const float* scores, int32_t* idx, int B, int Lq, int Lk, int q_pos0,
+                    int k, void* stream);
+
+/*
+ * dsa_sparse_mla_workspace_size - bytes of workspace dsa_sparse_mla_fwd needs for
+ * this shape (0 when it runs without key splitting).
+ */
+size_t dsa_sparse_mla_workspace_size(int B, int Lq, int Lk, int H, int Dqk, int Dv, int k);
+
+/*
+ * dsa_sparse_mla_fwd - MLA attention in MQA mode over the selected latent rows
+ * ("Key claims", section 2.1 Eq. 2 / Fig. 2; "Method": the latent vector is shared
+ * by all query heads of a token).
+ *   q    [B, Lq, H, Dqk] bf16 queries
+ *   kv   [B, Lk, Dqk] bf16 latent rows c_s; the values are c_s[0:Dv]
+ *   idx  [B, Lq, k] int32 selected keys; entries < 0 or >= Lk are skipped
+ *   out  [B, Lq, H, Dv] bf16 output (round to nearest even from fp32):
+ *          out[h] = sum_s softmax_s(sm_scale * q[h] . c_s) * c_s[0:Dv]
+ *   lse  [B, Lq, H] fp32 natural-log log-sum-exp of the scaled logits, or NULL.
+ *        A row with no valid key gets out = 0 and lse = -INFINITY.
+ *   ws   workspace of at least dsa_sparse_mla_workspace_size(...) bytes.
+ */
+int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t* out,
+                       float* lse, int B, int Lq, int Lk, int H, int Dqk, int Dv, int k,
+                       float sm_scale, void* ws, size_t ws_bytes, void* stream);
+
+/* Whole-path problem description for dsa_forward. */
+typedef struct dsa_problem {
+  int mode;        /* DSA_MODE_PREFILL or DSA_MODE_DECODE (informational; the
+                      shape decides the schedule) */
+  int B, Lq, Lk, q_pos0;
+  int H_I, d_I;    /* indexer heads, head dim */
+  int H, Dqk, Dv;  /* attention heads, latent key width, value width */
+  int k;           /* top-k */
+  float sm_scale;
+  int w_dtype;     /* DSA_DTYPE_F32 or DSA_DTYPE_BF16 */
+} dsa_problem;
+
+/* Tensors of one dsa_forward call; shapes as in the calls above. */
+typedef struct dsa_tensors {
+  const uint8_t* qI;
+  const float* qI_scale;
+  const uint8_t* kI;
+  const float* kI_scale;
+  const void* w;
+  const uint16_t* q;
+  const uint16_t* kv;
+  uint16_t* out;    /* [B, Lq, H, Dv] bf16 */
+  float* lse;       /* [B, Lq, H] fp32, optional (NULL) */
+  int32_t* idx_out; /* [B, Lq, k] int32, optional: the selected set */
+} dsa_tensors;
+
+/* Bytes of workspace dsa_forward needs for problem p (scores are streamed in
+ * query chunks, so this is far below B*Lq*Lk*4). */
+size_t dsa_forward_workspace_size(const dsa_problem* p);
+
+/*
+ * dsa_forward - the fused hot path: indexer -> top-k -> sparse MLA, for prefill
+ * (q_pos0 = 0) and decode (q_pos0 = Lk - Lq). Query rows with p + 1 <= k select
+ * every causal key without scoring (the top-k of at most k candidates is all of
+ * them). The score matrix is produced and consumed one query chunk at a time in
+ * the workspace. Results equal dsa_indexer_scores + dsa_topk_select +
+ * dsa_sparse_mla_fwd.
+ */
+int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                void* stream);
+
+/*
+ * dsa_forward_host - dsa_forward on HOST tensors: copies every input from host
+ * memory (pinned for asynchronous copies) into the caller's device staging
+ * buffers `dev` (same layout as dsa_tensors, all device pointers), runs
+ * dsa_forward, copies out (and lse/idx_out when both host and device pointers are
+ * given) back to host, and waits for the stream. `host` holds host pointers.
+ */
+int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_tensors* dev,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Kernel kinds reported by dsa_forward_profiled. */
+#define DSA_KIND_INDEXER 1
+#define DSA_KIND_TOPK 2
+#define DSA_KIND_SPARSE_MLA 3
+#define DSA_KIND_COMBINE 4
+
+/*
+ * dsa_forward_profiled - dsa_forward that also records a CUDA event around each
+ * kernel launch, for per-kernel timing on the launching stream.
+ *   events        max_launches + 1 caller-created cudaEvent_t (as void*): events[0]
+ *                 is recorded before the first launch, events[i + 1] after launch i
+ *   kinds         [max_launches] out: DSA_KIND_* of launch i
+ *   n_launches    out: number of kernel launches made
+ * Fails with DSA_ERR_INVALID_ARG (after enqueueing part of the work) if the call
+ * needs more than max_launches launches; results are otherwise identical to
+ * dsa_forward.
+ */
+int dsa_forward_profiled(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                         void* stream, void* const* events, int* kinds, int max_launches,
+                         int* n_launches);
+
+/*
+ * dsa_check_status - wait for `stream`, then read and clear the device status
+ * word. Returns DSA_OK, DSA_ERR_TIMEOUT (a bounded wait ran out; the message names
+ * the kernel) or DSA_ERR_CUDA (a launch or execution error).
+ */
+int dsa_check_status(void* stream);
+
+/*
+ * dsa_set_wait_limit_ns - bound on every device-side wait, in nanoseconds
+ * (default 2e9). Used by tests to make a wait run out on purpose.
+ */
+int dsa_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * dsa_debug_wait_timeout - launch one small kernel that waits on an mbarrier no
+ * one arrives at, bounded by the current wait limit, so that tests can check the
+ * timeout path: afterwards dsa_check_status() returns DSA_ERR_TIMEOUT.
+ */
+int dsa_debug_wait_timeout(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

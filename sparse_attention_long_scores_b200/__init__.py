@@ -1,0 +1,331 @@
+"""Python binding of the sm_100a DeepSeek Sparse Attention forward library.
+
+Thin ctypes layer over ``libdsa.so`` (C ABI in ``include/dsa.h``): it checks
+tensor dtypes, shapes and devices, passes raw device pointers and the current
+CUDA stream, and raises on a non-zero status. Every step of the path runs in
+the library's CUDA kernels; there is no fallback. If the library is missing the
+first call raises.
+
+The computation ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language
+Models", bud-325 paper digest, "Key claims", section 2.1 Eq. 1-2; "Method"):
+    I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])      (FP8 lightning indexer)
+    S_t    = top-k_s I[t,s]                               (k = 2048)
+    out[t] = softmax(sm_scale * q[t] . c_S^T) c_S[:, :Dv] (MLA, MQA mode)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_OK = 0
+DSA_ERR_INVALID_ARG = -1
+DSA_ERR_UNSUPPORTED_SHAPE = -2
+DSA_ERR_WORKSPACE_TOO_SMALL = -3
+DSA_ERR_CUDA = -4
+DSA_ERR_TIMEOUT = -5
+DSA_DTYPE_F32 = 0
+DSA_DTYPE_BF16 = 1
+DSA_MODE_PREFILL = 0
+DSA_MODE_DECODE = 1
+
+EXPORTED = [
+    "dsa_last_error", "dsa_version", "dsa_indexer_scores", "dsa_topk_select",
+    "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_fwd", "dsa_forward_workspace_size",
+    "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
+    "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout",
+]
+KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
+
+
+class DsaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"dsa error {code}: {msg}")
+        self.code = code
+
+
+class DsaProblem(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("B", ctypes.c_int), ("Lq", ctypes.c_int),
+                ("Lk", ctypes.c_int), ("q_pos0", ctypes.c_int), ("H_I", ctypes.c_int),
+                ("d_I", ctypes.c_int), ("H", ctypes.c_int), ("Dqk", ctypes.c_int),
+                ("Dv", ctypes.c_int), ("k", ctypes.c_int), ("sm_scale", ctypes.c_float),
+                ("w_dtype", ctypes.c_int)]
+
+
+class DsaTensors(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("qI", "qI_scale", "kI", "kI_scale", "w", "q", "kv", "out", "lse", "idx_out")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libdsa.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                           "(run python -m sparse_attention_long_scores_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.dsa_last_error.restype = ctypes.c_char_p
+    L.dsa_version.restype = ctypes.c_char_p
+    L.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, i, i, vp]
+    L.dsa_topk_select.argtypes = [vp, vp, i, i, i, i, i, vp]
+    L.dsa_sparse_mla_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.dsa_sparse_mla_workspace_size.restype = sz
+    L.dsa_sparse_mla_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, ctypes.c_float,
+                                     vp, sz, vp]
+    L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
+    L.dsa_forward_workspace_size.restype = sz
+    L.dsa_forward.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp, sz, vp]
+    L.dsa_forward_host.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors),
+                                   ctypes.POINTER(DsaTensors), vp, sz, vp]
+    L.dsa_forward_profiled.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp,
+                                       sz, vp, ctypes.POINTER(ctypes.c_void_p),
+                                       ctypes.POINTER(ctypes.c_int), i, ctypes.POINTER(ctypes.c_int)]
+    L.dsa_check_status.argtypes = [vp]
+    L.dsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    L.dsa_debug_wait_timeout.argtypes = [vp]
+    for name in ("dsa_indexer_scores", "dsa_topk_select", "dsa_sparse_mla_fwd", "dsa_forward",
+                 "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status", "dsa_set_wait_limit_ns",
+                 "dsa_debug_wait_timeout"):
+        getattr(L, name).restype = i
+    _lib = L
+    return L
+
+
+def _check(code: int) -> None:
+    if code != DSA_OK:
+        raise DsaError(code, lib().dsa_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None, cuda=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _w_dtype(w: torch.Tensor) -> int:
+    if w.dtype == torch.float32:
+        return DSA_DTYPE_F32
+    if w.dtype == torch.bfloat16:
+        return DSA_DTYPE_BF16
+    raise TypeError("w must be float32 or bfloat16")
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+
+def indexer_scores(qI, qI_scale, kI, kI_scale, w, q_pos0: int = 0, scores=None, stream=None):
+    """Lightning-indexer scores [B, Lq, Lk] fp32 (-inf above the causal limit)."""
+    B, Lq, H_I, d_I = qI.shape
+    Lk = kI.shape[1]
+    _need(qI, "qI", torch.uint8, (B, Lq, H_I, d_I))
+    _need(qI_scale, "qI_scale", torch.float32, (B, Lq, H_I))
+    _need(kI, "kI", torch.uint8, (B, Lk, d_I))
+    _need(kI_scale, "kI_scale", torch.float32, (B, Lk))
+    _need(w, "w", w.dtype, (B, Lq, H_I))
+    if scores is None:
+        scores = torch.empty((B, Lq, Lk), dtype=torch.float32, device=qI.device)
+    _need(scores, "scores", torch.float32, (B, Lq, Lk))
+    _check(lib().dsa_indexer_scores(_ptr(qI), _ptr(qI_scale), _ptr(kI), _ptr(kI_scale), _ptr(w),
+                                    _w_dtype(w), _ptr(scores), B, Lq, Lk, q_pos0, H_I, d_I,
+                                    _stream(stream)))
+    return scores
+
+
+def topk_select(scores, k: int, q_pos0: int = 0, idx=None, stream=None):
+    """Top-k key indices [B, Lq, k] int32, ascending, ties to the lowest index, -1 padded."""
+    B, Lq, Lk = scores.shape
+    _need(scores, "scores", torch.float32)
+    if idx is None:
+        idx = torch.empty((B, Lq, k), dtype=torch.int32, device=scores.device)
+    _need(idx, "idx", torch.int32, (B, Lq, k))
+    _check(lib().dsa_topk_select(_ptr(scores), _ptr(idx), B, Lq, Lk, q_pos0, k, _stream(stream)))
+    return idx
+
+
+def sparse_mla_workspace_size(B, Lq, Lk, H, Dqk, Dv, k) -> int:
+    return int(lib().dsa_sparse_mla_workspace_size(B, Lq, Lk, H, Dqk, Dv, k))
+
+
+def sparse_mla_fwd(q, kv, idx, sm_scale: float, Dv: int, out=None, lse=None, ws=None,
+                   with_lse: bool = True, stream=None):
+    """Sparse MQA attention over the selected latent rows; returns (out bf16, lse fp32|None)."""
+    B, Lq, H, Dqk = q.shape
+    Lk = kv.shape[1]
+    k = idx.shape[2]
+    _need(q, "q", torch.bfloat16)
+    _need(kv, "kv", torch.bfloat16, (B, Lk, Dqk))
+    _need(idx, "idx", torch.int32, (B, Lq, k))
+    if out is None:
+        out = torch.empty((B, Lq, H, Dv), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Lq, H, Dv))
+    if lse is None and with_lse:
+        lse = torch.empty((B, Lq, H), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Lq, H))
+    need = sparse_mla_workspace_size(B, Lq, Lk, H, Dqk, Dv, k)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(lse), B, Lq, Lk,
+                                    H, Dqk, Dv, k, float(sm_scale), _ptr(ws), ws_bytes,
+                                    _stream(stream)))
+    return out, lse
+
+
+@dataclass
+class Problem:
+    B: int
+    Lq: int
+    Lk: int
+    q_pos0: int
+    H_I: int
+    d_I: int
+    H: int
+    Dqk: int
+    Dv: int
+    k: int
+    sm_scale: float
+    w_dtype: int = DSA_DTYPE_BF16
+    mode: int = DSA_MODE_PREFILL
+
+    @classmethod
+    def from_config(cls, cfg) -> "Problem":
+        return cls(B=cfg.B, Lq=cfg.Lq, Lk=cfg.Lk, q_pos0=cfg.q_pos0, H_I=cfg.H_I, d_I=cfg.d_I,
+                   H=cfg.H, Dqk=cfg.Dqk, Dv=cfg.Dv, k=cfg.k, sm_scale=cfg.sm_scale,
+                   w_dtype=DSA_DTYPE_F32 if cfg.w_dtype == "f32" else DSA_DTYPE_BF16,
+                   mode=DSA_MODE_DECODE if cfg.mode == "decode" else DSA_MODE_PREFILL)
+
+    def c(self) -> DsaProblem:
+        return DsaProblem(self.mode, self.B, self.Lq, self.Lk, self.q_pos0, self.H_I, self.d_I,
+                          self.H, self.Dqk, self.Dv, self.k, self.sm_scale, self.w_dtype)
+
+
+def forward_workspace_size(p: Problem) -> int:
+    cp = p.c()
+    n = int(lib().dsa_forward_workspace_size(ctypes.byref(cp)))
+    if n == 0:
+        raise DsaError(DSA_ERR_INVALID_ARG, lib().dsa_last_error().decode())
+    return n
+
+
+def _tensors(inp: dict, out, lse, idx_out) -> DsaTensors:
+    return DsaTensors(*[None if x is None else x.data_ptr() for x in (
+        inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"], inp["q"], inp["kv"],
+        out, lse, idx_out)])
+
+
+def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, stream=None):
+    """Whole DSA forward (indexer -> top-k -> sparse MLA) on device tensors.
+
+    inp: dict with qI, qI_scale, kI, kI_scale, w, q, kv (see ``dsa_inputs.gen_inputs``).
+    Returns out [B, Lq, H, Dv] bf16 (lse / idx_out are filled when given).
+    """
+    dev = inp["q"].device
+    _need(inp["qI"], "qI", torch.uint8, (p.B, p.Lq, p.H_I, p.d_I))
+    _need(inp["qI_scale"], "qI_scale", torch.float32, (p.B, p.Lq, p.H_I))
+    _need(inp["kI"], "kI", torch.uint8, (p.B, p.Lk, p.d_I))
+    _need(inp["kI_scale"], "kI_scale", torch.float32, (p.B, p.Lk))
+    _need(inp["w"], "w", torch.float32 if p.w_dtype == DSA_DTYPE_F32 else torch.bfloat16,
+          (p.B, p.Lq, p.H_I))
+    _need(inp["q"], "q", torch.bfloat16, (p.B, p.Lq, p.H, p.Dqk))
+    _need(inp["kv"], "kv", torch.bfloat16, (p.B, p.Lk, p.Dqk))
+    if out is None:
+        out = torch.empty((p.B, p.Lq, p.H, p.Dv), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (p.B, p.Lq, p.H, p.Dv))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (p.B, p.Lq, p.H))
+    if idx_out is not None:
+        _need(idx_out, "idx_out", torch.int32, (p.B, p.Lq, p.k))
+    if ws is None:
+        ws = torch.empty(forward_workspace_size(p), dtype=torch.uint8, device=dev)
+    cp = p.c()
+    ct = _tensors(inp, out, lse, idx_out)
+    _check(lib().dsa_forward(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+class LaunchProfiler:
+    """Events for ``forward_profiled``: one CUDA event around each kernel launch."""
+
+    def __init__(self, max_launches: int = 4096):
+        self.max = max_launches
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(max_launches + 1)]
+        self._ev = (ctypes.c_void_p * (max_launches + 1))(*[e.cuda_event for e in self.events])
+        self._kinds = (ctypes.c_int * max_launches)()
+        self.n = 0
+
+    def durations(self):
+        """[(kind name, ms)] of the last profiled call (synchronises)."""
+        self.events[self.n].synchronize()
+        return [(KIND_NAMES.get(self._kinds[i], "?"), self.events[i].elapsed_time(self.events[i + 1]))
+                for i in range(self.n)]
+
+
+def forward_profiled(p: Problem, inp: dict, out, prof: LaunchProfiler, lse=None, idx_out=None,
+                     ws=None, stream=None):
+    """``forward`` that records an event after every kernel launch into ``prof``."""
+    if ws is None:
+        ws = torch.empty(forward_workspace_size(p), dtype=torch.uint8, device=out.device)
+    cp = p.c()
+    ct = _tensors(inp, out, lse, idx_out)
+    n = ctypes.c_int(0)
+    rc = lib().dsa_forward_profiled(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream), prof._ev,
+                                    prof._kinds, prof.max, ctypes.byref(n))
+    prof.n = n.value
+    _check(rc)
+    return out
+
+
+def forward_host(p: Problem, host: dict, dev: dict, host_out, dev_out, ws, stream=None):
+    """dsa_forward on host tensors: H2D copies, forward, D2H copy of out, synchronise."""
+    cp = p.c()
+    ch = _tensors(host, host_out, None, None)
+    cd = _tensors(dev, dev_out, None, None)
+    _check(lib().dsa_forward_host(ctypes.byref(cp), ctypes.byref(ch), ctypes.byref(cd), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)))
+    return host_out
+
+
+def check_status(stream=None) -> None:
+    """Synchronise and raise DsaError if a bounded device wait ran out."""
+    _check(lib().dsa_check_status(_stream(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _check(lib().dsa_set_wait_limit_ns(int(ns)))
+
+
+def debug_wait_timeout(stream=None) -> None:
+    _check(lib().dsa_debug_wait_timeout(_stream(stream)))

@@ -1,0 +1,611 @@
+// dsa_api.cu - the C ABI declared in include/dsa.h: argument validation, TMA
+// descriptor set-up, workspace carving and the launch schedule of the DSA
+// forward path (indexer -> top-k -> sparse MLA; "DeepSeek-V3.2: Pushing the
+// Frontier of Open Large Language Models", bud-325 paper digest, "Key claims",
+// section 2.1 Eq. 1-2, and "Method").
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/dsa.h"
+#include "dsa_kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+// Bound on device-side waits; DSA_WAIT_LIMIT_NS overrides the 2 s default.
+unsigned long long initial_wait_ns() {
+  const char* e = getenv("DSA_WAIT_LIMIT_NS");
+  if (e != nullptr) {
+    unsigned long long v = strtoull(e, nullptr, 10);
+    if (v > 0) return v;
+  }
+  return 2000000000ull;
+}
+unsigned long long g_wait_ns = initial_wait_ns();
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(DSA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define DSA_TRY_CUDA(expr, what)            \
+  do {                                      \
+    cudaError_t e_ = (expr);                \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+// Device status word: [0] code, [1] site, [2] block, [3] wait id.
+__device__ int g_status[4];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+
+int device_ctl(dsa::DevCtl& ctl, int& num_sms) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_status_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    DSA_TRY_CUDA(cudaGetSymbolAddress(&p, g_status), "cudaGetSymbolAddress(status)");
+    g_status_ptr[dev] = static_cast<int*>(p);
+    int sms = 0;
+    DSA_TRY_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count");
+    int major = 0, minor = 0;
+    DSA_TRY_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "cc");
+    DSA_TRY_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "cc");
+    if (major != 10 || minor != 0)
+      return fail(DSA_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a only",
+                  dev, major, minor);
+    g_num_sms[dev] = sms;
+  }
+  ctl.status = g_status_ptr[dev];
+  ctl.wait_ns = g_wait_ns;
+  num_sms = g_num_sms[dev];
+  return DSA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D tiled tensor map over a row-major [rows, inner] array.
+int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows,
+                CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (driver too old?)");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_ptr(const void* p, const char* name, bool optional = false) {
+  if (p == nullptr) {
+    if (optional) return DSA_OK;
+    return fail(DSA_ERR_INVALID_ARG, "%s is NULL", name);
+  }
+  if (!aligned16(p)) return fail(DSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return DSA_OK;
+}
+
+#define DSA_TRY(expr)          \
+  do {                         \
+    int r_ = (expr);           \
+    if (r_ != DSA_OK) return r_; \
+  } while (0)
+
+int check_seq(int B, int Lq, int Lk, int q_pos0) {
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1 (got %d, %d, %d)", B, Lq, Lk);
+  if (q_pos0 < 0 || (long long)q_pos0 + Lq > Lk)
+    return fail(DSA_ERR_INVALID_ARG, "need 0 <= q_pos0 and q_pos0 + Lq <= Lk (q_pos0=%d Lq=%d Lk=%d)", q_pos0, Lq, Lk);
+  if ((long long)B * Lk > (1LL << 30) || (long long)B * Lq > (1LL << 30))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lk and B*Lq must be <= 2^30");
+  return DSA_OK;
+}
+
+int check_indexer_shape(int H_I, int d_I, int B, int Lq) {
+  if (!((H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 32)))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "indexer (H_I, d_I) = (%d, %d) unsupported; use (64, 128) or (4, 32)", H_I, d_I);
+  if ((long long)B * Lq * H_I > (1LL << 31) - 1)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lq*H_I too large");
+  return DSA_OK;
+}
+
+int check_mla_shape(int H, int Dqk, int Dv, int B, int Lq) {
+  if (!((H == 128 && Dqk == 576 && Dv == 512) || (H == 8 && Dqk == 80 && Dv == 64)))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "attention (H, Dqk, Dv) = (%d, %d, %d) unsupported; use (128, 576, 512) or (8, 80, 64)", H, Dqk, Dv);
+  if ((long long)B * Lq * H > (1LL << 31) - 1)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lq*H too large");
+  return DSA_OK;
+}
+
+int check_k(int k, int kmax) {
+  if (k < 32 || k > kmax || (k % 32) != 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k = %d unsupported: need a multiple of 32 in [32, %d]", k, kmax);
+  return DSA_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Optional per-launch event recording (profiling entry point only).
+struct Recorder {
+  void* const* events = nullptr;  // events[0] before the first launch, events[i+1] after launch i
+  int* kinds = nullptr;
+  int cap = 0;
+  int n = 0;
+  int mark(int kind, cudaStream_t s) {
+    if (events == nullptr) return DSA_OK;
+    if (n >= cap) return fail(DSA_ERR_INVALID_ARG, "profiling: more than %d launches", cap);
+    kinds[n] = kind;
+    ++n;
+    DSA_TRY_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(events[n]), s), "cudaEventRecord");
+    return DSA_OK;
+  }
+};
+Recorder g_no_rec;
+
+// ---------------- schedule helpers ----------------
+int indexer_piece_keys(int B, int rows, int t_blk, int keys_max, int num_sms) {
+  int nblk = (rows + t_blk - 1) / t_blk;
+  int R = 4096;
+  while (R > 128 && (long long)B * nblk * ((keys_max + R - 1) / R) < 2LL * num_sms) R /= 2;
+  return R;
+}
+
+int mla_n_dv(int Dv) { return Dv == 512 ? 2 : 1; }
+
+int mla_splits(int B, int Lq, int Dv, int k, int num_sms) {
+  long long ctas = (long long)B * Lq * mla_n_dv(Dv);
+  int tiles = k / 32;
+  if (ctas >= 2LL * num_sms) return 1;
+  int s = (int)((4LL * num_sms + ctas - 1) / ctas);
+  int max_s = tiles / 4 > 1 ? tiles / 4 : 1;
+  if (s > max_s) s = max_s;
+  if (s > 16) s = 16;
+  return s < 1 ? 1 : s;
+}
+
+size_t mla_ws_bytes(int B, int Lq, int H, int Dv, int splits) {
+  if (splits <= 1) return 0;
+  size_t tok = (size_t)B * Lq;
+  return align_up(tok * splits * H * Dv * sizeof(float), 256) +
+         align_up(tok * splits * H * 2 * sizeof(float), 256);
+}
+
+int assumed_sms() {
+  // Workspace sizing must not depend on a device being present; size for the
+  // largest schedule (fewest SMs never needs more splits than this bound).
+  return 148;
+}
+
+int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t* out, float* lse,
+            int B, int Lq, int Lk, int H, int Dqk, int Dv, int k, float sm_scale, void* ws,
+            size_t ws_bytes, const dsa::DevCtl& ctl, int num_sms, cudaStream_t stream,
+            Recorder& rec = g_no_rec) {
+  (void)num_sms;
+  int splits = mla_splits(B, Lq, Dv, k, assumed_sms());
+  size_t need = mla_ws_bytes(B, Lq, H, Dv, splits);
+  if (ws_bytes < need)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "sparse MLA workspace: need %zu bytes, got %zu", need, ws_bytes);
+  CUtensorMap tq, tkv;
+  DSA_TRY(make_map_2d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Dqk,
+                      (uint64_t)B * Lq * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  DSA_TRY(make_map_2d(&tkv, kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Dqk,
+                      (uint64_t)B * Lk, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B));
+  dsa::MlaArgs a{};
+  a.idx = idx;
+  a.out = out;
+  a.lse = lse;
+  a.B = B; a.Lq = Lq; a.Lk = Lk; a.H = H; a.Dqk = Dqk; a.Dv = Dv; a.k = k;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.n_dv = mla_n_dv(Dv);
+  a.splits = splits;
+  a.ctl = ctl;
+  if (splits > 1) {
+    size_t tok = (size_t)B * Lq;
+    a.part_o = static_cast<float*>(ws);
+    a.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                         align_up(tok * splits * H * Dv * sizeof(float), 256));
+  }
+  DSA_TRY_CUDA(dsa::launch_sparse_mla(tq, tkv, a, stream), "sparse MLA launch");
+  DSA_TRY(rec.mark(DSA_KIND_SPARSE_MLA, stream));
+  if (splits > 1) {
+    DSA_TRY_CUDA(dsa::launch_mla_combine(a, stream), "split combine launch");
+    DSA_TRY(rec.mark(DSA_KIND_COMBINE, stream));
+  }
+  return DSA_OK;
+}
+
+struct ForwardPlan {
+  int chunk;         // query rows per chunk
+  long long ld;      // score row stride (floats)
+  size_t scores_bytes, idx_bytes, mla_bytes, total;
+};
+
+ForwardPlan plan_forward(const dsa_problem* p, bool need_idx, size_t ws_bytes_or_zero) {
+  ForwardPlan f{};
+  f.ld = (long long)align_up((size_t)p->Lk, 4);
+  const size_t row_bytes = (size_t)p->B * f.ld * sizeof(float);
+  f.idx_bytes = need_idx ? align_up((size_t)p->B * p->Lq * p->k * sizeof(int32_t), 256) : 0;
+  f.mla_bytes = align_up(mla_ws_bytes(p->B, p->Lq, p->H, p->Dv,
+                                      mla_splits(p->B, p->Lq, p->Dv, p->k, assumed_sms())), 256);
+  // Rows that need scores are those with q_pos0 + t + 1 > k.
+  int first_scored = p->k - p->q_pos0;
+  if (first_scored < 0) first_scored = 0;
+  int scored_rows = p->Lq - first_scored;
+  if (scored_rows <= 0) {
+    f.chunk = p->Lq;
+    f.scores_bytes = 0;
+  } else {
+    // default: about 64 MB of scores per chunk so one chunk stays in L2
+    long long c = (64ll << 20) / (long long)row_bytes;
+    if (ws_bytes_or_zero) {
+      size_t fixed = f.idx_bytes + f.mla_bytes;
+      long long avail = ws_bytes_or_zero > fixed + 256
+                            ? (long long)((ws_bytes_or_zero - fixed - 256) / row_bytes) : 0;
+      c = avail;
+    }
+    if (c > scored_rows) c = scored_rows;
+    if (c >= 4) c &= ~3ll;
+    if (c < 1) c = 0;
+    if (!ws_bytes_or_zero && c < 4) c = scored_rows < 4 ? scored_rows : 4;
+    f.chunk = (int)c;
+    f.scores_bytes = align_up((size_t)c * row_bytes, 256);
+  }
+  f.total = f.scores_bytes + f.idx_bytes + f.mla_bytes;
+  return f;
+}
+
+// Smallest workspace dsa_forward accepts: the fixed parts plus score rows for
+// one chunk of min(4, scored rows) query rows.
+size_t min_forward_bytes(const dsa_problem* p, const ForwardPlan& f) {
+  int first_scored = p->k - p->q_pos0;
+  if (first_scored < 0) first_scored = 0;
+  int scored_rows = p->Lq - first_scored;
+  size_t rows = scored_rows <= 0 ? 0 : (size_t)(scored_rows < 4 ? scored_rows : 4);
+  if (rows == 0) return f.idx_bytes + f.mla_bytes;
+  return f.idx_bytes + f.mla_bytes + rows * (size_t)p->B * f.ld * sizeof(float) + 256;
+}
+
+int validate_problem(const dsa_problem* p) {
+  if (!p) return fail(DSA_ERR_INVALID_ARG, "problem is NULL");
+  DSA_TRY(check_seq(p->B, p->Lq, p->Lk, p->q_pos0));
+  DSA_TRY(check_indexer_shape(p->H_I, p->d_I, p->B, p->Lq));
+  DSA_TRY(check_mla_shape(p->H, p->Dqk, p->Dv, p->B, p->Lq));
+  DSA_TRY(check_k(p->k, 2048));
+  if (p->w_dtype != DSA_DTYPE_F32 && p->w_dtype != DSA_DTYPE_BF16)
+    return fail(DSA_ERR_INVALID_ARG, "w_dtype must be DSA_DTYPE_F32 or DSA_DTYPE_BF16");
+  if (!(p->sm_scale > 0.f) || !std::isfinite(p->sm_scale))
+    return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+  if (p->mode != DSA_MODE_PREFILL && p->mode != DSA_MODE_DECODE)
+    return fail(DSA_ERR_INVALID_ARG, "mode must be DSA_MODE_PREFILL or DSA_MODE_DECODE");
+  return DSA_OK;
+}
+
+int validate_tensors(const dsa_tensors* t) {
+  if (!t) return fail(DSA_ERR_INVALID_ARG, "tensors is NULL");
+  DSA_TRY(check_ptr(t->qI, "qI"));
+  DSA_TRY(check_ptr(t->qI_scale, "qI_scale"));
+  DSA_TRY(check_ptr(t->kI, "kI"));
+  DSA_TRY(check_ptr(t->kI_scale, "kI_scale"));
+  DSA_TRY(check_ptr(t->w, "w"));
+  DSA_TRY(check_ptr(t->q, "q"));
+  DSA_TRY(check_ptr(t->kv, "kv"));
+  DSA_TRY(check_ptr(t->out, "out"));
+  DSA_TRY(check_ptr(t->lse, "lse", true));
+  DSA_TRY(check_ptr(t->idx_out, "idx_out", true));
+  return DSA_OK;
+}
+
+int launch_indexer_rows(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
+                        const float* kI_scale, const void* w, int w_dtype, float* scores,
+                        long long sc_ld, long long sc_bstride, int sc_t0, int B, int Lq, int Lk,
+                        int q_pos0, int H_I, int d_I, int t_lo, int t_hi, const dsa::DevCtl& ctl,
+                        int num_sms, cudaStream_t stream, Recorder& rec = g_no_rec) {
+  if (t_hi <= t_lo) return DSA_OK;
+  const int n_tok = (H_I == 64) ? ((t_hi - t_lo == 1) ? 1 : 4) : 64;
+  CUtensorMap tq, tk;
+  DSA_TRY(make_map_2d(&tq, qI, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)d_I,
+                      (uint64_t)B * Lq * H_I, (uint32_t)d_I, (uint32_t)(n_tok * H_I),
+                      d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B));
+  DSA_TRY(make_map_2d(&tk, kI, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)d_I, (uint64_t)B * Lk,
+                      (uint32_t)d_I, 128,
+                      d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B));
+  dsa::IndexerArgs a{};
+  a.qI_scale = qI_scale;
+  a.w = w;
+  a.w_bf16 = w_dtype == DSA_DTYPE_BF16;
+  a.kI_scale = kI_scale;
+  a.scores = scores;
+  a.sc_ld = sc_ld;
+  a.sc_bstride = sc_bstride;
+  a.sc_t0 = sc_t0;
+  a.B = B; a.Lq = Lq; a.Lk = Lk; a.q_pos0 = q_pos0;
+  a.t_lo = t_lo; a.t_hi = t_hi;
+  int keys_max = q_pos0 + t_hi < Lk ? q_pos0 + t_hi : Lk;
+  a.piece_keys = indexer_piece_keys(B, t_hi - t_lo, n_tok, keys_max, num_sms);
+  a.ctl = ctl;
+  DSA_TRY_CUDA(dsa::launch_indexer(tq, tk, a, H_I, d_I, num_sms, stream), "indexer launch");
+  DSA_TRY(rec.mark(DSA_KIND_INDEXER, stream));
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_last_error(void) { return g_err.c_str(); }
+
+const char* dsa_version(void) { return "dsa-b200 0.1 (sm_100a)"; }
+
+int dsa_indexer_scores(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
+                       const float* kI_scale, const void* w, int w_dtype, float* scores, int B,
+                       int Lq, int Lk, int q_pos0, int H_I, int d_I, void* stream) {
+  DSA_TRY(check_ptr(qI, "qI"));
+  DSA_TRY(check_ptr(qI_scale, "qI_scale"));
+  DSA_TRY(check_ptr(kI, "kI"));
+  DSA_TRY(check_ptr(kI_scale, "kI_scale"));
+  DSA_TRY(check_ptr(w, "w"));
+  DSA_TRY(check_ptr(scores, "scores"));
+  DSA_TRY(check_seq(B, Lq, Lk, q_pos0));
+  DSA_TRY(check_indexer_shape(H_I, d_I, B, Lq));
+  if (w_dtype != DSA_DTYPE_F32 && w_dtype != DSA_DTYPE_BF16)
+    return fail(DSA_ERR_INVALID_ARG, "w_dtype must be DSA_DTYPE_F32 or DSA_DTYPE_BF16");
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DSA_TRY_CUDA(dsa::launch_fill_noncausal(scores, B, Lq, Lk, q_pos0, s), "fill launch");
+  return launch_indexer_rows(qI, qI_scale, kI, kI_scale, w, w_dtype, scores, Lk, Lq, 0, B, Lq, Lk,
+                             q_pos0, H_I, d_I, 0, Lq, ctl, sms, s);
+}
+
+int dsa_topk_select(const float* scores, int32_t* idx, int B, int Lq, int Lk, int q_pos0, int k,
+                    void* stream) {
+  DSA_TRY(check_ptr(scores, "scores"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_seq(B, Lq, Lk, q_pos0));
+  DSA_TRY(check_k(k, 4096));
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  dsa::TopkArgs a{};
+  a.scores = scores;
+  a.sc_ld = Lk;
+  a.sc_bstride = Lq;
+  a.sc_t0 = 0;
+  a.idx = idx;
+  a.B = B; a.Lq = Lq; a.Lk = Lk; a.q_pos0 = q_pos0; a.k = k;
+  a.t_lo = 0; a.t_hi = Lq;
+  a.vec4 = (Lk % 4) == 0;
+  a.ctl = ctl;
+  DSA_TRY_CUDA(dsa::launch_topk(a, sms, static_cast<cudaStream_t>(stream)), "top-k launch");
+  return DSA_OK;
+}
+
+size_t dsa_sparse_mla_workspace_size(int B, int Lq, int Lk, int H, int Dqk, int Dv, int k) {
+  (void)Lk; (void)Dqk;
+  if (B < 1 || Lq < 1 || k < 32) return 0;
+  return mla_ws_bytes(B, Lq, H, Dv, mla_splits(B, Lq, Dv, k, assumed_sms()));
+}
+
+int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t* out,
+                       float* lse, int B, int Lq, int Lk, int H, int Dqk, int Dv, int k,
+                       float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(check_ptr(q, "q"));
+  DSA_TRY(check_ptr(kv, "kv"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(out, "out"));
+  DSA_TRY(check_ptr(lse, "lse", true));
+  DSA_TRY(check_ptr(ws, "ws", true));
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1");
+  if ((long long)B * Lk > (1LL << 30)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lk must be <= 2^30");
+  DSA_TRY(check_mla_shape(H, Dqk, Dv, B, Lq));
+  DSA_TRY(check_k(k, 4096));
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
+    return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+  if (ws == nullptr && ws_bytes != 0) return fail(DSA_ERR_INVALID_ARG, "ws is NULL but ws_bytes > 0");
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  return run_mla(q, kv, idx, out, lse, B, Lq, Lk, H, Dqk, Dv, k, sm_scale, ws, ws_bytes, ctl, sms,
+                 static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_forward_workspace_size(const dsa_problem* p) {
+  if (validate_problem(p) != DSA_OK) return 0;
+  return plan_forward(p, true, 0).total;
+}
+
+}  // extern "C"
+
+namespace {
+int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                 void* stream, Recorder& rec) {
+  DSA_TRY(validate_problem(p));
+  DSA_TRY(validate_tensors(t));
+  DSA_TRY(check_ptr(ws, "ws", true));
+  const bool need_idx = t->idx_out == nullptr;
+  ForwardPlan rec_plan = plan_forward(p, need_idx, 0);
+  const size_t min_bytes = min_forward_bytes(p, rec_plan);
+  if (ws_bytes < min_bytes)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL,
+                "dsa_forward workspace: need at least %zu bytes (recommended %zu), got %zu",
+                min_bytes, rec_plan.total, ws_bytes);
+  if (ws == nullptr) return fail(DSA_ERR_INVALID_ARG, "ws is NULL");
+  ForwardPlan f = plan_forward(p, need_idx, ws_bytes);
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  char* wsb = static_cast<char*>(ws);
+  float* scores = reinterpret_cast<float*>(wsb);
+  int32_t* idx = need_idx ? reinterpret_cast<int32_t*>(wsb + f.scores_bytes) : t->idx_out;
+  void* mla_ws = wsb + f.scores_bytes + f.idx_bytes;
+
+  int first_scored = p->k - p->q_pos0;
+  if (first_scored < 0) first_scored = 0;
+  if (f.scores_bytes > 0 && (f.chunk < 1 || f.total > ws_bytes))
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "dsa_forward workspace: no room for one score row");
+  const int C = f.chunk > 0 ? f.chunk : p->Lq;
+  for (int t0 = 0; t0 < p->Lq; t0 += C) {
+    const int t1 = t0 + C < p->Lq ? t0 + C : p->Lq;
+    const int ts = t0 > first_scored ? t0 : first_scored;
+    if (ts < t1) {
+      DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
+                                  f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
+                                  t1, ctl, sms, s, rec));
+    }
+    dsa::TopkArgs ta{};
+    ta.scores = scores;
+    ta.sc_ld = f.ld;
+    ta.sc_bstride = C;
+    ta.sc_t0 = t0;
+    ta.idx = idx;
+    ta.B = p->B; ta.Lq = p->Lq; ta.Lk = p->Lk; ta.q_pos0 = p->q_pos0; ta.k = p->k;
+    ta.t_lo = t0; ta.t_hi = t1;
+    ta.vec4 = 1;
+    ta.ctl = ctl;
+    DSA_TRY_CUDA(dsa::launch_topk(ta, sms, s), "top-k launch");
+    DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
+  }
+  return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
+                 p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec);
+}
+}  // namespace
+
+extern "C" {
+
+int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                void* stream) {
+  Recorder none;
+  return forward_impl(p, t, ws, ws_bytes, stream, none);
+}
+
+int dsa_forward_profiled(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                         void* stream, void* const* events, int* kinds, int max_launches,
+                         int* n_launches) {
+  if (events == nullptr || kinds == nullptr || n_launches == nullptr || max_launches < 1)
+    return fail(DSA_ERR_INVALID_ARG, "profiling arrays are NULL or empty");
+  for (int i = 0; i <= max_launches; ++i)
+    if (events[i] == nullptr) return fail(DSA_ERR_INVALID_ARG, "events[%d] is NULL", i);
+  *n_launches = 0;
+  Recorder rec;
+  rec.events = events;
+  rec.kinds = kinds;
+  rec.cap = max_launches;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DSA_TRY(validate_problem(p));
+  DSA_TRY_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s), "cudaEventRecord");
+  int r = forward_impl(p, t, ws, ws_bytes, stream, rec);
+  *n_launches = rec.n;
+  return r;
+}
+
+int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_tensors* dev,
+                     void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(validate_problem(p));
+  if (!host) return fail(DSA_ERR_INVALID_ARG, "host tensors is NULL");
+  DSA_TRY(validate_tensors(dev));
+  const char* names[7] = {"host qI", "host qI_scale", "host kI", "host kI_scale", "host w", "host q", "host kv"};
+  const void* hp[7] = {host->qI, host->qI_scale, host->kI, host->kI_scale, host->w, host->q, host->kv};
+  for (int i = 0; i < 7; ++i)
+    if (hp[i] == nullptr) return fail(DSA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+  if (host->out == nullptr) return fail(DSA_ERR_INVALID_ARG, "host out is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t B = p->B, Lq = p->Lq, Lk = p->Lk;
+  const size_t wbytes = p->w_dtype == DSA_DTYPE_BF16 ? 2 : 4;
+  struct Cp { void* d; const void* h; size_t n; } in[7] = {
+      {(void*)dev->qI, host->qI, B * Lq * p->H_I * p->d_I},
+      {(void*)dev->qI_scale, host->qI_scale, B * Lq * p->H_I * 4},
+      {(void*)dev->kI, host->kI, B * Lk * p->d_I},
+      {(void*)dev->kI_scale, host->kI_scale, B * Lk * 4},
+      {(void*)dev->w, host->w, B * Lq * p->H_I * wbytes},
+      {(void*)dev->q, host->q, B * Lq * p->H * p->Dqk * 2},
+      {(void*)dev->kv, host->kv, B * Lk * p->Dqk * 2}};
+  for (auto& c : in) DSA_TRY_CUDA(cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, s), "H2D copy");
+  DSA_TRY(dsa_forward(p, dev, ws, ws_bytes, stream));
+  DSA_TRY_CUDA(cudaMemcpyAsync(host->out, dev->out, B * Lq * p->H * p->Dv * 2, cudaMemcpyDeviceToHost, s), "D2H copy");
+  if (host->lse && dev->lse)
+    DSA_TRY_CUDA(cudaMemcpyAsync(host->lse, dev->lse, B * Lq * p->H * 4, cudaMemcpyDeviceToHost, s), "D2H copy");
+  if (host->idx_out && dev->idx_out)
+    DSA_TRY_CUDA(cudaMemcpyAsync(host->idx_out, dev->idx_out, B * Lq * p->k * 4, cudaMemcpyDeviceToHost, s), "D2H copy");
+  DSA_TRY_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+  return DSA_OK;
+}
+
+int dsa_check_status(void* stream) {
+  dsa::DevCtl ctl{nullptr, 0};
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DSA_TRY_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+  DSA_TRY_CUDA(cudaGetLastError(), "pending CUDA error");
+  int st[4] = {0, 0, 0, 0};
+  DSA_TRY_CUDA(cudaMemcpy(st, ctl.status, sizeof(st), cudaMemcpyDeviceToHost), "status read");
+  if (st[0] != 0) {
+    int zero[4] = {0, 0, 0, 0};
+    DSA_TRY_CUDA(cudaMemcpy(ctl.status, zero, sizeof(zero), cudaMemcpyHostToDevice), "status clear");
+    const char* site = st[1] == dsa::kSiteIndexer ? "indexer" : st[1] == dsa::kSiteTopk ? "top-k"
+                       : st[1] == dsa::kSiteMla ? "sparse MLA" : st[1] == dsa::kSiteDebug ? "debug wait" : "?";
+    return fail(DSA_ERR_TIMEOUT, "device wait timed out in %s kernel (block %d, wait %d)", site, st[2], st[3]);
+  }
+  return DSA_OK;
+}
+
+int dsa_set_wait_limit_ns(unsigned long long ns) {
+  if (ns == 0) return fail(DSA_ERR_INVALID_ARG, "wait limit must be > 0");
+  g_wait_ns = ns;
+  return DSA_OK;
+}
+
+int dsa_debug_wait_timeout(void* stream) {
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  DSA_TRY_CUDA(dsa::launch_debug_wait(ctl, static_cast<cudaStream_t>(stream)), "debug launch");
+  return DSA_OK;
+}
+
+}  // extern "C"

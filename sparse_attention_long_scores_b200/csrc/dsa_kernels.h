@@ -1,0 +1,74 @@
+// dsa_kernels.h - host-side launch interface of the DSA kernels (internal).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+// ---------------- lightning indexer (Eq. 1) ----------------
+struct IndexerArgs {
+  const float* qI_scale;  // [B, Lq, H_I]
+  const void* w;          // [B, Lq, H_I] fp32 or bf16
+  int w_bf16;
+  const float* kI_scale;  // [B, Lk]
+  float* scores;          // row (b, t) at scores + (b * sc_bstride + t - sc_t0) * sc_ld
+  long long sc_ld;
+  long long sc_bstride;
+  int sc_t0;
+  int B, Lq, Lk, q_pos0;
+  int t_lo, t_hi;    // query rows [t_lo, t_hi) of every sequence are scored
+  int piece_keys;    // keys per work unit (multiple of 128)
+  DevCtl ctl;
+};
+
+// Launch the tcgen05 FP8 indexer for (H_I, d_I) in {(4,32), (64,128)}.
+// `decode_like` selects the one-token-per-block variant (Lq == 1).
+cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                           const IndexerArgs& a, int H_I, int d_I, int num_sms,
+                           cudaStream_t stream);
+
+// scores[b,t,s] = -inf for s > q_pos0 + t (public score matrix only).
+cudaError_t launch_fill_noncausal(float* scores, int B, int Lq, int Lk, int q_pos0,
+                                  cudaStream_t stream);
+
+// ---------------- top-k selection ----------------
+struct TopkArgs {
+  const float* scores;  // row (b, t) at scores + (b * sc_bstride + t - sc_t0) * sc_ld
+  long long sc_ld;
+  long long sc_bstride;
+  int sc_t0;
+  int32_t* idx;  // [B, Lq, k]
+  int B, Lq, Lk, q_pos0, k;
+  int t_lo, t_hi;  // rows [t_lo, t_hi) of every sequence
+  int vec4;        // rows are 16-byte aligned (sc_ld % 4 == 0, aligned base)
+  DevCtl ctl;
+};
+cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream);
+
+// ---------------- sparse MLA (MQA mode) ----------------
+struct MlaArgs {
+  const int32_t* idx;  // [B, Lq, k]
+  uint16_t* out;       // [B, Lq, H, Dv] bf16
+  float* lse;          // [B, Lq, H] or null
+  float* part_o;       // [tokens, splits, H, Dv] fp32 (splits > 1)
+  float* part_ml;      // [tokens, splits, H, 2]   (splits > 1)
+  int B, Lq, Lk, H, Dqk, Dv, k;
+  float scale_log2;    // sm_scale * log2(e)
+  int n_dv;            // value chunks per token
+  int splits;          // key splits per token
+  DevCtl ctl;
+};
+// (H, Dqk, Dv) in {(8,80,64), (128,576,512)}.
+cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
+                              const MlaArgs& a, cudaStream_t stream);
+cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t stream);
+
+// ---------------- debug ----------------
+cudaError_t launch_debug_wait(DevCtl ctl, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,350 @@
+// indexer.cu - the lightning indexer on sm_100a tensor cores.
+//
+// Computes, for query rows t of every sequence and their causal keys s <= q_pos0+t,
+//     I[t,s] = kI_scale[s] * sum_j (w[t,j] * qI_scale[t,j]) * max(0, qhat[t,j] . khat[s])
+// which is the index score of "DeepSeek-V3.2: Pushing the Frontier of Open Large
+// Language Models" (bud-325 paper digest, "Key claims", section 2.1 Eq. 1) with
+// FP8 e4m3 inputs dequantised by positive per-row scales (a positive scale
+// commutes with ReLU, so both scales move outside it exactly).
+//
+// Design (one persistent CTA per SM):
+//   * The GEMM is transposed so the head reduction needs no cross-thread
+//     traffic: A = 128 indexer keys (M, one TMEM lane each), B = T_BLK query
+//     tokens x H_I heads (N = 256, or 64 for single-token decode blocks),
+//     K = d_I. One tcgen05.mma kind::f8f6f4 per 32 bytes of K.
+//   * Warp 0 streams key tiles with TMA into a STAGES-deep ring; warp 1 issues
+//     the MMAs into two TMEM accumulators; warps 2.. are the epilogue: each
+//     thread owns one key, reads its accumulator row with tcgen05.ld, applies
+//     ReLU and the folded weight w*s^q per column, reduces over heads in
+//     registers and writes one fp32 score per (token, key). The L x L score
+//     matrix never exists in full: the caller picks the rows and key range.
+//   * Work unit = (sequence, token block, piece of `piece_keys` keys); units are
+//     dealt to CTAs round robin.
+#include "dsa_kernels.h"
+
+namespace dsa {
+namespace {
+
+template <int D_I, int H_I, int N>
+struct IdxTraits {
+  static constexpr int T_BLK = N / H_I;
+  static constexpr int KT = 128;
+  static constexpr int KTILE_BYTES = KT * D_I;
+  static constexpr int QBLK_BYTES = N * D_I;
+  static constexpr int STAGES = (D_I == 128) ? 6 : 8;
+  static constexpr int ACC = 2;
+  static constexpr int TMEM_COLS = (ACC * N <= 32) ? 32 : (ACC * N <= 64) ? 64
+                                   : (ACC * N <= 128) ? 128 : (ACC * N <= 256) ? 256 : 512;
+  static constexpr int EPI_WARPS = (T_BLK >= 2) ? 8 : 4;
+  static constexpr int EPI_THREADS = EPI_WARPS * 32;
+  static constexpr int THREADS = 64 + EPI_THREADS;
+  static constexpr uint32_t SWZ = (D_I == 128) ? 2u : 6u;   // 128B / 32B swizzle
+  static constexpr uint32_t SBO = 8u * D_I;                  // bytes per 8-row group
+  static constexpr uint32_t IDESC = make_idesc(0, 0, 0, 0, N, 128);
+  // shared memory layout (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * QBLK_BYTES;
+  static constexpr int OFF_W = OFF_K + STAGES * KTILE_BYTES;
+  static constexpr int OFF_BAR = OFF_W + 4 * N * 4;  // EPI_WARPS x (N / HALVES) floats
+  static constexpr int NUM_BARS = 2 + 2 + 2 * STAGES + 2 * ACC + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(N % 16 == 0 && N <= 256, "N");
+  static_assert(ACC * N <= 512, "TMEM");
+  static_assert(H_I >= 32 ? (H_I % 32 == 0) : (32 % H_I == 0), "heads per chunk");
+};
+
+struct Unit {
+  int b, t_a, t_b, s_lo, s_hi;
+};
+
+template <int T_BLK>
+__device__ __forceinline__ int unit_count(const IndexerArgs& a, int& nblk, int& maxp) {
+  nblk = (a.t_hi - a.t_lo + T_BLK - 1) / T_BLK;
+  int keys_max = min(a.Lk, a.q_pos0 + a.t_hi);
+  maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
+  return a.B * nblk * maxp;
+}
+
+template <int T_BLK>
+__device__ __forceinline__ bool get_unit(const IndexerArgs& a, int u, int nblk, int maxp,
+                                         Unit& o) {
+  int piece = u % maxp;
+  int rest = u / maxp;
+  int blk = rest % nblk;
+  o.b = rest / nblk;
+  o.t_a = a.t_lo + blk * T_BLK;
+  o.t_b = min(o.t_a + T_BLK, a.t_hi);
+  int keys = min(a.Lk, a.q_pos0 + o.t_b);  // keys 0 .. q_pos0 + t_b - 1
+  o.s_lo = piece * a.piece_keys;
+  o.s_hi = min(keys, o.s_lo + a.piece_keys);
+  return o.s_lo < o.s_hi;
+}
+
+template <int D_I, int H_I, int N>
+__global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                   const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs a) {
+  using Tr = IdxTraits<D_I, H_I, N>;
+  constexpr int T_BLK = Tr::T_BLK;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+
+  uint8_t* q_smem = smem + Tr::OFF_Q;
+  uint8_t* k_smem = smem + Tr::OFF_K;
+  float* wq = reinterpret_cast<float*>(smem + Tr::OFF_W);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* k_full = bars + 4;
+  uint64_t* k_empty = k_full + Tr::STAGES;
+  uint64_t* acc_full = k_empty + Tr::STAGES;
+  uint64_t* acc_empty = acc_full + Tr::ACC;
+  uint64_t* done_bar = acc_empty + Tr::ACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::OFF_MISC + 4);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < Tr::STAGES; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < Tr::ACC; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], Tr::EPI_THREADS);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_map(&tmap_q);
+    tma_prefetch_map(&tmap_k);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, Tr::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  int nblk, maxp;
+  const int total = unit_count<T_BLK>(a, nblk, maxp);
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int kst = 0, kph = 0, qb = 0, qph = 0;
+      int k_pending[Tr::STAGES];
+      for (int i = 0; i < Tr::STAGES; ++i) k_pending[i] = -1;
+      int q_pending[2] = {-1, -1};
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        Unit un;
+        if (!get_unit<T_BLK>(a, u, nblk, maxp, un)) continue;
+        if (!mbar_wait(&q_empty[qb], qph ^ 1, a.ctl, abort_flag, kSiteIndexer, 1)) { ok = false; break; }
+        q_pending[qb] = -1;
+        mbar_arrive_expect_tx(&q_full[qb], Tr::QBLK_BYTES);
+        tma_load_2d(q_smem + qb * Tr::QBLK_BYTES, &tmap_q, 0,
+                    (un.b * a.Lq + un.t_a) * H_I, &q_full[qb]);
+        q_pending[qb] = qph;
+        if (++qb == 2) { qb = 0; qph ^= 1; }
+        for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
+          if (!mbar_wait(&k_empty[kst], kph ^ 1, a.ctl, abort_flag, kSiteIndexer, 2)) { ok = false; break; }
+          k_pending[kst] = -1;
+          mbar_arrive_expect_tx(&k_full[kst], Tr::KTILE_BYTES);
+          tma_load_2d(k_smem + kst * Tr::KTILE_BYTES, &tmap_k, 0, un.b * a.Lk + s0, &k_full[kst]);
+          k_pending[kst] = kph;
+          if (++kst == Tr::STAGES) { kst = 0; kph ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        // Let copies that are still in flight land before the CTA exits.
+        DevCtl drain = a.ctl;
+        volatile int never = 0;
+        for (int i = 0; i < Tr::STAGES; ++i)
+          if (k_pending[i] >= 0) mbar_wait(&k_full[i], k_pending[i], drain, &never, kSiteIndexer, 3);
+        for (int i = 0; i < 2; ++i)
+          if (q_pending[i] >= 0) mbar_wait(&q_full[i], q_pending[i], drain, &never, kSiteIndexer, 3);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int kst = 0, kph = 0, qb = 0, qph = 0, ac = 0, aph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        Unit un;
+        if (!get_unit<T_BLK>(a, u, nblk, maxp, un)) continue;
+        if (!mbar_wait(&q_full[qb], qph, a.ctl, abort_flag, kSiteIndexer, 4)) { ok = false; break; }
+        const uint32_t q_addr = smem_u32(q_smem + qb * Tr::QBLK_BYTES);
+        for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
+          if (!mbar_wait(&k_full[kst], kph, a.ctl, abort_flag, kSiteIndexer, 5)) { ok = false; break; }
+          if (!mbar_wait(&acc_empty[ac], aph ^ 1, a.ctl, abort_flag, kSiteIndexer, 6)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(k_smem + kst * Tr::KTILE_BYTES);
+          const uint32_t d_tmem = tbase + (uint32_t)(ac * N);
+#pragma unroll
+          for (int kk = 0; kk < D_I / 32; ++kk) {
+            uint64_t ad = make_sdesc(k_addr + kk * 32, 16, Tr::SBO, Tr::SWZ);
+            uint64_t bd = make_sdesc(q_addr + kk * 32, 16, Tr::SBO, Tr::SWZ);
+            mma_f8_ss(d_tmem, ad, bd, Tr::IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&k_empty[kst]);
+          mma_commit(&acc_full[ac]);
+          if (++kst == Tr::STAGES) { kst = 0; kph ^= 1; }
+          if (++ac == Tr::ACC) { ac = 0; aph ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&q_empty[qb]);
+        if (++qb == 2) { qb = 0; qph ^= 1; }
+      }
+      // every MMA issued by this thread has completed once done_bar flips
+      mma_commit(done_bar);
+      DevCtl drain = a.ctl;
+      volatile int never = 0;
+      mbar_wait(done_bar, 0, drain, &never, kSiteIndexer, 7);
+    }
+  } else {
+    // ------------------------------------------------ epilogue
+    const int ew = warp - 2;                 // 0 .. EPI_WARPS-1
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+    constexpr int HALVES = Tr::EPI_WARPS / 4;
+    const int half = ew / 4;
+    constexpr int COLS = N / HALVES;         // columns (token x head) handled by this warp
+    const int c_begin = half * COLS;
+    const int key_in_tile = quad * 32 + lane;
+    float* wbuf = wq + ew * COLS;           // this warp's folded weights
+    const uint32_t t_lane = tbase + ((uint32_t)(quad * 32) << 16);
+    int ac = 0, aph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      Unit un;
+      if (!get_unit<T_BLK>(a, u, nblk, maxp, un)) continue;
+      // folded per-(token, head) weight w * s^q of this warp's columns, in a
+      // buffer private to the warp (no cross-warp barrier)
+      __syncwarp();
+      for (int c = c_begin + lane; c < c_begin + COLS; c += 32) {
+        int t = un.t_a + c / H_I;
+        float v = 0.f;
+        if (t < un.t_b) {
+          size_t off = ((size_t)un.b * a.Lq + t) * H_I + (c % H_I);
+          float wv = a.w_bf16 ? __uint_as_float(((uint32_t)reinterpret_cast<const uint16_t*>(a.w)[off]) << 16)
+                              : reinterpret_cast<const float*>(a.w)[off];
+          v = wv * a.qI_scale[off];
+        }
+        wbuf[c - c_begin] = v;
+      }
+      __syncwarp();
+      for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
+        if (!mbar_wait(&acc_full[ac], aph, a.ctl, abort_flag, kSiteIndexer, 8)) { ok = false; break; }
+        tc_fence_after();
+        const int s = s0 + key_in_tile;
+        const bool key_ok = s < un.s_hi;
+        const float ks = key_ok ? a.kI_scale[(size_t)un.b * a.Lk + s] : 0.f;
+        float part = 0.f;
+#pragma unroll 1
+        for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(t_lane + (uint32_t)(ac * N + c0), r);
+          tmem_wait_ld();
+          const float4* wv4 = reinterpret_cast<const float4*>(wbuf + (c0 - c_begin));
+          if constexpr (H_I >= 32) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              float4 wv = wv4[g];
+              part = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * g + 0]), 0.f), part);
+              part = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * g + 1]), 0.f), part);
+              part = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * g + 2]), 0.f), part);
+              part = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * g + 3]), 0.f), part);
+            }
+            if (((c0 + 32) % H_I) == 0) {
+              const int t = un.t_a + c0 / H_I;
+              if (key_ok && t < un.t_b && s <= a.q_pos0 + t) {
+                a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = part * ks;
+              }
+              part = 0.f;
+            }
+          } else {
+            constexpr int TPC = 32 / H_I;  // tokens per 32-column chunk
+            const float* wv = wbuf + (c0 - c_begin);
+#pragma unroll
+            for (int g = 0; g < TPC; ++g) {
+              float acc = 0.f;
+#pragma unroll
+              for (int j = 0; j < H_I; ++j)
+                acc = fmaf(wv[g * H_I + j], fmaxf(__uint_as_float(r[g * H_I + j]), 0.f), acc);
+              const int t = un.t_a + c0 / H_I + g;
+              if (key_ok && t < un.t_b && s <= a.q_pos0 + t) {
+                a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = acc * ks;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[ac]);
+        if (++ac == Tr::ACC) { ac = 0; aph ^= 1; }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Tr::TMEM_COLS);
+  }
+}
+
+template <int D_I, int H_I, int N>
+cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
+                           int num_sms, cudaStream_t stream) {
+  using Tr = IdxTraits<D_I, H_I, N>;
+  auto kern = indexer_kernel<D_I, H_I, N>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Tr::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  int nblk = (a.t_hi - a.t_lo + Tr::T_BLK - 1) / Tr::T_BLK;
+  int keys_max = a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk;
+  long long maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
+  long long units = (long long)a.B * nblk * maxp;
+  if (units <= 0) return cudaSuccess;
+  int grid = (int)(units < num_sms ? units : num_sms);
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, stream>>>(tq, tk, a);
+  return cudaGetLastError();
+}
+
+__global__ void fill_noncausal_kernel(float* scores, int B, int Lq, int Lk, int q_pos0) {
+  const long long row = blockIdx.x;  // b * Lq + t
+  const int t = (int)(row % Lq);
+  const int first = q_pos0 + t + 1;
+  float* dst = scores + row * Lk;
+  for (int s = first + (int)threadIdx.x; s < Lk; s += blockDim.x) dst[s] = -__int_as_float(0x7f800000);
+}
+
+}  // namespace
+
+cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                           const IndexerArgs& a, int H_I, int d_I, int num_sms,
+                           cudaStream_t stream) {
+  if (a.t_hi <= a.t_lo) return cudaSuccess;
+  if (H_I == 64 && d_I == 128) {
+    if (a.t_hi - a.t_lo == 1) return launch_variant<128, 64, 64>(tmap_q, tmap_k, a, num_sms, stream);
+    return launch_variant<128, 64, 256>(tmap_q, tmap_k, a, num_sms, stream);
+  }
+  if (H_I == 4 && d_I == 32) return launch_variant<32, 4, 256>(tmap_q, tmap_k, a, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fill_noncausal(float* scores, int B, int Lq, int Lk, int q_pos0,
+                                  cudaStream_t stream) {
+  long long rows = (long long)B * Lq;
+  if (rows == 0) return cudaSuccess;
+  fill_noncausal_kernel<<<(unsigned)rows, 256, 0, stream>>>(scores, B, Lq, Lk, q_pos0);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

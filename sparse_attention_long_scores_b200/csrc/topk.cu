@@ -1,0 +1,214 @@
+// topk.cu - fine-grained token selection: the k largest index scores of each
+// query row ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language Models",
+// bud-325 paper digest, "Key claims", section 2.1, and "Method": k = 2048 key-value
+// entries per query token).
+//
+// One CTA per query row. Scores are mapped to order-preserving 32-bit keys
+// (-0.0 folded onto +0.0) and the exact k-th largest key T is found by a
+// three-digit radix select (11 + 11 + 10 bits, most significant first): each
+// pass histograms the keys that still match the selected prefix in shared
+// memory and a block scan picks the digit where the running count from the top
+// crosses k. A final ordered pass writes every key > T and the first
+// (k - #{key > T}) keys == T, in ascending index order: one block-wide scan of
+// packed (greater, equal) counts per 4096 candidates gives every element its
+// output slot. Ties therefore go to the lowest index and the output is sorted.
+// Rows of up to 48K candidates are staged once in shared memory as keys;
+// longer rows are re-read from global memory (L2) on each pass.
+// Rows with at most k candidates select all of them and pad with -1.
+#include "dsa_kernels.h"
+
+namespace dsa {
+namespace {
+
+constexpr int TK_THREADS = 512;
+constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_ITEMS = 8;                       // contiguous elements per thread, output pass
+constexpr int TK_SMEM_MAX = 48 * 1024;            // candidates staged in shared memory
+
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;                   // -0.0 == +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive block scan of one int per thread; also returns the block total.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t& total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) tmp[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t x = lane < TK_WARPS ? tmp[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t n = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += n;
+    }
+    if (lane < TK_WARPS) tmp[lane] = x;
+  }
+  __syncthreads();
+  uint32_t off = wid > 0 ? tmp[wid - 1] : 0u;
+  total = tmp[TK_WARPS - 1];
+  __syncthreads();
+  return off + incl - v;
+}
+
+template <bool SMEM_ROW>
+struct RowSrc {
+  const uint32_t* keys;  // shared-memory keys (SMEM_ROW)
+  const float* src;      // global scores
+  __device__ __forceinline__ uint32_t operator()(int i) const {
+    if constexpr (SMEM_ROW) return keys[i];
+    else return score_key(__ldg(src + i));
+  }
+};
+
+// One radix pass: histogram digit (key >> shift) & (nbins-1) of keys whose bits
+// above `shift + bits` equal `prefix`; then find the digit holding the `need`-th
+// largest key. Updates prefix/need in place (uniform across the block).
+template <bool SMEM_ROW, int BITS>
+__device__ __forceinline__ void radix_pass(const RowSrc<SMEM_ROW>& row, int n, int shift,
+                                           bool first, uint32_t& prefix, uint32_t& need,
+                                           uint32_t* hist, uint32_t* tmp, uint32_t* sel) {
+  constexpr int NB = 1 << BITS;
+  constexpr int BPT = NB / TK_THREADS;  // bins per thread
+  static_assert(BPT >= 1, "bins");
+  for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
+  __syncthreads();
+  const int hi_shift = shift + BITS;
+  for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+    uint32_t key = row(i);
+    if (first || (key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (NB - 1)], 1u);
+  }
+  __syncthreads();
+  uint32_t local = 0;
+  const int b0 = threadIdx.x * BPT;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) local += hist[b0 + j];
+  uint32_t total;
+  uint32_t before = block_excl_scan(local, tmp, total);
+  uint32_t above = total - before - local;  // keys in bins of higher-numbered threads
+#pragma unroll
+  for (int j = BPT - 1; j >= 0; --j) {
+    uint32_t h = hist[b0 + j];
+    if (above < need && need <= above + h) {
+      sel[0] = (uint32_t)(b0 + j);
+      sel[1] = need - above;
+    }
+    above += h;
+  }
+  __syncthreads();
+  prefix = first ? sel[0] : ((prefix << BITS) | sel[0]);
+  need = sel[1];
+  __syncthreads();
+}
+
+template <bool SMEM_ROW>
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
+  extern __shared__ uint32_t row_keys[];
+  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t tmp[32];
+  __shared__ uint32_t sel[2];
+  const int rows_per_b = a.t_hi - a.t_lo;
+  const long long nrows = (long long)a.B * rows_per_b;
+  for (long long r = blockIdx.x; r < nrows; r += gridDim.x) {
+    const int b = (int)(r / rows_per_b);
+    const int t = a.t_lo + (int)(r % rows_per_b);
+    const int n = min(a.Lk, a.q_pos0 + t + 1);
+    int32_t* dst = a.idx + ((long long)b * a.Lq + t) * a.k;
+    if (n <= a.k) {
+      for (int i = threadIdx.x; i < a.k; i += TK_THREADS) dst[i] = i < n ? i : -1;
+      continue;
+    }
+    const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld;
+    if constexpr (SMEM_ROW) {
+      for (int i = threadIdx.x; i < n; i += TK_THREADS) row_keys[i] = score_key(__ldg(src + i));
+      __syncthreads();
+    }
+    RowSrc<SMEM_ROW> row{row_keys, src};
+    uint32_t prefix = 0, need = (uint32_t)a.k;
+    radix_pass<SMEM_ROW, 11>(row, n, 21, true, prefix, need, hist, tmp, sel);
+    radix_pass<SMEM_ROW, 11>(row, n, 10, false, prefix, need, hist, tmp, sel);
+    radix_pass<SMEM_ROW, 10>(row, n, 0, false, prefix, need, hist, tmp, sel);
+    const uint32_t T = prefix;
+    const uint32_t need_eq = need;  // keys equal to T that are selected (lowest indices first)
+
+    uint32_t g_run = 0, e_run = 0;
+    for (int base = 0; base < n; base += TK_THREADS * TK_ITEMS) {
+      const int i0 = base + threadIdx.x * TK_ITEMS;
+      uint32_t keys[TK_ITEMS];
+      bool full = i0 + TK_ITEMS <= n;
+      if constexpr (!SMEM_ROW) {
+        if (full && a.vec4) {
+          float4 v0 = __ldg(reinterpret_cast<const float4*>(src + i0));
+          float4 v1 = __ldg(reinterpret_cast<const float4*>(src + i0 + 4));
+          keys[0] = score_key(v0.x); keys[1] = score_key(v0.y);
+          keys[2] = score_key(v0.z); keys[3] = score_key(v0.w);
+          keys[4] = score_key(v1.x); keys[5] = score_key(v1.y);
+          keys[6] = score_key(v1.z); keys[7] = score_key(v1.w);
+        } else {
+#pragma unroll
+          for (int j = 0; j < TK_ITEMS; ++j) keys[j] = (i0 + j < n) ? row(i0 + j) : 0u;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < TK_ITEMS; ++j) keys[j] = (i0 + j < n) ? row_keys[i0 + j] : 0u;
+      }
+      uint32_t g = 0, e = 0;
+#pragma unroll
+      for (int j = 0; j < TK_ITEMS; ++j) {
+        if (i0 + j < n) {
+          g += keys[j] > T;
+          e += keys[j] == T;
+        }
+      }
+      uint32_t total;
+      uint32_t excl = block_excl_scan((e << 16) | g, tmp, total);
+      uint32_t G = g_run + (excl & 0xFFFFu);
+      uint32_t E = e_run + (excl >> 16);
+#pragma unroll
+      for (int j = 0; j < TK_ITEMS; ++j) {
+        if (i0 + j < n) {
+          if (keys[j] > T) {
+            dst[G + min(E, need_eq)] = i0 + j;
+            ++G;
+          } else if (keys[j] == T) {
+            if (E < need_eq) dst[G + E] = i0 + j;
+            ++E;
+          }
+        }
+      }
+      g_run += total & 0xFFFFu;
+      e_run += total >> 16;
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream) {
+  const int rows_per_b = a.t_hi - a.t_lo;
+  if (rows_per_b <= 0 || a.B <= 0) return cudaSuccess;
+  long long nrows = (long long)a.B * rows_per_b;
+  const int n_max = a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk;
+  unsigned grid = (unsigned)(nrows < (1LL << 30) ? nrows : (1LL << 30));
+  if (n_max <= TK_SMEM_MAX) {
+    size_t smem = (size_t)((n_max + 3) & ~3) * 4;
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_kernel<true><<<grid, TK_THREADS, smem, stream>>>(a);
+  } else {
+    topk_kernel<false><<<grid, TK_THREADS, 0, stream>>>(a);
+  }
+  (void)num_sms;
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

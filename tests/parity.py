@@ -1,0 +1,84 @@
+"""Comparison helpers for the GPU-vs-oracle parity tests.
+
+Tolerances (written here once, used by every parity test):
+  * scores:    |I_gpu - I_ref| <= 1e-3 * max(|I_ref|, 1e-3 * max_s |I_ref[t, :]|)
+  * selection: identical sets, except keys whose oracle score lies within 1e-3
+               (relative) of the oracle k-th score; the GPU set must still hold
+               exactly min(k, p+1) unique causal keys, ascending, -1 padded
+  * attention: max-abs <= 2e-2, mean-abs <= 2e-3, relative L2 <= 1e-2 per row,
+               and |o_gpu| > 0.5 |o_ref| (an all-zero output would otherwise pass);
+               lse within 1e-4 absolute.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+SCORE_RTOL = 1e-3
+BAND_RTOL = 1e-3
+ATT_MAX_ABS = 2e-2
+ATT_MEAN_ABS = 2e-3
+ATT_REL_L2 = 1e-2
+LSE_ABS = 1e-4
+
+
+def check_scores(gpu_row: np.ndarray, ref_row: np.ndarray, where=""):
+    ref = np.asarray(ref_row, np.float64)
+    got = np.asarray(gpu_row, np.float64)
+    floor = 1e-3 * np.abs(ref).max() if ref.size else 0.0
+    tol = SCORE_RTOL * np.maximum(np.abs(ref), floor)
+    err = np.abs(got - ref)
+    bad = np.nonzero(err > tol)[0]
+    assert bad.size == 0, (f"{where}: {bad.size} scores out of tolerance, first s={bad[0]} "
+                           f"gpu={got[bad[0]]} ref={ref[bad[0]]}")
+
+
+def check_selection(gpu_idx: np.ndarray, ref_scores, ref_idx: np.ndarray, k: int, p: int, where=""):
+    gpu_idx = np.asarray(gpu_idx, np.int64)
+    n = p + 1
+    v = gpu_idx[gpu_idx >= 0]
+    m = min(k, n)
+    assert len(v) == m, f"{where}: {len(v)} selected, expected {m}"
+    assert (gpu_idx[m:] == -1).all(), f"{where}: padding"
+    assert (np.diff(v) > 0).all(), f"{where}: not ascending/unique"
+    assert v.min() >= 0 and v.max() <= p, f"{where}: non-causal index"
+    r = ref_idx[ref_idx >= 0]
+    if n <= k:
+        assert np.array_equal(v, np.arange(n)), f"{where}: short row must select every key"
+        return 0
+    sc = np.asarray(ref_scores, np.float64)
+    kth = np.sort(sc)[::-1][k - 1]
+    band = np.abs(sc - kth) <= BAND_RTOL * abs(kth)
+    diff = np.setxor1d(v, r)
+    outside = diff[~band[diff]]
+    assert outside.size == 0, (f"{where}: {outside.size} selection differences outside the tie band, "
+                               f"e.g. s={outside[:5]} scores={sc[outside[:5]]} kth={kth}")
+    return int(diff.size)
+
+
+def check_attention(gpu_out, ref_out, gpu_lse=None, ref_lse=None, where=""):
+    g = np.asarray(gpu_out, np.float64)
+    r = np.asarray(ref_out, np.float64)
+    err = np.abs(g - r)
+    assert err.max() <= ATT_MAX_ABS, f"{where}: max abs err {err.max()}"
+    assert err.mean() <= ATT_MEAN_ABS, f"{where}: mean abs err {err.mean()}"
+    rn = np.linalg.norm(r, axis=-1)
+    en = np.linalg.norm(g - r, axis=-1)
+    ok = rn > 0
+    if ok.any():
+        rel = (en[ok] / rn[ok]).max()
+        assert rel <= ATT_REL_L2, f"{where}: rel L2 err {rel}"
+        assert (np.linalg.norm(g, axis=-1)[ok] > 0.5 * rn[ok]).all(), f"{where}: output collapsed"
+    if gpu_lse is not None and ref_lse is not None:
+        gl = np.asarray(gpu_lse, np.float64)
+        rl = np.asarray(ref_lse, np.float64)
+        fin = np.isfinite(rl)
+        assert np.array_equal(np.isfinite(gl), fin), f"{where}: lse finiteness"
+        if fin.any():
+            lerr = np.abs(gl[fin] - rl[fin]).max()
+            assert lerr <= LSE_ABS, f"{where}: lse err {lerr}"
+    return float(err.max())
+
+
+def bf16_to_f64(t) -> np.ndarray:
+    import torch
+    return t.detach().to("cpu", torch.float32).double().numpy()

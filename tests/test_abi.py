@@ -1,0 +1,129 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before touching a GPU (no device needed)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import sparse_attention_long_scores_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_attention_long_scores_b200.build import build
+    build()
+    return dsa.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(dsa_[a-z0-9_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("dsa_indexer_scores", "dsa_topk_select", "dsa_sparse_mla_fwd", "dsa_forward",
+              "dsa_forward_workspace_size", "dsa_last_error", "dsa_check_status"):
+        assert n in names
+    assert sorted(dsa.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert L.dsa_version().decode().startswith("dsa-b200")
+
+
+FAKE = 0x10000   # aligned, never dereferenced: validation fails first
+
+
+def test_indexer_rejects_bad_args(L):
+    p = ctypes.c_void_p(FAKE)
+    # unsupported indexer shape
+    rc = L.dsa_indexer_scores(p, p, p, p, p, 0, p, 1, 8, 8, 0, 32, 64, None)
+    assert rc == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert "unsupported" in L.dsa_last_error().decode()
+    # null pointer
+    rc = L.dsa_indexer_scores(None, p, p, p, p, 0, p, 1, 8, 8, 0, 4, 32, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG and "qI" in L.dsa_last_error().decode()
+    # misaligned
+    rc = L.dsa_indexer_scores(ctypes.c_void_p(FAKE + 4), p, p, p, p, 0, p, 1, 8, 8, 0, 4, 32, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG and "aligned" in L.dsa_last_error().decode()
+    # causal window outside the keys
+    rc = L.dsa_indexer_scores(p, p, p, p, p, 0, p, 1, 8, 8, 1, 4, 32, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+    # bad w dtype
+    rc = L.dsa_indexer_scores(p, p, p, p, p, 7, p, 1, 8, 8, 0, 4, 32, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_topk_rejects_bad_k(L):
+    p = ctypes.c_void_p(FAKE)
+    for k in (0, 16, 33, 8192):
+        assert L.dsa_topk_select(p, p, 1, 8, 8, 0, k, None) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert L.dsa_topk_select(p, None, 1, 8, 8, 0, 32, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_sparse_mla_rejects_bad_args(L):
+    p = ctypes.c_void_p(FAKE)
+    rc = L.dsa_sparse_mla_fwd(p, p, p, p, None, 1, 4, 8, 16, 80, 64, 32, 0.1, None, 0, None)
+    assert rc == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    rc = L.dsa_sparse_mla_fwd(p, p, p, p, None, 1, 4, 8, 8, 80, 64, 32, -1.0, None, 0, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+    rc = L.dsa_sparse_mla_fwd(p, p, p, p, None, 1, 4, 8, 8, 80, 64, 32, float("nan"), None, 0, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(L):
+    from dsa_inputs import CONFIGS
+    for name, cfg in CONFIGS.items():
+        p = dsa.Problem.from_config(cfg)
+        n = dsa.forward_workspace_size(p)
+        assert n > 0
+        # never anywhere near the full score matrix
+        full = cfg.B * cfg.Lq * cfg.Lk * 4
+        idx = cfg.B * cfg.Lq * cfg.k * 4
+        assert n < idx + max(full // 8, 256 << 20), name
+    # decode splits keys: needs a partial-output buffer
+    d = CONFIGS["decode_128k"]
+    assert dsa.sparse_mla_workspace_size(d.B, d.Lq, d.Lk, d.H, d.Dqk, d.Dv, d.k) > 0
+    pf = CONFIGS["prefill_32k"]
+    assert dsa.sparse_mla_workspace_size(pf.B, pf.Lq, pf.Lk, pf.H, pf.Dqk, pf.Dv, pf.k) == 0
+
+
+def test_forward_rejects_bad_problem(L):
+    from dsa_inputs import CONFIGS
+    p = dsa.Problem.from_config(CONFIGS["tiny"])
+    p.k = 4096
+    cp = p.c()
+    assert L.dsa_forward_workspace_size(ctypes.byref(cp)) == 0
+    assert "k = 4096" in L.dsa_last_error().decode()
+    p = dsa.Problem.from_config(CONFIGS["tiny"])
+    cp = p.c()
+    t = dsa.DsaTensors(*([FAKE] * 8 + [None, None]))
+    rc = L.dsa_forward(ctypes.byref(cp), ctypes.byref(t), ctypes.c_void_p(FAKE), 16, None)
+    assert rc == dsa.DSA_ERR_WORKSPACE_TOO_SMALL
+    t.kv = None
+    rc = L.dsa_forward(ctypes.byref(cp), ctypes.byref(t), ctypes.c_void_p(FAKE), 1 << 30, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG and "kv" in L.dsa_last_error().decode()
+
+
+def test_wait_limit_validation(L):
+    assert L.dsa_set_wait_limit_ns(0) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_set_wait_limit_ns(2_000_000_000) == dsa.DSA_OK
+
+
+def test_no_cpu_fallback_in_binding():
+    """The binding has no compute of its own: every entry calls into the library."""
+    src = open(os.path.join(ROOT, "sparse_attention_long_scores_b200", "__init__.py")).read()
+    assert "import oracle" not in src and "from oracle" not in src
+    for banned in ("torch.topk", "torch.softmax", "torch.matmul", "@ ", "einsum"):
+        assert banned not in src, banned

@@ -1,0 +1,324 @@
+"""GPU parity: every kernel of the path against the fp64 oracle, through the C ABI.
+
+Small cases are compared element by element in full; the full-size workloads
+are compared on sampled query rows (the oracle computes them one by one), with
+``dsa_forward`` run in the launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as ORC
+import sparse_attention_long_scores_b200 as dsa
+from dsa_inputs import CONFIGS, gen_inputs, sample_rows
+from parity import bf16_to_f64, check_attention, check_scores, check_selection
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    from sparse_attention_long_scores_b200.build import build
+    build()
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+
+
+def _u16(t):
+    return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _np(t):
+    t = t.detach().to("cpu").contiguous()
+    return _u16(t) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+class Rows:
+    """Oracle evaluation of single query rows, copying only the slices it needs."""
+
+    def __init__(self, cfg, inp):
+        self.cfg, self.inp = cfg, inp
+        self._seq = {}
+
+    def seq(self, b):
+        if b not in self._seq:
+            self._seq = {b: (_np(self.inp["kI"][b]), _np(self.inp["kI_scale"][b]))}
+        return self._seq[b]
+
+    def scores(self, b, t):
+        cfg, inp = self.cfg, self.inp
+        n = cfg.q_pos0 + t + 1
+        kI, ks = self.seq(b)
+        return ORC.index_scores(_np(inp["qI"][b, t]), _np(inp["qI_scale"][b, t]),
+                                _np(inp["w"][b, t]), kI[:n], ks[:n])
+
+    def attention(self, b, t, idx):
+        """Oracle attention of row (b, t) over the key set ``idx`` (int array)."""
+        idx = np.asarray(idx)
+        v = idx[(idx >= 0) & (idx < self.cfg.Lk)]
+        if v.size == 0:
+            return ORC.sparse_mla(_np(self.inp["q"][b, t]), np.zeros((1, self.cfg.Dqk), np.uint16),
+                                  np.array([-1]), self.cfg.sm_scale, self.cfg.Dv)
+        rows = _np(self.inp["kv"][b][torch.as_tensor(v, device=self.inp["kv"].device)])
+        return ORC.sparse_mla(_np(self.inp["q"][b, t]), rows, np.arange(v.size), self.cfg.sm_scale,
+                              self.cfg.Dv)
+
+
+def _forward(cfg, inp, ws=None):
+    p = dsa.Problem.from_config(cfg)
+    out = torch.empty((cfg.B, cfg.Lq, cfg.H, cfg.Dv), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((cfg.B, cfg.Lq, cfg.H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.int32, device="cuda")
+    dsa.forward(p, inp, out=out, lse=lse, idx_out=idx, ws=ws)
+    dsa.check_status()
+    return out, lse, idx
+
+
+# ---------------------------------------------------------------------------
+# tiny workload: everything, every row
+# ---------------------------------------------------------------------------
+
+
+def test_tiny_all_stages_full():
+    cfg = CONFIGS["tiny"]
+    inp = gen_inputs(cfg, "cuda")
+    host = ORC.numpy_inputs(inp)
+    # indexer: the whole score matrix, -inf above the diagonal
+    sc = dsa.indexer_scores(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"])
+    dsa.check_status()
+    sc_h = sc.cpu().numpy()
+    ref = ORC.forward_rows(host, cfg, 0, range(cfg.Lq))
+    for t in range(cfg.Lq):
+        check_scores(sc_h[0, t, :t + 1], ref["scores"][t], f"t={t}")
+        assert np.all(np.isneginf(sc_h[0, t, t + 1:]))
+    # top-k on the GPU scores
+    idx = dsa.topk_select(sc, cfg.k)
+    dsa.check_status()
+    idx_h = idx.cpu().numpy()
+    for t in range(cfg.Lq):
+        check_selection(idx_h[0, t], ref["scores"][t], ref["idx"][t], cfg.k, t, f"t={t}")
+    # sparse MLA on the oracle's selection
+    ref_idx = torch.as_tensor(np.stack(ref["idx"])[None].astype(np.int32), device="cuda")
+    out, lse = dsa.sparse_mla_fwd(inp["q"], inp["kv"], ref_idx, cfg.sm_scale, cfg.Dv)
+    dsa.check_status()
+    check_attention(bf16_to_f64(out[0]), np.stack(ref["out"]), lse[0].cpu().numpy(),
+                    np.stack(ref["lse"]), "mla")
+    # fused forward: selection, then attention over the GPU's own selection
+    out, lse, idx = _forward(cfg, inp)
+    idx_h = idx.cpu().numpy()
+    rows = Rows(cfg, inp)
+    ro, rl = [], []
+    for t in range(cfg.Lq):
+        check_selection(idx_h[0, t], ref["scores"][t], ref["idx"][t], cfg.k, t, f"fwd t={t}")
+        o, l = rows.attention(0, t, idx_h[0, t])
+        ro.append(o)
+        rl.append(l)
+    check_attention(bf16_to_f64(out[0]), np.stack(ro), lse[0].cpu().numpy(), np.stack(rl), "fwd")
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 31, 32, 33, 257, 300])
+def test_tiny_odd_lengths(L):
+    cfg = CONFIGS["tiny"].with_(Lq=L, Lk=L, name="tiny")
+    inp = gen_inputs(cfg, "cuda", seed=77 + L)
+    host = ORC.numpy_inputs(inp)
+    ref = ORC.forward_rows(host, cfg, 0, range(L))
+    sc = dsa.indexer_scores(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"])
+    out, lse, idx = _forward(cfg, inp)
+    sc_h, idx_h = sc.cpu().numpy(), idx.cpu().numpy()
+    rows = Rows(cfg, inp)
+    ro, rl = [], []
+    for t in range(L):
+        check_scores(sc_h[0, t, :t + 1], ref["scores"][t], f"L={L} t={t}")
+        check_selection(idx_h[0, t], ref["scores"][t], ref["idx"][t], cfg.k, t, f"L={L} t={t}")
+        o, l = rows.attention(0, t, idx_h[0, t])
+        ro.append(o)
+        rl.append(l)
+    check_attention(bf16_to_f64(out[0]), np.stack(ro), lse[0].cpu().numpy(), np.stack(rl), f"L={L}")
+
+
+def test_tiny_decode_and_batch():
+    """Batched decode shape on tiny dims: B=5, Lq=1 against 300 cached keys, plus a
+    chunked prefill continuation (q_pos0 > 0, Lq = 40)."""
+    for cfg in (CONFIGS["tiny"].with_(B=5, Lq=1, Lk=300, q_pos0=299, mode="decode"),
+                CONFIGS["tiny"].with_(B=2, Lq=40, Lk=100, q_pos0=60)):
+        inp = gen_inputs(cfg, "cuda", seed=5)
+        host = ORC.numpy_inputs(inp)
+        out, lse, idx = _forward(cfg, inp)
+        idx_h = idx.cpu().numpy()
+        rows = Rows(cfg, inp)
+        for b in range(cfg.B):
+            ref = ORC.forward_rows(host, cfg, b, range(cfg.Lq))
+            ro, rl = [], []
+            for t in range(cfg.Lq):
+                p = cfg.q_pos0 + t
+                check_selection(idx_h[b, t], ref["scores"][t], ref["idx"][t], cfg.k, p, f"b={b} t={t}")
+                o, l = rows.attention(b, t, idx_h[b, t])
+                ro.append(o)
+                rl.append(l)
+            check_attention(bf16_to_f64(out[b]), np.stack(ro), lse[b].cpu().numpy(), np.stack(rl),
+                            f"b={b}")
+
+
+# ---------------------------------------------------------------------------
+# top-k edge cases
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("Lk,k,levels", [(3000, 2048, 4), (5000, 64, 0), (70000, 2048, 0),
+                                          (70000, 256, 3), (40000, 32, 1)])
+def test_topk_exact_ties_and_long_rows(Lk, k, levels):
+    """Scores with many exact ties (levels > 0 distinct values) must select the
+    lowest indices exactly; long rows exercise the global-memory path."""
+    g = torch.Generator(device="cuda").manual_seed(Lk + k)
+    B, Lq = 1, 3
+    q_pos0 = Lk - Lq
+    if levels:
+        sc = torch.randint(0, levels, (B, Lq, Lk), generator=g, device="cuda").float()
+        sc[..., ::7] = -0.0 if levels == 1 else sc[..., ::7]
+    else:
+        sc = torch.randn((B, Lq, Lk), generator=g, device="cuda")
+    idx = dsa.topk_select(sc, k, q_pos0=q_pos0)
+    dsa.check_status()
+    sc_h = sc.cpu().double().numpy()
+    idx_h = idx.cpu().numpy()
+    for t in range(Lq):
+        p = q_pos0 + t
+        ref = ORC.topk_select(sc_h[0, t, :p + 1], k)
+        assert np.array_equal(idx_h[0, t], ref), f"t={t}"
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads on sampled rows
+# ---------------------------------------------------------------------------
+
+
+def _check_big(cfg, n_rows, score_blocks=2):
+    inp = gen_inputs(cfg, "cuda")
+    out, lse, idx = _forward(cfg, inp)
+    rows = Rows(cfg, inp)
+    samples = sample_rows(cfg, n_rows)
+    n_band = 0
+    for b in range(cfg.B):
+        ro, rl, go, gl = [], [], [], []
+        for t in samples:
+            p = cfg.q_pos0 + t
+            gidx = idx[b, t].cpu().numpy()
+            if p + 1 > cfg.k:
+                sc = rows.scores(b, t)
+                ref_idx = ORC.topk_select(sc, cfg.k)
+            else:
+                sc, ref_idx = None, ORC.topk_select(np.zeros(p + 1), cfg.k)
+            n_band += check_selection(gidx, sc, ref_idx, cfg.k, p, f"{cfg.name} b={b} t={t}")
+            o, l = rows.attention(b, t, gidx)
+            ro.append(o)
+            rl.append(l)
+            go.append(bf16_to_f64(out[b, t]))
+            gl.append(lse[b, t].cpu().numpy())
+        check_attention(np.stack(go), np.stack(ro), np.stack(gl), np.stack(rl), f"{cfg.name} b={b}")
+    # indexer scores on blocks of rows through the public score entry point
+    for b in range(min(cfg.B, 2)):
+        for t0 in [samples[len(samples) // 2], samples[-1] - 7][:score_blocks]:
+            t0 = max(0, min(t0, cfg.Lq - 8))
+            nq = min(8, cfg.Lq)
+            sl = slice(t0, t0 + nq)
+            qpos = cfg.q_pos0 + t0
+            sc = dsa.indexer_scores(inp["qI"][b:b + 1, sl].contiguous(),
+                                    inp["qI_scale"][b:b + 1, sl].contiguous(), inp["kI"][b:b + 1],
+                                    inp["kI_scale"][b:b + 1], inp["w"][b:b + 1, sl].contiguous(),
+                                    q_pos0=qpos)
+            sc_h = sc.cpu().numpy()
+            for i in range(nq):
+                t = t0 + i
+                p = cfg.q_pos0 + t
+                check_scores(sc_h[0, i, :p + 1], rows.scores(b, t), f"{cfg.name} scores b={b} t={t}")
+    del inp, out, lse, idx
+    torch.cuda.empty_cache()
+    return n_band
+
+
+def test_prefill_8k():
+    _check_big(CONFIGS["prefill_8k"], 48)
+
+
+def test_prefill_32k_batch2():
+    _check_big(CONFIGS["prefill_32k"], 24)
+
+
+def test_prefill_128k():
+    _check_big(CONFIGS["prefill_128k"], 16)
+
+
+def test_decode_128k():
+    cfg = CONFIGS["decode_128k"]
+    inp = gen_inputs(cfg, "cuda")
+    out, lse, idx = _forward(cfg, inp)
+    rows = Rows(cfg, inp)
+    go, gl, ro, rl = [], [], [], []
+    for b in range(cfg.B):
+        gidx = idx[b, 0].cpu().numpy()
+        sc = rows.scores(b, 0)
+        check_selection(gidx, sc, ORC.topk_select(sc, cfg.k), cfg.k, cfg.q_pos0, f"decode b={b}")
+        o, l = rows.attention(b, 0, gidx)
+        ro.append(o)
+        rl.append(l)
+        go.append(bf16_to_f64(out[b, 0]))
+        gl.append(lse[b, 0].cpu().numpy())
+    check_attention(np.stack(go), np.stack(ro), np.stack(gl), np.stack(rl), "decode")
+
+
+# ---------------------------------------------------------------------------
+# invariances, determinism, bounded waits
+# ---------------------------------------------------------------------------
+
+
+def test_unselected_rows_do_not_matter_and_determinism():
+    cfg = CONFIGS["tiny"].with_(Lq=200, Lk=200)
+    inp = gen_inputs(cfg, "cuda", seed=11)
+    out1, lse1, idx1 = _forward(cfg, inp)
+    out2, lse2, idx2 = _forward(cfg, inp)
+    assert torch.equal(out1, out2) and torch.equal(idx1, idx2) and torch.equal(lse1, lse2)
+    t = cfg.Lq - 1
+    sel = idx1[0, t][idx1[0, t] >= 0].long()
+    mask = torch.ones(cfg.Lk, dtype=torch.bool, device="cuda")
+    mask[sel] = False
+    kv2 = inp["kv"].clone()
+    kv2[0, mask] = 1.0e4
+    o, l = dsa.sparse_mla_fwd(inp["q"][:, t:t + 1].contiguous(), kv2, idx1[:, t:t + 1].contiguous(),
+                              cfg.sm_scale, cfg.Dv)
+    o_ref, l_ref = dsa.sparse_mla_fwd(inp["q"][:, t:t + 1].contiguous(), inp["kv"],
+                                      idx1[:, t:t + 1].contiguous(), cfg.sm_scale, cfg.Dv)
+    assert torch.equal(o, o_ref) and torch.equal(l, l_ref)
+    assert torch.equal(o[0, 0], out1[0, t])
+
+
+def test_sparse_mla_skips_invalid_indices():
+    cfg = CONFIGS["tiny"].with_(Lq=4, Lk=64)
+    inp = gen_inputs(cfg, "cuda", seed=3)
+    idx = torch.full((1, 4, 32), -1, dtype=torch.int32, device="cuda")
+    idx[0, 0, 5] = 7          # a lone valid key in the middle
+    idx[0, 1, :3] = torch.tensor([1, 64, 2])   # 64 is out of range: skipped
+    idx[0, 2, 0] = -5
+    # row 3: no valid key at all
+    out, lse = dsa.sparse_mla_fwd(inp["q"], inp["kv"], idx, cfg.sm_scale, cfg.Dv)
+    dsa.check_status()
+    rows = Rows(cfg, inp)
+    for t in range(4):
+        o, l = rows.attention(0, t, idx[0, t].cpu().numpy())
+        check_attention(bf16_to_f64(out[0, t]), o, lse[0, t].cpu().numpy(), l, f"t={t}")
+    assert torch.all(out[0, 2:] == 0) and torch.all(torch.isneginf(lse[0, 2:]))
+
+
+def test_bounded_wait_reports_timeout():
+    dsa.set_wait_limit_ns(20_000_000)   # 20 ms
+    try:
+        dsa.debug_wait_timeout()
+        with pytest.raises(dsa.DsaError) as ei:
+            dsa.check_status()
+        assert ei.value.code == dsa.DSA_ERR_TIMEOUT
+        assert "debug wait" in str(ei.value)
+    finally:
+        dsa.set_wait_limit_ns(2_000_000_000)
+    dsa.check_status()   # cleared, context still usable
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
