@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA forward hot path on B200.
+
+Default workload: DSA prefill, batch 2 x 32768 tokens, causal, H_I=64 / d_I=128
+FP8 indexer, top-2048, 128-head MQA over 576-wide bf16 latent rows; plus the
+decode workload (64 sequences x 1 token against a 131072-token cache) in the
+same run. One step = one ``dsa_forward`` over the whole batch (indexer, top-k,
+sparse MLA). Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs the same
+per-GPU workload on its own GPU (weak scaling, no data-path collective); the
+reported time is the max over ranks. ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from dsa_inputs import CONFIG_ORDER, CONFIGS, gen_inputs  # noqa: E402
+
+METRIC = "DSA prefill tokens/s at 32K ctx; decode tokens/s at 128K ctx (k=2048), %roofline"
+DTYPE = "fp8_e4m3+bf16"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (what the method must do, not what a kernel happens to do)
+# ---------------------------------------------------------------------------
+
+
+def work(cfg) -> dict:
+    """Per-step algorithmic work of each stage.
+
+    indexer  flops = 2 * H_I * d_I per (query row, causal key) of rows that need
+             scoring (p + 1 > k); rows with p + 1 <= k select every key unscored.
+    topk     bytes = 4 per candidate score read + 4 * k per selected row written.
+    mla      flops = 2 * H * (Dqk + Dv) per (query row, selected key).
+    decode   bytes = indexer keys + scales + gathered latent rows + q, qI, w, out.
+    """
+    p = cfg.q_pos0 + np.arange(cfg.Lq, dtype=np.int64)
+    n = np.minimum(p + 1, cfg.Lk)
+    scored = n > cfg.k
+    pairs_idx = int(n[scored].sum()) * cfg.B
+    sel = int(np.minimum(n, cfg.k).sum()) * cfg.B
+    rows_scored = int(scored.sum()) * cfg.B
+    w_bytes = 4 if cfg.w_dtype == "f32" else 2
+    return {
+        "indexer_flops": 2.0 * cfg.H_I * cfg.d_I * pairs_idx,
+        "topk_bytes": 4.0 * pairs_idx + 4.0 * cfg.k * rows_scored,
+        "mla_flops": 2.0 * cfg.H * (cfg.Dqk + cfg.Dv) * sel,
+        "hbm_bytes": float(cfg.B * cfg.Lk * (cfg.d_I + 4)            # indexer keys + scales
+                           + sel * cfg.Dqk * 2                      # gathered latent rows
+                           + cfg.B * cfg.Lq * (cfg.H * cfg.Dqk * 2 + cfg.H_I * (cfg.d_I + 4 + w_bytes)
+                                               + cfg.H * cfg.Dv * 2)),
+    }
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        m = json.load(open(path))
+        return {"hbm": float(m["hbm_gbs"]), "bf16": float(m["bf16_tflops"]),
+                "bf16_sustained": float(m["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+
+def dist_max(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk: dict,
+                  sampler: ClockSampler | None, e2e: bool):
+    import sparse_attention_long_scores_b200 as dsa
+
+    cfg = CONFIGS[name]
+    inp = gen_inputs(cfg, "cuda", seed=1000 + CONFIG_ORDER.index(name) + 97 * rank)
+    p = dsa.Problem.from_config(cfg)
+    ws = torch.empty(dsa.forward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    out = torch.empty((cfg.B, cfg.Lq, cfg.H, cfg.Dv), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        dsa.forward(p, inp, out=out, ws=ws)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    profs = [dsa.LaunchProfiler(4096) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        dsa.forward_profiled(p, inp, out, profs[i], ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    dsa.check_status()
+    ms_local = e0.elapsed_time(e1) / steps
+    ms = dist_max(ms_local, world)
+    # per-kernel device time, from events on the launching stream
+    per_kind, launches = {}, 0
+    for pr in profs:
+        for kind, d in pr.durations():
+            c = per_kind.setdefault(kind, [0.0, 0])
+            c[0] += d
+            c[1] += 1
+        launches += pr.n
+    kernels = {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps,
+                   "avg_launch_ms": v[0] / v[1]} for k, v in per_kind.items()}
+    w = work(cfg)
+    fp8_peak = 2.0 * pk["bf16_sustained"]   # FP8 dense = 2 x bf16 dense (nominal ratio)
+    roof = {}
+    if "indexer" in kernels:
+        t = kernels["indexer"]["ms_per_step"] * 1e-3
+        a = w["indexer_flops"] / t / 1e12
+        roof["indexer"] = {"bound": "tensor", "achieved": a, "peak": fp8_peak, "unit": "TFLOP/s",
+                           "frac": a / fp8_peak, "peak_note": "fp8 = 2 x measured bf16 sustained"}
+    if "topk" in kernels:
+        t = kernels["topk"]["ms_per_step"] * 1e-3
+        a = w["topk_bytes"] / t / 1e9
+        roof["topk"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s",
+                        "frac": a / pk["hbm"]}
+    if "sparse_mla" in kernels:
+        t = kernels["sparse_mla"]["ms_per_step"] * 1e-3
+        a = w["mla_flops"] / t / 1e12
+        roof["sparse_mla"] = {"bound": "tensor", "achieved": a, "peak": pk["bf16_sustained"],
+                              "unit": "TFLOP/s", "frac": a / pk["bf16_sustained"],
+                              "peak_note": "measured bf16 sustained"}
+    tokens = cfg.B * cfg.Lq * world
+    res = {"cfg": cfg, "ms": ms, "tokens_per_s": tokens / (ms * 1e-3), "kernels": kernels,
+           "roof": roof, "launches": launches, "clocks": clocks, "work": w}
+    if cfg.mode == "decode":
+        a = w["hbm_bytes"] / (ms * 1e-3) / 1e9
+        res["step_roof"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s",
+                            "frac": a / pk["hbm"], "traffic": None}
+    if e2e:
+        res["e2e"] = time_e2e(cfg, p, inp, ws, world)
+    del inp, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_e2e(cfg, p, inp, ws, world, steps: int = 2):
+    """Same metric through dsa_forward_host: pinned host inputs -> device -> host out."""
+    import sparse_attention_long_scores_b200 as dsa
+
+    host = {k: v.cpu().pin_memory() for k, v in inp.items()}
+    host_out = torch.empty((cfg.B, cfg.Lq, cfg.H, cfg.Dv), dtype=torch.bfloat16).pin_memory()
+    dev_out = torch.empty((cfg.B, cfg.Lq, cfg.H, cfg.Dv), dtype=torch.bfloat16, device="cuda")
+    dsa.forward_host(p, host, inp, host_out, dev_out, ws)     # warm-up
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        dsa.forward_host(p, host, inp, host_out, dev_out, ws)
+    dt = (time.perf_counter() - t0) / steps
+    dt = dist_max(dt, world)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+    del host, host_out, dev_out
+    return {"value": cfg.B * cfg.Lq * world / dt, "unit": "tokens/s", "ms_per_step": dt * 1e3,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU) arm
+# ---------------------------------------------------------------------------
+
+
+def oracle_sample(cfg, rows: int, seed: int = 4242):
+    """A bounded sample of the workload for the fp64 oracle: one sequence with all
+    Lk keys and `rows` query rows at evenly spread positions (decode: the last)."""
+    import oracle as ORC
+
+    c1 = cfg.with_(B=1, Lq=rows, q_pos0=0)
+    inp = ORC.numpy_inputs(gen_inputs(c1, "cpu", seed=seed))
+    if cfg.mode == "decode":
+        pos = [cfg.Lk - 1] * rows
+    else:
+        pos = [min(cfg.Lk - 1, int((i + 0.5) * cfg.Lk / rows)) for i in range(rows)]
+
+    def run(i):
+        p = pos[i]
+        n = p + 1
+        if n > cfg.k:
+            sc = ORC.index_scores(inp["qI"][0, i], inp["qI_scale"][0, i], inp["w"][0, i],
+                                  inp["kI"][0, :n], inp["kI_scale"][0, :n])
+            idx = ORC.topk_select(sc, cfg.k)
+        else:
+            idx = ORC.topk_select(np.zeros(n), cfg.k)
+        ORC.sparse_mla(inp["q"][0, i], inp["kv"][0], idx, cfg.sm_scale, cfg.Dv)
+
+    return run, pos
+
+
+def cpu_baseline(cfg, budget_s: float = 15.0) -> dict:
+    run, pos = oracle_sample(cfg, 64)
+    t0 = time.perf_counter()
+    done = 0
+    for i in range(len(pos)):
+        run(i)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} query rows of {cfg.name} (one sequence, rows at evenly spread "
+                      f"positions, {dt:.1f} s), numpy fp64 with BLAS on {cores} host threads"}
+
+
+def reference_arm(args):
+    cfg = CONFIGS[args.workload]
+    rows_per_step = 8
+    run, pos = oracle_sample(cfg, rows_per_step * (args.steps + args.warmup))
+    i = 0
+    for _ in range(args.warmup):
+        for _ in range(rows_per_step):
+            run(i)
+            i += 1
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(rows_per_step):
+            run(i)
+            i += 1
+    dt = (time.perf_counter() - t0) / args.steps
+    v = rows_per_step / dt
+    cores = len(os.sched_getaffinity(0))
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": cfg.name, "global_batch": cfg.B, "seq_len": cfg.Lk,
+                       "step": f"{rows_per_step} query rows of the workload per step"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows_per_step} query rows per step at evenly spread "
+                                       f"positions of {cfg.name}, numpy fp64"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_32k", choices=sorted(CONFIGS))
+    ap.add_argument("--decode-workload", default="decode_128k")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args)
+        return
+
+    from sparse_attention_long_scores_b200.build import build
+    if rank == 0 or not os.path.exists(os.path.join(ROOT, "sparse_attention_long_scores_b200", "libdsa.so")):
+        build()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+        dist.barrier()
+
+    pk = peaks()
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local
+    sampler = ClockSampler(gpu_index) if rank == 0 else None
+    pre = time_workload(args.workload, args.steps, args.warmup, world, rank, pk, sampler,
+                        e2e=not args.no_e2e)
+    dec = None
+    if not args.no_decode:
+        dec = time_workload(args.decode_workload, args.steps, args.warmup, world, rank, pk,
+                            None, e2e=False)
+
+    if rank == 0:
+        cfg = pre["cfg"]
+        dom_name = max(pre["kernels"], key=lambda k: pre["kernels"][k]["ms_per_step"])
+        dom = dict(pre["roof"].get(dom_name, {}))
+        dom.update({"kernel": dom_name, "traffic": None,
+                    "peak_source": pk["source"]})
+        line = {
+            "metric": METRIC, "value": pre["tokens_per_s"], "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": pre["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
+            "config": {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.Lk,
+                       "per_gpu_batch": cfg.B, "indexer": f"H_I={cfg.H_I} d_I={cfg.d_I} e4m3",
+                       "topk": cfg.k, "attention": f"H={cfg.H} Dqk={cfg.Dqk} Dv={cfg.Dv} bf16",
+                       "parallelism": f"dp{world} (independent sequences per GPU)",
+                       "l2": "inputs larger than L2 (no flush needed)"},
+            "roofline": dom,
+            "kernels": {k: {**v, **({"roofline": pre["roof"][k]} if k in pre["roof"] else {})}
+                        for k, v in pre["kernels"].items()},
+            "gpu_launches": pre["launches"],
+            "clocks": pre["clocks"],
+        }
+        if "e2e" in pre:
+            line["e2e"] = pre["e2e"]
+        if dec is not None:
+            dc = dec["cfg"]
+            line["decode"] = {
+                "workload": dc.name, "value": dec["tokens_per_s"], "unit": "tokens/s",
+                "ms_per_step": dec["ms"], "roofline": dec.get("step_roof"),
+                "kernels": {k: {**v, **({"roofline": dec["roof"][k]} if k in dec["roof"] else {})}
+                            for k, v in dec["kernels"].items()},
+                "gpu_launches": dec["launches"],
+                "config": {"batch": dc.B, "cached_tokens": dc.Lk, "topk": dc.k},
+            }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -281,6 +281,8 @@ class LaunchProfiler:
     def __init__(self, max_launches: int = 4096):
         self.max = max_launches
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(max_launches + 1)]
+        for e in self.events:      # torch creates the underlying event on first record
+            e.record()
         self._ev = (ctypes.c_void_p * (max_launches + 1))(*[e.cuda_event for e in self.events])
         self._kinds = (ctypes.c_int * max_launches)()
         self.n = 0

@@ -196,7 +196,7 @@ int mla_n_dv(int Dv) { return Dv == 512 ? 2 : 1; }
 
 int mla_splits(int B, int Lq, int Dv, int k, int num_sms) {
   long long ctas = (long long)B * Lq * mla_n_dv(Dv);
-  int tiles = k / 32;
+  int tiles = k / 64 > 0 ? k / 64 : 1;   // 64-key tiles
   if (ctas >= 2LL * num_sms) return 1;
   int s = (int)((4LL * num_sms + ctas - 1) / ctas);
   int max_s = tiles / 4 > 1 ? tiles / 4 : 1;
@@ -227,12 +227,11 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
   size_t need = mla_ws_bytes(B, Lq, H, Dv, splits);
   if (ws_bytes < need)
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "sparse MLA workspace: need %zu bytes, got %zu", need, ws_bytes);
-  CUtensorMap tq, tkv;
+  CUtensorMap tq;
   DSA_TRY(make_map_2d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Dqk,
                       (uint64_t)B * Lq * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
-  DSA_TRY(make_map_2d(&tkv, kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Dqk,
-                      (uint64_t)B * Lk, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B));
   dsa::MlaArgs a{};
+  a.q = q;
   a.idx = idx;
   a.out = out;
   a.lse = lse;
@@ -247,7 +246,7 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
     a.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                          align_up(tok * splits * H * Dv * sizeof(float), 256));
   }
-  DSA_TRY_CUDA(dsa::launch_sparse_mla(tq, tkv, a, stream), "sparse MLA launch");
+  DSA_TRY_CUDA(dsa::launch_sparse_mla(tq, kv, a, stream), "sparse MLA launch");
   DSA_TRY(rec.mark(DSA_KIND_SPARSE_MLA, stream));
   if (splits > 1) {
     DSA_TRY_CUDA(dsa::launch_mla_combine(a, stream), "split combine launch");
@@ -292,7 +291,7 @@ ForwardPlan plan_forward(const dsa_problem* p, bool need_idx, size_t ws_bytes_or
     f.chunk = (int)c;
     f.scores_bytes = align_up((size_t)c * row_bytes, 256);
   }
-  f.total = f.scores_bytes + f.idx_bytes + f.mla_bytes;
+  f.total = f.scores_bytes + f.idx_bytes + f.mla_bytes + (f.scores_bytes ? 256 : 0);
   return f;
 }
 

@@ -253,6 +253,18 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t afmt, uint32_t bfmt, 
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// acc += a * b on a pair of floats with one packed fma.rn.f32x2.
+DSA_DEVICE_INLINE void ffma2(float2& acc, float2 a, float2 b) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+}
+
 // Warp-uniform role helpers.
 DSA_DEVICE_INLINE int warp_id() { return __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0); }
 DSA_DEVICE_INLINE int lane_id() { return (int)(threadIdx.x & 31); }

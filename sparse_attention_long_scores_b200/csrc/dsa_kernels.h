@@ -52,6 +52,7 @@ cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream);
 
 // ---------------- sparse MLA (MQA mode) ----------------
 struct MlaArgs {
+  const uint16_t* q;   // [B, Lq, H, Dqk] bf16
   const int32_t* idx;  // [B, Lq, k]
   uint16_t* out;       // [B, Lq, H, Dv] bf16
   float* lse;          // [B, Lq, H] or null
@@ -64,8 +65,8 @@ struct MlaArgs {
   DevCtl ctl;
 };
 // (H, Dqk, Dv) in {(8,80,64), (128,576,512)}.
-cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
-                              const MlaArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const uint16_t* kv, const MlaArgs& a,
+                              cudaStream_t stream);
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t stream);
 
 // ---------------- debug ----------------

@@ -246,7 +246,9 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, 1)
         const int s = s0 + key_in_tile;
         const bool key_ok = s < un.s_hi;
         const float ks = key_ok ? a.kI_scale[(size_t)un.b * a.Lk + s] : 0.f;
-        float part = 0.f;
+        // four independent packed partial sums: no serial FMA chain
+        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
 #pragma unroll 1
         for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 32) {
           uint32_t r[32];
@@ -256,18 +258,23 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, 1)
           if constexpr (H_I >= 32) {
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
-              float4 wv = wv4[g];
-              part = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * g + 0]), 0.f), part);
-              part = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * g + 1]), 0.f), part);
-              part = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * g + 2]), 0.f), part);
-              part = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * g + 3]), 0.f), part);
+              const float4 wv = wv4[g];
+              const float2 x01 = make_float2(fmaxf(__uint_as_float(r[4 * g + 0]), 0.f),
+                                             fmaxf(__uint_as_float(r[4 * g + 1]), 0.f));
+              const float2 x23 = make_float2(fmaxf(__uint_as_float(r[4 * g + 2]), 0.f),
+                                             fmaxf(__uint_as_float(r[4 * g + 3]), 0.f));
+              ffma2(acc2[(2 * g) & 3], make_float2(wv.x, wv.y), x01);
+              ffma2(acc2[(2 * g + 1) & 3], make_float2(wv.z, wv.w), x23);
             }
             if (((c0 + 32) % H_I) == 0) {
+              const float part = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
+                                 ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
               const int t = un.t_a + c0 / H_I;
               if (key_ok && t < un.t_b && s <= a.q_pos0 + t) {
                 a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = part * ks;
               }
-              part = 0.f;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) acc2[q] = make_float2(0.f, 0.f);
             }
           } else {
             constexpr int TPC = 32 / H_I;  // tokens per 32-column chunk

@@ -5,17 +5,20 @@
 // all query heads, so one gathered KV row serves every head).
 //
 // One CTA computes, for one query token and one chunk of DVC value columns:
-//     z[h,s] = sm_scale * q[h] . c_s        (tcgen05, M = 128 heads, N = 32 keys,
+//     z[h,s] = sm_scale * q[h] . c_s        (tcgen05, M = 128 heads, N = 64 keys,
 //                                            K = Dqk in 16-wide steps)
 //     online softmax over the key tiles     (base 2, lazy rescale of O)
-//     O[h, chunk] += P[h,s] . c_s[chunk]    (tcgen05, M = 128, N = DVC, K = 32 keys)
+//     O[h, chunk] += P[h,s] . c_s[chunk]    (tcgen05, M = 128, N = DVC, K = 64 keys)
 // Layout of the work:
-//   warp 0      producer: Q once (TMA tiles), then the selected latent rows of each
-//               32-key tile with TMA gather4 (4 rows per instruction, 64-column
-//               128-byte-swizzled boxes) into a 2-stage ring;
-//   warp 1      tcgen05 issuer: S_i = Q K_i^T into one of two TMEM buffers,
-//               then O += P_{i-1} V_{i-1};
-//   warps 2..5  softmax: one head (TMEM lane) per thread. Writes P (bf16) to
+//   warp 0      tcgen05 issuer: Q once (TMA tiles), then S_i = Q K_i^T into one of
+//               two TMEM buffers, then O += P_{i-1} V_{i-1};
+//   warps 5..12 gather producers: the selected latent rows of each 32-key tile,
+//               16 bytes per thread per load (register-staged, several rows in
+//               flight per thread), stored straight into the 128-byte-swizzled
+//               K-major layout the tensor core reads, into a 2-stage ring. A TMA
+//               gather4 costs about as much issue time per 512 bytes as these
+//               warps need for a whole tile, so the rows are gathered by threads;
+//   warps 1..4  softmax: one head (TMEM lane) per thread. Writes P (bf16) to
 //               shared memory in the 64-byte-swizzled K-major layout, rescales O
 //               in TMEM only when the running max grew by more than 2^8, and
 //               normalises at the end.
@@ -28,8 +31,10 @@
 namespace dsa {
 namespace {
 
-constexpr int MLA_THREADS = 192;
-constexpr int KEYS = 32;                       // keys per tile
+constexpr int KEYS = 64;                       // keys per tile (N of the S MMA)
+constexpr int PROD_WARPS = 8;                  // gather warps
+constexpr int MLA_THREADS = 32 + 128 + PROD_WARPS * 32;
+constexpr int PROD_T0 = 160;                   // first producer thread
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -43,28 +48,76 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 template <int NKB, int DVC>
 struct MlaTraits {
   static constexpr int QBLK = 128 * 128;            // one 64-column block of Q: 128 rows x 128 B
   static constexpr int KVBLK = KEYS * 128;          // one 64-column block of a KV tile
+  static constexpr int QT_KB = (NKB == 9) ? 6 : 1;  // Q column blocks held in TMEM
+  static constexpr int QS_KB = NKB - QT_KB;         // Q column blocks held in shared memory
+  static constexpr int STAGES = 2;                  // KV ring depth
+  static constexpr int LAG = 0;                     // cp.async groups a producer keeps pending
+  static constexpr int CPR = NKB * 8;               // 16-byte chunks per gathered row
+  static constexpr int CHUNKS = KEYS * CPR;         // chunks per tile
+  static constexpr int NP = PROD_WARPS * 32;
+  static constexpr int CPT = (CHUNKS + NP - 1) / NP;  // chunks per producer thread per tile
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + NKB * QBLK;
-  static constexpr int OFF_P = OFF_KV + 2 * NKB * KVBLK;
-  static constexpr int OFF_BAR = OFF_P + 128 * 64;
-  static constexpr int NUM_BARS = 1 + 2 + 2 + 2 + 2 + 1 + 1 + 1;
+  static constexpr int OFF_KV = OFF_Q + QS_KB * QBLK;
+  static constexpr int OFF_P = OFF_KV + STAGES * NKB * KVBLK;
+  static constexpr int PBYTES = 128 * KEYS * 2;    // one P buffer (bf16, 128 heads x KEYS)
+  static constexpr int OFF_BAR = OFF_P + 2 * PBYTES;
+  // mbarrier slots (8 bytes each), in this order
+  static constexpr int BAR_Q = 0;                     // Q part in shared memory landed
+  static constexpr int BAR_QT = 1;                    // Q part in TMEM written
+  static constexpr int BAR_KV_FULL = 2;               // [STAGES]
+  static constexpr int BAR_KV_EMPTY = BAR_KV_FULL + STAGES;   // [STAGES]
+  static constexpr int BAR_S_FULL = BAR_KV_EMPTY + STAGES;
+  static constexpr int BAR_S_EMPTY = BAR_S_FULL + 1;
+  static constexpr int BAR_P_FULL = BAR_S_EMPTY + 1;  // [2]
+  static constexpr int BAR_P_FREE = BAR_P_FULL + 2;   // [2]
+  static constexpr int BAR_DONE = BAR_P_FREE + 2;
+  static constexpr int NUM_BARS = BAR_DONE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
-  static constexpr int TMEM_COLS = (DVC + 2 * KEYS) <= 128 ? 128 : (DVC + 2 * KEYS) <= 256 ? 256 : 512;
+  static constexpr int SMEM_BYTES = OFF_MISC + 48 + 1024;
+  // TMEM columns: O [0, DVC), S [DVC, DVC + KEYS), Q part [DVC + KEYS, ... + 32 * QT_KB)
+  static constexpr int COL_S = DVC;
+  static constexpr int COL_Q = DVC + KEYS;
+  static constexpr int COLS_USED = COL_Q + 32 * QT_KB;
+  static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_S = make_idesc(1, 1, 0, 0, KEYS, 128);   // bf16, K-major both
+  static_assert(KEYS == 64, "P layout assumes 128-byte rows");
   static constexpr uint32_t IDESC_PV = make_idesc(1, 1, 0, 1, DVC, 128);   // B (values) MN-major
   static_assert(DVC % 64 == 0 && DVC <= 256, "DVC");
+  static_assert(COLS_USED <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 template <int NKB, int DVC>
 __global__ void __launch_bounds__(MLA_THREADS, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                      const __grid_constant__ CUtensorMap tmap_kv, const MlaArgs a) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ kv,
+                      const MlaArgs a) {
   using Tr = MlaTraits<NKB, DVC>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -73,19 +126,20 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   uint8_t* kv_smem = smem + Tr::OFF_KV;
   uint8_t* p_smem = smem + Tr::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_empty = bars + 7;
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;
-  uint64_t* done_bar = bars + 11;
+  uint64_t* q_full = bars + Tr::BAR_Q;          // Q part in shared memory (TMA)
+  uint64_t* qt_full = bars + Tr::BAR_QT;        // Q part in TMEM (softmax warps)
+  uint64_t* kv_full = bars + Tr::BAR_KV_FULL;   // [STAGES]
+  uint64_t* kv_empty = bars + Tr::BAR_KV_EMPTY; // [STAGES]
+  uint64_t* s_full = bars + Tr::BAR_S_FULL;
+  uint64_t* s_empty = bars + Tr::BAR_S_EMPTY;
+  uint64_t* p_full = bars + Tr::BAR_P_FULL;     // [2] P buffer written
+  uint64_t* p_free = bars + Tr::BAR_P_FREE;     // [2] PV that read the P buffer is done
+  uint64_t* done_bar = bars + Tr::BAR_DONE;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Tr::OFF_MISC);
   uint32_t* tmem_slot = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  volatile uint32_t* masks = misc + 2;   // [2]
-  volatile int* ntiles_slot = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* ntiles_slot = reinterpret_cast<volatile int*>(misc + 2);   // [2]
+  volatile uint32_t* masks = misc + 4;   // [STAGES][2]: valid-key bits of the tile in each stage
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -99,21 +153,23 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
+    mbar_init(qt_full, 128);
+    for (int i = 0; i < Tr::STAGES; ++i) {
+      mbar_init(&kv_full[i], Tr::NP);
       mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_free[i], 1);
+    }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tmap_q);
-    tma_prefetch_map(&tmap_kv);
   }
-  if (warp == 0) {
+  if (warp == 1) {
     // number of 32-key tiles this CTA covers: trailing invalid entries are trimmed
     int last = -1;
     for (int base = ((a.k - 1) / 32) * 32; base >= 0 && last < 0; base -= 32) {
@@ -131,146 +187,224 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       ntiles_slot[1] = t_lo;
     }
   }
-  if (warp == 1) tmem_alloc(tmem_slot, Tr::TMEM_COLS);
+  if (warp == 0) tmem_alloc(tmem_slot, Tr::TMEM_COLS);
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const int ntiles = ntiles_slot[0];
   const int tile0 = ntiles_slot[1];
   const uint32_t o_tmem = tbase;
-  const uint32_t s_tmem = tbase + DVC;
+  const uint32_t s_tmem = tbase + Tr::COL_S;
+  const uint32_t qt_tmem = tbase + Tr::COL_Q;
 
   if (warp == 0) {
-    // ------------------------------------------------ producer
-    bool ok = true;
-    int kv_pending[2] = {-1, -1};
-    int q_pending = -1;
-    if (ntiles > 0 && lane == 0) {
-      mbar_arrive_expect_tx(q_full, NKB * Tr::QBLK);
-      for (int kb = 0; kb < NKB; ++kb)
-        tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, kb * 64, (int)(token * a.H), q_full);
-      q_pending = 0;
-    }
-    for (int i = 0; i < ntiles && ok; ++i) {
-      const int st = i & 1;
-      const int ph = (i >> 1) & 1;
-      const int pos = (tile0 + i) * KEYS + lane;
-      const int v = pos < a.k ? idx_row[pos] : -1;
-      const bool valid = v >= 0 && v < a.Lk;
-      const int row = b * a.Lk + (valid ? v : 0);
-      const unsigned m = __ballot_sync(0xffffffffu, valid);
-      int rows[KEYS];
-#pragma unroll
-      for (int j = 0; j < KEYS; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j);
-      if (lane == 0) {
-        if (!mbar_wait(&kv_empty[st], ph ^ 1, a.ctl, abort_flag, kSiteMla, 1)) {
-          ok = false;
-        } else {
-          kv_pending[st] = -1;
-          masks[st] = m;
-          mbar_arrive_expect_tx(&kv_full[st], NKB * Tr::KVBLK);
-          uint8_t* dst = kv_smem + st * NKB * Tr::KVBLK;
-#pragma unroll
-          for (int g = 0; g < KEYS / 4; ++g)
-#pragma unroll
-            for (int kb = 0; kb < NKB; ++kb)
-              tma_gather4(dst + kb * Tr::KVBLK + g * 512, &tmap_kv, kb * 64, rows[4 * g],
-                          rows[4 * g + 1], rows[4 * g + 2], rows[4 * g + 3], &kv_full[st]);
-          kv_pending[st] = ph;
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    }
-    if (lane == 0 && *abort_flag) {
-      DevCtl drain = a.ctl;
-      volatile int never = 0;
-      for (int i = 0; i < 2; ++i)
-        if (kv_pending[i] >= 0) mbar_wait(&kv_full[i], kv_pending[i], drain, &never, kSiteMla, 2);
-      if (q_pending >= 0) mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
+    // ------------------------------------------------ MMA issuer (and the Q load)
     if (lane == 0) {
-      bool ok = ntiles == 0 || mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 3);
-      const uint32_t q_addr = smem_u32(q_smem);
-      const uint32_t p_addr = smem_u32(p_smem);
-      const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(p_full, j & 1, a.ctl, abort_flag, kSiteMla, 4)) return false;
-        tc_fence_after();
-        const int stj = j & 1;
-        const uint32_t kv_addr = smem_u32(kv_smem + stj * NKB * Tr::KVBLK);
-#pragma unroll
-        for (int kk = 0; kk < KEYS / 16; ++kk) {
-          uint64_t ad = make_sdesc(p_addr + kk * 32, 16, 512, 4);
-          uint64_t bd = make_sdesc(kv_addr + v_off + kk * 2048, Tr::KVBLK, 1024, 2);
-          mma_f16_ss(o_tmem, ad, bd, Tr::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+      bool ok = true;
+      if (ntiles > 0) {
+        mbar_arrive_expect_tx(q_full, Tr::QS_KB * Tr::QBLK);
+        for (int kb = 0; kb < Tr::QS_KB; ++kb)
+          tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, (Tr::QT_KB + kb) * 64, (int)(token * a.H),
+                      q_full);
+        ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 3);
+        if (!ok) {
+          DevCtl drain = a.ctl;
+          volatile int never = 0;
+          mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
         }
-        mma_commit(&kv_empty[stj]);
-        mma_commit(o_done);
-        return true;
-      };
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int st = i & 1;
-        const int ph = (i >> 1) & 1;
-        if (!mbar_wait(&kv_full[st], ph, a.ctl, abort_flag, kSiteMla, 5)) { ok = false; break; }
-        if (!mbar_wait(&s_empty[st], ph ^ 1, a.ctl, abort_flag, kSiteMla, 6)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kv_addr = smem_u32(kv_smem + st * NKB * Tr::KVBLK);
-        const uint32_t d = s_tmem + st * KEYS;
+        ok = ok && mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 12);
+      }
+      // Descriptors are built once; per MMA only the start-address field moves
+      // (byte offset / 16 added to the low bits, which never carry: smem < 256 KB).
+      const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
+      const uint64_t pd0 = make_sdesc(smem_u32(p_smem), 16, 1024, 2);
+      const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
+      auto issue_s = [&](int i) {
+        const int st = i % Tr::STAGES;
+        const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + st * NKB * Tr::KVBLK), 16, 1024, 2);
+        // S = Q K^T: the first QT_KB column blocks of Q come from TMEM, the rest from smem
 #pragma unroll
-        for (int kb = 0; kb < NKB; ++kb) {
+        for (int kb = 0; kb < Tr::QT_KB; ++kb) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            uint64_t ad = make_sdesc(q_addr + kb * Tr::QBLK + kk * 32, 16, 1024, 2);
-            uint64_t bd = make_sdesc(kv_addr + kb * Tr::KVBLK + kk * 32, 16, 1024, 2);
-            mma_f16_ss(d, ad, bd, Tr::IDESC_S, (kb | kk) ? 1u : 0u);
+            mma_f16_ts(s_tmem, qt_tmem + kb * 32 + kk * 8,
+                       kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S,
+                       (kb | kk) ? 1u : 0u);
           }
         }
-        mma_commit(&s_full[st]);
-        if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
+#pragma unroll
+        for (int kb = Tr::QT_KB; kb < NKB; ++kb) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_f16_ss(s_tmem, qd0 + (uint64_t)(((kb - Tr::QT_KB) * Tr::QBLK + kk * 32) >> 4),
+                       kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S, 1u);
+          }
+        }
+        mma_commit(s_full);
+      };
+      auto issue_pv = [&](int j) {
+        const int stj = j % Tr::STAGES;
+        const uint64_t bd0 = make_sdesc(smem_u32(kv_smem + stj * NKB * Tr::KVBLK) + v_off,
+                                        Tr::KVBLK, 1024, 2);
+        const uint64_t pd = pd0 + (uint64_t)(((j & 1) * Tr::PBYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < KEYS / 16; ++kk)
+          mma_f16_ss(o_tmem, pd + (uint64_t)(kk * 32 >> 4), bd0 + (uint64_t)(kk * 16 * 128 >> 4),
+                     Tr::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&kv_empty[stj]);
+        mma_commit(&p_free[j & 1]);
+      };
+      // Issue S_i and PV_j in whichever order their inputs become ready: S_i needs
+      // tile i in shared memory and the S buffer drained by the softmax warps; PV_j
+      // needs P_j. Bounded like every other wait.
+      int ns = 0, npv = 0;
+      uint64_t t_mark = globaltimer_ns();
+      uint32_t spins = 0;
+      while (ok && npv < ntiles) {
+        bool did = false;
+        if (ns < ntiles &&
+            mbar_try_wait(smem_u32(&kv_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1) &&
+            mbar_try_wait(smem_u32(s_empty), (ns & 1) ^ 1)) {
+          tc_fence_after();
+          issue_s(ns);
+          ++ns;
+          did = true;
+        }
+        if (npv < ns && mbar_try_wait(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1)) {
+          tc_fence_after();
+          issue_pv(npv);
+          ++npv;
+          did = true;
+        }
+        if (did) {
+          spins = 0;
+          t_mark = globaltimer_ns();
+        } else if ((++spins & 63u) == 0) {
+          if (*abort_flag || *reinterpret_cast<volatile int*>(a.ctl.status) != 0) {
+            *abort_flag = 1;
+            ok = false;
+          } else if (globaltimer_ns() - t_mark > a.ctl.wait_ns) {
+            report_timeout(a.ctl, kSiteMla, 4);
+            *abort_flag = 1;
+            ok = false;
+          }
+        }
       }
-      if (ok && ntiles > 0) issue_pv(ntiles - 1);
       mma_commit(done_bar);
       DevCtl drain = a.ctl;
       volatile int never = 0;
       mbar_wait(done_bar, 0, drain, &never, kSiteMla, 7);
     }
+  } else if (warp >= PROD_T0 / 32) {
+    // ------------------------------------------------ gather producers
+    // Chunk c of a tile is 16 bytes: row r = c / CPR, chunk q = c % CPR of that row.
+    // It lands in the 128-byte-swizzled K-major layout the tensor core reads:
+    // column block q / 8, row r, 16-byte slot (q % 8) ^ (r % 8). Chunks past the
+    // end of a row (padding up to the 64-column block) are written as zeros.
+    // Each thread keeps LAG tiles of cp.async groups in flight; once a group is
+    // complete it makes the writes visible to the tensor core (proxy fence) and
+    // arrives on that tile's full barrier.
+    const int ptid = threadIdx.x - PROD_T0;
+    const int row_bytes = a.Dqk * 2;
+    const uint8_t* kv_b = reinterpret_cast<const uint8_t*>(kv) + (size_t)b * a.Lk * row_bytes;
+    const uint32_t kv_base = smem_u32(kv_smem);
+    int issued = 0;
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % Tr::STAGES;
+      if (!mbar_wait(&kv_empty[st], ((i / Tr::STAGES) & 1) ^ 1, a.ctl, abort_flag, kSiteMla, 1)) break;
+      const uint32_t stage = kv_base + st * NKB * Tr::KVBLK;
+#pragma unroll
+      for (int j = 0; j < Tr::CPT; ++j) {
+        const int c = ptid + j * Tr::NP;
+        if (c < Tr::CHUNKS) {
+          const int r = c / Tr::CPR, q = c % Tr::CPR;
+          const int pos = (tile0 + i) * KEYS + r;
+          const int v = pos < a.k ? __ldg(idx_row + pos) : -1;
+          const int row = (v >= 0 && v < a.Lk) ? v : 0;   // invalid keys read row 0, masked later
+          const bool in_row = q * 16 < row_bytes;
+          cp_async16(stage + (q >> 3) * Tr::KVBLK + r * 128 + (((q & 7) ^ (r & 7)) << 4),
+                     kv_b + (size_t)row * row_bytes + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if (ptid < 32) {
+#pragma unroll
+        for (int hw = 0; hw < KEYS / 32; ++hw) {
+          const int pos = (tile0 + i) * KEYS + hw * 32 + lane;
+          const int vi = pos < a.k ? __ldg(idx_row + pos) : -1;
+          const unsigned m = __ballot_sync(0xffffffffu, vi >= 0 && vi < a.Lk);
+          if (ptid == 0) masks[st * 2 + hw] = m;   // slot free: PV of its previous tile is done
+        }
+      }
+      ++issued;
+      if (i >= Tr::LAG) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(Tr::LAG) : "memory");
+        fence_proxy_async_smem();
+        mbar_arrive(&kv_full[(i - Tr::LAG) % Tr::STAGES]);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (!*abort_flag) {
+      fence_proxy_async_smem();
+      for (int i = (issued > Tr::LAG ? issued - Tr::LAG : 0); i < issued; ++i)
+        mbar_arrive(&kv_full[i % Tr::STAGES]);
+    }
   } else {
-    // ------------------------------------------------ softmax / epilogue
+    // ------------------------------------------------ softmax / epilogue (warps 1..4)
     const int quad = warp & 3;
     const int h = quad * 32 + lane;  // head = TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    // this head's first QT_KB * 64 query columns go to TMEM (the MMA's A operand:
+    // lane = head, 32-bit column = two consecutive bf16 of the row)
+    if (ntiles > 0) {
+      const long long qrow = token * a.H + h;
+      const bool have = qrow < (long long)a.B * a.Lq * a.H;
+      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) + (have ? qrow : 0) * (long long)a.Dqk * 2;
+#pragma unroll 1
+      for (int kb = 0; kb < Tr::QT_KB; ++kb) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 u = have ? *reinterpret_cast<const uint4*>(qsrc + kb * 128 + c * 16) : make_uint4(0u, 0u, 0u, 0u);
+          qv[4 * c] = u.x; qv[4 * c + 1] = u.y; qv[4 * c + 2] = u.z; qv[4 * c + 3] = u.w;
+        }
+        tmem_st32(qt_tmem + lane_off + kb * 32, qv);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(qt_full);
+    }
     float m_used = -INFINITY;  // running max (log2 domain) that P is relative to
     float l = 0.f;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      const int st = i & 1;
-      const int ph = (i >> 1) & 1;
-      if (!mbar_wait(&s_full[st], ph, a.ctl, abort_flag, kSiteMla, 8)) { ok = false; break; }
-      if (!mbar_wait(&kv_full[st], ph, a.ctl, abort_flag, kSiteMla, 9)) { ok = false; break; }
+      const int st = i % Tr::STAGES;
+      if (!mbar_wait(s_full, i & 1, a.ctl, abort_flag, kSiteMla, 8)) { ok = false; break; }
+      if (!mbar_wait(&kv_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 9)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(s_tmem + lane_off + st * KEYS, r);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_empty[st]);
-      const uint32_t m = masks[st];
-      float x[32];
+      float x[KEYS];
       float tmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] = ((m >> j) & 1u) ? __uint_as_float(r[j]) * a.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, x[j]);
+      for (int hw = 0; hw < KEYS / 32; ++hw) {
+        uint32_t r[32];
+        tmem_ld32(s_tmem + lane_off + hw * 32, r);
+        tmem_wait_ld();
+        const uint32_t m = masks[st * 2 + hw];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          x[hw * 32 + j] = ((m >> j) & 1u) ? __uint_as_float(r[j]) * a.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, x[hw * 32 + j]);
+        }
       }
-      if (i > 0) {
-        if (!mbar_wait(o_done, (i - 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
-        tc_fence_after();
-      }
+      tc_fence_before();
+      mbar_arrive(s_empty);
       const bool grow = tmax > m_used + 8.0f;
       const float m_new = grow ? tmax : m_used;
       const bool need_o = grow && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
+        // O is rescaled in place: PV_{i-1} (the last one issued) must be done
+        if (!mbar_wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
+        tc_fence_after();
         const float alpha = need_o ? ex2(m_used - m_new) : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < DVC; c0 += 32) {
@@ -285,30 +419,33 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         l *= alpha;
       }
       m_used = m_new;
-      uint32_t pk[16];
-      float psum = 0.f;
+      uint32_t pk[KEYS / 2];
+      float psum0 = 0.f, psum1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < KEYS / 2; ++j) {
         float p0 = ex2(x[2 * j] - m_used);
         float p1 = ex2(x[2 * j + 1] - m_used);
         if (m_used == -INFINITY) { p0 = 0.f; p1 = 0.f; }
-        psum += p0 + p1;
+        psum0 += p0;
+        psum1 += p1;
         pk[j] = pack_bf16x2(p0, p1);
       }
-      l += psum;
-      // P row h: 32 bf16 = four 16-byte chunks, 64-byte swizzle (chunk ^= (h >> 1) & 3)
-      uint8_t* prow = p_smem + h * 64;
+      l += psum0 + psum1;
+      // P buffer i % 2 is free once PV_{i-2} is done
+      if (i >= 2 && !mbar_wait(&p_free[i & 1], ((i >> 1) & 1) ^ 1, a.ctl, abort_flag, kSiteMla, 13)) { ok = false; break; }
+      // P row h: 64 bf16 = eight 16-byte chunks, 128-byte swizzle (chunk ^= h % 8)
+      uint8_t* prow = p_smem + (i & 1) * Tr::PBYTES + h * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int pc = c ^ ((h >> 1) & 3);
+      for (int c = 0; c < 8; ++c) {
+        const int pc = c ^ (h & 7);
         *reinterpret_cast<uint4*>(prow + pc * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[i & 1]);
     }
     if (ok && ntiles > 0) {
-      ok = mbar_wait(o_done, (ntiles - 1) & 1, a.ctl, abort_flag, kSiteMla, 11);
+      ok = mbar_wait(&p_free[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 11);
       tc_fence_after();
     }
     if (ok) {
@@ -369,7 +506,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, Tr::TMEM_COLS);
   }
@@ -410,7 +547,7 @@ __global__ void mla_combine_kernel(const MlaArgs a) {
 }
 
 template <int NKB, int DVC>
-cudaError_t launch_mla_variant(const CUtensorMap& tq, const CUtensorMap& tkv, const MlaArgs& a,
+cudaError_t launch_mla_variant(const CUtensorMap& tq, const uint16_t* kv, const MlaArgs& a,
                                cudaStream_t stream) {
   using Tr = MlaTraits<NKB, DVC>;
   auto kern = sparse_mla_kernel<NKB, DVC>;
@@ -419,16 +556,16 @@ cudaError_t launch_mla_variant(const CUtensorMap& tq, const CUtensorMap& tkv, co
   if (e != cudaSuccess) return e;
   long long grid = (long long)a.B * a.Lq * a.n_dv * a.splits;
   if (grid <= 0) return cudaSuccess;
-  kern<<<(unsigned)grid, MLA_THREADS, Tr::SMEM_BYTES, stream>>>(tq, tkv, a);
+  kern<<<(unsigned)grid, MLA_THREADS, Tr::SMEM_BYTES, stream>>>(tq, kv, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
-                              const MlaArgs& a, cudaStream_t stream) {
-  if (a.H == 128 && a.Dqk == 576 && a.Dv == 512) return launch_mla_variant<9, 256>(tmap_q, tmap_kv, a, stream);
-  if (a.H == 8 && a.Dqk == 80 && a.Dv == 64) return launch_mla_variant<2, 64>(tmap_q, tmap_kv, a, stream);
+cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const uint16_t* kv, const MlaArgs& a,
+                              cudaStream_t stream) {
+  if (a.H == 128 && a.Dqk == 576 && a.Dv == 512) return launch_mla_variant<9, 256>(tmap_q, kv, a, stream);
+  if (a.H == 8 && a.Dqk == 80 && a.Dv == 64) return launch_mla_variant<2, 64>(tmap_q, kv, a, stream);
   return cudaErrorInvalidValue;
 }
 

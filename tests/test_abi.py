@@ -127,3 +127,22 @@ def test_no_cpu_fallback_in_binding():
     assert "import oracle" not in src and "from oracle" not in src
     for banned in ("torch.topk", "torch.softmax", "torch.matmul", "@ ", "einsum"):
         assert banned not in src, banned
+
+
+def test_recommended_workspace_passes_validation(L):
+    """The recommended size passes validation and a tiny one does not. With fake
+    device pointers a valid call gets past validation and then fails for want of
+    a GPU, so this runs only where no GPU is visible."""
+    import torch
+    from dsa_inputs import CONFIGS
+    if torch.cuda.is_available():
+        pytest.skip("uses fake device pointers")
+    for name, cfg in CONFIGS.items():
+        p = dsa.Problem.from_config(cfg)
+        cp = p.c()
+        n = L.dsa_forward_workspace_size(ctypes.byref(cp))
+        t = dsa.DsaTensors(*([FAKE] * 8 + [None, None]))
+        rc = L.dsa_forward(ctypes.byref(cp), ctypes.byref(t), ctypes.c_void_p(FAKE), n, None)
+        assert rc == dsa.DSA_ERR_CUDA, (name, rc, L.dsa_last_error().decode())
+        rc = L.dsa_forward(ctypes.byref(cp), ctypes.byref(t), ctypes.c_void_p(FAKE), 64, None)
+        assert rc == dsa.DSA_ERR_WORKSPACE_TOO_SMALL, name
