@@ -115,6 +115,30 @@ int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
                        float* lse, int B, int Lq, int Lk, int H, int Dqk, int Dv, int k,
                        float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * dsa_sparse_mla_fwd_noalloc - dsa_sparse_mla_fwd for callers that cannot
+ * allocate device memory. (The paper has no counterpart: this is a deployment
+ * convenience of this library.) Some callers cannot call cudaMalloc or hand
+ * over a workspace: plugins running inside a host framework that reserves all
+ * device memory up front, or code paths where the implicit synchronisation of
+ * an allocation is not acceptable. This entry point takes the same inputs and
+ * outputs as dsa_sparse_mla_fwd and calls no allocator: the key-split partial
+ * results live in a 16 MiB array compiled into the library, which every GPU
+ * that loads the library holds until the process exits.
+ *   - Shapes whose split partials need more than 16 MiB are rejected with
+ *     DSA_ERR_UNSUPPORTED_SHAPE (for H = 128, Dv = 512, k = 2048 that is 8 to
+ *     147 query tokens; up to 7 tokens, and 148 or more, are accepted).
+ *   - The first call on a device looks up the array's device address with the
+ *     device current; make that first call before any stream capture.
+ *   - All calls share the one array and every call fully overwrites the part it
+ *     uses (nothing needs clearing), so calls that overlap on the GPU (other
+ *     streams, other host threads) race with each other: serialise them.
+ *   - Results equal dsa_sparse_mla_fwd for the same shape.
+ */
+int dsa_sparse_mla_fwd_noalloc(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                               uint16_t* out, float* lse, int B, int Lq, int Lk, int H, int Dqk,
+                               int Dv, int k, float sm_scale, void* stream);
+
 /* Whole-path problem description for dsa_forward. */
 typedef struct dsa_problem {
   int mode;        /* DSA_MODE_PREFILL or DSA_MODE_DECODE (informational; the

@@ -38,7 +38,7 @@ EXPORTED = [
     "dsa_last_error", "dsa_version", "dsa_indexer_scores", "dsa_topk_select",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_fwd", "dsa_forward_workspace_size",
     "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
-    "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout",
+    "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout", "dsa_sparse_mla_fwd_noalloc",
 ]
 KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
 
@@ -83,6 +83,9 @@ def lib() -> ctypes.CDLL:
     L.dsa_sparse_mla_workspace_size.restype = sz
     L.dsa_sparse_mla_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, ctypes.c_float,
                                      vp, sz, vp]
+    L.dsa_sparse_mla_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
+                                             ctypes.c_float, vp]
+    L.dsa_sparse_mla_fwd_noalloc.restype = i
     L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
     L.dsa_forward_workspace_size.restype = sz
     L.dsa_forward.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp, sz, vp]

@@ -451,6 +451,68 @@ int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
                  static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of dsa_sparse_mla_fwd.
+//
+// Its key-split partials live in a fixed device array compiled into the
+// library instead of a caller-provided workspace. Every GPU that loads the
+// library holds this array until the process exits. Host code only sees a
+// host-side stand-in for the symbol, so the device address is looked up once
+// per device with cudaGetSymbolAddress (device current) and cached.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    DSA_TRY_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int dsa_sparse_mla_fwd_noalloc(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                               uint16_t* out, float* lse, int B, int Lq, int Lk, int H, int Dqk,
+                               int Dv, int k, float sm_scale, void* stream) {
+  DSA_TRY(check_ptr(q, "q"));
+  DSA_TRY(check_ptr(kv, "kv"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(out, "out"));
+  DSA_TRY(check_ptr(lse, "lse", true));
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1");
+  if ((long long)B * Lk > (1LL << 30)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lk must be <= 2^30");
+  DSA_TRY(check_mla_shape(H, Dqk, Dv, B, Lq));
+  DSA_TRY(check_k(k, 4096));
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
+    return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+  const size_t need = mla_ws_bytes(B, Lq, H, Dv, mla_splits(B, Lq, Dv, k, assumed_sms()));
+  if (need > kNoAllocScratchBytes)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE,
+                "dsa_sparse_mla_fwd_noalloc: this shape needs %zu bytes of scratch but the built-in "
+                "scratch holds %zu; use dsa_sparse_mla_fwd with a workspace",
+                need, kNoAllocScratchBytes);
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  void* scratch = nullptr;
+  DSA_TRY(noalloc_scratch(&scratch));
+  return run_mla(q, kv, idx, out, lse, B, Lq, Lk, H, Dqk, Dv, k, sm_scale, scratch,
+                 kNoAllocScratchBytes, ctl, sms, static_cast<cudaStream_t>(stream));
+}
+
 size_t dsa_forward_workspace_size(const dsa_problem* p) {
   if (validate_problem(p) != DSA_OK) return 0;
   return plan_forward(p, true, 0).total;
