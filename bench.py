@@ -141,12 +141,24 @@ class ClockSampler:
 
 
 def dist_max(x: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (the step time of a weak-scaling run)."""
     if world <= 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(name: str, rank: int) -> int:
+    """Seed of this rank's share of the workload: every rank gets its own sequences."""
+    return 1000 + CONFIG_ORDER.index(name) + 97 * rank
+
+
+def aggregate_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
 
 
 def barrier(world: int):
@@ -160,7 +172,7 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     import sparse_attention_long_scores_b200 as dsa
 
     cfg = CONFIGS[name]
-    inp = gen_inputs(cfg, "cuda", seed=1000 + CONFIG_ORDER.index(name) + 97 * rank)
+    inp = gen_inputs(cfg, "cuda", seed=rank_seed(name, rank))
     p = dsa.Problem.from_config(cfg)
     ws = torch.empty(dsa.forward_workspace_size(p), dtype=torch.uint8, device="cuda")
     out = torch.empty((cfg.B, cfg.Lq, cfg.H, cfg.Dv), dtype=torch.bfloat16, device="cuda")
@@ -215,8 +227,8 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
         roof["sparse_mla"] = {"bound": "tensor", "achieved": a, "peak": pk["bf16_sustained"],
                               "unit": "TFLOP/s", "frac": a / pk["bf16_sustained"],
                               "peak_note": "measured bf16 sustained"}
-    tokens = cfg.B * cfg.Lq * world
-    res = {"cfg": cfg, "ms": ms, "tokens_per_s": tokens / (ms * 1e-3), "kernels": kernels,
+    res = {"cfg": cfg, "ms": ms, "tokens_per_s": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, ms),
+           "kernels": kernels,
            "roof": roof, "launches": launches, "clocks": clocks, "work": w}
     if cfg.mode == "decode":
         a = w["hbm_bytes"] / (ms * 1e-3) / 1e9
