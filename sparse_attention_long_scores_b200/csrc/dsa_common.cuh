@@ -79,6 +79,19 @@ DSA_DEVICE_INLINE bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (for polling several barriers in turn).
+DSA_DEVICE_INLINE bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete. Bounded: gives up when
 // `*abort` becomes non-zero (another role of this CTA gave up), when the device
 // status word is set (another CTA gave up), or after ctl.wait_ns nanoseconds,
@@ -263,6 +276,112 @@ DSA_DEVICE_INLINE void ffma2(float2& acc, float2 a, float2 b) {
       "mov.b64 {%0, %1}, rc;\n\t}"
       : "+f"(acc.x), "+f"(acc.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+}
+
+// 2^x on the special-function unit (ex2.approx: ~2 ulp, -inf -> +0).
+DSA_DEVICE_INLINE float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two floats -> packed bf16x2 (round to nearest even); `lo` in the low half.
+DSA_DEVICE_INLINE uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 16-byte global -> shared copy; src_bytes = 0 writes zeros (no read).
+DSA_DEVICE_INLINE void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+DSA_DEVICE_INLINE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+DSA_DEVICE_INLINE void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+DSA_DEVICE_INLINE void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] x B[smem]^T (bf16 A operand held in tensor memory).
+DSA_DEVICE_INLINE void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters (distributed shared memory)
+// ---------------------------------------------------------------------------
+DSA_DEVICE_INLINE uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared-memory address of the same variable in CTA `rank` of this cluster.
+DSA_DEVICE_INLINE uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+
+DSA_DEVICE_INLINE void st_cluster_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster, releasing this thread's
+// prior (distributed) shared-memory writes to it.
+DSA_DEVICE_INLINE void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+DSA_DEVICE_INLINE bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait (as mbar_wait) that acquires at cluster scope: for barriers
+// that other CTAs of the cluster arrive on.
+DSA_DEVICE_INLINE bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const DevCtl& ctl,
+                                         volatile int* abort, int site, int wait_id) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait_cluster(addr, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(addr, parity)) return true;
+    if (*abort) return false;
+    if (*reinterpret_cast<volatile int*>(ctl.status) != 0) {
+      *abort = 1;
+      return false;
+    }
+    if (globaltimer_ns() - t0 > ctl.wait_ns) {
+      report_timeout(ctl, site, wait_id);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// All threads of all CTAs of the cluster.
+DSA_DEVICE_INLINE void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
 }
 
 // Warp-uniform role helpers.

@@ -322,3 +322,28 @@ def test_bounded_wait_reports_timeout():
     dsa.check_status()   # cleared, context still usable
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+@pytest.mark.parametrize("tokens,Lk", [(6, 5000), (160, 3000)])
+def test_mla_128_heads_every_row(tokens, Lk):
+    """128-head / 576-wide attention on random selections, every row against the
+    oracle: few tokens take the key-split path, many tokens the direct one. Row 0
+    holds a short selection padded with -1, row 1 an out-of-range index."""
+    cfg = CONFIGS["prefill_8k"].with_(B=1, Lq=tokens, Lk=Lk, q_pos0=Lk - tokens)
+    inp = gen_inputs(cfg, "cuda", seed=tokens, only=("q", "kv"))
+    g = torch.Generator(device="cuda").manual_seed(tokens + Lk)
+    rows = [torch.sort(torch.randperm(Lk, generator=g, device="cuda")[:cfg.k]).values
+            for _ in range(tokens)]
+    idx = torch.stack(rows).view(1, tokens, cfg.k).to(torch.int32)
+    idx[0, 0, 100:] = -1
+    idx[0, 1, 7] = Lk + 5
+    out, lse = dsa.sparse_mla_fwd(inp["q"], inp["kv"], idx.contiguous(), cfg.sm_scale, cfg.Dv)
+    dsa.check_status()
+    q_h, kv_h, idx_h = _np(inp["q"][0]), _np(inp["kv"][0]), idx[0].cpu().numpy()
+    ro, rl = [], []
+    for t in range(tokens):
+        o, l = ORC.sparse_mla(q_h[t], kv_h, idx_h[t], cfg.sm_scale, cfg.Dv)
+        ro.append(o)
+        rl.append(l)
+    check_attention(bf16_to_f64(out[0]), np.stack(ro), lse[0].cpu().numpy(), np.stack(rl),
+                    f"mla128 tokens={tokens}")
