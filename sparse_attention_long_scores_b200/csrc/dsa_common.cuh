@@ -329,6 +329,12 @@ DSA_DEVICE_INLINE uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
   return r;
 }
 
+DSA_DEVICE_INLINE uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 DSA_DEVICE_INLINE void st_cluster_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)
