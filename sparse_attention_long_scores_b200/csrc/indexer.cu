@@ -31,11 +31,13 @@ struct IdxTraits {
   static constexpr int KT = 128;
   static constexpr int KTILE_BYTES = KT * D_I;
   static constexpr int QBLK_BYTES = N * D_I;
-  static constexpr int STAGES = (D_I == 128) ? 6 : 8;
+  // key-tile ring depth; the single-token variant keeps two CTAs per SM in smem
+  static constexpr int STAGES = (D_I == 128) ? (N == 64 ? 5 : 6) : 8;
   static constexpr int ACC = 2;
   static constexpr int TMEM_COLS = (ACC * N <= 32) ? 32 : (ACC * N <= 64) ? 64
                                    : (ACC * N <= 128) ? 128 : (ACC * N <= 256) ? 256 : 512;
   static constexpr int EPI_WARPS = (T_BLK >= 2) ? 8 : 4;
+  static constexpr int MIN_CTAS = (N == 64) ? 2 : 1;        // CTAs per SM the registers must allow
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
   static constexpr int THREADS = 64 + EPI_THREADS;
   static constexpr uint32_t SWZ = (D_I == 128) ? 2u : 6u;   // 128B / 32B swizzle
@@ -51,7 +53,7 @@ struct IdxTraits {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N <= 256, "N");
   static_assert(ACC * N <= 512, "TMEM");
-  static_assert(H_I >= 32 ? (H_I % 32 == 0) : (32 % H_I == 0), "heads per chunk");
+  static_assert(H_I == 64 || (H_I < 32 && 32 % H_I == 0), "heads per chunk");
 };
 
 struct Unit {
@@ -82,7 +84,7 @@ __device__ __forceinline__ bool get_unit(const IndexerArgs& a, int u, int nblk, 
 }
 
 template <int D_I, int H_I, int N>
-__global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, 1)
+__global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I, H_I, N>::MIN_CTAS)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs a) {
   using Tr = IdxTraits<D_I, H_I, N>;
@@ -240,25 +242,41 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, 1)
         wbuf[c - c_begin] = v;
       }
       __syncwarp();
+      // single-token blocks (decode): this unit's 64 folded weights stay in registers
+      float wr[(T_BLK == 1 && H_I == 64) ? 64 : 1];
+      if constexpr (T_BLK == 1 && H_I == 64) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) wr[j] = wbuf[j];
+      }
+      // key scales are fetched one tile ahead so their latency hides behind a tile
+      const float* ks_row = a.kI_scale + (size_t)un.b * a.Lk;
+      float ks_next = (un.s_lo + key_in_tile < un.s_hi) ? __ldg(ks_row + un.s_lo + key_in_tile) : 0.f;
       for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
-        if (!mbar_wait(&acc_full[ac], aph, a.ctl, abort_flag, kSiteIndexer, 8)) { ok = false; break; }
-        tc_fence_after();
         const int s = s0 + key_in_tile;
         const bool key_ok = s < un.s_hi;
-        const float ks = key_ok ? a.kI_scale[(size_t)un.b * a.Lk + s] : 0.f;
-        // four independent packed partial sums: no serial FMA chain
-        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                          make_float2(0.f, 0.f)};
+        const float ks = ks_next;
+        ks_next = (s + Tr::KT < un.s_hi) ? __ldg(ks_row + s + Tr::KT) : 0.f;
+        if (!mbar_wait(&acc_full[ac], aph, a.ctl, abort_flag, kSiteIndexer, 8)) { ok = false; break; }
+        tc_fence_after();
+        if constexpr (H_I == 64) {
+          // one token (64 heads) per step: both TMEM loads in flight, one wait
 #pragma unroll 1
-        for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + (uint32_t)(ac * N + c0), r);
-          tmem_wait_ld();
-          const float4* wv4 = reinterpret_cast<const float4*>(wbuf + (c0 - c_begin));
-          if constexpr (H_I >= 32) {
+          for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 64) {
+            uint32_t r[64];
+            tmem_ld32(t_lane + (uint32_t)(ac * N + c0), *reinterpret_cast<uint32_t(*)[32]>(r));
+            tmem_ld32(t_lane + (uint32_t)(ac * N + c0 + 32), *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+            tmem_wait_ld();
+            // four independent packed partial sums: no serial FMA chain
+            float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                              make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              const float4 wv = wv4[g];
+            for (int g = 0; g < 16; ++g) {
+              float4 wv;
+              if constexpr (T_BLK == 1) {
+                wv = make_float4(wr[4 * g], wr[4 * g + 1], wr[4 * g + 2], wr[4 * g + 3]);
+              } else {
+                wv = reinterpret_cast<const float4*>(wbuf + (c0 - c_begin))[g];
+              }
               const float2 x01 = make_float2(fmaxf(__uint_as_float(r[4 * g + 0]), 0.f),
                                              fmaxf(__uint_as_float(r[4 * g + 1]), 0.f));
               const float2 x23 = make_float2(fmaxf(__uint_as_float(r[4 * g + 2]), 0.f),
@@ -266,17 +284,18 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, 1)
               ffma2(acc2[(2 * g) & 3], make_float2(wv.x, wv.y), x01);
               ffma2(acc2[(2 * g + 1) & 3], make_float2(wv.z, wv.w), x23);
             }
-            if (((c0 + 32) % H_I) == 0) {
-              const float part = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
-                                 ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
-              const int t = un.t_a + c0 / H_I;
-              if (key_ok && t < un.t_b && s <= a.q_pos0 + t) {
-                a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = part * ks;
-              }
-#pragma unroll
-              for (int q = 0; q < 4; ++q) acc2[q] = make_float2(0.f, 0.f);
-            }
-          } else {
+            const float part = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
+                               ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
+            const int t = un.t_a + c0 / 64;
+            if (key_ok && t < un.t_b && s <= a.q_pos0 + t)
+              a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = part * ks;
+          }
+        } else {
+#pragma unroll 1
+          for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(t_lane + (uint32_t)(ac * N + c0), r);
+            tmem_wait_ld();
             constexpr int TPC = 32 / H_I;  // tokens per 32-column chunk
             const float* wv = wbuf + (c0 - c_begin);
 #pragma unroll
@@ -319,7 +338,10 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const I
   long long maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
   long long units = (long long)a.B * nblk * maxp;
   if (units <= 0) return cudaSuccess;
-  int grid = (int)(units < num_sms ? units : num_sms);
+  // persistent CTAs: as many as fit on the SMs at once (smem and TMEM allow two
+  // of the single-token variant per SM)
+  const int per_sm = (2 * Tr::SMEM_BYTES <= 227 * 1024 && 2 * Tr::TMEM_COLS <= 512) ? 2 : 1;
+  int grid = (int)(units < (long long)per_sm * num_sms ? units : (long long)per_sm * num_sms);
   kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, stream>>>(tq, tk, a);
   return cudaGetLastError();
 }
