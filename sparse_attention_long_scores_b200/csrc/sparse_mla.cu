@@ -26,6 +26,8 @@
 // columns are split over CTAs (DVC = 256): each CTA recomputes S for its token.
 // With several key splits (decode) each CTA writes an unnormalised partial
 // (O, running max, sum) and a combine kernel merges them.
+#include <type_traits>
+
 #include "dsa_kernels.h"
 
 namespace dsa {
@@ -51,11 +53,15 @@ struct MlaTraits {
   static constexpr int QT_KB = (NKB == 9) ? 6 : 1;  // Q column blocks held in TMEM
   static constexpr int QS_KB = NKB - QT_KB;         // Q column blocks held in shared memory
   static constexpr int STAGES = 2;                  // KV ring depth
-  static constexpr int LAG = 0;                     // cp.async groups a producer keeps pending
-  static constexpr int CPR = NKB * 8;               // 16-byte chunks per gathered row
-  static constexpr int CHUNKS = KEYS * CPR;         // chunks per tile
+  // A tile's column blocks come in two parts: part B = the DVC / 64 value blocks
+  // this CTA multiplies with P (read by S and by PV), part A = the others (read
+  // by S only). Part A of a stage is refilled as soon as S of its tile is done.
+  static constexpr int NB_B = DVC / 64;
+  static constexpr int NB_A = NKB - NB_B;
   static constexpr int NP = PROD_WARPS * 32;
-  static constexpr int CPT = (CHUNKS + NP - 1) / NP;  // chunks per producer thread per tile
+  static constexpr int CPT_A = (KEYS * NB_A * 8 + NP - 1) / NP;   // chunks per thread, part A
+  static constexpr int CPT_B = (KEYS * NB_B * 8 + NP - 1) / NP;   // chunks per thread, part B
+  static_assert(NB_A >= 1 && NB_B >= 1, "both parts must be non-empty");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + QS_KB * QBLK;
   static constexpr int OFF_P = OFF_KV + STAGES * NKB * KVBLK;
@@ -64,9 +70,9 @@ struct MlaTraits {
   // mbarrier slots (8 bytes each), in this order
   static constexpr int BAR_Q = 0;                     // Q part in shared memory landed
   static constexpr int BAR_QT = 1;                    // Q part in TMEM written
-  static constexpr int BAR_KV_FULL = 2;               // [STAGES]
-  static constexpr int BAR_KV_EMPTY = BAR_KV_FULL + STAGES;   // [STAGES]
-  static constexpr int BAR_S_FULL = BAR_KV_EMPTY + STAGES;
+  static constexpr int BAR_KV_FULL = 2;               // [2 parts][STAGES]
+  static constexpr int BAR_KV_EMPTY = BAR_KV_FULL + 2 * STAGES;   // [2 parts][STAGES]
+  static constexpr int BAR_S_FULL = BAR_KV_EMPTY + 2 * STAGES;
   static constexpr int BAR_S_EMPTY = BAR_S_FULL + 1;
   static constexpr int BAR_P_FULL = BAR_S_EMPTY + 1;  // [2]
   static constexpr int BAR_P_FREE = BAR_P_FULL + 2;   // [2]
@@ -101,8 +107,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
   uint64_t* q_full = bars + Tr::BAR_Q;          // Q part in shared memory (TMA)
   uint64_t* qt_full = bars + Tr::BAR_QT;        // Q part in TMEM (softmax warps)
-  uint64_t* kv_full = bars + Tr::BAR_KV_FULL;   // [STAGES]
-  uint64_t* kv_empty = bars + Tr::BAR_KV_EMPTY; // [STAGES]
+  uint64_t* kvA_full = bars + Tr::BAR_KV_FULL;                  // [STAGES]
+  uint64_t* kvB_full = bars + Tr::BAR_KV_FULL + Tr::STAGES;     // [STAGES]
+  uint64_t* kvA_empty = bars + Tr::BAR_KV_EMPTY;                // [STAGES]
+  uint64_t* kvB_empty = bars + Tr::BAR_KV_EMPTY + Tr::STAGES;   // [STAGES]
   uint64_t* s_full = bars + Tr::BAR_S_FULL;
   uint64_t* s_empty = bars + Tr::BAR_S_EMPTY;
   uint64_t* p_full = bars + Tr::BAR_P_FULL;     // [2] P buffer written
@@ -128,8 +136,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     mbar_init(q_full, 1);
     mbar_init(qt_full, 128);
     for (int i = 0; i < Tr::STAGES; ++i) {
-      mbar_init(&kv_full[i], Tr::NP);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kvA_full[i], Tr::NP);
+      mbar_init(&kvB_full[i], Tr::NP);
+      mbar_init(&kvA_empty[i], 1);
+      mbar_init(&kvB_empty[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, 128);
@@ -192,28 +202,35 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
       const uint64_t pd0 = make_sdesc(smem_u32(p_smem), 16, 1024, 2);
       const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
-      auto issue_s = [&](int i) {
+      // column block at position j of part (0 = A, 1 = B) of this CTA's tiles
+      const int vb0 = dvc * Tr::NB_B;
+      auto blk_of = [&](int part, int j) { return part ? vb0 + j : (j < vb0 ? j : j + Tr::NB_B); };
+      // S = Q K^T over one part's column blocks; the first QT_KB column blocks of
+      // Q come from TMEM, the rest from smem. Part A is issued first (it starts
+      // the accumulation) and releases its blocks; part B completes S.
+      auto issue_s_part = [&](int i, int part) {
         const int st = i % Tr::STAGES;
         const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + st * NKB * Tr::KVBLK), 16, 1024, 2);
-        // S = Q K^T: the first QT_KB column blocks of Q come from TMEM, the rest from smem
+        const int nb = part ? Tr::NB_B : Tr::NB_A;
+#pragma unroll 1
+        for (int j = 0; j < nb; ++j) {
+          const int kb = blk_of(part, j);
+          if (kb < Tr::QT_KB) {
 #pragma unroll
-        for (int kb = 0; kb < Tr::QT_KB; ++kb) {
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts(s_tmem, qt_tmem + kb * 32 + kk * 8,
+                         kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S,
+                         (part | j | kk) ? 1u : 0u);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_f16_ts(s_tmem, qt_tmem + kb * 32 + kk * 8,
-                       kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S,
-                       (kb | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss(s_tmem, qd0 + (uint64_t)(((kb - Tr::QT_KB) * Tr::QBLK + kk * 32) >> 4),
+                         kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S,
+                         (part | j | kk) ? 1u : 0u);
           }
         }
-#pragma unroll
-        for (int kb = Tr::QT_KB; kb < NKB; ++kb) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_f16_ss(s_tmem, qd0 + (uint64_t)(((kb - Tr::QT_KB) * Tr::QBLK + kk * 32) >> 4),
-                       kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S, 1u);
-          }
-        }
-        mma_commit(s_full);
+        if (part == 0) mma_commit(&kvA_empty[st]);
+        else mma_commit(s_full);
       };
       auto issue_pv = [&](int j) {
         const int stj = j % Tr::STAGES;
@@ -224,22 +241,30 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         for (int kk = 0; kk < KEYS / 16; ++kk)
           mma_f16_ss(o_tmem, pd + (uint64_t)(kk * 32 >> 4), bd0 + (uint64_t)(kk * 16 * 128 >> 4),
                      Tr::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[stj]);
+        mma_commit(&kvB_empty[stj]);
         mma_commit(&p_free[j & 1]);
       };
       // Issue S_i and PV_j in whichever order their inputs become ready: S_i needs
       // tile i in shared memory and the S buffer drained by the softmax warps; PV_j
       // needs P_j. Bounded like every other wait.
-      int ns = 0, npv = 0;
+      int ns = 0, npv = 0, spart = 0;
       uint64_t t_mark = globaltimer_ns();
       uint32_t spins = 0;
       while (ok && npv < ntiles) {
         bool did = false;
-        if (ns < ntiles &&
-            mbar_try_wait(smem_u32(&kv_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1) &&
+        if (ns < ntiles && spart == 0 &&
+            mbar_try_wait(smem_u32(&kvA_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1) &&
             mbar_try_wait(smem_u32(s_empty), (ns & 1) ^ 1)) {
           tc_fence_after();
-          issue_s(ns);
+          issue_s_part(ns, 0);
+          spart = 1;
+          did = true;
+        }
+        if (ns < ntiles && spart == 1 &&
+            mbar_try_wait(smem_u32(&kvB_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1)) {
+          tc_fence_after();
+          issue_s_part(ns, 1);
+          spart = 0;
           ++ns;
           did = true;
         }
@@ -274,32 +299,50 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     // It lands in the 128-byte-swizzled K-major layout the tensor core reads:
     // column block q / 8, row r, 16-byte slot (q % 8) ^ (r % 8). Chunks past the
     // end of a row (padding up to the 64-column block) are written as zeros.
-    // Each thread keeps LAG tiles of cp.async groups in flight; once a group is
-    // complete it makes the writes visible to the tensor core (proxy fence) and
-    // arrives on that tile's full barrier.
+    // Once its copies of a part have landed, a thread makes them visible to the
+    // tensor core (proxy fence) and arrives on that part's full barrier.
     const int ptid = threadIdx.x - PROD_T0;
     const int row_bytes = a.Dqk * 2;
     const uint8_t* kv_b = reinterpret_cast<const uint8_t*>(kv) + (size_t)b * a.Lk * row_bytes;
     const uint32_t kv_base = smem_u32(kv_smem);
-    int issued = 0;
-    for (int i = 0; i < ntiles; ++i) {
-      const int st = i % Tr::STAGES;
-      if (!mbar_wait(&kv_empty[st], ((i / Tr::STAGES) & 1) ^ 1, a.ctl, abort_flag, kSiteMla, 1)) break;
-      const uint32_t stage = kv_base + st * NKB * Tr::KVBLK;
+    const int vb0 = dvc * Tr::NB_B;
+    // copy this thread's chunks of one part of tile i into its stage
+    auto gather_part = [&](int i, auto part_c) {
+      constexpr int PART = decltype(part_c)::value;
+      constexpr int NB = PART ? Tr::NB_B : Tr::NB_A;
+      constexpr int CPT = PART ? Tr::CPT_B : Tr::CPT_A;
+      const uint32_t stage = kv_base + (i % Tr::STAGES) * NKB * Tr::KVBLK;
 #pragma unroll
-      for (int j = 0; j < Tr::CPT; ++j) {
-        const int c = ptid + j * Tr::NP;
-        if (c < Tr::CHUNKS) {
-          const int r = c / Tr::CPR, q = c % Tr::CPR;
+      for (int jj = 0; jj < CPT; ++jj) {
+        const int c = ptid + jj * Tr::NP;
+        if (c < KEYS * NB * 8) {
+          const int r = c / (NB * 8);
+          const int rem = c - r * NB * 8;
+          const int j = rem >> 3, q8 = rem & 7;
+          const int kb = PART ? vb0 + j : (j < vb0 ? j : j + Tr::NB_B);
+          const int q = kb * 8 + q8;                  // 16-byte chunk within the row
           const int pos = (tile0 + i) * KEYS + r;
           const int v = pos < a.k ? __ldg(idx_row + pos) : -1;
           const int row = (v >= 0 && v < a.Lk) ? v : 0;   // invalid keys read row 0, masked later
           const bool in_row = q * 16 < row_bytes;
-          cp_async16(stage + (q >> 3) * Tr::KVBLK + r * 128 + (((q & 7) ^ (r & 7)) << 4),
+          cp_async16(stage + kb * Tr::KVBLK + r * 128 + ((q8 ^ (r & 7)) << 4),
                      kv_b + (size_t)row * row_bytes + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
         }
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
+      cp_async_commit();
+    };
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % Tr::STAGES;
+      const uint32_t ph = ((i / Tr::STAGES) & 1) ^ 1;
+      // part A is free once S of the tile that last used this stage is done ...
+      if (!mbar_wait(&kvA_empty[st], ph, a.ctl, abort_flag, kSiteMla, 1)) break;
+      gather_part(i, std::integral_constant<int, 0>{});
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(&kvA_full[st]);
+      // ... part B (the values) once PV of that tile is done
+      if (!mbar_wait(&kvB_empty[st], ph, a.ctl, abort_flag, kSiteMla, 14)) break;
+      gather_part(i, std::integral_constant<int, 1>{});
       if (ptid < 32) {
 #pragma unroll
         for (int hw = 0; hw < KEYS / 32; ++hw) {
@@ -309,19 +352,11 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
           if (ptid == 0) masks[st * 2 + hw] = m;   // slot free: PV of its previous tile is done
         }
       }
-      ++issued;
-      if (i >= Tr::LAG) {
-        asm volatile("cp.async.wait_group %0;" ::"n"(Tr::LAG) : "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(&kv_full[(i - Tr::LAG) % Tr::STAGES]);
-      }
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (!*abort_flag) {
+      cp_async_wait<0>();
       fence_proxy_async_smem();
-      for (int i = (issued > Tr::LAG ? issued - Tr::LAG : 0); i < issued; ++i)
-        mbar_arrive(&kv_full[i % Tr::STAGES]);
+      mbar_arrive(&kvB_full[st]);
     }
+    cp_async_wait_all();
   } else {
     // ------------------------------------------------ softmax / epilogue (warps 1..4)
     const int quad = warp & 3;
@@ -353,7 +388,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
       if (!mbar_wait(s_full, i & 1, a.ctl, abort_flag, kSiteMla, 8)) { ok = false; break; }
-      if (!mbar_wait(&kv_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 9)) { ok = false; break; }
+      if (!mbar_wait(&kvB_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 9)) { ok = false; break; }
       tc_fence_after();
       float x[KEYS];
       float tmax = -INFINITY;
