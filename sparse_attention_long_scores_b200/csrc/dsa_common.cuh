@@ -79,6 +79,21 @@ DSA_DEVICE_INLINE bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread is suspended for at most about `ns`
+// nanoseconds (the suspend-time hint) before the test fails. Lets one thread
+// poll several barriers in turn without sleeping on one of them for long.
+DSA_DEVICE_INLINE bool mbar_try_wait_for(uint32_t bar_addr, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking test of a phase (for polling several barriers in turn).
 DSA_DEVICE_INLINE bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
   uint32_t ok;

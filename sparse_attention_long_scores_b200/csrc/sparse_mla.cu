@@ -38,13 +38,9 @@ constexpr int PROD_WARPS = 8;                  // gather warps
 constexpr int MLA_THREADS = 32 + 128 + PROD_WARPS * 32;
 constexpr int PROD_T0 = 160;                   // first producer thread
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+// How long the MMA thread may sleep on one barrier while it polls the inputs of
+// S and PV in turn: short, so that whichever becomes ready first is issued.
+constexpr uint32_t kMmaPollNs = 100;
 
 template <int NKB, int DVC>
 struct MlaTraits {
@@ -253,22 +249,22 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       while (ok && npv < ntiles) {
         bool did = false;
         if (ns < ntiles && spart == 0 &&
-            mbar_try_wait(smem_u32(&kvA_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1) &&
-            mbar_try_wait(smem_u32(s_empty), (ns & 1) ^ 1)) {
+            mbar_try_wait_for(smem_u32(&kvA_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1, kMmaPollNs) &&
+            mbar_try_wait_for(smem_u32(s_empty), (ns & 1) ^ 1, kMmaPollNs)) {
           tc_fence_after();
           issue_s_part(ns, 0);
           spart = 1;
           did = true;
         }
         if (ns < ntiles && spart == 1 &&
-            mbar_try_wait(smem_u32(&kvB_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1)) {
+            mbar_try_wait_for(smem_u32(&kvB_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1, kMmaPollNs)) {
           tc_fence_after();
           issue_s_part(ns, 1);
           spart = 0;
           ++ns;
           did = true;
         }
-        if (npv < ns && mbar_try_wait(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1)) {
+        if (npv < ns && mbar_try_wait_for(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1, kMmaPollNs)) {
           tc_fence_after();
           issue_pv(npv);
           ++npv;
@@ -295,10 +291,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     }
   } else if (warp >= PROD_T0 / 32) {
     // ------------------------------------------------ gather producers
-    // Chunk c of a tile is 16 bytes: row r = c / CPR, chunk q = c % CPR of that row.
-    // It lands in the 128-byte-swizzled K-major layout the tensor core reads:
-    // column block q / 8, row r, 16-byte slot (q % 8) ^ (r % 8). Chunks past the
-    // end of a row (padding up to the 64-column block) are written as zeros.
+    // Chunk c of a part is 16 bytes: row r = c / (8 NB), then column block j and
+    // 16-byte chunk q8 within it. It lands in the 128-byte-swizzled K-major layout
+    // the tensor core reads: column block kb, row r, 16-byte slot q8 ^ (r % 8).
+    // Chunks past the end of a row (padding up to the 64-column block) are zeros.
     // Once its copies of a part have landed, a thread makes them visible to the
     // tensor core (proxy fence) and arrives on that part's full barrier.
     const int ptid = threadIdx.x - PROD_T0;
