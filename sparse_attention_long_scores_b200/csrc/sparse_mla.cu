@@ -89,6 +89,35 @@ struct MlaTraits {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
+// One part of S = Q K^T for a tile whose stage starts at descriptor kd0: part
+// A (PART = 0, the column blocks only S reads) or part B (PART = 1, the value
+// blocks of the CTA's slice DVCI of the output columns). Block order, offsets and
+// the operand form of every MMA are compile-time constants: Q's first QT_KB
+// column blocks are read from TMEM, the rest from shared memory. Issue from a
+// fully unrolled sequence costs about as much as the MMAs take to run; the same
+// sequence built from a runtime block index costs up to twice as much per MMA.
+template <int NKB, int DVC, int DVCI, int PART>
+__device__ __forceinline__ void issue_s_part(uint32_t s_tmem, uint32_t qt_tmem, uint64_t qd0, uint64_t kd0) {
+  using Tr = MlaTraits<NKB, DVC>;
+  constexpr int VB0 = DVCI * Tr::NB_B;
+  constexpr int NB = PART ? Tr::NB_B : Tr::NB_A;
+  static_assert(VB0 + Tr::NB_B <= NKB, "value blocks of the slice");
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    const int kb = PART ? VB0 + j : (j < VB0 ? j : j + Tr::NB_B);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t acc = (PART | j | kk) ? 1u : 0u;   // the first MMA of part A overwrites S
+      const uint64_t kdesc = kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4);
+      if (kb < Tr::QT_KB)
+        mma_f16_ts(s_tmem, qt_tmem + kb * 32 + kk * 8, kdesc, Tr::IDESC_S, acc);
+      else
+        mma_f16_ss(s_tmem, qd0 + (uint64_t)(((kb - Tr::QT_KB) * Tr::QBLK + kk * 32) >> 4), kdesc,
+                   Tr::IDESC_S, acc);
+    }
+  }
+}
+
 template <int NKB, int DVC>
 __global__ void __launch_bounds__(MLA_THREADS, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ kv,
@@ -198,35 +227,18 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
       const uint64_t pd0 = make_sdesc(smem_u32(p_smem), 16, 1024, 2);
       const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
-      // column block at position j of part (0 = A, 1 = B) of this CTA's tiles
-      const int vb0 = dvc * Tr::NB_B;
-      auto blk_of = [&](int part, int j) { return part ? vb0 + j : (j < vb0 ? j : j + Tr::NB_B); };
-      // S = Q K^T over one part's column blocks; the first QT_KB column blocks of
-      // Q come from TMEM, the rest from smem. Part A is issued first (it starts
-      // the accumulation) and releases its blocks; part B completes S.
-      auto issue_s_part = [&](int i, int part) {
-        const int st = i % Tr::STAGES;
-        const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + st * NKB * Tr::KVBLK), 16, 1024, 2);
-        const int nb = part ? Tr::NB_B : Tr::NB_A;
-#pragma unroll 1
-        for (int j = 0; j < nb; ++j) {
-          const int kb = blk_of(part, j);
-          if (kb < Tr::QT_KB) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ts(s_tmem, qt_tmem + kb * 32 + kk * 8,
-                         kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S,
-                         (part | j | kk) ? 1u : 0u);
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ss(s_tmem, qd0 + (uint64_t)(((kb - Tr::QT_KB) * Tr::QBLK + kk * 32) >> 4),
-                         kd0 + (uint64_t)((kb * Tr::KVBLK + kk * 32) >> 4), Tr::IDESC_S,
-                         (part | j | kk) ? 1u : 0u);
-          }
+      // S for tile i, part A (then part B): the slice index selects one of the
+      // compile-time block orders (output columns are split in at most two slices)
+      auto issue_s = [&](int i, int part) {
+        const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + (i % Tr::STAGES) * NKB * Tr::KVBLK), 16, 1024, 2);
+        if (dvc == 0) {
+          if (part == 0) issue_s_part<NKB, DVC, 0, 0>(s_tmem, qt_tmem, qd0, kd0);
+          else issue_s_part<NKB, DVC, 0, 1>(s_tmem, qt_tmem, qd0, kd0);
+        } else {
+          if (part == 0) issue_s_part<NKB, DVC, 1, 0>(s_tmem, qt_tmem, qd0, kd0);
+          else issue_s_part<NKB, DVC, 1, 1>(s_tmem, qt_tmem, qd0, kd0);
         }
-        if (part == 0) mma_commit(&kvA_empty[st]);
-        else mma_commit(s_full);
+        mma_commit(part == 0 ? &kvA_empty[i % Tr::STAGES] : s_full);
       };
       auto issue_pv = [&](int j) {
         const int stj = j % Tr::STAGES;
@@ -252,14 +264,14 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
             mbar_try_wait_for(smem_u32(&kvA_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1, kMmaPollNs) &&
             mbar_try_wait_for(smem_u32(s_empty), (ns & 1) ^ 1, kMmaPollNs)) {
           tc_fence_after();
-          issue_s_part(ns, 0);
+          issue_s(ns, 0);
           spart = 1;
           did = true;
         }
         if (ns < ntiles && spart == 1 &&
             mbar_try_wait_for(smem_u32(&kvB_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1, kMmaPollNs)) {
           tc_fence_after();
-          issue_s_part(ns, 1);
+          issue_s(ns, 1);
           spart = 0;
           ++ns;
           did = true;
