@@ -40,7 +40,7 @@ constexpr int PROD_T0 = 160;                   // first producer thread
 
 // How long the MMA thread may sleep on one barrier while it polls the inputs of
 // S and PV in turn: short, so that whichever becomes ready first is issued.
-constexpr uint32_t kMmaPollNs = 100;
+constexpr uint32_t kMmaPollNs = 40;
 
 template <int NKB, int DVC>
 struct MlaTraits {
@@ -91,11 +91,13 @@ struct MlaTraits {
 
 // One part of S = Q K^T for a tile whose stage starts at descriptor kd0: part
 // A (PART = 0, the column blocks only S reads) or part B (PART = 1, the value
-// blocks of the CTA's slice DVCI of the output columns). Block order, offsets and
-// the operand form of every MMA are compile-time constants: Q's first QT_KB
-// column blocks are read from TMEM, the rest from shared memory. Issue from a
-// fully unrolled sequence costs about as much as the MMAs take to run; the same
-// sequence built from a runtime block index costs up to twice as much per MMA.
+// blocks of the CTA's slice DVCI of the output columns).
+// Block order, offsets and the operand form of every MMA are compile-time
+// constants: Q's first QT_KB column blocks are read from TMEM, the rest from
+// shared memory. Issue from a fully unrolled sequence costs about as much as
+// the MMAs take to run; the same sequence built from a runtime block index
+// costs up to twice as much per MMA, and so does a part split into shorter
+// sequences with other work between them.
 template <int NKB, int DVC, int DVCI, int PART>
 __device__ __forceinline__ void issue_s_part(uint32_t s_tmem, uint32_t qt_tmem, uint64_t qd0, uint64_t kd0) {
   using Tr = MlaTraits<NKB, DVC>;
@@ -227,8 +229,9 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
       const uint64_t pd0 = make_sdesc(smem_u32(p_smem), 16, 1024, 2);
       const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
-      // S for tile i, part A (then part B): the slice index selects one of the
-      // compile-time block orders (output columns are split in at most two slices)
+      // Part `part` of S for tile i: the slice index selects one of the
+      // compile-time block orders (output columns are split in at most two
+      // slices). Part A ends by releasing its blocks, part B by handing S over.
       auto issue_s = [&](int i, int part) {
         const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + (i % Tr::STAGES) * NKB * Tr::KVBLK), 16, 1024, 2);
         if (dvc == 0) {
@@ -252,40 +255,52 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         mma_commit(&kvB_empty[stj]);
         mma_commit(&p_free[j & 1]);
       };
-      // Issue S_i and PV_j in whichever order their inputs become ready: S_i needs
-      // tile i in shared memory and the S buffer drained by the softmax warps; PV_j
-      // needs P_j. Bounded like every other wait.
+      // Issue S_i and PV_j in whichever order their inputs become ready, a ready
+      // PV first: S_i needs part A of tile i in shared memory and the S buffer
+      // drained by the softmax warps, then part B; PV_j needs P_j. The barriers
+      // are tested without blocking; only when nothing is ready does the thread
+      // sleep briefly. Bounded like every other wait.
       int ns = 0, npv = 0, spart = 0;
       uint64_t t_mark = globaltimer_ns();
       uint32_t spins = 0;
       while (ok && npv < ntiles) {
         bool did = false;
-        if (ns < ntiles && spart == 0 &&
-            mbar_try_wait_for(smem_u32(&kvA_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1, kMmaPollNs) &&
-            mbar_try_wait_for(smem_u32(s_empty), (ns & 1) ^ 1, kMmaPollNs)) {
-          tc_fence_after();
-          issue_s(ns, 0);
-          spart = 1;
-          did = true;
-        }
-        if (ns < ntiles && spart == 1 &&
-            mbar_try_wait_for(smem_u32(&kvB_full[ns % Tr::STAGES]), (ns / Tr::STAGES) & 1, kMmaPollNs)) {
-          tc_fence_after();
-          issue_s(ns, 1);
-          spart = 0;
-          ++ns;
-          did = true;
-        }
-        if (npv < ns && mbar_try_wait_for(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1, kMmaPollNs)) {
+        if (npv < ns && mbar_test_wait(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1)) {
           tc_fence_after();
           issue_pv(npv);
           ++npv;
           did = true;
         }
+        if (ns < ntiles) {
+          const int st = ns % Tr::STAGES;
+          const uint32_t ph = (ns / Tr::STAGES) & 1;
+          const bool ready = spart == 0 ? mbar_test_wait(smem_u32(&kvA_full[st]), ph) &&
+                                              mbar_test_wait(smem_u32(s_empty), (ns & 1) ^ 1)
+                                        : mbar_test_wait(smem_u32(&kvB_full[st]), ph);
+          if (ready) {
+            tc_fence_after();
+            issue_s(ns, spart);
+            if (spart) ++ns;
+            spart ^= 1;
+            did = true;
+          }
+        }
         if (did) {
           spins = 0;
           t_mark = globaltimer_ns();
-        } else if ((++spins & 63u) == 0) {
+          continue;
+        }
+        // nothing ready: sleep briefly on the barrier S waits for (else P's)
+        if (ns < ntiles) {
+          const int st = ns % Tr::STAGES;
+          const uint32_t ph = (ns / Tr::STAGES) & 1;
+          if (spart == 1) mbar_try_wait_for(smem_u32(&kvB_full[st]), ph, kMmaPollNs);
+          else if (!mbar_test_wait(smem_u32(&kvA_full[st]), ph)) mbar_try_wait_for(smem_u32(&kvA_full[st]), ph, kMmaPollNs);
+          else mbar_try_wait_for(smem_u32(s_empty), (ns & 1) ^ 1, kMmaPollNs);
+        } else {
+          mbar_try_wait_for(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1, kMmaPollNs);
+        }
+        if ((++spins & 63u) == 0) {
           if (*abort_flag || *reinterpret_cast<volatile int*>(a.ctl.status) != 0) {
             *abort_flag = 1;
             ok = false;
