@@ -10,16 +10,16 @@
 //     online softmax over the key tiles     (base 2, lazy rescale of O)
 //     O[h, chunk] += P[h,s] . c_s[chunk]    (tcgen05, M = 128, N = DVC, K = 64 keys)
 // Layout of the work:
-//   warp 0      tcgen05 issuer: Q once (TMA tiles), then S_i = Q K_i^T into one of
-//               two TMEM buffers, then O += P_{i-1} V_{i-1};
-//   warps 5..12 gather producers: the selected latent rows of each 32-key tile,
-//               16 bytes per thread per load (register-staged, several rows in
-//               flight per thread), stored straight into the 128-byte-swizzled
-//               K-major layout the tensor core reads, into a 2-stage ring. A TMA
-//               gather4 costs about as much issue time per 512 bytes as these
-//               warps need for a whole tile, so the rows are gathered by threads;
-//   warps 1..4  softmax: one head (TMEM lane) per thread. Writes P (bf16) to
-//               shared memory in the 64-byte-swizzled K-major layout, rescales O
+//   warp 0      tcgen05 issuer: Q's shared-memory part once (TMA tiles), then for
+//               each 64-key tile S_i = Q K_i^T into one of two TMEM buffers and
+//               O += P_i V_i with P read from TMEM;
+//   warps 5..12 gather producers: the selected latent rows of each tile, 16 bytes
+//               per thread per cp.async, stored straight into the 128-byte-
+//               swizzled K-major layout the tensor core reads, into a 2-stage
+//               ring. A TMA gather4 costs about as much issue time per 512 bytes
+//               as these warps need for a whole tile, so threads gather the rows;
+//   warps 1..4  softmax: one head (TMEM lane) per thread. Reads S_i, writes P_i
+//               (bf16) over the first half of S_i's own TMEM buffer, rescales O
 //               in TMEM only when the running max grew by more than 2^8, and
 //               normalises at the end.
 // O for 128 heads x 512 values in fp32 would fill all of TMEM, so the value
@@ -46,7 +46,7 @@ template <int NKB, int DVC>
 struct MlaTraits {
   static constexpr int QBLK = 128 * 128;            // one 64-column block of Q: 128 rows x 128 B
   static constexpr int KVBLK = KEYS * 128;          // one 64-column block of a KV tile
-  static constexpr int QT_KB = (NKB == 9) ? 6 : 1;  // Q column blocks held in TMEM
+  static constexpr int QT_KB = (NKB == 9) ? 4 : 1;  // Q column blocks held in TMEM
   static constexpr int QS_KB = NKB - QT_KB;         // Q column blocks held in shared memory
   static constexpr int STAGES = 2;                  // KV ring depth
   // A tile's column blocks come in two parts: part B = the DVC / 64 value blocks
@@ -60,30 +60,29 @@ struct MlaTraits {
   static_assert(NB_A >= 1 && NB_B >= 1, "both parts must be non-empty");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + QS_KB * QBLK;
-  static constexpr int OFF_P = OFF_KV + STAGES * NKB * KVBLK;
-  static constexpr int PBYTES = 128 * KEYS * 2;    // one P buffer (bf16, 128 heads x KEYS)
-  static constexpr int OFF_BAR = OFF_P + 2 * PBYTES;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * NKB * KVBLK;
   // mbarrier slots (8 bytes each), in this order
   static constexpr int BAR_Q = 0;                     // Q part in shared memory landed
   static constexpr int BAR_QT = 1;                    // Q part in TMEM written
   static constexpr int BAR_KV_FULL = 2;               // [2 parts][STAGES]
   static constexpr int BAR_KV_EMPTY = BAR_KV_FULL + 2 * STAGES;   // [2 parts][STAGES]
-  static constexpr int BAR_S_FULL = BAR_KV_EMPTY + 2 * STAGES;
-  static constexpr int BAR_S_EMPTY = BAR_S_FULL + 1;
-  static constexpr int BAR_P_FULL = BAR_S_EMPTY + 1;  // [2]
-  static constexpr int BAR_P_FREE = BAR_P_FULL + 2;   // [2]
-  static constexpr int BAR_DONE = BAR_P_FREE + 2;
+  static constexpr int BAR_S_FULL = BAR_KV_EMPTY + 2 * STAGES;   // [2] S buffer computed
+  static constexpr int BAR_P_FULL = BAR_S_FULL + 2;   // [2] P written over its S buffer
+  static constexpr int BAR_PV_DONE = BAR_P_FULL + 2;  // [2] PV of a tile of that parity done
+  static constexpr int BAR_DONE = BAR_PV_DONE + 2;
   static constexpr int NUM_BARS = BAR_DONE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 48 + 1024;
-  // TMEM columns: O [0, DVC), S [DVC, DVC + KEYS), Q part [DVC + KEYS, ... + 32 * QT_KB)
+  // TMEM columns: O [0, DVC), two S buffers [DVC, DVC + 2 KEYS) (P_i, bf16, is
+  // written over the first KEYS / 2 columns of S_i's buffer), Q part after them
   static constexpr int COL_S = DVC;
-  static constexpr int COL_Q = DVC + KEYS;
+  static constexpr int COL_Q = DVC + 2 * KEYS;
   static constexpr int COLS_USED = COL_Q + 32 * QT_KB;
   static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_S = make_idesc(1, 1, 0, 0, KEYS, 128);   // bf16, K-major both
-  static_assert(KEYS == 64, "P layout assumes 128-byte rows");
-  static constexpr uint32_t IDESC_PV = make_idesc(1, 1, 0, 1, DVC, 128);   // B (values) MN-major
+  static_assert(KEYS == 64, "masks hold two 32-key words per tile");
+  // PV: A = P from TMEM, B = values MN-major
+  static constexpr uint32_t IDESC_PV = make_idesc(1, 1, 0, 1, DVC, 128);
   static_assert(DVC % 64 == 0 && DVC <= 256, "DVC");
   static_assert(COLS_USED <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -130,7 +129,6 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* q_smem = smem + Tr::OFF_Q;
   uint8_t* kv_smem = smem + Tr::OFF_KV;
-  uint8_t* p_smem = smem + Tr::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
   uint64_t* q_full = bars + Tr::BAR_Q;          // Q part in shared memory (TMA)
   uint64_t* qt_full = bars + Tr::BAR_QT;        // Q part in TMEM (softmax warps)
@@ -138,10 +136,9 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   uint64_t* kvB_full = bars + Tr::BAR_KV_FULL + Tr::STAGES;     // [STAGES]
   uint64_t* kvA_empty = bars + Tr::BAR_KV_EMPTY;                // [STAGES]
   uint64_t* kvB_empty = bars + Tr::BAR_KV_EMPTY + Tr::STAGES;   // [STAGES]
-  uint64_t* s_full = bars + Tr::BAR_S_FULL;
-  uint64_t* s_empty = bars + Tr::BAR_S_EMPTY;
-  uint64_t* p_full = bars + Tr::BAR_P_FULL;     // [2] P buffer written
-  uint64_t* p_free = bars + Tr::BAR_P_FREE;     // [2] PV that read the P buffer is done
+  uint64_t* s_full = bars + Tr::BAR_S_FULL;     // [2] S_i computed (buffer i % 2)
+  uint64_t* p_full = bars + Tr::BAR_P_FULL;     // [2] P_i written over S_i
+  uint64_t* pv_done = bars + Tr::BAR_PV_DONE;   // [2] PV_i done (tile parity)
   uint64_t* done_bar = bars + Tr::BAR_DONE;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Tr::OFF_MISC);
   uint32_t* tmem_slot = misc;
@@ -168,11 +165,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       mbar_init(&kvA_empty[i], 1);
       mbar_init(&kvB_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, 128);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
-      mbar_init(&p_free[i], 1);
+      mbar_init(&pv_done[i], 1);
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -227,39 +223,42 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       // Descriptors are built once; per MMA only the start-address field moves
       // (byte offset / 16 added to the low bits, which never carry: smem < 256 KB).
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
-      const uint64_t pd0 = make_sdesc(smem_u32(p_smem), 16, 1024, 2);
       const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
-      // Part `part` of S for tile i: the slice index selects one of the
-      // compile-time block orders (output columns are split in at most two
-      // slices). Part A ends by releasing its blocks, part B by handing S over.
+      // Part `part` of S for tile i into buffer i % 2: the slice index selects
+      // one of the compile-time block orders (output columns are split in at
+      // most two slices). Part A ends by releasing its blocks, part B by handing
+      // S over.
       auto issue_s = [&](int i, int part) {
         const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + (i % Tr::STAGES) * NKB * Tr::KVBLK), 16, 1024, 2);
+        const uint32_t sb = s_tmem + (uint32_t)((i & 1) * KEYS);
         if (dvc == 0) {
-          if (part == 0) issue_s_part<NKB, DVC, 0, 0>(s_tmem, qt_tmem, qd0, kd0);
-          else issue_s_part<NKB, DVC, 0, 1>(s_tmem, qt_tmem, qd0, kd0);
+          if (part == 0) issue_s_part<NKB, DVC, 0, 0>(sb, qt_tmem, qd0, kd0);
+          else issue_s_part<NKB, DVC, 0, 1>(sb, qt_tmem, qd0, kd0);
         } else {
-          if (part == 0) issue_s_part<NKB, DVC, 1, 0>(s_tmem, qt_tmem, qd0, kd0);
-          else issue_s_part<NKB, DVC, 1, 1>(s_tmem, qt_tmem, qd0, kd0);
+          if (part == 0) issue_s_part<NKB, DVC, 1, 0>(sb, qt_tmem, qd0, kd0);
+          else issue_s_part<NKB, DVC, 1, 1>(sb, qt_tmem, qd0, kd0);
         }
-        mma_commit(part == 0 ? &kvA_empty[i % Tr::STAGES] : s_full);
+        mma_commit(part == 0 ? &kvA_empty[i % Tr::STAGES] : &s_full[i & 1]);
       };
       auto issue_pv = [&](int j) {
         const int stj = j % Tr::STAGES;
         const uint64_t bd0 = make_sdesc(smem_u32(kv_smem + stj * NKB * Tr::KVBLK) + v_off,
                                         Tr::KVBLK, 1024, 2);
-        const uint64_t pd = pd0 + (uint64_t)(((j & 1) * Tr::PBYTES) >> 4);
+        const uint32_t pt = s_tmem + (uint32_t)((j & 1) * KEYS);   // P_j: 16 keys per 8 columns
 #pragma unroll
         for (int kk = 0; kk < KEYS / 16; ++kk)
-          mma_f16_ss(o_tmem, pd + (uint64_t)(kk * 32 >> 4), bd0 + (uint64_t)(kk * 16 * 128 >> 4),
-                     Tr::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_f16_ts(o_tmem, pt + kk * 8, bd0 + (uint64_t)(kk * 16 * 128 >> 4), Tr::IDESC_PV,
+                     (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&kvB_empty[stj]);
-        mma_commit(&p_free[j & 1]);
+        mma_commit(&pv_done[j & 1]);
       };
       // Issue S_i and PV_j in whichever order their inputs become ready, a ready
-      // PV first: S_i needs part A of tile i in shared memory and the S buffer
-      // drained by the softmax warps, then part B; PV_j needs P_j. The barriers
-      // are tested without blocking; only when nothing is ready does the thread
-      // sleep briefly. Bounded like every other wait.
+      // PV first: S_i needs part A of tile i in shared memory and its TMEM buffer
+      // free, which it is once PV_{i-2} (the reader of P_{i-2}, written over the
+      // same buffer) has been issued: the tensor pipe runs the MMAs in order.
+      // Then part B. PV_j needs P_j. The barriers are tested without blocking;
+      // only when nothing is ready does the thread sleep briefly. Bounded like
+      // every other wait.
       int ns = 0, npv = 0, spart = 0;
       uint64_t t_mark = globaltimer_ns();
       uint32_t spins = 0;
@@ -274,8 +273,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         if (ns < ntiles) {
           const int st = ns % Tr::STAGES;
           const uint32_t ph = (ns / Tr::STAGES) & 1;
-          const bool ready = spart == 0 ? mbar_test_wait(smem_u32(&kvA_full[st]), ph) &&
-                                              mbar_test_wait(smem_u32(s_empty), (ns & 1) ^ 1)
+          const bool ready = spart == 0 ? npv >= ns - 1 && mbar_test_wait(smem_u32(&kvA_full[st]), ph)
                                         : mbar_test_wait(smem_u32(&kvB_full[st]), ph);
           if (ready) {
             tc_fence_after();
@@ -291,15 +289,14 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
           continue;
         }
         // nothing ready: sleep briefly on the barrier S waits for (else P's)
-        if (ns < ntiles) {
-          const int st = ns % Tr::STAGES;
-          const uint32_t ph = (ns / Tr::STAGES) & 1;
-          if (spart == 1) mbar_try_wait_for(smem_u32(&kvB_full[st]), ph, kMmaPollNs);
-          else if (!mbar_test_wait(smem_u32(&kvA_full[st]), ph)) mbar_try_wait_for(smem_u32(&kvA_full[st]), ph, kMmaPollNs);
-          else mbar_try_wait_for(smem_u32(s_empty), (ns & 1) ^ 1, kMmaPollNs);
-        } else {
+        const int st_n = ns % Tr::STAGES;
+        const uint32_t ph_n = (ns / Tr::STAGES) & 1;
+        if (ns < ntiles && spart == 1)
+          mbar_try_wait_for(smem_u32(&kvB_full[st_n]), ph_n, kMmaPollNs);
+        else if (ns < ntiles && npv >= ns - 1)
+          mbar_try_wait_for(smem_u32(&kvA_full[st_n]), ph_n, kMmaPollNs);
+        else
           mbar_try_wait_for(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1, kMmaPollNs);
-        }
         if ((++spins & 63u) == 0) {
           if (*abort_flag || *reinterpret_cast<volatile int*>(a.ctl.status) != 0) {
             *abort_flag = 1;
@@ -410,15 +407,16 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
-      if (!mbar_wait(s_full, i & 1, a.ctl, abort_flag, kSiteMla, 8)) { ok = false; break; }
+      if (!mbar_wait(&s_full[i & 1], (i >> 1) & 1, a.ctl, abort_flag, kSiteMla, 8)) { ok = false; break; }
       if (!mbar_wait(&kvB_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 9)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t sbuf = s_tmem + (uint32_t)((i & 1) * KEYS) + lane_off;   // this head's S_i
       float x[KEYS];
       float tmax = -INFINITY;
 #pragma unroll
       for (int hw = 0; hw < KEYS / 32; ++hw) {
         uint32_t r[32];
-        tmem_ld32(s_tmem + lane_off + hw * 32, r);
+        tmem_ld32(sbuf + hw * 32, r);
         tmem_wait_ld();
         const uint32_t m = masks[st * 2 + hw];
 #pragma unroll
@@ -427,14 +425,12 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
           tmax = fmaxf(tmax, x[hw * 32 + j]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(s_empty);
       const bool grow = tmax > m_used + 8.0f;
       const float m_new = grow ? tmax : m_used;
       const bool need_o = grow && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
         // O is rescaled in place: PV_{i-1} (the last one issued) must be done
-        if (!mbar_wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
+        if (!mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
         tc_fence_after();
         const float alpha = need_o ? ex2(m_used - m_new) : 1.f;
 #pragma unroll 1
@@ -462,21 +458,15 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         pk[j] = pack_bf16x2(p0, p1);
       }
       l += psum0 + psum1;
-      // P buffer i % 2 is free once PV_{i-2} is done
-      if (i >= 2 && !mbar_wait(&p_free[i & 1], ((i >> 1) & 1) ^ 1, a.ctl, abort_flag, kSiteMla, 13)) { ok = false; break; }
-      // P row h: 64 bf16 = eight 16-byte chunks, 128-byte swizzle (chunk ^= h % 8)
-      uint8_t* prow = p_smem + (i & 1) * Tr::PBYTES + h * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int pc = c ^ (h & 7);
-        *reinterpret_cast<uint4*>(prow + pc * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      // P_i over the first half of S_i's buffer (S_i is in registers already;
+      // PV_{i-2}, the last reader of this buffer, finished before S_i did)
+      tmem_st32(sbuf, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[i & 1]);
     }
     if (ok && ntiles > 0) {
-      ok = mbar_wait(&p_free[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 11);
+      ok = mbar_wait(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 11);
       tc_fence_after();
     }
     if (ok) {
