@@ -17,6 +17,7 @@ oracle on a bounded sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -35,6 +36,16 @@ import torch  # noqa: E402
 from dsa_inputs import CONFIG_ORDER, CONFIGS, gen_inputs  # noqa: E402
 
 METRIC = "DSA prefill tokens/s at 32K ctx; decode tokens/s at 128K ctx (k=2048), %roofline"
+CSRC = os.path.join(ROOT, "sparse_attention_long_scores_b200", "csrc")
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum from one ncu
+# capture of the small profile case, see --profile-case), with the query rows that
+# launch processed and the SHA-256 of the kernel's source file when it was taken. A
+# full launch's traffic is scaled from it by the rows it processes (the per-row Q read
+# and output write dominate; the once-per-sequence latent rows are under 1 %). When
+# the source has changed since the capture the figure no longer describes the kernel,
+# and the traffic is reported as null.
+TRAFFIC = {}
 DTYPE = "fp8_e4m3+bf16"
 
 
@@ -167,6 +178,16 @@ def barrier(world: int):
         dist.barrier()
 
 
+def traffic_per_launch(kernel: str, mode: str, rows_per_launch: float):
+    ent = TRAFFIC.get((kernel, mode))
+    if not ent:
+        return None
+    with open(os.path.join(CSRC, ent["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != ent["sha256"]:
+            return None
+    return ent["bytes"] * rows_per_launch / ent["rows"]
+
+
 def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk: dict,
                   sampler: ClockSampler | None, e2e: bool):
     import sparse_attention_long_scores_b200 as dsa
@@ -227,6 +248,8 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
         roof["sparse_mla"] = {"bound": "tensor", "achieved": a, "peak": pk["bf16_sustained"],
                               "unit": "TFLOP/s", "frac": a / pk["bf16_sustained"],
                               "peak_note": "measured bf16 sustained"}
+    for k, r in roof.items():
+        r["traffic"] = traffic_per_launch(k, cfg.mode, cfg.B * cfg.Lq / kernels[k]["launches_per_step"])
     res = {"cfg": cfg, "ms": ms, "tokens_per_s": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, ms),
            "kernels": kernels,
            "roof": roof, "launches": launches, "clocks": clocks, "work": w}
@@ -293,8 +316,8 @@ def oracle_sample(cfg, rows: int, seed: int = 4242):
     return run, pos
 
 
-def cpu_baseline(cfg, budget_s: float = 15.0) -> dict:
-    run, pos = oracle_sample(cfg, 64)
+def cpu_baseline(cfg, budget_s: float = 20.0) -> dict:
+    run, pos = oracle_sample(cfg, 1024)
     t0 = time.perf_counter()
     done = 0
     for i in range(len(pos)):
@@ -343,6 +366,33 @@ def reference_arm(args):
 # ---------------------------------------------------------------------------
 
 
+PROFILE_CASES = {
+    # one 2048-row prefill chunk of the 8K workload (rows 6144..8191, all keys causal)
+    "prefill_chunk": ("prefill_8k", dict(Lq=2048, q_pos0=6144)),
+    # 16 decode sequences against 131072 cached keys
+    "decode_small": ("decode_128k", dict(B=16)),
+}
+
+
+def profile_case(name: str) -> None:
+    """Two untimed forwards of a small case, for an ncu capture of its kernels
+    (the second forward's launches are the ones to capture)."""
+    import sparse_attention_long_scores_b200 as dsa
+    from sparse_attention_long_scores_b200.build import build
+
+    build()
+    torch.cuda.set_device(0)
+    base, kw = PROFILE_CASES[name]
+    cfg = CONFIGS[base].with_(**kw)
+    inp = gen_inputs(cfg, "cuda")
+    p = dsa.Problem.from_config(cfg)
+    for _ in range(2):
+        dsa.forward(p, inp)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    print(f"profile case {name}: {cfg}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -354,7 +404,12 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run a small untimed case for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -391,8 +446,8 @@ def main():
         cfg = pre["cfg"]
         dom_name = max(pre["kernels"], key=lambda k: pre["kernels"][k]["ms_per_step"])
         dom = dict(pre["roof"].get(dom_name, {}))
-        dom.update({"kernel": dom_name, "traffic": None,
-                    "peak_source": pk["source"]})
+        dom.update({"kernel": dom_name, "peak_source": pk["source"]})
+        dom.setdefault("traffic", None)
         line = {
             "metric": METRIC, "value": pre["tokens_per_s"], "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
