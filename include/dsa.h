@@ -125,15 +125,18 @@ int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
  * outputs as dsa_sparse_mla_fwd and calls no allocator: the key-split partial
  * results live in a 16 MiB array compiled into the library, which every GPU
  * that loads the library holds until the process exits.
- *   - Shapes whose split partials need more than 16 MiB are rejected with
- *     DSA_ERR_UNSUPPORTED_SHAPE (for H = 128, Dv = 512, k = 2048 that is 8 to
- *     147 query tokens; up to 7 tokens, and 148 or more, are accepted).
+ *   - When the partials of the recommended number of key splits (the one
+ *     dsa_sparse_mla_workspace_size sizes for) need more than 16 MiB, the
+ *     largest number of splits whose partials fit is used instead (one split
+ *     needs none), so every shape dsa_sparse_mla_fwd accepts is accepted.
  *   - The first call on a device looks up the array's device address with the
  *     device current; make that first call before any stream capture.
  *   - All calls share the one array and every call fully overwrites the part it
  *     uses (nothing needs clearing), so calls that overlap on the GPU (other
  *     streams, other host threads) race with each other: serialise them.
- *   - Results equal dsa_sparse_mla_fwd for the same shape.
+ *   - Results equal dsa_sparse_mla_fwd's for the same shape when the
+ *     recommended splits fit, and otherwise differ from them only by the
+ *     rounding of a different merge order.
  */
 int dsa_sparse_mla_fwd_noalloc(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
                                uint16_t* out, float* lse, int B, int Lq, int Lk, int H, int Dqk,

@@ -194,11 +194,15 @@ int indexer_piece_keys(int B, int rows, int t_blk, int keys_max, int num_sms) {
 
 int mla_n_dv(int Dv) { return Dv == 512 ? 2 : 1; }
 
+// Key splits of the attention: as many as keep all CTAs in one wave. Every CTA
+// pays a fixed cost (Q staging, pipeline fill, epilogue) of about three key
+// tiles, so a second wave of short CTAs costs more than it saves; each split
+// keeps at least 4 tiles, and at most 16 splits (the combine kernel's limit).
 int mla_splits(int B, int Lq, int Dv, int k, int num_sms) {
   long long ctas = (long long)B * Lq * mla_n_dv(Dv);
+  if (ctas >= num_sms) return 1;
   int tiles = k / 64 > 0 ? k / 64 : 1;   // 64-key tiles
-  if (ctas >= 2LL * num_sms) return 1;
-  int s = (int)((4LL * num_sms + ctas - 1) / ctas);
+  int s = (int)(num_sms / ctas);
   int max_s = tiles / 4 > 1 ? tiles / 4 : 1;
   if (s > max_s) s = max_s;
   if (s > 16) s = 16;
@@ -221,9 +225,12 @@ int assumed_sms() {
 int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t* out, float* lse,
             int B, int Lq, int Lk, int H, int Dqk, int Dv, int k, float sm_scale, void* ws,
             size_t ws_bytes, const dsa::DevCtl& ctl, int num_sms, cudaStream_t stream,
-            Recorder& rec = g_no_rec) {
+            Recorder& rec = g_no_rec, bool fit_splits = false) {
   (void)num_sms;
   int splits = mla_splits(B, Lq, Dv, k, assumed_sms());
+  // fit_splits: use fewer key splits rather than fail when the partials of the
+  // recommended count do not fit (one split needs none)
+  while (fit_splits && splits > 1 && mla_ws_bytes(B, Lq, H, Dv, splits) > ws_bytes) --splits;
   size_t need = mla_ws_bytes(B, Lq, H, Dv, splits);
   if (ws_bytes < need)
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "sparse MLA workspace: need %zu bytes, got %zu", need, ws_bytes);
@@ -498,19 +505,14 @@ int dsa_sparse_mla_fwd_noalloc(const uint16_t* q, const uint16_t* kv, const int3
   DSA_TRY(check_k(k, 4096));
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
     return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
-  const size_t need = mla_ws_bytes(B, Lq, H, Dv, mla_splits(B, Lq, Dv, k, assumed_sms()));
-  if (need > kNoAllocScratchBytes)
-    return fail(DSA_ERR_UNSUPPORTED_SHAPE,
-                "dsa_sparse_mla_fwd_noalloc: this shape needs %zu bytes of scratch but the built-in "
-                "scratch holds %zu; use dsa_sparse_mla_fwd with a workspace",
-                need, kNoAllocScratchBytes);
   dsa::DevCtl ctl;
   int sms = 0;
   DSA_TRY(device_ctl(ctl, sms));
   void* scratch = nullptr;
   DSA_TRY(noalloc_scratch(&scratch));
   return run_mla(q, kv, idx, out, lse, B, Lq, Lk, H, Dqk, Dv, k, sm_scale, scratch,
-                 kNoAllocScratchBytes, ctl, sms, static_cast<cudaStream_t>(stream));
+                 kNoAllocScratchBytes, ctl, sms, static_cast<cudaStream_t>(stream), g_no_rec,
+                 /*fit_splits=*/true);
 }
 
 size_t dsa_forward_workspace_size(const dsa_problem* p) {

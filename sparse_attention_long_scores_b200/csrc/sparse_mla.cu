@@ -534,34 +534,53 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
 }
 
 // Merge key-split partials: out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-__global__ void mla_combine_kernel(const MlaArgs a) {
+// One CTA per (token, head) row, four value columns per thread; the weights of
+// the (at most kMaxSplits) partials are computed once and all partial loads of a
+// thread are issued before any is used. Dv is a multiple of 4 (512 or 64).
+constexpr int kMaxSplits = 16;
+constexpr int kCombineThreads = 128;
+__global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const MlaArgs a) {
   const long long row = blockIdx.x;  // token * H + h
   const long long token = row / a.H;
   const int h = (int)(row % a.H);
+  const float* ml0 = a.part_ml + (token * a.splits * a.H + h) * 2;
+  const long long ml_stride = (long long)a.H * 2;
   float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) {
-    const float* ml = a.part_ml + ((token * a.splits + s) * a.H + h) * 2;
-    if (ml[1] > 0.f) M = fmaxf(M, ml[0]);
-  }
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s)
+    if (s < a.splits && ml0[s * ml_stride + 1] > 0.f) M = fmaxf(M, ml0[s * ml_stride]);
+  float f[kMaxSplits];
   float L = 0.f;
-  for (int s = 0; s < a.splits; ++s) {
-    const float* ml = a.part_ml + ((token * a.splits + s) * a.H + h) * 2;
-    if (ml[1] > 0.f) L += ml[1] * ex2(ml[0] - M);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    f[s] = 0.f;
+    if (s < a.splits && ml0[s * ml_stride + 1] > 0.f) {
+      f[s] = ex2(ml0[s * ml_stride] - M);
+      L += ml0[s * ml_stride + 1] * f[s];
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
+  const float* o0 = a.part_o + (token * a.splits * a.H + h) * (long long)a.Dv;
+  const long long o_stride = (long long)a.H * a.Dv;
   uint16_t* orow = a.out + row * (long long)a.Dv;
-  for (int c = threadIdx.x * 2; c < a.Dv; c += blockDim.x * 2) {
-    float acc0 = 0.f, acc1 = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
-      const long long pr = (token * a.splits + s) * a.H + h;
-      const float* ml = a.part_ml + pr * 2;
-      if (!(ml[1] > 0.f)) continue;
-      const float f = ex2(ml[0] - M);
-      const float2 v = *reinterpret_cast<const float2*>(a.part_o + pr * a.Dv + c);
-      acc0 = fmaf(v.x, f, acc0);
-      acc1 = fmaf(v.y, f, acc1);
+  for (int c = threadIdx.x * 4; c < a.Dv; c += kCombineThreads * 4) {
+    float4 v[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+      v[s] = f[s] != 0.f ? __ldcs(reinterpret_cast<const float4*>(o0 + s * o_stride + c))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      acc.x = fmaf(v[s].x, f[s], acc.x);
+      acc.y = fmaf(v[s].y, f[s], acc.y);
+      acc.z = fmaf(v[s].z, f[s], acc.z);
+      acc.w = fmaf(v[s].w, f[s], acc.w);
     }
-    *reinterpret_cast<uint32_t*>(orow + c) = pack_bf16x2(acc0 * inv, acc1 * inv);
+    uint2 packed;
+    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(orow + c) = packed;
   }
   if (threadIdx.x == 0 && a.lse != nullptr)
     a.lse[row] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
@@ -593,7 +612,7 @@ cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const uint16_t* kv, con
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t stream) {
   long long rows = (long long)a.B * a.Lq * a.H;
   if (rows <= 0) return cudaSuccess;
-  mla_combine_kernel<<<(unsigned)rows, 128, 0, stream>>>(a);
+  mla_combine_kernel<<<(unsigned)rows, kCombineThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

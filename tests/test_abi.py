@@ -92,9 +92,11 @@ def test_workspace_sizes(L):
         full = cfg.B * cfg.Lq * cfg.Lk * 4
         idx = cfg.B * cfg.Lq * cfg.k * 4
         assert n < idx + max(full // 8, 256 << 20), name
-    # decode splits keys: needs a partial-output buffer
+    # a small decode batch splits keys (one wave of CTAs): needs a partial-output
+    # buffer; 64 sequences already fill the SMs with one split
     d = CONFIGS["decode_128k"]
-    assert dsa.sparse_mla_workspace_size(d.B, d.Lq, d.Lk, d.H, d.Dqk, d.Dv, d.k) > 0
+    assert dsa.sparse_mla_workspace_size(8, d.Lq, d.Lk, d.H, d.Dqk, d.Dv, d.k) > 0
+    assert dsa.sparse_mla_workspace_size(d.B, d.Lq, d.Lk, d.H, d.Dqk, d.Dv, d.k) == 0
     pf = CONFIGS["prefill_32k"]
     assert dsa.sparse_mla_workspace_size(pf.B, pf.Lq, pf.Lk, pf.H, pf.Dqk, pf.Dv, pf.k) == 0
 
