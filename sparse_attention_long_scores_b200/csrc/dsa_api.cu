@@ -246,6 +246,7 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
   a.scale_log2 = sm_scale * 1.4426950408889634f;
   a.n_dv = mla_n_dv(Dv);
   a.splits = splits;
+  a.wave = num_sms > 0 ? num_sms : assumed_sms();
   a.ctl = ctl;
   if (splits > 1) {
     size_t tok = (size_t)B * Lq;

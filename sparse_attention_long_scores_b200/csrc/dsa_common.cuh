@@ -137,6 +137,12 @@ DSA_DEVICE_INLINE bool mbar_wait(uint64_t* bar, uint32_t parity, const DevCtl& c
 // ---------------------------------------------------------------------------
 // TMA (the tensor map lives in kernel parameter space: __grid_constant__)
 // ---------------------------------------------------------------------------
+// A hint that pulls `bytes` of global memory at `p` into L2 ahead of use (no data
+// is returned); both must be multiples of 16 (the caller checks).
+DSA_DEVICE_INLINE void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 DSA_DEVICE_INLINE void tma_prefetch_map(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

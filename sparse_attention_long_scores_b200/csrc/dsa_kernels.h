@@ -62,6 +62,8 @@ struct MlaArgs {
   float scale_log2;    // sm_scale * log2(e)
   int n_dv;            // value chunks per token
   int splits;          // key splits per token
+  int wave;            // CTAs resident at once (one per SM): the next CTA an SM runs
+                       // is about this many block indices further on
   DevCtl ctl;
 };
 // (H, Dqk, Dv) in {(8,80,64), (128,576,512)}.

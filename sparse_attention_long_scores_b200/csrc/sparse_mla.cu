@@ -156,6 +156,20 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   const int b = (int)(token / a.Lq);
   const int32_t* idx_row = a.idx + token * a.k;
 
+  // Warm L2 for the Q and index rows of the CTA that will probably run next on
+  // this SM (one wave of block indices further on): its prologue waits on them.
+  if (warp == 5 && lane == 0) {
+    const long long nb = (long long)blockIdx.x + a.wave;
+    if (nb < (long long)gridDim.x) {
+      const long long ntok = nb / per_token;
+      const uint8_t* qn = reinterpret_cast<const uint8_t*>(a.q) + ntok * a.H * (long long)a.Dqk * 2;
+      const uint32_t qbytes = (uint32_t)(a.H * a.Dqk * 2);
+      if ((reinterpret_cast<uintptr_t>(qn) & 15) == 0 && (qbytes & 15) == 0) bulk_prefetch_l2(qn, qbytes);
+      const int32_t* in = a.idx + ntok * a.k;
+      const uint32_t ibytes = (uint32_t)a.k * 4u;
+      if ((reinterpret_cast<uintptr_t>(in) & 15) == 0 && (ibytes & 15) == 0) bulk_prefetch_l2(in, ibytes);
+    }
+  }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(qt_full, 128);
