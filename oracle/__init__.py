@@ -5,5 +5,5 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 """
 from .dsa_oracle import (  # noqa: F401
     e4m3_table, decode_e4m3, decode_bf16, to_f64, index_scores, topk_select,
-    sparse_mla, dense_causal_mqa, forward_rows, numpy_inputs,
+    sparse_mla, dense_causal_mqa, forward_rows, numpy_inputs, indexer_kl_target,
 )

@@ -13,7 +13,11 @@ Models", bud-325 paper digest):
   * same passage, §2.1 Eq. 2 / Fig. 2: attention runs only on the top-k key-value
     entries selected by I[t,:], in MLA's MQA mode (one latent row shared by all
     query heads);
-  * "Method": k = 2048, one latent vector per token shared by all heads.
+  * "Method": k = 2048, one latent vector per token shared by all heads;
+  * "Key claims" (paper section 2.1.1, Eq. 3-4, in words) and "Method": the
+    indexer is trained with a KL loss toward the head-aggregated main attention
+    distribution, on the selected tokens in the sparse stage
+    (``indexer_kl_target``, forward only).
 The eu.36kr.com article (section 02) adds that candidates are the query's
 preceding tokens and that top-k index scores pick the entries that are read.
 
@@ -150,6 +154,54 @@ def sparse_mla(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, sm_scale: float, 
     out = (p @ c[:, :Dv]) / denom
     lse = m[:, 0] + np.log(denom[:, 0])
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Indexer alignment target (training objective, forward only)
+# ---------------------------------------------------------------------------
+
+
+def indexer_kl_target(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, sel_scores: np.ndarray,
+                      sm_scale: float):
+    """KL divergence between the aggregated main-attention distribution and the
+    lightning indexer's distribution over one query token's key set.
+
+    Follows "DeepSeek-V3.2: Pushing the Frontier of Open Large Language Models"
+    (bud-325 paper digest): "Key claims" (paper section 2.1.1, Eq. 3-4, given in
+    words only) has a KL-divergence loss align the indexer output with the main
+    attention distribution aggregated over heads; "Method" restricts that KL to
+    the selected tokens in the sparse stage. The eu.36kr.com article (section 02)
+    says the indexer learns to mimic the original attention's distribution.
+    Reading (the pages print neither equation):
+      * the key set is the valid entries of ``idx`` (all causal keys for the dense
+        warm-up, the top-k set for the sparse stage);
+      * main attention of head h: a[h,s] = softmax over the set of sm_scale q[h].c_s;
+      * target p = sum_h a[h,:], L1-normalised over the set;
+      * indexer distribution r = softmax over the set of sel_scores;
+      * loss KL(p || r) = sum_s p_s (ln p_s - ln r_s), natural log; terms with
+        p_s = 0 are 0.
+    q: [H, Dqk]; kv: [n_keys, Dqk]; idx: [k] (entries < 0 or >= n_keys are not in
+    the set); sel_scores: [k] index scores I[t, idx[j]] aligned with idx.
+    Returns (p float64 [k] with 0 at the slots outside the set, kl float64).
+    """
+    qf = to_f64(q)
+    idx = np.asarray(idx)
+    ok = (idx >= 0) & (idx < kv.shape[0])
+    p_out = np.zeros(idx.shape[0])
+    if not ok.any():
+        return p_out, 0.0
+    c = to_f64(kv[idx[ok]])                                   # [n, Dqk]
+    z = sm_scale * (qf @ c.T)                                 # [H, n]
+    a = np.exp(z - z.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)                         # each head's attention
+    agg = a.sum(axis=0)
+    p = agg / agg.sum()                                       # L1-normalised aggregate
+    sc = np.asarray(sel_scores, dtype=np.float64)[ok]
+    log_r = sc - (sc.max() + np.log(np.exp(sc - sc.max()).sum()))
+    nz = p > 0
+    kl = float(np.sum(p[nz] * (np.log(p[nz]) - log_r[nz])))
+    p_out[ok] = p
+    return p_out, kl
 
 
 def dense_causal_mqa(q: np.ndarray, kv: np.ndarray, sm_scale: float, Dv: int, q_pos0: int = 0):

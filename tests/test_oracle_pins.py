@@ -32,7 +32,8 @@ def e4m3_codes(values) -> np.ndarray:
 def real_oracle():
     return types.SimpleNamespace(index_scores=ORC.index_scores, topk_select=ORC.topk_select,
                                  sparse_mla=ORC.sparse_mla, dense_causal_mqa=ORC.dense_causal_mqa,
-                                 decode_e4m3=ORC.decode_e4m3)
+                                 decode_e4m3=ORC.decode_e4m3,
+                                 indexer_kl_target=ORC.indexer_kl_target)
 
 
 # ---------------------------------------------------------------------------
@@ -231,9 +232,62 @@ def pin_invariances(orc):
     assert np.array_equal(orc.topk_select(sc2, cfg.k), idx)
 
 
+def _golden_value(v):
+    """Evaluate a fixture entry: a number or an expression in ln(), ln3 and fractions."""
+    if isinstance(v, (int, float)):
+        return float(v)
+    return float(eval(v, {"__builtins__": {}}, {"ln": math.log, "ln3": math.log(3.0)}))
+
+
+def pin_kl_golden(orc):
+    """Hand-worked KL targets over two keys (tests/golden/kl_two_keys.json)."""
+    g = json.load(open(os.path.join(GOLDEN, "kl_two_keys.json")))
+    kv = np.array([[_golden_value(x) for x in g["keys"]["c0"]],
+                   [_golden_value(x) for x in g["keys"]["c1"]]])
+    for case in g["cases"]:
+        q = np.array([[_golden_value(x) for x in row] for row in case["q"]])
+        idx = np.array(case.get("idx", [0, 1]))
+        sc = np.array([_golden_value(x) for x in case["scores"]])
+        p, kl = orc.indexer_kl_target(q, kv, idx, sc, g["sm_scale"])
+        assert np.allclose(p, [_golden_value(x) for x in case["p"]], rtol=0, atol=1e-15), case["note"]
+        assert abs(kl - _golden_value(case["kl"])) < 1e-15, case["note"]
+
+
+def pin_kl_properties(orc):
+    """Gibbs' inequality, invariances, and the dense-warm-up reading checked against
+    the separately written dense attention (linearity of the head average)."""
+    cfg = CONFIGS["tiny"]
+    inp = ORC.numpy_inputs(gen_inputs(cfg, "cpu"))
+    rng = np.random.default_rng(21)
+    b = 0
+    for t in (0, 5, 40, 255):
+        n = t + 1
+        idx = rng.permutation(n)[: min(n, cfg.k)]
+        sc = rng.standard_normal(idx.shape[0]) * 3.0
+        p, kl = orc.indexer_kl_target(inp["q"][b, t], inp["kv"][b], idx, sc, cfg.sm_scale)
+        assert kl >= -1e-15 and abs(p.sum() - 1.0) < 1e-12 and (p > 0).all()
+        # shifting the scores changes nothing; permuting the set permutes p
+        p2, kl2 = orc.indexer_kl_target(inp["q"][b, t], inp["kv"][b], idx, sc + 17.0, cfg.sm_scale)
+        assert abs(kl2 - kl) < 1e-12 and np.allclose(p2, p, rtol=0, atol=1e-15)
+        perm = rng.permutation(idx.shape[0])
+        p3, kl3 = orc.indexer_kl_target(inp["q"][b, t], inp["kv"][b], idx[perm], sc[perm], cfg.sm_scale)
+        assert abs(kl3 - kl) < 1e-12 and np.allclose(p3, p[perm], rtol=0, atol=1e-15)
+    # dense warm-up: the set is every causal key; sum_s p_s c_s[:Dv] must be the head
+    # mean of the dense attention outputs of the independently written routine
+    Lq = 12
+    dense, _ = orc.dense_causal_mqa(inp["q"][b, :Lq], inp["kv"][b, :Lq], cfg.sm_scale, cfg.Dv)
+    c = ORC.to_f64(inp["kv"][b, :Lq])
+    for t in range(Lq):
+        idx = np.arange(t + 1)
+        p, kl = orc.indexer_kl_target(inp["q"][b, t], inp["kv"][b], idx, np.zeros(t + 1), cfg.sm_scale)
+        assert np.allclose(p @ c[: t + 1, : cfg.Dv], dense[t].mean(axis=0), rtol=0, atol=1e-13)
+        # equal scores: r is uniform, so KL = sum p ln p + ln n
+        assert abs(kl - (float(np.sum(p * np.log(p))) + math.log(t + 1))) < 1e-13
+
+
 PINS = [pin_three_token, pin_e4m3_table, pin_indexer_closed_forms, pin_indexer_mixed_signs,
         pin_topk_bruteforce, pin_topk_properties, pin_attention_special_cases,
-        pin_dense_equivalence, pin_invariances]
+        pin_dense_equivalence, pin_invariances, pin_kl_golden, pin_kl_properties]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -326,7 +380,52 @@ def _mut_e4m3_bias8(codes):
     return ORC.decode_e4m3(codes) * 0.5
 
 
+def _mut_kl_reversed(q, kv, idx, sc, sm_scale):
+    """KL(r || p) instead of KL(p || r)."""
+    p, _ = ORC.indexer_kl_target(q, kv, idx, sc, sm_scale)
+    ok = np.asarray(idx) >= 0
+    s = np.asarray(sc, dtype=np.float64)[ok]
+    r = np.exp(s - s.max())
+    r /= r.sum()
+    return p, float(np.sum(r * (np.log(r) - np.log(p[ok]))))
+
+
+def _mut_kl_head_max(q, kv, idx, sc, sm_scale):
+    """Aggregate heads by their largest weight instead of the sum."""
+    qf = ORC.to_f64(q)
+    ok = np.asarray(idx) >= 0
+    c = ORC.to_f64(kv[np.asarray(idx)[ok]])
+    z = sm_scale * (qf @ c.T)
+    a = np.exp(z - z.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)
+    agg = a.max(axis=0)
+    p = agg / agg.sum()
+    s = np.asarray(sc, dtype=np.float64)[ok]
+    log_r = s - (s.max() + np.log(np.exp(s - s.max()).sum()))
+    out = np.zeros(len(idx))
+    out[ok] = p
+    return out, float(np.sum(p * (np.log(p) - log_r)))
+
+
+def _mut_kl_raw_scores(q, kv, idx, sc, sm_scale):
+    """Uses the index scores as log-probabilities without normalising them."""
+    p, _ = ORC.indexer_kl_target(q, kv, idx, sc, sm_scale)
+    ok = np.asarray(idx) >= 0
+    s = np.asarray(sc, dtype=np.float64)[ok]
+    pp = p[ok]
+    nz = pp > 0
+    return p, float(np.sum(pp[nz] * (np.log(pp[nz]) - s[nz])))
+
+
+def _mut_kl_no_scale(q, kv, idx, sc, sm_scale):
+    return ORC.indexer_kl_target(q, kv, idx, sc, 1.0)
+
+
 MUTANTS = {
+    "kl_reversed": dict(indexer_kl_target=_mut_kl_reversed),
+    "kl_heads_by_max": dict(indexer_kl_target=_mut_kl_head_max),
+    "kl_unnormalised_scores": dict(indexer_kl_target=_mut_kl_raw_scores),
+    "kl_no_softmax_scale": dict(indexer_kl_target=_mut_kl_no_scale),
     "no_relu": dict(index_scores=_mut_no_relu),
     "relu_after_head_sum": dict(index_scores=_mut_relu_after_sum),
     "dropped_q_scale": dict(index_scores=_mut_no_qscale),
