@@ -207,3 +207,28 @@ def sample_rows(cfg: DsaConfig, n_per_seq: int = 64) -> list:
     for i in range(rest):
         rows.add(int(round(i * (Lq - 1) / max(1, rest - 1))))
     return sorted(r for r in rows if 0 <= r < Lq)
+
+
+def random_key_sets(B: int, Lq: int, k: int, q_pos0: int, seed: int, holes: float = 0.0) -> torch.Tensor:
+    """Seeded random key sets shaped like a top-k selection: for query row t (absolute
+    position p = q_pos0 + t) a uniformly random subset of the causal keys 0..p of size
+    min(k, p + 1), ascending, padded with -1. With holes > 0 that fraction of the kept
+    entries is replaced by -1 as well (entries outside the set may sit anywhere).
+    Returns int32 [B, Lq, k] on the CPU."""
+    rng = np.random.default_rng(seed)
+    out = np.full((B, Lq, k), -1, dtype=np.int32)
+    for b in range(B):
+        for t in range(Lq):
+            n = q_pos0 + t + 1
+            m = min(k, n)
+            sel = np.sort(rng.choice(n, size=m, replace=False)) if m < n else np.arange(n)
+            if holes > 0.0:
+                sel = np.where(rng.random(m) < holes, -1, sel)
+            out[b, t, :m] = sel
+    return torch.from_numpy(out)
+
+
+def random_scores(shape, seed: int, std: float = 2.0) -> torch.Tensor:
+    """Seeded N(0, std^2) fp32 values (stand-ins for index scores). CPU tensor."""
+    rng = np.random.default_rng(seed)
+    return torch.from_numpy((rng.standard_normal(shape) * std).astype(np.float32))

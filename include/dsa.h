@@ -142,6 +142,42 @@ int dsa_sparse_mla_fwd_noalloc(const uint16_t* q, const uint16_t* kv, const int3
                                uint16_t* out, float* lse, int B, int Lq, int Lk, int H, int Dqk,
                                int Dv, int k, float sm_scale, void* stream);
 
+/*
+ * dsa_indexer_kl - the indexer alignment target, forward only: for every query
+ * token, KL(p || r) between the main attention aggregated over heads and the
+ * lightning indexer's distribution, both over the token's key set.
+ * ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language Models", bud-325
+ * paper digest: "Key claims", paper section 2.1.1 Eq. 3-4, given in words - a
+ * KL-divergence loss aligns the indexer output with the main attention
+ * aggregated over heads, in the dense warm-up; "Method" - in the sparse stage
+ * the KL is taken on the selected tokens. The equations are not printed; this is
+ * the plain reading.) For token t with key set S = the valid entries of idx[t,:]:
+ *     a[h,s] = exp(sm_scale * q[t,h] . kv[s] - lse[t,h])   (attention of head h)
+ *     p_s    = sum_h a[h,s] / H                           (L1-normalised aggregate)
+ *     r_s    = exp(sel[t,s]) / sum_{s' in S} exp(sel[t,s'])
+ *     KL_t   = sum_{s in S} p_s (ln p_s - ln r_s)          (terms with p_s = 0 are 0)
+ * For the dense warm-up pass every causal key in idx (k >= the token's position
+ * + 1); for the sparse stage pass the top-k set of dsa_forward.
+ *   q          [B, Lq, H, Dqk] bf16                  (as dsa_sparse_mla_fwd)
+ *   kv         [B, Lk, Dqk] bf16 latent rows
+ *   idx        [B, Lq, k] int32; entries < 0 or >= Lk are not in the set
+ *   lse        [B, Lq, H] fp32: natural-log log-sum-exp over S of the scaled
+ *              logits, as dsa_sparse_mla_fwd / dsa_forward return it for the
+ *              same idx (it makes each head's a[h,:] sum to 1)
+ *   sel_scores [B, Lq, k] fp32: index scores I[t, idx[t,j]], aligned with idx
+ *              (entries outside the set are ignored)
+ *   p_out      [B, Lq, k] fp32 or NULL: p at each slot of idx, 0 outside the set
+ *   kl_out     [B, Lq] fp32: KL_t (0 for a token with an empty set)
+ *   (H, Dqk) in {(128, 576), (8, 80)}; k a multiple of 32 in [32, 4096].
+ * All pointers are caller-owned device memory, 16-byte aligned; nothing is
+ * allocated. Errors: DSA_ERR_INVALID_ARG (null or misaligned pointer, bad
+ * sm_scale), DSA_ERR_UNSUPPORTED_SHAPE, DSA_ERR_CUDA (launch), and a device
+ * wait that ran out is reported by dsa_check_status.
+ */
+int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, const float* lse,
+                   const float* sel_scores, float* p_out, float* kl_out, int B, int Lq, int Lk,
+                   int H, int Dqk, int k, float sm_scale, void* stream);
+
 /* Whole-path problem description for dsa_forward. */
 typedef struct dsa_problem {
   int mode;        /* DSA_MODE_PREFILL or DSA_MODE_DECODE (informational; the

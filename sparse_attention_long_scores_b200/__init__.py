@@ -39,6 +39,7 @@ EXPORTED = [
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_fwd", "dsa_forward_workspace_size",
     "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
     "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout", "dsa_sparse_mla_fwd_noalloc",
+    "dsa_indexer_kl",
 ]
 KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
 
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
     L.dsa_sparse_mla_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
                                              ctypes.c_float, vp]
     L.dsa_sparse_mla_fwd_noalloc.restype = i
+    L.dsa_indexer_kl.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float, vp]
     L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
     L.dsa_forward_workspace_size.restype = sz
     L.dsa_forward.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp, sz, vp]
@@ -203,6 +205,33 @@ def sparse_mla_fwd(q, kv, idx, sm_scale: float, Dv: int, out=None, lse=None, ws=
                                     H, Dqk, Dv, k, float(sm_scale), _ptr(ws), ws_bytes,
                                     _stream(stream)))
     return out, lse
+
+
+def indexer_kl(q, kv, idx, lse, sel_scores, sm_scale: float, p_out=None, kl_out=None,
+               with_p: bool = True, stream=None):
+    """Indexer alignment target (forward): per query token KL(p || r) between the
+    head-aggregated attention p over the key set idx and the softmax r of the index
+    scores sel_scores over the same set; lse is the forward's per-head lse over that
+    set. Returns (kl fp32 [B, Lq], p fp32 [B, Lq, k] | None)."""
+    B, Lq, H, Dqk = q.shape
+    Lk = kv.shape[1]
+    k = idx.shape[2]
+    _need(q, "q", torch.bfloat16)
+    _need(kv, "kv", torch.bfloat16, (B, Lk, Dqk))
+    _need(idx, "idx", torch.int32, (B, Lq, k))
+    _need(lse, "lse", torch.float32, (B, Lq, H))
+    _need(sel_scores, "sel_scores", torch.float32, (B, Lq, k))
+    if kl_out is None:
+        kl_out = torch.empty((B, Lq), dtype=torch.float32, device=q.device)
+    _need(kl_out, "kl_out", torch.float32, (B, Lq))
+    if p_out is None and with_p:
+        p_out = torch.empty((B, Lq, k), dtype=torch.float32, device=q.device)
+    if p_out is not None:
+        _need(p_out, "p_out", torch.float32, (B, Lq, k))
+    _check(lib().dsa_indexer_kl(_ptr(q), _ptr(kv), _ptr(idx), _ptr(lse), _ptr(sel_scores),
+                                _ptr(p_out), _ptr(kl_out), B, Lq, Lk, H, Dqk, k,
+                                float(sm_scale), _stream(stream)))
+    return kl_out, p_out
 
 
 @dataclass

@@ -459,6 +459,42 @@ int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
                  static_cast<cudaStream_t>(stream));
 }
 
+int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, const float* lse,
+                   const float* sel_scores, float* p_out, float* kl_out, int B, int Lq, int Lk,
+                   int H, int Dqk, int k, float sm_scale, void* stream) {
+  DSA_TRY(check_ptr(q, "q"));
+  DSA_TRY(check_ptr(kv, "kv"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(lse, "lse"));
+  DSA_TRY(check_ptr(sel_scores, "sel_scores"));
+  DSA_TRY(check_ptr(p_out, "p_out", true));
+  DSA_TRY(check_ptr(kl_out, "kl_out"));
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1");
+  if ((long long)B * Lk > (1LL << 30)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lk must be <= 2^30");
+  if (!((H == 128 && Dqk == 576) || (H == 8 && Dqk == 80)))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "(H, Dqk) = (%d, %d) unsupported; use (128, 576) or (8, 80)", H, Dqk);
+  if ((long long)B * Lq * H > (1LL << 31) - 1 || (long long)B * Lq > (1LL << 31) - 1)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lq*H too large");
+  DSA_TRY(check_k(k, 4096));
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
+    return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  dsa::KlArgs a{};
+  a.q = q;
+  a.idx = idx;
+  a.lse = lse;
+  a.sel = sel_scores;
+  a.p_out = p_out;
+  a.kl_out = kl_out;
+  a.B = B; a.Lq = Lq; a.Lk = Lk; a.H = H; a.Dqk = Dqk; a.k = k;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.ctl = ctl;
+  DSA_TRY_CUDA(dsa::launch_indexer_kl(kv, a, static_cast<cudaStream_t>(stream)), "indexer KL launch");
+  return DSA_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

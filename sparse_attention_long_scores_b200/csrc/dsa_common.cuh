@@ -20,6 +20,7 @@ enum : int {
   kSiteIndexer = 1,
   kSiteTopk = 2,
   kSiteMla = 3,
+  kSiteKl = 4,
   kSiteDebug = 9,
 };
 

@@ -71,6 +71,21 @@ cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const uint16_t* kv, con
                               cudaStream_t stream);
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t stream);
 
+// ---------------- indexer alignment target (KL, forward) ----------------
+struct KlArgs {
+  const uint16_t* q;   // [B, Lq, H, Dqk] bf16
+  const int32_t* idx;  // [B, Lq, k] key set of each query token (entries < 0 are not in it)
+  const float* lse;    // [B, Lq, H] natural-log log-sum-exp of the scaled logits over the set
+  const float* sel;    // [B, Lq, k] index scores of the selected keys, aligned with idx
+  float* p_out;        // [B, Lq, k] or null: aggregated attention target (0 outside the set)
+  float* kl_out;       // [B, Lq]
+  int B, Lq, Lk, H, Dqk, k;
+  float scale_log2;    // sm_scale * log2(e)
+  DevCtl ctl;
+};
+// (H, Dqk) in {(8, 80), (128, 576)}.
+cudaError_t launch_indexer_kl(const uint16_t* kv, const KlArgs& a, cudaStream_t stream);
+
 // ---------------- debug ----------------
 cudaError_t launch_debug_wait(DevCtl ctl, cudaStream_t stream);
 

@@ -82,3 +82,32 @@ def check_attention(gpu_out, ref_out, gpu_lse=None, ref_lse=None, where=""):
 def bf16_to_f64(t) -> np.ndarray:
     import torch
     return t.detach().to("cpu", torch.float32).double().numpy()
+
+
+# Indexer alignment target (KL). The GPU forms a = exp(z - lse) from fp32-accumulated
+# bf16 logits and the forward's lse; the log-domain error of both together stays under
+# 2e-4 (the attention tests bound lse to LSE_ABS = 1e-4), so p is within about 2e-4
+# relative. Tolerances: p within KL_P_RTOL relative (plus a 1e-9 floor for p ~ 0);
+# since dKL = sum_s dp_s (ln p_s - ln r_s + 1), KL within
+# KL_P_RTOL * (1 + sum_s p_s (|ln p_s| + |ln r_s|)) of the oracle's value.
+KL_P_RTOL = 1e-3
+
+
+def check_kl(gpu_kl, gpu_p, ref_kl, ref_p, sel, idx, where=""):
+    gk = float(gpu_kl)
+    gp = np.asarray(gpu_p, np.float64)
+    rp = np.asarray(ref_p, np.float64)
+    ok = (np.asarray(idx) >= 0)
+    assert np.all(gp[~ok] == 0.0), f"{where}: p outside the set"
+    perr = np.abs(gp - rp)
+    assert (perr <= KL_P_RTOL * rp + 1e-9).all(), f"{where}: p err {perr.max()} (rel {(perr / np.maximum(rp, 1e-30)).max()})"
+    s = np.asarray(sel, np.float64)[ok]
+    if ok.any():
+        log_r = s - (s.max() + np.log(np.exp(s - s.max()).sum()))
+        pp = rp[ok]
+        nz = pp > 0
+        bound = KL_P_RTOL * (1.0 + float(np.sum(pp[nz] * (np.abs(np.log(pp[nz])) + np.abs(log_r[nz])))))
+    else:
+        bound = 1e-12
+    assert abs(gk - ref_kl) <= bound, f"{where}: kl {gk} vs {ref_kl} (bound {bound})"
+    return abs(gk - ref_kl)

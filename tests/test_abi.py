@@ -82,6 +82,25 @@ def test_sparse_mla_rejects_bad_args(L):
     assert rc == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_indexer_kl_rejects_bad_args(L):
+    p = ctypes.c_void_p(FAKE)
+    # (H, Dqk) outside the supported pair
+    rc = L.dsa_indexer_kl(p, p, p, p, p, None, p, 1, 4, 8, 16, 80, 32, 0.1, None)
+    assert rc == dsa.DSA_ERR_UNSUPPORTED_SHAPE and "unsupported" in L.dsa_last_error().decode()
+    # k not a multiple of 32
+    rc = L.dsa_indexer_kl(p, p, p, p, p, None, p, 1, 4, 8, 8, 80, 40, 0.1, None)
+    assert rc == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    # missing lse (required), missing kl_out, misaligned scores, bad scale
+    rc = L.dsa_indexer_kl(p, p, p, None, p, None, p, 1, 4, 8, 8, 80, 32, 0.1, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG and "lse" in L.dsa_last_error().decode()
+    rc = L.dsa_indexer_kl(p, p, p, p, p, None, None, 1, 4, 8, 8, 80, 32, 0.1, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG and "kl_out" in L.dsa_last_error().decode()
+    rc = L.dsa_indexer_kl(p, p, p, p, ctypes.c_void_p(FAKE + 8), None, p, 1, 4, 8, 8, 80, 32, 0.1, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG and "aligned" in L.dsa_last_error().decode()
+    rc = L.dsa_indexer_kl(p, p, p, p, p, None, p, 1, 4, 8, 8, 80, 32, 0.0, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+
+
 def test_workspace_sizes(L):
     from dsa_inputs import CONFIGS
     for name, cfg in CONFIGS.items():
