@@ -297,6 +297,55 @@ def time_e2e(cfg, p, inp, ws, world, steps: int = 2):
 # ---------------------------------------------------------------------------
 
 
+def time_indexer_kl(name: str, steps: int, warmup: int, world: int, rank: int, pk: dict):
+    """The indexer alignment target (dsa_indexer_kl, forward) on the workload's own
+    selected sets: one forward gives idx and the per-head lse, the index scores of the
+    selected keys are seeded random stand-ins (the kernel's cost does not depend on
+    their values). Timed with CUDA events on the launching stream, p written."""
+    import sparse_attention_long_scores_b200 as dsa
+    from dsa_inputs import random_scores
+
+    cfg = CONFIGS[name]
+    inp = gen_inputs(cfg, "cuda", seed=rank_seed(name, rank))
+    p = dsa.Problem.from_config(cfg)
+    lse = torch.empty((cfg.B, cfg.Lq, cfg.H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.int32, device="cuda")
+    dsa.forward(p, inp, lse=lse, idx_out=idx)
+    q, kv = inp["q"], inp["kv"]
+    del inp
+    sel = random_scores((cfg.B, cfg.Lq, cfg.k), seed=77 + rank).cuda()
+    kl = torch.empty((cfg.B, cfg.Lq), dtype=torch.float32, device="cuda")
+    pt = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        dsa.indexer_kl(q, kv, idx, lse, sel, cfg.sm_scale, p_out=pt, kl_out=kl)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        dsa.indexer_kl(q, kv, idx, lse, sel, cfg.sm_scale, p_out=pt, kl_out=kl)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    dsa.check_status()
+    ms = dist_max(e0.elapsed_time(e1) / steps, world)
+    pairs = work(cfg)["mla_flops"] / (2.0 * cfg.H * (cfg.Dqk + cfg.Dv))
+    flops = 2.0 * cfg.H * cfg.Dqk * pairs
+    a = flops / (ms * 1e-3) / 1e12
+    res = {"workload": cfg.name, "value": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, ms),
+           "unit": "tokens/s", "ms_per_step": ms, "launches_per_step": 1,
+           "roofline": {"bound": "tensor", "achieved": a, "peak": pk["bf16_sustained"],
+                        "unit": "TFLOP/s", "frac": a / pk["bf16_sustained"], "traffic": None,
+                        "peak_note": "measured bf16 sustained; work = 2 H Dqk per selected pair"},
+           "note": "KL(p || softmax(index scores)) over the forward's top-k sets, p written"}
+    del q, kv, idx, lse, sel, kl, pt
+    torch.cuda.empty_cache()
+    return res
+
+
 def oracle_sample(cfg, rows: int, seed: int = 4242):
     """A bounded sample of the workload for the fp64 oracle: one sequence with all
     Lk keys and `rows` query rows at evenly spread positions (decode: the last)."""
@@ -409,6 +458,7 @@ def main():
     ap.add_argument("--workload", default="prefill_32k", choices=sorted(CONFIGS))
     ap.add_argument("--decode-workload", default="decode_128k")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-kl", action="store_true", help="skip the indexer KL target line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
@@ -444,6 +494,9 @@ def main():
     sampler = ClockSampler(gpu_index) if rank == 0 else None
     pre = time_workload(args.workload, args.steps, args.warmup, world, rank, pk, sampler,
                         e2e=not args.no_e2e)
+    kl = None
+    if not args.no_kl:
+        kl = time_indexer_kl(args.workload, args.steps, args.warmup, world, rank, pk)
     dec = None
     if not args.no_decode:
         dec = time_workload(args.decode_workload, args.steps, args.warmup, world, rank, pk,
@@ -483,6 +536,8 @@ def main():
                 "gpu_launches": dec["launches"],
                 "config": {"batch": dc.B, "cached_tokens": dc.Lk, "topk": dc.k},
             }
+        if kl is not None:
+            line["indexer_kl"] = kl
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
