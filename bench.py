@@ -209,7 +209,6 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
         dsa.forward(p, inp, out=out, ws=ws)
     torch.cuda.synchronize()
     dsa.check_status()
-    profs = [dsa.LaunchProfiler(4096) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     if sampler:
@@ -217,8 +216,10 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    timed_launches = 0
     for i in range(steps):
-        dsa.forward_profiled(p, inp, out, profs[i], ws=ws)
+        dsa.forward(p, inp, out=out, ws=ws)
+        timed_launches += dsa.last_launch_count()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -226,7 +227,14 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     dsa.check_status()
     ms_local = e0.elapsed_time(e1) / steps
     ms = dist_max(ms_local, world)
-    # per-kernel device time, from events on the launching stream
+    # per-kernel device time: the same steps again through dsa_forward_profiled,
+    # which keeps every launch on the caller's stream (no top-k / indexer overlap)
+    # so that the events around a launch time that launch alone
+    profs = [dsa.LaunchProfiler(4096) for _ in range(steps)]
+    for i in range(steps):
+        dsa.forward_profiled(p, inp, out, profs[i], ws=ws)
+    torch.cuda.synchronize()
+    dsa.check_status()
     per_kind, launches = {}, 0
     for pr in profs:
         for kind, d in pr.durations():
@@ -259,7 +267,7 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
         r["traffic"] = traffic_per_launch(k, cfg.mode, cfg.B * cfg.Lq / kernels[k]["launches_per_step"])
     res = {"cfg": cfg, "ms": ms, "tokens_per_s": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, ms),
            "kernels": kernels,
-           "roof": roof, "launches": launches, "clocks": clocks, "work": w}
+           "roof": roof, "launches": timed_launches, "clocks": clocks, "work": w}
     if cfg.mode == "decode":
         a = w["hbm_bytes"] / (ms * 1e-3) / 1e9
         res["step_roof"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s",

@@ -178,6 +178,15 @@ int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, co
                    const float* sel_scores, float* p_out, float* kl_out, int B, int Lq, int Lk,
                    int H, int Dqk, int k, float sm_scale, void* stream);
 
+/*
+ * dsa_last_launch_count - number of kernel launches that the calling thread's
+ * last dsa_forward, dsa_forward_host or dsa_forward_profiled call enqueued
+ * (all of this library's kernels, on the caller's stream and on the library's
+ * internal side stream). 0 before the first call. For benchmarks that report
+ * how many of the library's kernels ran in a timed region.
+ */
+int dsa_last_launch_count(void);
+
 /* Whole-path problem description for dsa_forward. */
 typedef struct dsa_problem {
   int mode;        /* DSA_MODE_PREFILL or DSA_MODE_DECODE (informational; the

@@ -39,7 +39,7 @@ EXPORTED = [
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_fwd", "dsa_forward_workspace_size",
     "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
     "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout", "dsa_sparse_mla_fwd_noalloc",
-    "dsa_indexer_kl",
+    "dsa_indexer_kl", "dsa_last_launch_count",
 ]
 KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
 
@@ -350,6 +350,11 @@ def forward_host(p: Problem, host: dict, dev: dict, host_out, dev_out, ws, strea
     _check(lib().dsa_forward_host(ctypes.byref(cp), ctypes.byref(ch), ctypes.byref(cd), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)))
     return host_out
+
+
+def last_launch_count() -> int:
+    """Kernel launches of this thread's last forward call (see dsa_last_launch_count)."""
+    return int(lib().dsa_last_launch_count())
 
 
 def check_status(stream=None) -> None:

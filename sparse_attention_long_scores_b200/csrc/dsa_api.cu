@@ -173,7 +173,9 @@ struct Recorder {
   int* kinds = nullptr;
   int cap = 0;
   int n = 0;
+  int launched = 0;               // kernel launches so far (counted with or without events)
   int mark(int kind, cudaStream_t s) {
+    ++launched;
     if (events == nullptr) return DSA_OK;
     if (n >= cap) return fail(DSA_ERR_INVALID_ARG, "profiling: more than %d launches", cap);
     kinds[n] = kind;
@@ -183,6 +185,7 @@ struct Recorder {
   }
 };
 Recorder g_no_rec;
+thread_local int g_last_launches = 0;   // kernel launches of this thread's last forward call
 
 // ---------------- schedule helpers ----------------
 int indexer_piece_keys(int B, int rows, int t_blk, int keys_max, int num_sms) {
@@ -560,6 +563,52 @@ size_t dsa_forward_workspace_size(const dsa_problem* p) {
 }  // extern "C"
 
 namespace {
+// Per-device side stream and events on which dsa_forward overlaps the top-k of
+// one score chunk with the indexer of the next. Created on first use and kept for
+// the life of the process; the mutex keeps one call's sequence of records and
+// waits on them from interleaving with another call's.
+struct SideStream {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t scored[2] = {nullptr, nullptr};    // indexer of the chunk in buffer b done
+  cudaEvent_t selected[2] = {nullptr, nullptr};  // top-k of the chunk in buffer b done
+};
+SideStream g_side[kMaxDevices];
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "device index %d", dev);
+  SideStream& r = g_side[dev];
+  std::lock_guard<std::mutex> lk(r.mu);
+  if (!r.ready) {
+    DSA_TRY_CUDA(cudaStreamCreateWithFlags(&r.side, cudaStreamNonBlocking), "cudaStreamCreate");
+    for (int b = 0; b < 2; ++b) {
+      DSA_TRY_CUDA(cudaEventCreateWithFlags(&r.scored[b], cudaEventDisableTiming), "cudaEventCreate");
+      DSA_TRY_CUDA(cudaEventCreateWithFlags(&r.selected[b], cudaEventDisableTiming), "cudaEventCreate");
+    }
+    r.ready = true;
+  }
+  *out = &r;
+  return DSA_OK;
+}
+
+dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld, int bstride,
+                        int t0, int t1, int32_t* idx, const dsa::DevCtl& ctl) {
+  dsa::TopkArgs ta{};
+  ta.scores = scores;
+  ta.sc_ld = ld;
+  ta.sc_bstride = bstride;
+  ta.sc_t0 = t0;
+  ta.idx = idx;
+  ta.B = p->B; ta.Lq = p->Lq; ta.Lk = p->Lk; ta.q_pos0 = p->q_pos0; ta.k = p->k;
+  ta.t_lo = t0; ta.t_hi = t1;
+  ta.vec4 = 1;
+  ta.ctl = ctl;
+  return ta;
+}
+
 int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
                  void* stream, Recorder& rec) {
   DSA_TRY(validate_problem(p));
@@ -589,26 +638,52 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
   if (f.scores_bytes > 0 && (f.chunk < 1 || f.total > ws_bytes))
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "dsa_forward workspace: no room for one score row");
   const int C = f.chunk > 0 ? f.chunk : p->Lq;
-  for (int t0 = 0; t0 < p->Lq; t0 += C) {
-    const int t1 = t0 + C < p->Lq ? t0 + C : p->Lq;
-    const int ts = t0 > first_scored ? t0 : first_scored;
-    if (ts < t1) {
-      DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
-                                  f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
-                                  t1, ctl, sms, s, rec));
+  // Overlapped schedule: the score area holds two half-size chunk buffers; the
+  // top-k of a chunk runs on the side stream while the indexer scores the next
+  // chunk into the other buffer (their CTAs fit on one SM together). The
+  // profiling entry point keeps the serial schedule so that each launch's events
+  // time that launch alone.
+  const int C2 = (C / 2) & ~3;
+  if (rec.events == nullptr && f.scores_bytes > 0 && C2 >= 4) {
+    SideStream* r = nullptr;
+    DSA_TRY(side_stream(&r));
+    std::lock_guard<std::mutex> lk(r->mu);
+    const size_t half = (size_t)p->B * C2 * (size_t)f.ld;   // floats per buffer
+    int c = 0;
+    for (int t0 = 0; t0 < p->Lq; t0 += C2, ++c) {
+      const int t1 = t0 + C2 < p->Lq ? t0 + C2 : p->Lq;
+      const int ts = t0 > first_scored ? t0 : first_scored;
+      const int b = c & 1;
+      float* sb = scores + b * half;
+      // the buffer's previous chunk must have been selected before it is rewritten
+      if (c >= 2) DSA_TRY_CUDA(cudaStreamWaitEvent(s, r->selected[b], 0), "cudaStreamWaitEvent");
+      if (ts < t1) {
+        DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, sb,
+                                    f.ld, C2, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
+                                    t1, ctl, sms, s, rec));
+      }
+      DSA_TRY_CUDA(cudaEventRecord(r->scored[b], s), "cudaEventRecord");
+      DSA_TRY_CUDA(cudaStreamWaitEvent(r->side, r->scored[b], 0), "cudaStreamWaitEvent");
+      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl), sms, r->side),
+                   "top-k launch");
+      DSA_TRY(rec.mark(DSA_KIND_TOPK, r->side));   // counts it (no events on this path)
+      DSA_TRY_CUDA(cudaEventRecord(r->selected[b], r->side), "cudaEventRecord");
     }
-    dsa::TopkArgs ta{};
-    ta.scores = scores;
-    ta.sc_ld = f.ld;
-    ta.sc_bstride = C;
-    ta.sc_t0 = t0;
-    ta.idx = idx;
-    ta.B = p->B; ta.Lq = p->Lq; ta.Lk = p->Lk; ta.q_pos0 = p->q_pos0; ta.k = p->k;
-    ta.t_lo = t0; ta.t_hi = t1;
-    ta.vec4 = 1;
-    ta.ctl = ctl;
-    DSA_TRY_CUDA(dsa::launch_topk(ta, sms, s), "top-k launch");
-    DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
+    // top-k launches run in order on the side stream: the last one covers all
+    if (c >= 1) DSA_TRY_CUDA(cudaStreamWaitEvent(s, r->selected[(c - 1) & 1], 0), "cudaStreamWaitEvent");
+  } else {
+    for (int t0 = 0; t0 < p->Lq; t0 += C) {
+      const int t1 = t0 + C < p->Lq ? t0 + C : p->Lq;
+      const int ts = t0 > first_scored ? t0 : first_scored;
+      if (ts < t1) {
+        DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
+                                    f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
+                                    t1, ctl, sms, s, rec));
+      }
+      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl), sms, s),
+                   "top-k launch");
+      DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
+    }
   }
   return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
                  p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec);
@@ -620,8 +695,12 @@ extern "C" {
 int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
                 void* stream) {
   Recorder none;
-  return forward_impl(p, t, ws, ws_bytes, stream, none);
+  const int rc = forward_impl(p, t, ws, ws_bytes, stream, none);
+  g_last_launches = none.launched;
+  return rc;
 }
+
+int dsa_last_launch_count(void) { return g_last_launches; }
 
 int dsa_forward_profiled(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
                          void* stream, void* const* events, int* kinds, int max_launches,
@@ -640,6 +719,7 @@ int dsa_forward_profiled(const dsa_problem* p, const dsa_tensors* t, void* ws, s
   DSA_TRY_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s), "cudaEventRecord");
   int r = forward_impl(p, t, ws, ws_bytes, stream, rec);
   *n_launches = rec.n;
+  g_last_launches = rec.launched;
   return r;
 }
 

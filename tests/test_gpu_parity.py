@@ -292,6 +292,27 @@ def test_unselected_rows_do_not_matter_and_determinism():
     assert torch.equal(o[0, 0], out1[0, t])
 
 
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("prefill_8k", dict(Lq=2048, q_pos0=6144))])
+def test_overlapped_schedule_matches_serial(name, kw):
+    """dsa_forward runs the top-k of a score chunk on a side stream while the indexer
+    scores the next half-size chunk; dsa_forward_profiled keeps the serial schedule with
+    full-size chunks. Every score is computed the same way in both, so the selections
+    and outputs must be identical."""
+    cfg = CONFIGS[name].with_(**kw)
+    inp = gen_inputs(cfg, "cuda", seed=23)
+    out1, lse1, idx1 = _forward(cfg, inp)
+    launches = dsa.last_launch_count()
+    p = dsa.Problem.from_config(cfg)
+    out2 = torch.empty_like(out1)
+    prof = dsa.LaunchProfiler(4096)
+    dsa.forward_profiled(p, inp, out2, prof)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    assert torch.equal(out1, out2)
+    # the overlapped schedule splits the score chunks in two: more top-k launches
+    assert launches > prof.n and dsa.last_launch_count() == prof.n
+
+
 def test_sparse_mla_skips_invalid_indices():
     cfg = CONFIGS["tiny"].with_(Lq=4, Lk=64)
     inp = gen_inputs(cfg, "cuda", seed=3)
