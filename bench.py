@@ -435,6 +435,8 @@ PROFILE_CASES = {
     "prefill_chunk": ("prefill_8k", dict(Lq=2048, q_pos0=6144)),
     # 16 decode sequences against 131072 cached keys
     "decode_small": ("decode_128k", dict(B=16)),
+    # the indexer KL target over the forward's top-k sets of the prefill chunk above
+    "kl_chunk": ("prefill_8k", dict(Lq=2048, q_pos0=6144)),
 }
 
 
@@ -450,8 +452,17 @@ def profile_case(name: str) -> None:
     cfg = CONFIGS[base].with_(**kw)
     inp = gen_inputs(cfg, "cuda")
     p = dsa.Problem.from_config(cfg)
-    for _ in range(2):
-        dsa.forward(p, inp)
+    if name == "kl_chunk":
+        from dsa_inputs import random_scores
+        lse = torch.empty((cfg.B, cfg.Lq, cfg.H), dtype=torch.float32, device="cuda")
+        idx = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.int32, device="cuda")
+        dsa.forward(p, inp, lse=lse, idx_out=idx)
+        sel = random_scores((cfg.B, cfg.Lq, cfg.k), seed=77).cuda()
+        for _ in range(2):
+            dsa.indexer_kl(inp["q"], inp["kv"], idx, lse, sel, cfg.sm_scale)
+    else:
+        for _ in range(2):
+            dsa.forward(p, inp)
     torch.cuda.synchronize()
     dsa.check_status()
     print(f"profile case {name}: {cfg}")
