@@ -229,6 +229,41 @@ int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_
                 void* stream);
 
 /*
+ * Paged, variable-length caches (a serving layout; the pages describe the method
+ * only, so this is a plain reading: each sequence's keys are the tokens of its
+ * own cache, "Key claims" section 2.1, and the query rows are its newest tokens).
+ * The latent rows kv, index keys kI and key scales kI_scale of every sequence live
+ * in shared pools of num_pages pages of page_size tokens. Logical key s of sequence
+ * b is pool row block_table[b][s / page_size] * page_size + s % page_size.
+ */
+typedef struct dsa_paged_cache {
+  const int32_t* block_table; /* [B, max_blocks] device: pool page of each logical block */
+  const int32_t* seq_lens;    /* [B] device: tokens in each sequence's cache, its Lq query
+                                 rows included (query row t sits at seq_lens[b] - Lq + t) */
+  int max_blocks;             /* logical blocks per sequence; Lk = max_blocks * page_size */
+  int page_size;              /* tokens per page: a positive multiple of 128 */
+  int num_pages;              /* pages in each pool */
+} dsa_paged_cache;
+
+/*
+ * dsa_forward_paged - dsa_forward over a paged cache with per-sequence lengths.
+ * p: as for dsa_forward with Lk = max_blocks * page_size (the capacity of one
+ * sequence); q_pos0 is ignored (the positions come from seq_lens). t: qI,
+ * qI_scale, w, q as for dsa_forward ([B, Lq, ...]); kv [num_pages * page_size,
+ * Dqk], kI [num_pages * page_size, d_I] and kI_scale [num_pages * page_size] are
+ * the pools. Each row's candidates are keys 0 .. seq_lens[b] - Lq + t of its own
+ * sequence, selected by the same top-k rule; idx_out holds logical key positions.
+ * ws: at least dsa_forward_paged_workspace_size(p) bytes. Device-side contents are
+ * not validated: seq_lens outside [Lq, Lk] or page numbers outside [0, num_pages)
+ * give unspecified results but never an out-of-bounds access (a page number
+ * outside the pool reads pool row 0 or zeros). Errors as for dsa_forward, plus
+ * DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED_SHAPE for the cache description.
+ */
+size_t dsa_forward_paged_workspace_size(const dsa_problem* p);
+int dsa_forward_paged(const dsa_problem* p, const dsa_tensors* t, const dsa_paged_cache* c,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
  * dsa_forward_host - dsa_forward on HOST tensors: copies every input from host
  * memory (pinned for asynchronous copies) into the caller's device staging
  * buffers `dev` (same layout as dsa_tensors, all device pointers), runs

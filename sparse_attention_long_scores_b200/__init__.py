@@ -39,7 +39,8 @@ EXPORTED = [
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_fwd", "dsa_forward_workspace_size",
     "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
     "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout", "dsa_sparse_mla_fwd_noalloc",
-    "dsa_indexer_kl", "dsa_last_launch_count",
+    "dsa_indexer_kl", "dsa_last_launch_count", "dsa_forward_paged_workspace_size",
+    "dsa_forward_paged",
 ]
 KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
 
@@ -61,6 +62,12 @@ class DsaProblem(ctypes.Structure):
 class DsaTensors(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("qI", "qI_scale", "kI", "kI_scale", "w", "q", "kv", "out", "lse", "idx_out")]
+
+
+class DsaPagedCache(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("max_blocks", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("num_pages", ctypes.c_int)]
 
 
 _lib = None
@@ -91,6 +98,10 @@ def lib() -> ctypes.CDLL:
     L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
     L.dsa_forward_workspace_size.restype = sz
     L.dsa_forward.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp, sz, vp]
+    L.dsa_forward_paged_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
+    L.dsa_forward_paged_workspace_size.restype = sz
+    L.dsa_forward_paged.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors),
+                                    ctypes.POINTER(DsaPagedCache), vp, sz, vp]
     L.dsa_forward_host.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors),
                                    ctypes.POINTER(DsaTensors), vp, sz, vp]
     L.dsa_forward_profiled.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp,
@@ -304,6 +315,39 @@ def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, st
     ct = _tensors(inp, out, lse, idx_out)
     _check(lib().dsa_forward(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def forward_paged_workspace_size(p: Problem) -> int:
+    cp = p.c()
+    return int(lib().dsa_forward_paged_workspace_size(ctypes.byref(cp)))
+
+
+def forward_paged(p: Problem, inp: dict, block_table, seq_lens, page_size: int, out=None,
+                  lse=None, idx_out=None, ws=None, stream=None):
+    """dsa_forward over a paged cache with per-sequence lengths.
+
+    inp: qI, qI_scale, w, q as for ``forward`` ([B, Lq, ...]); kv, kI, kI_scale are
+    pools of num_pages * page_size rows. block_table int32 [B, max_blocks], seq_lens
+    int32 [B] (device). p.Lk must be max_blocks * page_size; p.q_pos0 is ignored.
+    """
+    dev = inp["q"].device
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (p.B,))
+    B, max_blocks = block_table.shape
+    rows = inp["kv"].shape[0]
+    if rows % page_size:
+        raise ValueError("pool rows must be a multiple of page_size")
+    if out is None:
+        out = torch.empty((p.B, p.Lq, p.H, p.Dv), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = torch.empty(forward_paged_workspace_size(p), dtype=torch.uint8, device=dev)
+    cp = p.c()
+    ct = _tensors(inp, out, lse, idx_out)
+    cc = DsaPagedCache(block_table.data_ptr(), seq_lens.data_ptr(), max_blocks, page_size,
+                       rows // page_size)
+    _check(lib().dsa_forward_paged(ctypes.byref(cp), ctypes.byref(ct), ctypes.byref(cc), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)))
     return out
 
 

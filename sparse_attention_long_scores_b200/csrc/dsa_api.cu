@@ -228,7 +228,8 @@ int assumed_sms() {
 int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t* out, float* lse,
             int B, int Lq, int Lk, int H, int Dqk, int Dv, int k, float sm_scale, void* ws,
             size_t ws_bytes, const dsa::DevCtl& ctl, int num_sms, cudaStream_t stream,
-            Recorder& rec = g_no_rec, bool fit_splits = false) {
+            Recorder& rec = g_no_rec, bool fit_splits = false,
+            const dsa_paged_cache* pc = nullptr) {
   (void)num_sms;
   int splits = mla_splits(B, Lq, Dv, k, assumed_sms());
   // fit_splits: use fewer key splits rather than fail when the partials of the
@@ -250,6 +251,12 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
   a.n_dv = mla_n_dv(Dv);
   a.splits = splits;
   a.wave = num_sms > 0 ? num_sms : assumed_sms();
+  if (pc != nullptr) {   // kv is a pool of pages
+    a.block_table = pc->block_table;
+    a.max_blocks = pc->max_blocks;
+    a.page_size = pc->page_size;
+    a.num_pages = pc->num_pages;
+  }
   a.ctl = ctl;
   if (splits > 1) {
     size_t tok = (size_t)B * Lq;
@@ -351,14 +358,17 @@ int launch_indexer_rows(const uint8_t* qI, const float* qI_scale, const uint8_t*
                         const float* kI_scale, const void* w, int w_dtype, float* scores,
                         long long sc_ld, long long sc_bstride, int sc_t0, int B, int Lq, int Lk,
                         int q_pos0, int H_I, int d_I, int t_lo, int t_hi, const dsa::DevCtl& ctl,
-                        int num_sms, cudaStream_t stream, Recorder& rec = g_no_rec) {
+                        int num_sms, cudaStream_t stream, Recorder& rec = g_no_rec,
+                        const dsa_paged_cache* pc = nullptr) {
   if (t_hi <= t_lo) return DSA_OK;
   const int n_tok = (H_I == 64) ? ((t_hi - t_lo == 1) ? 1 : 4) : 64;
   CUtensorMap tq, tk;
   DSA_TRY(make_map_2d(&tq, qI, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)d_I,
                       (uint64_t)B * Lq * H_I, (uint32_t)d_I, (uint32_t)(n_tok * H_I),
                       d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B));
-  DSA_TRY(make_map_2d(&tk, kI, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)d_I, (uint64_t)B * Lk,
+  // key rows: the sequences one after another, or the page pool
+  const uint64_t k_rows = pc != nullptr ? (uint64_t)pc->num_pages * pc->page_size : (uint64_t)B * Lk;
+  DSA_TRY(make_map_2d(&tk, kI, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)d_I, k_rows,
                       (uint32_t)d_I, 128,
                       d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B));
   dsa::IndexerArgs a{};
@@ -372,6 +382,13 @@ int launch_indexer_rows(const uint8_t* qI, const float* qI_scale, const uint8_t*
   a.sc_t0 = sc_t0;
   a.B = B; a.Lq = Lq; a.Lk = Lk; a.q_pos0 = q_pos0;
   a.t_lo = t_lo; a.t_hi = t_hi;
+  if (pc != nullptr) {
+    a.seq_lens = pc->seq_lens;
+    a.block_table = pc->block_table;
+    a.max_blocks = pc->max_blocks;
+    a.page_size = pc->page_size;
+    a.num_pages = pc->num_pages;
+  }
   int keys_max = q_pos0 + t_hi < Lk ? q_pos0 + t_hi : Lk;
   a.piece_keys = indexer_piece_keys(B, t_hi - t_lo, n_tok, keys_max, num_sms);
   a.ctl = ctl;
@@ -595,7 +612,8 @@ int side_stream(SideStream** out) {
 }
 
 dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld, int bstride,
-                        int t0, int t1, int32_t* idx, const dsa::DevCtl& ctl) {
+                        int t0, int t1, int32_t* idx, const dsa::DevCtl& ctl,
+                        const dsa_paged_cache* pc) {
   dsa::TopkArgs ta{};
   ta.scores = scores;
   ta.sc_ld = ld;
@@ -605,12 +623,13 @@ dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld,
   ta.B = p->B; ta.Lq = p->Lq; ta.Lk = p->Lk; ta.q_pos0 = p->q_pos0; ta.k = p->k;
   ta.t_lo = t0; ta.t_hi = t1;
   ta.vec4 = 1;
+  ta.seq_lens = pc != nullptr ? pc->seq_lens : nullptr;
   ta.ctl = ctl;
   return ta;
 }
 
 int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
-                 void* stream, Recorder& rec) {
+                 void* stream, Recorder& rec, const dsa_paged_cache* pc = nullptr) {
   DSA_TRY(validate_problem(p));
   DSA_TRY(validate_tensors(t));
   DSA_TRY(check_ptr(ws, "ws", true));
@@ -660,11 +679,11 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
       if (ts < t1) {
         DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, sb,
                                     f.ld, C2, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
-                                    t1, ctl, sms, s, rec));
+                                    t1, ctl, sms, s, rec, pc));
       }
       DSA_TRY_CUDA(cudaEventRecord(r->scored[b], s), "cudaEventRecord");
       DSA_TRY_CUDA(cudaStreamWaitEvent(r->side, r->scored[b], 0), "cudaStreamWaitEvent");
-      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl), sms, r->side),
+      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl, pc), sms, r->side),
                    "top-k launch");
       DSA_TRY(rec.mark(DSA_KIND_TOPK, r->side));   // counts it (no events on this path)
       DSA_TRY_CUDA(cudaEventRecord(r->selected[b], r->side), "cudaEventRecord");
@@ -678,15 +697,40 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
       if (ts < t1) {
         DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
                                     f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
-                                    t1, ctl, sms, s, rec));
+                                    t1, ctl, sms, s, rec, pc));
       }
-      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl), sms, s),
+      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl, pc), sms, s),
                    "top-k launch");
       DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
     }
   }
   return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
-                 p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec);
+                 p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+}
+
+// A paged problem is scheduled as the uniform problem whose rows sit as late as
+// the capacity allows (q_pos0 = Lk - Lq): a row that needs no scores there needs
+// none in any sequence, since every sequence is at most Lk tokens long.
+dsa_problem paged_schedule_problem(const dsa_problem* p) {
+  dsa_problem pp = *p;
+  pp.q_pos0 = p->Lk - p->Lq;
+  return pp;
+}
+
+int validate_paged(const dsa_problem* p, const dsa_paged_cache* pc) {
+  if (pc == nullptr) return fail(DSA_ERR_INVALID_ARG, "paged cache is NULL");
+  DSA_TRY(check_ptr(pc->block_table, "block_table"));
+  DSA_TRY(check_ptr(pc->seq_lens, "seq_lens"));
+  if (pc->page_size < 128 || pc->page_size % 128 != 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "page_size = %d: need a multiple of 128", pc->page_size);
+  if (pc->max_blocks < 1 || pc->num_pages < 1)
+    return fail(DSA_ERR_INVALID_ARG, "max_blocks and num_pages must be >= 1");
+  if ((long long)pc->max_blocks * pc->page_size != p->Lk)
+    return fail(DSA_ERR_INVALID_ARG, "Lk = %d must equal max_blocks * page_size = %lld", p->Lk,
+                (long long)pc->max_blocks * pc->page_size);
+  if ((long long)pc->num_pages * pc->page_size > (1LL << 30))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "num_pages * page_size must be <= 2^30");
+  return DSA_OK;
 }
 }  // namespace
 
@@ -701,6 +745,24 @@ int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_
 }
 
 int dsa_last_launch_count(void) { return g_last_launches; }
+
+size_t dsa_forward_paged_workspace_size(const dsa_problem* p) {
+  if (p == nullptr) return 0;
+  const dsa_problem pp = paged_schedule_problem(p);
+  return dsa_forward_workspace_size(&pp);
+}
+
+int dsa_forward_paged(const dsa_problem* p, const dsa_tensors* t, const dsa_paged_cache* pc,
+                      void* ws, size_t ws_bytes, void* stream) {
+  if (p == nullptr) return fail(DSA_ERR_INVALID_ARG, "problem is NULL");
+  const dsa_problem pp = paged_schedule_problem(p);
+  DSA_TRY(validate_problem(&pp));
+  DSA_TRY(validate_paged(&pp, pc));
+  Recorder none;
+  const int rc = forward_impl(&pp, t, ws, ws_bytes, stream, none, pc);
+  g_last_launches = none.launched;
+  return rc;
+}
 
 int dsa_forward_profiled(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
                          void* stream, void* const* events, int* kinds, int max_launches,

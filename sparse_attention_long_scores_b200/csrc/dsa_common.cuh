@@ -413,6 +413,24 @@ DSA_DEVICE_INLINE void cluster_sync() {
 }
 
 // Warp-uniform role helpers.
+// Paged key caches: logical key s of sequence b lives in page
+// block_table[b][s / page_size] at offset s % page_size of a pool of num_pages
+// pages. Returns the pool row, b * Lk + s when there is no block table, and -1
+// for a page number outside the pool (the caller reads nothing there).
+DSA_DEVICE_INLINE long long key_row(const int32_t* block_table, int max_blocks, int page_size,
+                                    int num_pages, int b, int Lk, int s) {
+  if (block_table == nullptr) return (long long)b * Lk + s;
+  const int pg = __ldg(block_table + (long long)b * max_blocks + s / page_size);
+  if (pg < 0 || pg >= num_pages) return -1;
+  return (long long)pg * page_size + s % page_size;
+}
+
+// Position of query row 0 of sequence b: the shared q_pos0, or, with per-sequence
+// lengths, seq_lens[b] - Lq (the rows are the last Lq tokens of the sequence).
+DSA_DEVICE_INLINE int seq_pos0(const int32_t* seq_lens, int q_pos0, int Lq, int b) {
+  return seq_lens == nullptr ? q_pos0 : __ldg(seq_lens + b) - Lq;
+}
+
 DSA_DEVICE_INLINE int warp_id() { return __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0); }
 DSA_DEVICE_INLINE int lane_id() { return (int)(threadIdx.x & 31); }
 

@@ -23,6 +23,11 @@ struct IndexerArgs {
   int B, Lq, Lk, q_pos0;
   int t_lo, t_hi;    // query rows [t_lo, t_hi) of every sequence are scored
   int piece_keys;    // keys per work unit (multiple of 128)
+  // optional paged cache (see key_row / seq_pos0): kI and kI_scale are then pools of
+  // num_pages * page_size rows, and sequence b's rows sit at seq_lens[b] - Lq + t
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  int max_blocks, page_size, num_pages;
   DevCtl ctl;
 };
 
@@ -46,6 +51,7 @@ struct TopkArgs {
   int B, Lq, Lk, q_pos0, k;
   int t_lo, t_hi;  // rows [t_lo, t_hi) of every sequence
   int vec4;        // rows are 16-byte aligned (sc_ld % 4 == 0, aligned base)
+  const int32_t* seq_lens;   // [B] or null: per-sequence lengths (row t at seq_lens[b] - Lq + t)
   DevCtl ctl;
 };
 cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream);
@@ -64,6 +70,10 @@ struct MlaArgs {
   int splits;          // key splits per token
   int wave;            // CTAs resident at once (one per SM): the next CTA an SM runs
                        // is about this many block indices further on
+  // optional paged latent cache (see key_row): kv is then a pool of
+  // num_pages * page_size rows
+  const int32_t* block_table;
+  int max_blocks, page_size, num_pages;
   DevCtl ctl;
 };
 // (H, Dqk, Dv) in {(8,80,64), (128,576,512)}.

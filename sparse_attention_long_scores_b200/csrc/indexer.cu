@@ -63,7 +63,8 @@ struct Unit {
 template <int T_BLK>
 __device__ __forceinline__ int unit_count(const IndexerArgs& a, int& nblk, int& maxp) {
   nblk = (a.t_hi - a.t_lo + T_BLK - 1) / T_BLK;
-  int keys_max = min(a.Lk, a.q_pos0 + a.t_hi);
+  // with per-sequence lengths every sequence may use the whole capacity
+  int keys_max = a.seq_lens != nullptr ? a.Lk : min(a.Lk, a.q_pos0 + a.t_hi);
   maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
   return a.B * nblk * maxp;
 }
@@ -77,7 +78,7 @@ __device__ __forceinline__ bool get_unit(const IndexerArgs& a, int u, int nblk, 
   o.b = rest / nblk;
   o.t_a = a.t_lo + blk * T_BLK;
   o.t_b = min(o.t_a + T_BLK, a.t_hi);
-  int keys = min(a.Lk, a.q_pos0 + o.t_b);  // keys 0 .. q_pos0 + t_b - 1
+  int keys = min(a.Lk, seq_pos0(a.seq_lens, a.q_pos0, a.Lq, o.b) + o.t_b);  // keys 0 .. q_pos0 + t_b - 1
   o.s_lo = piece * a.piece_keys;
   o.s_hi = min(keys, o.s_lo + a.piece_keys);
   return o.s_lo < o.s_hi;
@@ -159,7 +160,11 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
           if (!mbar_wait(&k_empty[kst], kph ^ 1, a.ctl, abort_flag, kSiteIndexer, 2)) { ok = false; break; }
           k_pending[kst] = -1;
           mbar_arrive_expect_tx(&k_full[kst], Tr::KTILE_BYTES);
-          tma_load_2d(k_smem + kst * Tr::KTILE_BYTES, &tmap_k, 0, un.b * a.Lk + s0, &k_full[kst]);
+          // a tile of 128 keys never crosses a page (page_size is a multiple of 128); a
+          // page number outside the pool points past the tensor map: the tile reads zeros
+          long long krow = key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, un.b, a.Lk, s0);
+          if (krow < 0) krow = (long long)a.num_pages * a.page_size;
+          tma_load_2d(k_smem + kst * Tr::KTILE_BYTES, &tmap_k, 0, (int)krow, &k_full[kst]);
           k_pending[kst] = kph;
           if (++kst == Tr::STAGES) { kst = 0; kph ^= 1; }
         }
@@ -249,13 +254,17 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
         for (int j = 0; j < 64; ++j) wr[j] = wbuf[j];
       }
       // key scales are fetched one tile ahead so their latency hides behind a tile
-      const float* ks_row = a.kI_scale + (size_t)un.b * a.Lk;
-      float ks_next = (un.s_lo + key_in_tile < un.s_hi) ? __ldg(ks_row + un.s_lo + key_in_tile) : 0.f;
+      auto ks_at = [&](int s) -> float {   // scale of logical key s of this unit's sequence
+        const long long r = key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, un.b, a.Lk, s);
+        return r >= 0 ? __ldg(a.kI_scale + r) : 0.f;
+      };
+      const int qp = seq_pos0(a.seq_lens, a.q_pos0, a.Lq, un.b);
+      float ks_next = (un.s_lo + key_in_tile < un.s_hi) ? ks_at(un.s_lo + key_in_tile) : 0.f;
       for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
         const int s = s0 + key_in_tile;
         const bool key_ok = s < un.s_hi;
         const float ks = ks_next;
-        ks_next = (s + Tr::KT < un.s_hi) ? __ldg(ks_row + s + Tr::KT) : 0.f;
+        ks_next = (s + Tr::KT < un.s_hi) ? ks_at(s + Tr::KT) : 0.f;
         if (!mbar_wait(&acc_full[ac], aph, a.ctl, abort_flag, kSiteIndexer, 8)) { ok = false; break; }
         tc_fence_after();
         if constexpr (H_I == 64) {
@@ -287,7 +296,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
             const float part = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
                                ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
             const int t = un.t_a + c0 / 64;
-            if (key_ok && t < un.t_b && s <= a.q_pos0 + t)
+            if (key_ok && t < un.t_b && s <= qp + t)
               a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = part * ks;
           }
         } else {
@@ -305,7 +314,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
               for (int j = 0; j < H_I; ++j)
                 acc = fmaf(wv[g * H_I + j], fmaxf(__uint_as_float(r[g * H_I + j]), 0.f), acc);
               const int t = un.t_a + c0 / H_I + g;
-              if (key_ok && t < un.t_b && s <= a.q_pos0 + t) {
+              if (key_ok && t < un.t_b && s <= qp + t) {
                 a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = acc * ks;
               }
             }
@@ -334,7 +343,7 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const I
                                        Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   int nblk = (a.t_hi - a.t_lo + Tr::T_BLK - 1) / Tr::T_BLK;
-  int keys_max = a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk;
+  int keys_max = a.seq_lens != nullptr ? a.Lk : (a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk);
   long long maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
   long long units = (long long)a.B * nblk * maxp;
   if (units <= 0) return cudaSuccess;

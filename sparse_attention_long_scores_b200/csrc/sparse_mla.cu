@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     // tensor core (proxy fence) and arrives on that part's full barrier.
     const int ptid = threadIdx.x - PROD_T0;
     const int row_bytes = a.Dqk * 2;
-    const uint8_t* kv_b = reinterpret_cast<const uint8_t*>(kv) + (size_t)b * a.Lk * row_bytes;
+    const uint8_t* kv_g = reinterpret_cast<const uint8_t*>(kv);
     const uint32_t kv_base = smem_u32(kv_smem);
     const int vb0 = dvc * Tr::NB_B;
     // copy this thread's chunks of one part of tile i into its stage
@@ -357,10 +357,15 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
           const int q = kb * 8 + q8;                  // 16-byte chunk within the row
           const int pos = (tile0 + i) * KEYS + r;
           const int v = pos < a.k ? __ldg(idx_row + pos) : -1;
-          const int row = (v >= 0 && v < a.Lk) ? v : 0;   // invalid keys read row 0, masked later
+          // pool row of the key (sequence b's row v, or its page's row); invalid keys and
+          // pages outside the pool read pool row 0, and invalid keys are masked later
+          long long row = (v >= 0 && v < a.Lk)
+                              ? key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, b, a.Lk, v)
+                              : 0;
+          if (row < 0) row = 0;
           const bool in_row = q * 16 < row_bytes;
           cp_async16(stage + kb * Tr::KVBLK + r * 128 + ((q8 ^ (r & 7)) << 4),
-                     kv_b + (size_t)row * row_bytes + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
+                     kv_g + (size_t)row * row_bytes + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
         }
       }
       cp_async_commit();

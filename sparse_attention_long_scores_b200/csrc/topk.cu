@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
   for (long long r = blockIdx.x; r < nrows; r += gridDim.x) {
     const int b = (int)(r / rows_per_b);
     const int t = a.t_lo + (int)(r % rows_per_b);
-    const int n = min(a.Lk, a.q_pos0 + t + 1);
+    const int n = min(a.Lk, seq_pos0(a.seq_lens, a.q_pos0, a.Lq, b) + t + 1);
     int32_t* dst = a.idx + ((long long)b * a.Lq + t) * a.k;
     if (n <= a.k) {
       for (int i = threadIdx.x; i < a.k; i += TK_THREADS) dst[i] = i < n ? i : -1;
@@ -288,7 +288,7 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   const long long r = blockIdx.x / TKC;
   const int b = (int)(r / rows_per_b);
   const int t = a.t_lo + (int)(r % rows_per_b);
-  const int n = min(a.Lk, a.q_pos0 + t + 1);
+  const int n = min(a.Lk, seq_pos0(a.seq_lens, a.q_pos0, a.Lq, b) + t + 1);
   int32_t* dst = a.idx + ((long long)b * a.Lq + t) * a.k;
   if (n <= a.k) {   // the same decision in every CTA of the cluster: no shared traffic below
     if (rank == 0)
@@ -378,7 +378,7 @@ cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream) {
   const int rows_per_b = a.t_hi - a.t_lo;
   if (rows_per_b <= 0 || a.B <= 0) return cudaSuccess;
   long long nrows = (long long)a.B * rows_per_b;
-  const int n_max = a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk;
+  const int n_max = a.seq_lens != nullptr ? a.Lk : (a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk);
   unsigned grid = (unsigned)(nrows < (1LL << 30) ? nrows : (1LL << 30));
   const bool cluster = n_max <= TKC * TK_SMEM_MAX &&
                        (n_max > TK_SMEM_MAX || (nrows < num_sms && n_max > 4096));

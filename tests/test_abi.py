@@ -101,6 +101,23 @@ def test_indexer_kl_rejects_bad_args(L):
     assert rc == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_forward_paged_rejects_bad_cache(L):
+    from dsa_inputs import CONFIGS
+    p = dsa.Problem.from_config(CONFIGS["tiny"].with_(Lq=1, Lk=512, q_pos0=511))
+    cp = p.c()
+    t = dsa.DsaTensors(*([FAKE] * 8 + [None, None]))
+    ws = ctypes.c_void_p(FAKE)
+    assert L.dsa_forward_paged_workspace_size(ctypes.byref(cp)) > 0
+    good = dict(block_table=FAKE, seq_lens=FAKE, max_blocks=4, page_size=128, num_pages=8)
+    for change, code, text in ((dict(page_size=100), dsa.DSA_ERR_UNSUPPORTED_SHAPE, "page_size"),
+                               (dict(max_blocks=3), dsa.DSA_ERR_INVALID_ARG, "max_blocks * page_size"),
+                               (dict(block_table=None), dsa.DSA_ERR_INVALID_ARG, "block_table"),
+                               (dict(num_pages=0), dsa.DSA_ERR_INVALID_ARG, "num_pages")):
+        c = dsa.DsaPagedCache(**dict(good, **change))
+        rc = L.dsa_forward_paged(ctypes.byref(cp), ctypes.byref(t), ctypes.byref(c), ws, 1 << 30, None)
+        assert rc == code and text in L.dsa_last_error().decode(), (change, L.dsa_last_error())
+
+
 def test_workspace_sizes(L):
     from dsa_inputs import CONFIGS
     for name, cfg in CONFIGS.items():
