@@ -60,16 +60,16 @@ struct Unit {
   int b, t_a, t_b, s_lo, s_hi;
 };
 
-template <int T_BLK>
+template <int T_BLK, bool PAGED>
 __device__ __forceinline__ int unit_count(const IndexerArgs& a, int& nblk, int& maxp) {
   nblk = (a.t_hi - a.t_lo + T_BLK - 1) / T_BLK;
   // with per-sequence lengths every sequence may use the whole capacity
-  int keys_max = a.seq_lens != nullptr ? a.Lk : min(a.Lk, a.q_pos0 + a.t_hi);
+  int keys_max = PAGED ? a.Lk : min(a.Lk, a.q_pos0 + a.t_hi);
   maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
   return a.B * nblk * maxp;
 }
 
-template <int T_BLK>
+template <int T_BLK, bool PAGED>
 __device__ __forceinline__ bool get_unit(const IndexerArgs& a, int u, int nblk, int maxp,
                                          Unit& o) {
   int piece = u % maxp;
@@ -78,13 +78,16 @@ __device__ __forceinline__ bool get_unit(const IndexerArgs& a, int u, int nblk, 
   o.b = rest / nblk;
   o.t_a = a.t_lo + blk * T_BLK;
   o.t_b = min(o.t_a + T_BLK, a.t_hi);
-  int keys = min(a.Lk, seq_pos0(a.seq_lens, a.q_pos0, a.Lq, o.b) + o.t_b);  // keys 0 .. q_pos0 + t_b - 1
+  const int qp = PAGED ? seq_pos0(a.seq_lens, a.q_pos0, a.Lq, o.b) : a.q_pos0;
+  int keys = min(a.Lk, qp + o.t_b);  // keys 0 .. q_pos0 + t_b - 1
   o.s_lo = piece * a.piece_keys;
   o.s_hi = min(keys, o.s_lo + a.piece_keys);
   return o.s_lo < o.s_hi;
 }
 
-template <int D_I, int H_I, int N>
+// PAGED: keys, key scales and causal bounds come through the paged-cache fields
+// (block table, per-sequence lengths); the unpaged instantiation has none of it.
+template <int D_I, int H_I, int N, bool PAGED>
 __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I, H_I, N>::MIN_CTAS)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs a) {
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
   const uint32_t tbase = *tmem_slot;
 
   int nblk, maxp;
-  const int total = unit_count<T_BLK>(a, nblk, maxp);
+  const int total = unit_count<T_BLK, PAGED>(a, nblk, maxp);
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
       bool ok = true;
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
         Unit un;
-        if (!get_unit<T_BLK>(a, u, nblk, maxp, un)) continue;
+        if (!get_unit<T_BLK, PAGED>(a, u, nblk, maxp, un)) continue;
         if (!mbar_wait(&q_empty[qb], qph ^ 1, a.ctl, abort_flag, kSiteIndexer, 1)) { ok = false; break; }
         q_pending[qb] = -1;
         mbar_arrive_expect_tx(&q_full[qb], Tr::QBLK_BYTES);
@@ -162,8 +165,11 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
           mbar_arrive_expect_tx(&k_full[kst], Tr::KTILE_BYTES);
           // a tile of 128 keys never crosses a page (page_size is a multiple of 128); a
           // page number outside the pool points past the tensor map: the tile reads zeros
-          long long krow = key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, un.b, a.Lk, s0);
-          if (krow < 0) krow = (long long)a.num_pages * a.page_size;
+          long long krow = (long long)un.b * a.Lk + s0;
+          if constexpr (PAGED) {
+            krow = key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, un.b, a.Lk, s0);
+            if (krow < 0) krow = (long long)a.num_pages * a.page_size;
+          }
           tma_load_2d(k_smem + kst * Tr::KTILE_BYTES, &tmap_k, 0, (int)krow, &k_full[kst]);
           k_pending[kst] = kph;
           if (++kst == Tr::STAGES) { kst = 0; kph ^= 1; }
@@ -186,7 +192,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
       bool ok = true;
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
         Unit un;
-        if (!get_unit<T_BLK>(a, u, nblk, maxp, un)) continue;
+        if (!get_unit<T_BLK, PAGED>(a, u, nblk, maxp, un)) continue;
         if (!mbar_wait(&q_full[qb], qph, a.ctl, abort_flag, kSiteIndexer, 4)) { ok = false; break; }
         const uint32_t q_addr = smem_u32(q_smem + qb * Tr::QBLK_BYTES);
         for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       Unit un;
-      if (!get_unit<T_BLK>(a, u, nblk, maxp, un)) continue;
+      if (!get_unit<T_BLK, PAGED>(a, u, nblk, maxp, un)) continue;
       // folded per-(token, head) weight w * s^q of this warp's columns, in a
       // buffer private to the warp (no cross-warp barrier)
       __syncwarp();
@@ -254,11 +260,16 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
         for (int j = 0; j < 64; ++j) wr[j] = wbuf[j];
       }
       // key scales are fetched one tile ahead so their latency hides behind a tile
+      const float* ks_row = a.kI_scale + (size_t)un.b * a.Lk;
       auto ks_at = [&](int s) -> float {   // scale of logical key s of this unit's sequence
-        const long long r = key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, un.b, a.Lk, s);
-        return r >= 0 ? __ldg(a.kI_scale + r) : 0.f;
+        if constexpr (PAGED) {
+          const long long r = key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, un.b, a.Lk, s);
+          return r >= 0 ? __ldg(a.kI_scale + r) : 0.f;
+        } else {
+          return __ldg(ks_row + s);
+        }
       };
-      const int qp = seq_pos0(a.seq_lens, a.q_pos0, a.Lq, un.b);
+      const int qp = PAGED ? seq_pos0(a.seq_lens, a.q_pos0, a.Lq, un.b) : a.q_pos0;
       float ks_next = (un.s_lo + key_in_tile < un.s_hi) ? ks_at(un.s_lo + key_in_tile) : 0.f;
       for (int s0 = un.s_lo; s0 < un.s_hi; s0 += Tr::KT) {
         const int s = s0 + key_in_tile;
@@ -338,7 +349,8 @@ template <int D_I, int H_I, int N>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                            int num_sms, cudaStream_t stream) {
   using Tr = IdxTraits<D_I, H_I, N>;
-  auto kern = indexer_kernel<D_I, H_I, N>;
+  const bool paged = a.block_table != nullptr || a.seq_lens != nullptr;
+  auto kern = paged ? indexer_kernel<D_I, H_I, N, true> : indexer_kernel<D_I, H_I, N, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -119,7 +119,9 @@ __device__ __forceinline__ void issue_s_part(uint32_t s_tmem, uint32_t qt_tmem, 
   }
 }
 
-template <int NKB, int DVC>
+// PAGED: latent rows are gathered through the block table (pool rows); the
+// unpaged instantiation reads sequence b's rows directly.
+template <int NKB, int DVC, bool PAGED>
 __global__ void __launch_bounds__(MLA_THREADS, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ kv,
                       const MlaArgs a) {
@@ -338,6 +340,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     const int ptid = threadIdx.x - PROD_T0;
     const int row_bytes = a.Dqk * 2;
     const uint8_t* kv_g = reinterpret_cast<const uint8_t*>(kv);
+    const uint8_t* kv_b = kv_g + (size_t)b * a.Lk * row_bytes;   // unpaged: sequence b's rows
     const uint32_t kv_base = smem_u32(kv_smem);
     const int vb0 = dvc * Tr::NB_B;
     // copy this thread's chunks of one part of tile i into its stage
@@ -357,15 +360,22 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
           const int q = kb * 8 + q8;                  // 16-byte chunk within the row
           const int pos = (tile0 + i) * KEYS + r;
           const int v = pos < a.k ? __ldg(idx_row + pos) : -1;
-          // pool row of the key (sequence b's row v, or its page's row); invalid keys and
-          // pages outside the pool read pool row 0, and invalid keys are masked later
-          long long row = (v >= 0 && v < a.Lk)
-                              ? key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, b, a.Lk, v)
-                              : 0;
-          if (row < 0) row = 0;
+          // invalid keys read row 0 and are masked later; paged: the key's pool row,
+          // and a page outside the pool reads pool row 0
+          const uint8_t* src;
+          if constexpr (PAGED) {
+            long long prow = (v >= 0 && v < a.Lk)
+                                 ? key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, b, a.Lk, v)
+                                 : 0;
+            if (prow < 0) prow = 0;
+            src = kv_g + (size_t)prow * row_bytes;
+          } else {
+            const int row = (v >= 0 && v < a.Lk) ? v : 0;
+            src = kv_b + (size_t)row * row_bytes;
+          }
           const bool in_row = q * 16 < row_bytes;
           cp_async16(stage + kb * Tr::KVBLK + r * 128 + ((q8 ^ (r & 7)) << 4),
-                     kv_g + (size_t)row * row_bytes + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
+                     src + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
         }
       }
       cp_async_commit();
@@ -609,7 +619,7 @@ template <int NKB, int DVC>
 cudaError_t launch_mla_variant(const CUtensorMap& tq, const uint16_t* kv, const MlaArgs& a,
                                cudaStream_t stream) {
   using Tr = MlaTraits<NKB, DVC>;
-  auto kern = sparse_mla_kernel<NKB, DVC>;
+  auto kern = a.block_table != nullptr ? sparse_mla_kernel<NKB, DVC, true> : sparse_mla_kernel<NKB, DVC, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -313,6 +313,44 @@ def test_overlapped_schedule_matches_serial(name, kw):
     assert launches > prof.n and dsa.last_launch_count() == prof.n
 
 
+@pytest.mark.parametrize("name,L,rows", [("tiny", 32, None), ("prefill_8k", 2048, (0, 1, 700, 2047))])
+def test_short_context_is_dense_attention_without_indexer(name, L, rows):
+    """L <= k: every row selects all of its causal keys without scores (the top-k of at
+    most k candidates is all of them), so DSA is dense causal MQA and no indexer or
+    score work is launched."""
+    cfg = CONFIGS[name].with_(Lq=L, Lk=L, q_pos0=0)
+    assert L <= cfg.k
+    inp = gen_inputs(cfg, "cuda", seed=91)
+    p = dsa.Problem.from_config(cfg)
+    out = torch.empty((1, L, cfg.H, cfg.Dv), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, L, cfg.H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((1, L, cfg.k), dtype=torch.int32, device="cuda")
+    prof = dsa.LaunchProfiler(64)
+    dsa.forward_profiled(p, inp, out, prof, lse=lse, idx_out=idx)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    kinds = [k for k, _ in prof.durations()]
+    assert "indexer" not in kinds and "sparse_mla" in kinds, kinds
+    host = ORC.numpy_inputs(inp)
+    idx_h = idx.cpu().numpy()
+    check_rows = range(L) if rows is None else rows
+    if rows is None:
+        dense, dlse = ORC.dense_causal_mqa(host["q"][0], host["kv"][0], cfg.sm_scale, cfg.Dv)
+    ro, rl = [], []
+    for t in check_rows:
+        assert np.array_equal(idx_h[0, t][: t + 1], np.arange(t + 1)) and (idx_h[0, t][t + 1:] == -1).all()
+        if rows is None:
+            ro.append(dense[t])
+            rl.append(dlse[t])
+        else:
+            o, l = ORC.sparse_mla(host["q"][0, t], host["kv"][0], np.arange(t + 1), cfg.sm_scale, cfg.Dv)
+            ro.append(o)
+            rl.append(l)
+    sel = list(check_rows)
+    check_attention(bf16_to_f64(out[0, sel]), np.stack(ro), lse[0, sel].cpu().numpy(), np.stack(rl),
+                    f"short {name}")
+
+
 def test_sparse_mla_skips_invalid_indices():
     cfg = CONFIGS["tiny"].with_(Lq=4, Lk=64)
     inp = gen_inputs(cfg, "cuda", seed=3)
