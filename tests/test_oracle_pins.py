@@ -321,6 +321,27 @@ def test_generator_is_seeded_and_shaped():
     assert torch.all(vals == 448.0)
 
 
+def test_random_key_sets_look_like_selections():
+    from dsa_inputs import random_key_sets, random_scores
+    idx = random_key_sets(2, 40, 16, 5, seed=3)
+    assert idx.shape == (2, 40, 16) and idx.dtype == torch.int32
+    for b in range(2):
+        for t in range(40):
+            row = idx[b, t].numpy()
+            m = min(16, 5 + t + 1)
+            v = row[:m]
+            assert (row[m:] == -1).all() and (v >= 0).all() and (v <= 5 + t).all()
+            assert (np.diff(v) > 0).all()                       # ascending and unique
+            if m == 5 + t + 1:
+                assert np.array_equal(v, np.arange(m))          # short rows keep every key
+    assert torch.equal(idx, random_key_sets(2, 40, 16, 5, seed=3))
+    holes = random_key_sets(1, 40, 16, 5, seed=3, holes=0.5).numpy()
+    kept = holes[holes >= 0]
+    assert 0 < kept.size < (idx[0] >= 0).sum().item() and (kept <= 5 + 39).all()
+    sc = random_scores((3, 4), seed=9, std=2.0)
+    assert sc.dtype == torch.float32 and torch.equal(sc, random_scores((3, 4), seed=9, std=2.0))
+
+
 # ---------------------------------------------------------------------------
 # planted mistakes: each must be caught by at least one pin
 # ---------------------------------------------------------------------------
