@@ -269,6 +269,15 @@ int dsa_forward_paged(const dsa_problem* p, const dsa_tensors* t, const dsa_page
  * buffers `dev` (same layout as dsa_tensors, all device pointers), runs
  * dsa_forward, copies out (and lse/idx_out when both host and device pointers are
  * given) back to host, and waits for the stream. `host` holds host pointers.
+ * With Lq >= 1024 the call is pipelined per sequence in blocks of 4096 query rows
+ * (a remainder under 1024 rows joins the block before it): a block's query rows
+ * and the keys it newly needs are copied in on a library-owned stream while the
+ * previous block computes on `stream`, and its results are copied out on a second
+ * library-owned stream while later blocks compute. Rows are independent, so the
+ * results equal one dsa_forward over all rows. The copies begin after the work
+ * already queued on `stream`; the call returns when all of them are done. ws:
+ * as for dsa_forward over the whole problem. Errors as for dsa_forward; a failed
+ * copy returns DSA_ERR_CUDA.
  */
 int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_tensors* dev,
                      void* ws, size_t ws_bytes, void* stream);

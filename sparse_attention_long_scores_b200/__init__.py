@@ -386,11 +386,14 @@ def forward_profiled(p: Problem, inp: dict, out, prof: LaunchProfiler, lse=None,
     return out
 
 
-def forward_host(p: Problem, host: dict, dev: dict, host_out, dev_out, ws, stream=None):
-    """dsa_forward on host tensors: H2D copies, forward, D2H copy of out, synchronise."""
+def forward_host(p: Problem, host: dict, dev: dict, host_out, dev_out, ws, stream=None,
+                 host_lse=None, dev_lse=None, host_idx=None, dev_idx=None):
+    """dsa_forward on host tensors: H2D copies, forward, D2H copies of out (and of lse
+    / idx_out when both their host and device tensors are given), synchronise. With
+    Lq >= 1024 the library pipelines the copies with the compute by blocks of rows."""
     cp = p.c()
-    ch = _tensors(host, host_out, None, None)
-    cd = _tensors(dev, dev_out, None, None)
+    ch = _tensors(host, host_out, host_lse, host_idx)
+    cd = _tensors(dev, dev_out, dev_lse, dev_idx)
     _check(lib().dsa_forward_host(ctypes.byref(cp), ctypes.byref(ch), ctypes.byref(cd), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)))
     return host_out

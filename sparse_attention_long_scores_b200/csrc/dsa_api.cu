@@ -611,6 +611,40 @@ int side_stream(SideStream** out) {
   return DSA_OK;
 }
 
+// Copy streams of dsa_forward_host's pipeline, per device, created on first use.
+constexpr int kHostPipeRows = 4096;      // query rows per pipelined block
+constexpr int kHostPipeMinRows = 1024;   // shorter problems are not split
+constexpr int kHostPipeEvents = 64;      // ring of events (reused in order)
+struct HostPipe {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t in_done[kHostPipeEvents] = {};
+  cudaEvent_t computed[kHostPipeEvents] = {};
+};
+HostPipe g_host_pipe[kMaxDevices];
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "device index %d", dev);
+  HostPipe& r = g_host_pipe[dev];
+  std::lock_guard<std::mutex> lk(r.mu);
+  if (!r.ready) {
+    DSA_TRY_CUDA(cudaStreamCreateWithFlags(&r.in, cudaStreamNonBlocking), "cudaStreamCreate");
+    DSA_TRY_CUDA(cudaStreamCreateWithFlags(&r.out, cudaStreamNonBlocking), "cudaStreamCreate");
+    DSA_TRY_CUDA(cudaEventCreateWithFlags(&r.start, cudaEventDisableTiming), "cudaEventCreate");
+    for (int i = 0; i < kHostPipeEvents; ++i) {
+      DSA_TRY_CUDA(cudaEventCreateWithFlags(&r.in_done[i], cudaEventDisableTiming), "cudaEventCreate");
+      DSA_TRY_CUDA(cudaEventCreateWithFlags(&r.computed[i], cudaEventDisableTiming), "cudaEventCreate");
+    }
+    r.ready = true;
+  }
+  *out = &r;
+  return DSA_OK;
+}
+
 dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld, int bstride,
                         int t0, int t1, int32_t* idx, const dsa::DevCtl& ctl,
                         const dsa_paged_cache* pc) {
@@ -798,22 +832,124 @@ int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_te
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t B = p->B, Lq = p->Lq, Lk = p->Lk;
   const size_t wbytes = p->w_dtype == DSA_DTYPE_BF16 ? 2 : 4;
-  struct Cp { void* d; const void* h; size_t n; } in[7] = {
-      {(void*)dev->qI, host->qI, B * Lq * p->H_I * p->d_I},
-      {(void*)dev->qI_scale, host->qI_scale, B * Lq * p->H_I * 4},
-      {(void*)dev->kI, host->kI, B * Lk * p->d_I},
-      {(void*)dev->kI_scale, host->kI_scale, B * Lk * 4},
-      {(void*)dev->w, host->w, B * Lq * p->H_I * wbytes},
-      {(void*)dev->q, host->q, B * Lq * p->H * p->Dqk * 2},
-      {(void*)dev->kv, host->kv, B * Lk * p->Dqk * 2}};
-  for (auto& c : in) DSA_TRY_CUDA(cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, s), "H2D copy");
-  DSA_TRY(dsa_forward(p, dev, ws, ws_bytes, stream));
-  DSA_TRY_CUDA(cudaMemcpyAsync(host->out, dev->out, B * Lq * p->H * p->Dv * 2, cudaMemcpyDeviceToHost, s), "D2H copy");
-  if (host->lse && dev->lse)
-    DSA_TRY_CUDA(cudaMemcpyAsync(host->lse, dev->lse, B * Lq * p->H * 4, cudaMemcpyDeviceToHost, s), "D2H copy");
-  if (host->idx_out && dev->idx_out)
-    DSA_TRY_CUDA(cudaMemcpyAsync(host->idx_out, dev->idx_out, B * Lq * p->k * 4, cudaMemcpyDeviceToHost, s), "D2H copy");
-  DSA_TRY_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+  // bytes per query row and per key of each tensor
+  const size_t r_qI = (size_t)p->H_I * p->d_I, r_qs = (size_t)p->H_I * 4, r_w = (size_t)p->H_I * wbytes;
+  const size_t r_q = (size_t)p->H * p->Dqk * 2, r_out = (size_t)p->H * p->Dv * 2;
+  const size_t r_lse = (size_t)p->H * 4, r_idx = (size_t)p->k * 4;
+  const size_t k_kI = (size_t)p->d_I, k_ks = 4, k_kv = (size_t)p->Dqk * 2;
+  auto h2d = [&](void* d, const void* h, size_t off, size_t n, cudaStream_t st) -> int {
+    if (n == 0) return DSA_OK;
+    DSA_TRY_CUDA(cudaMemcpyAsync(static_cast<char*>(d) + off, static_cast<const char*>(h) + off, n,
+                                 cudaMemcpyHostToDevice, st), "H2D copy");
+    return DSA_OK;
+  };
+  auto d2h = [&](void* h, const void* d, size_t off, size_t n, cudaStream_t st) -> int {
+    if (n == 0) return DSA_OK;
+    DSA_TRY_CUDA(cudaMemcpyAsync(static_cast<char*>(h) + off, static_cast<const char*>(d) + off, n,
+                                 cudaMemcpyDeviceToHost, st), "D2H copy");
+    return DSA_OK;
+  };
+  int launched = 0;
+  if (Lq < (size_t)kHostPipeMinRows) {
+    // short problems: everything in, one forward, everything out
+    DSA_TRY(h2d((void*)dev->qI, host->qI, 0, B * Lq * r_qI, s));
+    DSA_TRY(h2d((void*)dev->qI_scale, host->qI_scale, 0, B * Lq * r_qs, s));
+    DSA_TRY(h2d((void*)dev->kI, host->kI, 0, B * Lk * k_kI, s));
+    DSA_TRY(h2d((void*)dev->kI_scale, host->kI_scale, 0, B * Lk * k_ks, s));
+    DSA_TRY(h2d((void*)dev->w, host->w, 0, B * Lq * r_w, s));
+    DSA_TRY(h2d((void*)dev->q, host->q, 0, B * Lq * r_q, s));
+    DSA_TRY(h2d((void*)dev->kv, host->kv, 0, B * Lk * k_kv, s));
+    DSA_TRY(dsa_forward(p, dev, ws, ws_bytes, stream));
+    launched = g_last_launches;
+    DSA_TRY(d2h(host->out, dev->out, 0, B * Lq * r_out, s));
+    if (host->lse && dev->lse) DSA_TRY(d2h(host->lse, dev->lse, 0, B * Lq * r_lse, s));
+    if (host->idx_out && dev->idx_out) DSA_TRY(d2h(host->idx_out, dev->idx_out, 0, B * Lq * r_idx, s));
+    DSA_TRY_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    g_last_launches = launched;
+    return DSA_OK;
+  }
+  // Pipelined: per sequence, blocks of kHostPipeRows query rows. Block c's rows (and
+  // the keys it newly needs) are copied in on the library's copy-in stream while
+  // block c - 1 computes on the caller's stream and block c - 2's results go out
+  // on the copy-out stream. Each block is an ordinary forward over one sequence
+  // (B = 1) whose rows start at q_pos0 + t0: rows are independent, so the results
+  // equal one forward over everything.
+  HostPipe* hpipe = nullptr;
+  DSA_TRY(host_pipe(&hpipe));
+  std::lock_guard<std::mutex> lk(hpipe->mu);
+  // the copies start after whatever the caller queued on its stream before
+  DSA_TRY_CUDA(cudaEventRecord(hpipe->start, s), "cudaEventRecord");
+  DSA_TRY_CUDA(cudaStreamWaitEvent(hpipe->in, hpipe->start, 0), "cudaStreamWaitEvent");
+  auto run = [&]() -> int {
+    int c = 0;
+    for (size_t b = 0; b < B; ++b) {
+      size_t keys_in = 0;
+      for (size_t t0 = 0, t1 = 0; t0 < Lq; t0 = t1, ++c) {
+        // a short remainder joins this block, so that every block has at least
+        // kHostPipeMinRows rows (enough CTAs that the attention needs no key splits)
+        t1 = t0 + kHostPipeRows;
+        if (t1 + kHostPipeMinRows > Lq) t1 = Lq;
+        // keys the block's rows can see (<= Lk, checked by validate_problem); the
+        // sequence's last block brings in the rest of its keys too
+        const size_t keys = t1 == Lq ? Lk : (size_t)p->q_pos0 + t1;
+        cudaEvent_t ev_in = hpipe->in_done[c % kHostPipeEvents];
+        cudaEvent_t ev_out = hpipe->computed[c % kHostPipeEvents];
+        // A block's copies write only its own query rows and the keys that earlier
+        // blocks did not need, which no launch in flight reads: they wait for nothing.
+        const size_t row0 = b * Lq + t0, nrow = t1 - t0;
+        DSA_TRY(h2d((void*)dev->qI, host->qI, row0 * r_qI, nrow * r_qI, hpipe->in));
+        DSA_TRY(h2d((void*)dev->qI_scale, host->qI_scale, row0 * r_qs, nrow * r_qs, hpipe->in));
+        DSA_TRY(h2d((void*)dev->w, host->w, row0 * r_w, nrow * r_w, hpipe->in));
+        DSA_TRY(h2d((void*)dev->q, host->q, row0 * r_q, nrow * r_q, hpipe->in));
+        const size_t key0 = b * Lk + keys_in, nkey = keys - keys_in;
+        DSA_TRY(h2d((void*)dev->kI, host->kI, key0 * k_kI, nkey * k_kI, hpipe->in));
+        DSA_TRY(h2d((void*)dev->kI_scale, host->kI_scale, key0 * k_ks, nkey * k_ks, hpipe->in));
+        DSA_TRY(h2d((void*)dev->kv, host->kv, key0 * k_kv, nkey * k_kv, hpipe->in));
+        keys_in = keys;
+        DSA_TRY_CUDA(cudaEventRecord(ev_in, hpipe->in), "cudaEventRecord");
+        DSA_TRY_CUDA(cudaStreamWaitEvent(s, ev_in, 0), "cudaStreamWaitEvent");
+        dsa_problem sp = *p;
+        sp.B = 1;
+        sp.Lq = (int)nrow;
+        sp.Lk = (int)keys;
+        sp.q_pos0 = p->q_pos0 + (int)t0;
+        dsa_tensors st = *dev;
+        st.qI = dev->qI + row0 * r_qI;
+        st.qI_scale = dev->qI_scale + row0 * p->H_I;
+        st.kI = dev->kI + b * Lk * k_kI;
+        st.kI_scale = dev->kI_scale + b * Lk;
+        st.w = static_cast<const char*>(dev->w) + row0 * r_w;
+        st.q = dev->q + row0 * (size_t)p->H * p->Dqk;
+        st.kv = dev->kv + b * Lk * (size_t)p->Dqk;
+        st.out = dev->out + row0 * (size_t)p->H * p->Dv;
+        st.lse = dev->lse ? dev->lse + row0 * p->H : nullptr;
+        st.idx_out = dev->idx_out ? dev->idx_out + row0 * p->k : nullptr;
+        // at most the block's recommended workspace, so that its score chunks keep
+        // the default size (a larger area would only make them spill out of L2)
+        const size_t sub_rec = dsa_forward_workspace_size(&sp);
+        DSA_TRY(dsa_forward(&sp, &st, ws, ws_bytes < sub_rec ? ws_bytes : sub_rec, stream));
+        launched += g_last_launches;
+        DSA_TRY_CUDA(cudaEventRecord(ev_out, s), "cudaEventRecord");
+        DSA_TRY_CUDA(cudaStreamWaitEvent(hpipe->out, ev_out, 0), "cudaStreamWaitEvent");
+        DSA_TRY(d2h(host->out, dev->out, row0 * r_out, nrow * r_out, hpipe->out));
+        if (host->lse && dev->lse) DSA_TRY(d2h(host->lse, dev->lse, row0 * r_lse, nrow * r_lse, hpipe->out));
+        if (host->idx_out && dev->idx_out)
+          DSA_TRY(d2h(host->idx_out, dev->idx_out, row0 * r_idx, nrow * r_idx, hpipe->out));
+      }
+    }
+    return DSA_OK;
+  };
+  const int rc = run();
+  // Wait for all three streams even after a failure, so that no copy still reads
+  // or writes the caller's host buffers once the call has returned.
+  const cudaError_t e_in = cudaStreamSynchronize(hpipe->in);
+  const cudaError_t e_s = cudaStreamSynchronize(s);
+  const cudaError_t e_out = cudaStreamSynchronize(hpipe->out);
+  if (rc != DSA_OK) return rc;
+  DSA_TRY_CUDA(e_in, "stream synchronize");
+  DSA_TRY_CUDA(e_s, "stream synchronize");
+  DSA_TRY_CUDA(e_out, "stream synchronize");
+  g_last_launches = launched;
   return DSA_OK;
 }
 

@@ -406,3 +406,33 @@ def test_mla_128_heads_every_row(tokens, Lk):
         rl.append(l)
     check_attention(bf16_to_f64(out[0]), np.stack(ro), lse[0].cpu().numpy(), np.stack(rl),
                     f"mla128 tokens={tokens}")
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=2, Lq=5596, Lk=5596, q_pos0=0),      # blocks of 4096 + 1500 rows per sequence
+    dict(B=1, Lq=4596, Lk=9000, q_pos0=4404),   # a 500-row remainder joins the first block
+    dict(B=2, Lq=700, Lk=3000, q_pos0=2300),    # too short to pipeline
+])
+def test_host_entry_point_matches_device_forward(kw):
+    """dsa_forward_host pipelines its copies with the compute by blocks of query rows,
+    each block an ordinary forward over one sequence. Rows are independent, so out,
+    lse and idx_out must equal one dsa_forward over the device tensors bit for bit."""
+    cfg = CONFIGS["tiny"].with_(**kw)
+    inp = gen_inputs(cfg, "cuda", seed=57)
+    out1, lse1, idx1 = _forward(cfg, inp)
+    p = dsa.Problem.from_config(cfg)
+    host = {k: v.cpu().pin_memory() for k, v in inp.items()}
+    dev = {k: torch.zeros_like(v) for k, v in inp.items()}   # staging, filled by the call
+    h_out = torch.empty(tuple(out1.shape), dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(tuple(lse1.shape), dtype=torch.float32).pin_memory()
+    h_idx = torch.empty(tuple(idx1.shape), dtype=torch.int32).pin_memory()
+    d_out, d_lse, d_idx = torch.empty_like(out1), torch.empty_like(lse1), torch.empty_like(idx1)
+    ws = torch.empty(dsa.forward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    dsa.forward_host(p, host, dev, h_out, d_out, ws, host_lse=h_lse, dev_lse=d_lse,
+                     host_idx=h_idx, dev_idx=d_idx)
+    dsa.check_status()
+    for k in inp:
+        assert torch.equal(dev[k].cpu(), host[k]), k
+    assert torch.equal(h_idx, idx1.cpu())
+    assert torch.equal(h_lse, lse1.cpu())
+    assert torch.equal(h_out, out1.cpu())
