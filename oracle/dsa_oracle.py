@@ -1,4 +1,5 @@
-"""Plain fp64 CPU oracle for the DeepSeek Sparse Attention (DSA) forward path.
+"""Plain fp64 CPU oracle for the DeepSeek Sparse Attention (DSA) path: the
+forward and the gradients of its sparse training stage.
 
 TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this module. The CUDA library
@@ -17,7 +18,10 @@ Models", bud-325 paper digest):
   * "Key claims" (paper section 2.1.1, Eq. 3-4, in words) and "Method": the
     indexer is trained with a KL loss toward the head-aggregated main attention
     distribution, on the selected tokens in the sparse stage
-    (``indexer_kl_target``, forward only).
+    (``indexer_kl_target``, and its score gradient ``indexer_kl_score_grad``);
+  * "Method": in the sparse stage the main model learns through the sparse
+    attention and the indexer through its own detached inputs
+    (``sparse_mla_backward``, ``indexer_backward``).
 The eu.36kr.com article (section 02) adds that candidates are the query's
 preceding tokens and that top-k index scores pick the entries that are read.
 
@@ -101,8 +105,16 @@ def index_scores(qI: np.ndarray, qI_scale: np.ndarray, w: np.ndarray,
     """
     q = decode_e4m3(qI) * to_f64(qI_scale)[:, None]          # [H_I, d_I]
     kk = decode_e4m3(kI) * to_f64(kI_scale)[:, None]         # [n, d_I]
-    dots = q @ kk.T                                          # [H_I, n]
-    return to_f64(w) @ np.maximum(dots, 0.0)                 # [n]
+    return index_scores_dequantised(q, to_f64(w), kk)
+
+
+def index_scores_dequantised(q: np.ndarray, w: np.ndarray, kk: np.ndarray) -> np.ndarray:
+    """Eq. 1 on real-valued vectors: I[s] = sum_j w_j * ReLU(q_j . k_s).
+
+    q: [H_I, d_I]; w: [H_I]; kk: [n, d_I]. Returns float64 [n].
+    """
+    dots = np.asarray(q, np.float64) @ np.asarray(kk, np.float64).T    # [H_I, n]
+    return np.asarray(w, np.float64) @ np.maximum(dots, 0.0)
 
 
 # ---------------------------------------------------------------------------
@@ -202,6 +214,113 @@ def indexer_kl_target(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, sel_scores
     kl = float(np.sum(p[nz] * (np.log(p[nz]) - log_r[nz])))
     p_out[ok] = p
     return p_out, kl
+
+
+def indexer_kl_score_grad(p: np.ndarray, sel_scores: np.ndarray, idx: np.ndarray,
+                          n_keys: int) -> np.ndarray:
+    """Gradient of KL(p || r) with respect to the selected index scores, p held fixed.
+
+    The bud-325 digest ("Method") trains the indexer on the KL toward the main
+    attention with the indexer's input detached from the main model's graph, so p
+    is a constant for this loss. With r = softmax over the set of the scores,
+    ln r_s = I_s - logsumexp(I) and sum_s p_s = 1 give
+        d KL / d I_u = -p_u + sum_s p_s r_u = r_u - p_u.
+    p, sel_scores, idx: [k] aligned slots; slots whose idx lies outside
+    [0, n_keys) are not in the set and get 0. Returns float64 [k].
+    """
+    idx = np.asarray(idx)
+    ok = (idx >= 0) & (idx < n_keys)
+    g = np.zeros(idx.shape[0])
+    if not ok.any():
+        return g
+    s = np.asarray(sel_scores, np.float64)[ok]
+    r = np.exp(s - s.max())
+    r /= r.sum()
+    g[ok] = r - np.asarray(p, np.float64)[ok]
+    return g
+
+
+# ---------------------------------------------------------------------------
+# Sparse training stage: gradients
+# ---------------------------------------------------------------------------
+
+
+def sparse_mla_backward(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, dout: np.ndarray,
+                        sm_scale: float, Dv: int):
+    """Gradients of one query token's sparse attention with respect to its query
+    and the latent rows, given dL/d(out).
+
+    The bud-325 digest ("Method") trains the main model in the sparse stage through
+    attention over the selected entries only, so the gradient is the ordinary
+    softmax-attention gradient restricted to the set. With
+    z[h,s] = sm_scale q[h].c_s, a = softmax_s(z), out[h] = sum_s a[h,s] c_s[:Dv]:
+        dA[h,s] = dout[h] . c_s[:Dv]
+        dz[h,s] = a[h,s] (dA[h,s] - dout[h] . out[h])        (softmax Jacobian)
+        dq[h]   = sm_scale sum_s dz[h,s] c_s
+        dc_s    = sm_scale sum_h dz[h,s] q[h], plus sum_h a[h,s] dout[h] on the
+                  first Dv columns (the value part of the shared latent row).
+    q: [H, Dqk]; kv: [n_keys, Dqk]; idx: [k] (entries outside [0, n_keys) are
+    skipped; an index listed twice counts twice, as in the forward); dout: [H, Dv].
+    Returns (dq float64 [H, Dqk], dkv float64 [n_keys, Dqk]).
+    """
+    qf = to_f64(q)
+    H, Dqk = qf.shape
+    idx = np.asarray(idx)
+    valid = idx[(idx >= 0) & (idx < kv.shape[0])]
+    dq = np.zeros((H, Dqk))
+    dkv = np.zeros((kv.shape[0], Dqk))
+    if valid.size == 0:
+        return dq, dkv
+    c = to_f64(kv[valid])                                    # [n, Dqk]
+    do = to_f64(dout)                                        # [H, Dv]
+    z = sm_scale * (qf @ c.T)                                # [H, n]
+    a = np.exp(z - z.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)
+    out = a @ c[:, :Dv]                                      # [H, Dv]
+    dA = do @ c[:, :Dv].T                                    # [H, n]
+    dz = a * (dA - np.sum(do * out, axis=1, keepdims=True))
+    dq = sm_scale * (dz @ c)
+    dc = sm_scale * (dz.T @ qf)                              # [n, Dqk]
+    dc[:, :Dv] += a.T @ do
+    np.add.at(dkv, valid, dc)
+    return dq, dkv
+
+
+def indexer_backward(qI: np.ndarray, qI_scale: np.ndarray, w: np.ndarray, kI: np.ndarray,
+                     kI_scale: np.ndarray, idx: np.ndarray, dI: np.ndarray):
+    """Gradients of L = sum_j dI[j] * I[idx[j]] (one query row) with respect to the
+    dequantised indexer query q^I, the dequantised keys k^I and the weights w.
+
+    The bud-325 digest ("Method") keeps training the indexer in the sparse stage
+    on the KL over the selected tokens, with its input detached: the loss reaches
+    only the indexer's own q^I, k^I and w. From Eq. 1, x[j,s] = q^I_j . k^I_s and
+    I_s = sum_j w_j ReLU(x[j,s]):
+        dw_j   = sum_s dI_s ReLU(x[j,s])
+        g[j,s] = dI_s w_j [x[j,s] > 0]            (ReLU'(0) taken as 0)
+        dq^I_j = sum_s g[j,s] k^I_s
+        dk^I_s = sum_j g[j,s] q^I_j
+    The FP8 rounding is passed through as the identity (gradients are with respect
+    to the dequantised values q^I = s^q qhat and k^I = s^k khat).
+    qI: uint8 [H_I, d_I]; qI_scale, w: [H_I]; kI: uint8 [n_keys, d_I]; kI_scale:
+    [n_keys]; idx, dI: [k] aligned (slots outside [0, n_keys) skipped).
+    Returns (dqI float64 [H_I, d_I], dkI float64 [n_keys, d_I], dw float64 [H_I]).
+    """
+    q = decode_e4m3(qI) * to_f64(qI_scale)[:, None]
+    kk = decode_e4m3(kI) * to_f64(kI_scale)[:, None]
+    wf = to_f64(w)
+    idx = np.asarray(idx)
+    ok = (idx >= 0) & (idx < kk.shape[0])
+    valid = idx[ok]
+    d = np.asarray(dI, np.float64)[ok]
+    dk = np.zeros_like(kk)
+    if valid.size == 0:
+        return np.zeros_like(q), dk, np.zeros_like(wf)
+    x = q @ kk[valid].T                                      # [H_I, n]
+    dw = np.maximum(x, 0.0) @ d
+    g = (x > 0) * wf[:, None] * d[None, :]
+    dq = g @ kk[valid]
+    np.add.at(dk, valid, g.T @ q)
+    return dq, dk, dw
 
 
 def dense_causal_mqa(q: np.ndarray, kv: np.ndarray, sm_scale: float, Dv: int, q_pos0: int = 0):

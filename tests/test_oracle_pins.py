@@ -33,7 +33,11 @@ def real_oracle():
     return types.SimpleNamespace(index_scores=ORC.index_scores, topk_select=ORC.topk_select,
                                  sparse_mla=ORC.sparse_mla, dense_causal_mqa=ORC.dense_causal_mqa,
                                  decode_e4m3=ORC.decode_e4m3,
-                                 indexer_kl_target=ORC.indexer_kl_target)
+                                 indexer_kl_target=ORC.indexer_kl_target,
+                                 index_scores_dequantised=ORC.index_scores_dequantised,
+                                 indexer_kl_score_grad=ORC.indexer_kl_score_grad,
+                                 sparse_mla_backward=ORC.sparse_mla_backward,
+                                 indexer_backward=ORC.indexer_backward)
 
 
 # ---------------------------------------------------------------------------
@@ -285,9 +289,113 @@ def pin_kl_properties(orc):
         assert abs(kl - (float(np.sum(p * np.log(p))) + math.log(t + 1))) < 1e-13
 
 
+def _fd_grad(f, x, eps=1e-6):
+    """Central differences of the scalar function f() in every element of x (x is
+    perturbed in place and restored)."""
+    g = np.zeros_like(x)
+    for i in np.ndindex(*x.shape):
+        old = x[i]
+        x[i] = old + eps
+        fp = f()
+        x[i] = old - eps
+        fm = f()
+        x[i] = old
+        g[i] = (fp - fm) / (2 * eps)
+    return g
+
+
+def pin_mla_backward_finite_differences(orc):
+    """The attention gradients against central differences of the forward, for the
+    loss sum(dout * out), on a set with a padded slot and keys outside the set."""
+    rng = np.random.default_rng(31)
+    H, Dqk, Dv, n, scale = 3, 6, 4, 7, 0.7
+    q = rng.standard_normal((H, Dqk))
+    kv = rng.standard_normal((n, Dqk))
+    idx = np.array([5, 0, -1, 2, 6])
+    dout = rng.standard_normal((H, Dv))
+
+    def loss():
+        return float(np.sum(dout * orc.sparse_mla(q, kv, idx, scale, Dv)[0]))
+
+    dq, dkv = orc.sparse_mla_backward(q, kv, idx, dout, scale, Dv)
+    assert np.allclose(dq, _fd_grad(loss, q), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dkv, _fd_grad(loss, kv), rtol=1e-6, atol=1e-8)
+    assert not dkv[[1, 3, 4]].any()
+
+
+def pin_mla_backward_closed_forms(orc):
+    """One selected key: out = c_s[:Dv] whatever q is, so dq = 0 and the row receives
+    sum_h dout[h] on its value columns and nothing on the others. Adding one vector
+    to the columns past Dv of every selected row adds the same logit to each key of
+    a head, which the softmax ignores, so those columns of dkv sum to 0 over the
+    set. An empty set gives zeros."""
+    rng = np.random.default_rng(32)
+    H, Dqk, Dv, n = 4, 10, 6, 9
+    q = rng.standard_normal((H, Dqk))
+    kv = rng.standard_normal((n, Dqk))
+    dout = rng.standard_normal((H, Dv))
+    dq, dkv = orc.sparse_mla_backward(q, kv, np.array([4, -1, -1]), dout, 0.5, Dv)
+    want = np.zeros((n, Dqk))
+    want[4, :Dv] = dout.sum(axis=0)
+    assert np.allclose(dq, 0.0, rtol=0, atol=1e-14)
+    assert np.allclose(dkv, want, rtol=0, atol=1e-14)
+    idx = rng.permutation(n)[:6]
+    dq, dkv = orc.sparse_mla_backward(q, kv, idx, dout, 0.5, Dv)
+    assert np.allclose(dkv[:, Dv:].sum(axis=0), 0.0, rtol=0, atol=1e-13)
+    assert np.abs(dkv[:, Dv:]).max() > 1e-3
+    dq, dkv = orc.sparse_mla_backward(q, kv, np.array([-1, n]), dout, 0.5, Dv)
+    assert not dq.any() and not dkv.any()
+
+
+def pin_indexer_backward_finite_differences(orc):
+    """Indexer gradients against central differences of Eq. 1 on the dequantised
+    values (loss sum_j dI_j I[idx_j]); heads with every dot <= 0 get nothing."""
+    qc, qs, w, kc, ks, qd, kd = _random_indexer(41, H_I=3, d_I=5, n=8)
+    qf = qd * qs.astype(np.float64)[:, None]
+    kf = kd * ks.astype(np.float64)[:, None]
+    wf = w.astype(np.float64)
+    idx = np.array([6, -1, 1, 3, 0])
+    dI = np.random.default_rng(42).standard_normal(idx.shape[0])
+    ok = idx >= 0
+
+    def loss():
+        return float(np.sum(dI[ok] * orc.index_scores_dequantised(qf, wf, kf)[idx[ok]]))
+
+    dq, dk, dw = orc.indexer_backward(qc, qs, w, kc, ks, idx, dI)
+    x = qf @ kf[idx[ok]].T
+    assert (np.abs(x) > 1e-3).all()          # no dot near the ReLU kink
+    assert np.allclose(dq, _fd_grad(loss, qf), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dk, _fd_grad(loss, kf), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dw, _fd_grad(loss, wf), rtol=1e-6, atol=1e-8)
+    qc, qs, w, kc, ks, _, _ = _random_indexer(43, qsign=1.0, ksign=-1.0)
+    dq, dk, dw = orc.indexer_backward(qc, qs, w, kc, ks, np.arange(10), np.ones(10))
+    assert not dq.any() and not dk.any() and not dw.any()
+
+
+def pin_kl_score_grad_finite_differences(orc):
+    """r - p against central differences of KL(p || r) in the selected scores (p does
+    not depend on them); slots outside the set get 0 and the gradient sums to 0."""
+    cfg = CONFIGS["tiny"]
+    inp = ORC.numpy_inputs(gen_inputs(cfg, "cpu"))
+    rng = np.random.default_rng(44)
+    t = 60
+    idx = np.concatenate([rng.permutation(t + 1)[:20], [-1, -1]])
+    sc = rng.standard_normal(idx.shape[0]) * 2.0
+
+    def kl():
+        return orc.indexer_kl_target(inp["q"][0, t], inp["kv"][0], idx, sc, cfg.sm_scale)[1]
+
+    p, _ = orc.indexer_kl_target(inp["q"][0, t], inp["kv"][0], idx, sc, cfg.sm_scale)
+    g = orc.indexer_kl_score_grad(p, sc, idx, inp["kv"].shape[1])
+    assert np.allclose(g, _fd_grad(kl, sc), rtol=1e-6, atol=1e-9)
+    assert g[-2:].tolist() == [0.0, 0.0] and abs(g.sum()) < 1e-14
+
+
 PINS = [pin_three_token, pin_e4m3_table, pin_indexer_closed_forms, pin_indexer_mixed_signs,
         pin_topk_bruteforce, pin_topk_properties, pin_attention_special_cases,
-        pin_dense_equivalence, pin_invariances, pin_kl_golden, pin_kl_properties]
+        pin_dense_equivalence, pin_invariances, pin_kl_golden, pin_kl_properties,
+        pin_mla_backward_finite_differences, pin_mla_backward_closed_forms,
+        pin_indexer_backward_finite_differences, pin_kl_score_grad_finite_differences]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -442,7 +550,71 @@ def _mut_kl_no_scale(q, kv, idx, sc, sm_scale):
     return ORC.indexer_kl_target(q, kv, idx, sc, 1.0)
 
 
+def _mut_mla_bwd_no_out_term(q, kv, idx, dout, sm_scale, Dv):
+    """Drops the dout . out term of the softmax Jacobian."""
+    qf = ORC.to_f64(q)
+    idx = np.asarray(idx)
+    valid = idx[(idx >= 0) & (idx < kv.shape[0])]
+    dq = np.zeros_like(qf)
+    dkv = np.zeros((kv.shape[0], qf.shape[1]))
+    if valid.size == 0:
+        return dq, dkv
+    c = ORC.to_f64(kv[valid])
+    z = sm_scale * (qf @ c.T)
+    a = np.exp(z - z.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)
+    dz = a * (ORC.to_f64(dout) @ c[:, :Dv].T)
+    dc = sm_scale * (dz.T @ qf)
+    dc[:, :Dv] += a.T @ ORC.to_f64(dout)
+    np.add.at(dkv, valid, dc)
+    return sm_scale * (dz @ c), dkv
+
+
+def _mut_mla_bwd_no_value_grad(q, kv, idx, dout, sm_scale, Dv):
+    """Forgets that the value part of a latent row is the same row as its key."""
+    dq, dkv = ORC.sparse_mla_backward(q, kv, idx, dout, sm_scale, Dv)
+    valid = np.asarray(idx)[(np.asarray(idx) >= 0) & (np.asarray(idx) < kv.shape[0])]
+    qf = ORC.to_f64(q)
+    c = ORC.to_f64(kv[valid])
+    z = sm_scale * (qf @ c.T)
+    a = np.exp(z - z.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)
+    np.add.at(dkv[:, :Dv], valid, -(a.T @ ORC.to_f64(dout)))
+    return dq, dkv
+
+
+def _mut_mla_bwd_transposed_dq(q, kv, idx, dout, sm_scale, Dv):
+    """Scales dq by 1/sm_scale instead of sm_scale."""
+    dq, dkv = ORC.sparse_mla_backward(q, kv, idx, dout, sm_scale, Dv)
+    return dq / (sm_scale * sm_scale), dkv
+
+
+def _mut_idx_bwd_no_w(qI, qs, w, kI, ks, idx, dI):
+    """Leaves the head weight out of the ReLU branch gradient."""
+    return ORC.indexer_backward(qI, qs, np.ones_like(np.asarray(w, np.float64)), kI, ks, idx, dI)[:2] + \
+        (ORC.indexer_backward(qI, qs, w, kI, ks, idx, dI)[2],)
+
+
+def _mut_idx_bwd_dw_no_relu(qI, qs, w, kI, ks, idx, dI):
+    """dw from the raw dots, without the ReLU."""
+    dq, dk, _ = ORC.indexer_backward(qI, qs, w, kI, ks, idx, dI)
+    q = ORC.decode_e4m3(qI) * ORC.to_f64(qs)[:, None]
+    kk = ORC.decode_e4m3(kI) * ORC.to_f64(ks)[:, None]
+    ok = np.asarray(idx) >= 0
+    return dq, dk, (q @ kk[np.asarray(idx)[ok]].T) @ np.asarray(dI, np.float64)[ok]
+
+
+def _mut_kl_grad_sign(p, sc, idx, n_keys):
+    return -ORC.indexer_kl_score_grad(p, sc, idx, n_keys)
+
+
 MUTANTS = {
+    "mla_bwd_no_out_term": dict(sparse_mla_backward=_mut_mla_bwd_no_out_term),
+    "mla_bwd_no_value_grad": dict(sparse_mla_backward=_mut_mla_bwd_no_value_grad),
+    "mla_bwd_dq_wrong_scale": dict(sparse_mla_backward=_mut_mla_bwd_transposed_dq),
+    "idx_bwd_no_head_weight": dict(indexer_backward=_mut_idx_bwd_no_w),
+    "idx_bwd_dw_no_relu": dict(indexer_backward=_mut_idx_bwd_dw_no_relu),
+    "kl_grad_sign": dict(indexer_kl_score_grad=_mut_kl_grad_sign),
     "kl_reversed": dict(indexer_kl_target=_mut_kl_reversed),
     "kl_heads_by_max": dict(indexer_kl_target=_mut_kl_head_max),
     "kl_unnormalised_scores": dict(indexer_kl_target=_mut_kl_raw_scores),
