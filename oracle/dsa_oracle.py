@@ -301,12 +301,20 @@ def indexer_backward(qI: np.ndarray, qI_scale: np.ndarray, w: np.ndarray, kI: np
         dk^I_s = sum_j g[j,s] q^I_j
     The FP8 rounding is passed through as the identity (gradients are with respect
     to the dequantised values q^I = s^q qhat and k^I = s^k khat).
+    The positive scales factor out of the dot, x = s^q s^k (qhat . khat), and the
+    dot of two rows of e4m3 codes is exact in float64 (each product needs at most
+    8 significant bits and every partial sum is a multiple of 2^-18 below 2^25),
+    so the ReLU mask is decided on that exact value.
     qI: uint8 [H_I, d_I]; qI_scale, w: [H_I]; kI: uint8 [n_keys, d_I]; kI_scale:
     [n_keys]; idx, dI: [k] aligned (slots outside [0, n_keys) skipped).
     Returns (dqI float64 [H_I, d_I], dkI float64 [n_keys, d_I], dw float64 [H_I]).
     """
-    q = decode_e4m3(qI) * to_f64(qI_scale)[:, None]
-    kk = decode_e4m3(kI) * to_f64(kI_scale)[:, None]
+    sq = to_f64(qI_scale)
+    sk = to_f64(kI_scale)
+    qh = decode_e4m3(qI)
+    kh = decode_e4m3(kI)
+    q = qh * sq[:, None]
+    kk = kh * sk[:, None]
     wf = to_f64(w)
     idx = np.asarray(idx)
     ok = (idx >= 0) & (idx < kk.shape[0])
@@ -315,9 +323,10 @@ def indexer_backward(qI: np.ndarray, qI_scale: np.ndarray, w: np.ndarray, kI: np
     dk = np.zeros_like(kk)
     if valid.size == 0:
         return np.zeros_like(q), dk, np.zeros_like(wf)
-    x = q @ kk[valid].T                                      # [H_I, n]
+    xhat = qh @ kh[valid].T                                  # [H_I, n], exact
+    x = xhat * sq[:, None] * sk[valid][None, :]
     dw = np.maximum(x, 0.0) @ d
-    g = (x > 0) * wf[:, None] * d[None, :]
+    g = (xhat > 0) * wf[:, None] * d[None, :]
     dq = g @ kk[valid]
     np.add.at(dk, valid, g.T @ q)
     return dq, dk, dw

@@ -372,6 +372,28 @@ def pin_indexer_backward_finite_differences(orc):
     assert not dq.any() and not dk.any() and not dw.any()
 
 
+def pin_code_dots_exact(orc):
+    """The indexer backward decides its ReLU mask on dots of e4m3 codes in float64,
+    which must be exact: every e4m3 value times 2^9 is an integer, so the dot times
+    2^18 is an integer sum, checked here with Python integers on the extreme codes."""
+    rng = np.random.default_rng(45)
+    table = orc.decode_e4m3(np.arange(256, dtype=np.uint8))
+    finite = np.flatnonzero(np.isfinite(table)).astype(np.uint8)
+    for d_I in (32, 128):
+        a = rng.choice(finite, size=(6, d_I))
+        b = rng.choice(finite, size=(9, d_I))
+        a[0] = 0x7E              # 448, the largest code, in every column
+        b[0] = 0x7E
+        b[1] = 0x01              # the smallest subnormal, 2^-9
+        got = orc.decode_e4m3(a) @ orc.decode_e4m3(b).T
+        ia = (orc.decode_e4m3(a) * 512).astype(np.int64)
+        ib = (orc.decode_e4m3(b) * 512).astype(np.int64)
+        for i in range(a.shape[0]):
+            for j in range(b.shape[0]):
+                exact = sum(int(x) * int(y) for x, y in zip(ia[i], ib[j]))
+                assert got[i, j] * 2.0 ** 18 == exact, (d_I, i, j)
+
+
 def pin_kl_score_grad_finite_differences(orc):
     """r - p against central differences of KL(p || r) in the selected scores (p does
     not depend on them); slots outside the set get 0 and the gradient sums to 0."""
@@ -395,7 +417,8 @@ PINS = [pin_three_token, pin_e4m3_table, pin_indexer_closed_forms, pin_indexer_m
         pin_topk_bruteforce, pin_topk_properties, pin_attention_special_cases,
         pin_dense_equivalence, pin_invariances, pin_kl_golden, pin_kl_properties,
         pin_mla_backward_finite_differences, pin_mla_backward_closed_forms,
-        pin_indexer_backward_finite_differences, pin_kl_score_grad_finite_differences]
+        pin_indexer_backward_finite_differences, pin_code_dots_exact,
+        pin_kl_score_grad_finite_differences]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
