@@ -354,6 +354,102 @@ def time_indexer_kl(name: str, steps: int, warmup: int, world: int, rank: int, p
     return res
 
 
+FP64_NOMINAL_TFLOPS = 37.0   # B200 datasheet fp64, for context (no measured fp64 peak)
+
+
+def time_backward(name: str, steps: int, warmup: int, world: int, rank: int, pk: dict):
+    """The sparse-stage gradients on the workload's own selected sets, each timed with
+    CUDA events on the launching stream: the attention backward (dsa_sparse_mla_bwd,
+    dq and dkv from a seeded output gradient) and the indexer backward
+    (dsa_indexer_kl_grad on the KL target's p, then dsa_indexer_bwd)."""
+    import sparse_attention_long_scores_b200 as dsa
+    from dsa_inputs import output_gradient, random_scores
+
+    cfg = CONFIGS[name]
+    dev = "cuda"
+    inp = gen_inputs(cfg, dev, seed=rank_seed(name, rank))
+    p = dsa.Problem.from_config(cfg)
+    B, Lq, Lk = cfg.B, cfg.Lq, cfg.Lk
+    out = torch.empty((B, Lq, cfg.H, cfg.Dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Lq, cfg.H), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Lq, cfg.k), dtype=torch.int32, device=dev)
+    dsa.forward(p, inp, out=out, lse=lse, idx_out=idx)
+    dout = output_gradient((B, Lq, cfg.H, cfg.Dv), seed=5 + rank, device=dev)
+    sel = random_scores((B, Lq, cfg.k), seed=77 + rank).to(dev)
+    _, pt = dsa.indexer_kl(inp["q"], inp["kv"], idx, lse, sel, cfg.sm_scale)
+    dq = torch.empty((B, Lq, cfg.H, cfg.Dqk), dtype=torch.float32, device=dev)
+    dkv = torch.empty((B, Lk, cfg.Dqk), dtype=torch.float32, device=dev)
+    ws = torch.empty(dsa.lib().dsa_sparse_mla_bwd_workspace_size(B, Lq, cfg.H, cfg.Dqk, cfg.Dv,
+                                                                 cfg.k), dtype=torch.uint8, device=dev)
+    dI = torch.empty_like(sel)
+    dqI = torch.empty((B, Lq, cfg.H_I, cfg.d_I), dtype=torch.float32, device=dev)
+    dkI = torch.empty((B, Lk, cfg.d_I), dtype=torch.float32, device=dev)
+    dw = torch.empty((B, Lq, cfg.H_I), dtype=torch.float32, device=dev)
+    wsi = torch.empty(dsa.lib().dsa_indexer_bwd_workspace_size(B, Lq, cfg.H_I, cfg.d_I, cfg.k),
+                      dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    launches = {}
+
+    def attention():
+        dsa.sparse_mla_bwd(inp["q"], inp["kv"], idx, out, lse, dout, cfg.sm_scale, dq=dq, dkv=dkv,
+                           ws=ws)
+        launches["attention"] = dsa.last_launch_count()
+
+    def indexer():
+        dsa.indexer_kl_grad(sel, pt, idx, Lk, dI=dI)
+        n = dsa.last_launch_count()
+        dsa.indexer_bwd(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"], idx, dI,
+                        dqI=dqI, dkI=dkI, dw=dw, ws=wsi)
+        launches["indexer"] = n + dsa.last_launch_count()
+
+    n_steps = max(1, min(steps, 5))
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        dsa.check_status()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        dsa.check_status()
+        return dist_max(e0.elapsed_time(e1) / n_steps, world)
+
+    ms_att = timed(attention)
+    ms_idx = timed(indexer)
+    pairs = work(cfg)["mla_flops"] / (2.0 * cfg.H * (cfg.Dqk + cfg.Dv))
+    att_tf = pairs * 2.0 * cfg.H * (3 * cfg.Dqk + 2 * cfg.Dv) / (ms_att * 1e-3) / 1e12
+    idx_tf = pairs * 6.0 * cfg.H_I * cfg.d_I / (ms_idx * 1e-3) / 1e12
+    res = {"workload": cfg.name,
+           "value": aggregate_tokens_per_s(B * Lq, world, ms_att + ms_idx), "unit": "tokens/s",
+           "ms_per_step": ms_att + ms_idx, "steps": n_steps,
+           "attention": {"ms_per_step": ms_att, "launches_per_step": launches.get("attention"),
+                         "roofline": {"bound": "tensor", "achieved": att_tf,
+                                      "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                                      "frac": att_tf / pk["bf16_sustained"], "traffic": None,
+                                      "peak_note": "measured bf16 sustained; work = "
+                                                   "2 H (3 Dqk + 2 Dv) per selected pair"}},
+           "indexer": {"ms_per_step": ms_idx, "launches_per_step": launches.get("indexer"),
+                       "roofline": {"bound": "fp64", "achieved": idx_tf,
+                                    "peak": FP64_NOMINAL_TFLOPS, "unit": "TFLOP/s",
+                                    "frac": idx_tf / FP64_NOMINAL_TFLOPS, "traffic": None,
+                                    "peak_note": "nominal B200 fp64 (not measured); work = "
+                                                 "6 H_I d_I per selected pair"}},
+           "note": "gradients of the sparse training stage: cuBLAS strided-batched GEMMs over "
+                   "gathered rows (bf16 for attention, fp64 for the indexer) with this library's "
+                   "gather, softmax/ReLU-gradient and scatter-add kernels; launches count this "
+                   "library's kernels only"}
+    del inp, out, lse, idx, dout, sel, pt, dq, dkv, ws, dI, dqI, dkI, dw, wsi
+    torch.cuda.empty_cache()
+    return res
+
+
 def oracle_sample(cfg, rows: int, seed: int = 4242):
     """A bounded sample of the workload for the fp64 oracle: one sequence with all
     Lk keys and `rows` query rows at evenly spread positions (decode: the last)."""
@@ -478,6 +574,7 @@ def main():
     ap.add_argument("--decode-workload", default="decode_128k")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-kl", action="store_true", help="skip the indexer KL target line")
+    ap.add_argument("--no-backward", action="store_true", help="skip the sparse-stage gradient line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
@@ -516,6 +613,9 @@ def main():
     kl = None
     if not args.no_kl:
         kl = time_indexer_kl(args.workload, args.steps, args.warmup, world, rank, pk)
+    bwd = None
+    if not args.no_backward:
+        bwd = time_backward(args.workload, args.steps, args.warmup, world, rank, pk)
     dec = None
     if not args.no_decode:
         dec = time_workload(args.decode_workload, args.steps, args.warmup, world, rank, pk,
@@ -557,6 +657,8 @@ def main():
             }
         if kl is not None:
             line["indexer_kl"] = kl
+        if bwd is not None:
+            line["backward"] = bwd
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)

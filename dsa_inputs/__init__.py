@@ -190,6 +190,13 @@ def gen_inputs(cfg: DsaConfig, device: str = "cpu", seed: int | None = None,
     return out
 
 
+def output_gradient(shape, seed: int, device: str = "cpu", std: float = 1.0) -> torch.Tensor:
+    """Seeded N(0, std^2) bf16 stand-in for dL/d(out), the loss gradient that reaches
+    the attention output in the sparse training stage. numpy PCG64 on the CPU, torch
+    Philox on a CUDA device (the same seed gives different values on the two)."""
+    return _fill_normal_bf16(_Source(np.random.SeedSequence(seed), device), shape, std)
+
+
 def sample_rows(cfg: DsaConfig, n_per_seq: int = 64) -> list:
     """Query rows checked against the oracle at full size.
 

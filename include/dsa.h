@@ -179,11 +179,88 @@ int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, co
                    int H, int Dqk, int k, float sm_scale, void* stream);
 
 /*
+ * Sparse training stage: gradients. ("DeepSeek-V3.2: Pushing the Frontier of
+ * Open Large Language Models", bud-325 paper digest, "Method": in the sparse
+ * stage the main model is trained through attention over the top-k selected
+ * entries, and the indexer keeps training on the KL over the selected tokens with
+ * its input detached from the main model's graph.) The contractions run as
+ * strided-batched cuBLAS GEMMs (bf16 operands with fp32 accumulation for the
+ * attention, fp64 for the indexer) over the selected rows, gathered per chunk of
+ * up to 64 tokens into the workspace; the gathers, the softmax / ReLU gradients and
+ * the scatter-add of key gradients are this library's kernels. The first call on
+ * a device creates a cuBLAS handle, which keeps a small device allocation of
+ * cuBLAS's own until the process exits; GEMM scratch comes from `ws`. Key
+ * gradients are accumulated with atomics, so their last bits may differ from
+ * run to run. All pointers are caller-owned device memory, 16-byte aligned.
+ * Errors: DSA_ERR_INVALID_ARG (null or misaligned pointer, bad scalar),
+ * DSA_ERR_UNSUPPORTED_SHAPE, DSA_ERR_WORKSPACE_TOO_SMALL (below one token's
+ * share), DSA_ERR_CUDA (a launch or cuBLAS call failed).
+ *
+ * dsa_sparse_mla_bwd - gradients of the sparse attention (dsa_sparse_mla_fwd)
+ * with respect to q and the latent rows, given dout = dL/d(out). With
+ * z[h,s] = sm_scale q[h].c_s over the valid slots s of idx[t,:] and
+ * P = exp(z - lse):
+ *     D[h]    = dout[h] . out[h]
+ *     dz[h,s] = sm_scale P[h,s] (dout[h] . c_s[:Dv] - D[h])
+ *     dq[h]   = sum_s dz[h,s] c_s                      (all Dqk columns)
+ *     dkv[s] += sum_h dz[h,s] q[h]   and, on columns < Dv, sum_h P[h,s] dout[h]
+ *   q [B, Lq, H, Dqk], kv [B, Lk, Dqk], out and dout [B, Lq, H, Dv]: bf16;
+ *   idx [B, Lq, k] int32 (slots < 0 or >= Lk skipped); lse [B, Lq, H] fp32 as
+ *   the forward returned it; dq [B, Lq, H, Dqk] fp32 (overwritten);
+ *   dkv [B, Lk, Dqk] fp32, zeroed first unless accumulate_dkv != 0.
+ *   (H, Dqk, Dv) in {(8, 80, 64), (128, 576, 512)}; k a multiple of 32 in
+ *   [32, 4096]. P and dz enter their GEMMs rounded to bf16.
+ *   ws: dsa_sparse_mla_bwd_workspace_size(...) bytes (about 10 MB per token of a
+ *   chunk at H = 128, k = 2048); less makes smaller chunks.
+ */
+size_t dsa_sparse_mla_bwd_workspace_size(int B, int Lq, int H, int Dqk, int Dv, int k);
+int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                       const uint16_t* out, const float* lse, const uint16_t* dout, float* dq,
+                       float* dkv, int accumulate_dkv, int B, int Lq, int Lk, int H, int Dqk,
+                       int Dv, int k, float sm_scale, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dsa_indexer_kl_grad - dI = loss_scale * (r - p): the gradient of
+ * loss_scale * KL(p || r) (dsa_indexer_kl) with respect to the selected index
+ * scores, p held fixed (the indexer's input is detached), r = softmax over the
+ * set of sel_scores. sel_scores, p (dsa_indexer_kl's p_out), dI: [B, Lq, k] fp32;
+ * idx [B, Lq, k] int32, slots < 0 or >= Lk get 0. k a multiple of 32 in
+ * [32, 4096]; loss_scale finite.
+ */
+int dsa_indexer_kl_grad(const float* sel_scores, const float* p, const int32_t* idx, float* dI,
+                        int B, int Lq, int Lk, int k, float loss_scale, void* stream);
+
+/*
+ * dsa_indexer_bwd - gradients of L = sum_{t,j} dI[t,j] I[t, idx[t,j]] (Eq. 1) with
+ * respect to the dequantised indexer inputs q^I = s^q qhat, k^I = s^k khat and
+ * the weights w; the FP8 rounding is passed through as the identity. With
+ * x[j,s] = q^I[t,j] . k^I[s]:
+ *     dw[t,j]   = sum_s dI[t,s] max(x[j,s], 0)
+ *     g[j,s]    = dI[t,s] w[t,j] [x[j,s] > 0]
+ *     dqI[t,j]  = sum_s g[j,s] k^I[s]
+ *     dkI[s]   += sum_{t,j} g[j,s] q^I[t,j]
+ *   qI [B, Lq, H_I, d_I] and kI [B, Lk, d_I] e4m3 codes, qI_scale [B, Lq, H_I],
+ *   kI_scale [B, Lk], w [B, Lq, H_I] (w_dtype) as for dsa_indexer_scores;
+ *   idx, dI [B, Lq, k] aligned (slots < 0 or >= Lk skipped); dqI
+ *   [B, Lq, H_I, d_I], dw [B, Lq, H_I] fp32 (overwritten); dkI [B, Lk, d_I] fp32,
+ *   zeroed first unless accumulate_dkI != 0. The contractions run in fp64, where
+ *   the dots of the e4m3 codes are exact, so the ReLU mask is decided exactly.
+ *   ws: dsa_indexer_bwd_workspace_size(...) bytes; less makes smaller chunks.
+ */
+size_t dsa_indexer_bwd_workspace_size(int B, int Lq, int H_I, int d_I, int k);
+int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
+                    const float* kI_scale, const void* w, int w_dtype, const int32_t* idx,
+                    const float* dI, float* dqI, float* dkI, float* dw, int accumulate_dkI, int B,
+                    int Lq, int Lk, int H_I, int d_I, int k, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
  * dsa_last_launch_count - number of kernel launches that the calling thread's
- * last dsa_forward, dsa_forward_host or dsa_forward_profiled call enqueued
- * (all of this library's kernels, on the caller's stream and on the library's
- * internal side stream). 0 before the first call. For benchmarks that report
- * how many of the library's kernels ran in a timed region.
+ * last dsa_forward, dsa_forward_host, dsa_forward_profiled, dsa_sparse_mla_bwd,
+ * dsa_indexer_bwd or dsa_indexer_kl_grad call enqueued (all of this library's
+ * kernels, on the caller's stream and on the library's internal side stream;
+ * not cuBLAS's). 0 before the first call. For benchmarks that report how many
+ * of the library's kernels ran in a timed region.
  */
 int dsa_last_launch_count(void);
 

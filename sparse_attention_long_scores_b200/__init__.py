@@ -40,7 +40,8 @@ EXPORTED = [
     "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
     "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout", "dsa_sparse_mla_fwd_noalloc",
     "dsa_indexer_kl", "dsa_last_launch_count", "dsa_forward_paged_workspace_size",
-    "dsa_forward_paged",
+    "dsa_forward_paged", "dsa_sparse_mla_bwd_workspace_size", "dsa_sparse_mla_bwd",
+    "dsa_indexer_kl_grad", "dsa_indexer_bwd_workspace_size", "dsa_indexer_bwd",
 ]
 KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
 
@@ -107,12 +108,22 @@ def lib() -> ctypes.CDLL:
     L.dsa_forward_profiled.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp,
                                        sz, vp, ctypes.POINTER(ctypes.c_void_p),
                                        ctypes.POINTER(ctypes.c_int), i, ctypes.POINTER(ctypes.c_int)]
+    L.dsa_sparse_mla_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.dsa_sparse_mla_bwd_workspace_size.restype = sz
+    L.dsa_sparse_mla_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                     ctypes.c_float, vp, sz, vp]
+    L.dsa_indexer_kl_grad.argtypes = [vp, vp, vp, vp, i, i, i, i, ctypes.c_float, vp]
+    L.dsa_indexer_bwd_workspace_size.argtypes = [i, i, i, i, i]
+    L.dsa_indexer_bwd_workspace_size.restype = sz
+    L.dsa_indexer_bwd.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
+                                  vp, sz, vp]
     L.dsa_check_status.argtypes = [vp]
     L.dsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     L.dsa_debug_wait_timeout.argtypes = [vp]
     for name in ("dsa_indexer_scores", "dsa_topk_select", "dsa_sparse_mla_fwd", "dsa_forward",
                  "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status", "dsa_set_wait_limit_ns",
-                 "dsa_debug_wait_timeout"):
+                 "dsa_debug_wait_timeout", "dsa_sparse_mla_bwd", "dsa_indexer_kl_grad",
+                 "dsa_indexer_bwd"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -243,6 +254,93 @@ def indexer_kl(q, kv, idx, lse, sel_scores, sm_scale: float, p_out=None, kl_out=
                                 _ptr(p_out), _ptr(kl_out), B, Lq, Lk, H, Dqk, k,
                                 float(sm_scale), _stream(stream)))
     return kl_out, p_out
+
+
+def _workspace(nbytes: int, device):
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def sparse_mla_bwd(q, kv, idx, out, lse, dout, sm_scale: float, dq=None, dkv=None,
+                   accumulate_dkv: bool = False, ws=None, stream=None):
+    """Sparse-stage attention gradients: dq [B, Lq, H, Dqk] fp32 and dkv [B, Lk, Dqk]
+    fp32 from dout = dL/d(out) [B, Lq, H, Dv] bf16, given the forward's idx, out and
+    lse. dkv is overwritten unless accumulate_dkv. Returns (dq, dkv)."""
+    B, Lq, H, Dqk = q.shape
+    Lk = kv.shape[1]
+    k = idx.shape[2]
+    Dv = dout.shape[3]
+    _need(q, "q", torch.bfloat16)
+    _need(kv, "kv", torch.bfloat16, (B, Lk, Dqk))
+    _need(idx, "idx", torch.int32, (B, Lq, k))
+    _need(out, "out", torch.bfloat16, (B, Lq, H, Dv))
+    _need(lse, "lse", torch.float32, (B, Lq, H))
+    _need(dout, "dout", torch.bfloat16, (B, Lq, H, Dv))
+    if dq is None:
+        dq = torch.empty((B, Lq, H, Dqk), dtype=torch.float32, device=q.device)
+    if dkv is None:
+        dkv = torch.empty((B, Lk, Dqk), dtype=torch.float32, device=q.device)
+    _need(dq, "dq", torch.float32, (B, Lq, H, Dqk))
+    _need(dkv, "dkv", torch.float32, (B, Lk, Dqk))
+    if ws is None:
+        ws = _workspace(lib().dsa_sparse_mla_bwd_workspace_size(B, Lq, H, Dqk, Dv, k), q.device)
+    _check(lib().dsa_sparse_mla_bwd(_ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(lse),
+                                    _ptr(dout), _ptr(dq), _ptr(dkv), int(bool(accumulate_dkv)),
+                                    B, Lq, Lk, H, Dqk, Dv, k, float(sm_scale), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)))
+    return dq, dkv
+
+
+def indexer_kl_grad(sel_scores, p, idx, Lk: int, loss_scale: float = 1.0, dI=None, stream=None):
+    """dI = loss_scale (softmax over the set of sel_scores - p) [B, Lq, k] fp32: the
+    gradient of the KL alignment loss in the selected index scores."""
+    B, Lq, k = idx.shape
+    _need(idx, "idx", torch.int32)
+    _need(sel_scores, "sel_scores", torch.float32, (B, Lq, k))
+    _need(p, "p", torch.float32, (B, Lq, k))
+    if dI is None:
+        dI = torch.empty((B, Lq, k), dtype=torch.float32, device=idx.device)
+    _need(dI, "dI", torch.float32, (B, Lq, k))
+    _check(lib().dsa_indexer_kl_grad(_ptr(sel_scores), _ptr(p), _ptr(idx), _ptr(dI), B, Lq, int(Lk),
+                                     k, float(loss_scale), _stream(stream)))
+    return dI
+
+
+def indexer_bwd(qI, qI_scale, kI, kI_scale, w, idx, dI, dqI=None, dkI=None, dw=None,
+                accumulate_dkI: bool = False, ws=None, stream=None):
+    """Indexer gradients with respect to the dequantised q^I [B, Lq, H_I, d_I], k^I
+    [B, Lk, d_I] and the weights w [B, Lq, H_I] (all fp32), from dI = dL/dI at the
+    selected slots [B, Lq, k]. dkI is overwritten unless accumulate_dkI. Returns
+    (dqI, dkI, dw)."""
+    B, Lq, H_I, d_I = qI.shape
+    Lk = kI.shape[1]
+    k = idx.shape[2]
+    _need(qI, "qI", torch.uint8)
+    _need(qI_scale, "qI_scale", torch.float32, (B, Lq, H_I))
+    _need(kI, "kI", torch.uint8, (B, Lk, d_I))
+    _need(kI_scale, "kI_scale", torch.float32, (B, Lk))
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("w must be float32 or bfloat16")
+    _need(w, "w", w.dtype, (B, Lq, H_I))
+    _need(idx, "idx", torch.int32, (B, Lq, k))
+    _need(dI, "dI", torch.float32, (B, Lq, k))
+    dev = qI.device
+    if dqI is None:
+        dqI = torch.empty((B, Lq, H_I, d_I), dtype=torch.float32, device=dev)
+    if dkI is None:
+        dkI = torch.empty((B, Lk, d_I), dtype=torch.float32, device=dev)
+    if dw is None:
+        dw = torch.empty((B, Lq, H_I), dtype=torch.float32, device=dev)
+    _need(dqI, "dqI", torch.float32, (B, Lq, H_I, d_I))
+    _need(dkI, "dkI", torch.float32, (B, Lk, d_I))
+    _need(dw, "dw", torch.float32, (B, Lq, H_I))
+    if ws is None:
+        ws = _workspace(lib().dsa_indexer_bwd_workspace_size(B, Lq, H_I, d_I, k), dev)
+    wd = DSA_DTYPE_BF16 if w.dtype == torch.bfloat16 else DSA_DTYPE_F32
+    _check(lib().dsa_indexer_bwd(_ptr(qI), _ptr(qI_scale), _ptr(kI), _ptr(kI_scale), _ptr(w), wd,
+                                 _ptr(idx), _ptr(dI), _ptr(dqI), _ptr(dkI), _ptr(dw),
+                                 int(bool(accumulate_dkI)), B, Lq, Lk, H_I, d_I, k, _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)))
+    return dqI, dkI, dw
 
 
 @dataclass

@@ -18,10 +18,13 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libdsa.so")
-SOURCES = ["dsa_api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "indexer_kl.cu"]
+SOURCES = ["dsa_api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "indexer_kl.cu", "backward.cu"]
 HEADERS = ["dsa_common.cuh", "dsa_kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# cuBLAS runs the batched GEMMs of the sparse-stage gradients.
+CUDA_LIB = "/usr/local/cuda/lib64"
+LINK = ["-L" + CUDA_LIB, "-lcublas", "-Xlinker", "-rpath=" + CUDA_LIB]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
@@ -69,7 +72,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
     if force or jobs or _stale(LIB, objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs]
+        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, *LINK]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)

@@ -1,0 +1,379 @@
+// backward.cu - the memory-bound kernels of the sparse training stage's
+// gradients ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language
+// Models", bud-325 paper digest, "Method": in the sparse stage the main model
+// learns through attention over the selected entries, and the indexer through
+// its own detached inputs with the KL on the selected tokens).
+//
+// The contractions of both gradients run as batched GEMMs (dsa_api.cu) over
+// the selected rows gathered here into a dense per-token block; these kernels
+// do the gathers, the softmax / ReLU gradient in between and the scatter-add of
+// the per-token key gradients back into the shared rows. Every kernel is a
+// grid-stride loop over rows with one warp per row, so any grid size is correct.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "dsa_kernels.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kRowThreads = 256;   // 8 warps per block, one row per warp
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t u) {
+  return __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t code) {
+  __nv_fp8_e4m3 x;
+  x.__x = code;
+  return static_cast<float>(x);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ long long warp_id_global() {
+  return (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+}
+
+__device__ __forceinline__ long long warps_in_grid() {
+  return (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+}
+
+// Rows (tt, j) of a chunk of T tokens starting at token tok0: the selected key
+// s = idx[tok][j] of sequence b = tok / Lq, or none when s is outside [0, Lk).
+__device__ __forceinline__ int selected_key(const int32_t* idx, long long tok, int j, int k,
+                                            int Lk) {
+  const int s = idx[tok * k + j];
+  return (s >= 0 && s < Lk) ? s : -1;
+}
+
+// out[tt][j][:] = kv[b][idx[tok][j]][:] (bf16 rows of V 16-byte vectors), zeros
+// for a slot without a valid key.
+__global__ void gather_rows_bf16_kernel(const uint4* __restrict__ kv,
+                                        const int32_t* __restrict__ idx, uint4* __restrict__ out,
+                                        long long tok0, int T, int Lq, int Lk, int k, int V) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * k;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / k;
+    const int j = static_cast<int>(r % k);
+    const int s = selected_key(idx, tok, j, k, Lk);
+    const long long b = tok / Lq;
+    uint4* dst = out + r * V;
+    if (s < 0) {
+      for (int v = lane; v < V; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      const uint4* src = kv + (b * Lk + s) * V;
+      for (int v = lane; v < V; v += 32) dst[v] = src[v];
+    }
+  }
+}
+
+// Softmax gradient of one (token, head) row over its k slots:
+//   D = dout . out,  P_s = exp(sm_scale S_s - lse),  dz_s = sm_scale P_s (dP_s - D)
+// with S and dP the raw q.c_s and dout.c_s[:Dv] of the batched GEMMs. P and dz are
+// written as bf16 for the GEMMs that follow; slots without a valid key get 0.
+__global__ void mla_bwd_softmax_kernel(const float* __restrict__ S, const float* __restrict__ dP,
+                                       const uint16_t* __restrict__ out,
+                                       const uint16_t* __restrict__ dout,
+                                       const float* __restrict__ lse,
+                                       const int32_t* __restrict__ idx, uint16_t* __restrict__ P16,
+                                       uint16_t* __restrict__ dz16, long long tok0, int T, int H,
+                                       int Dv, int k, int Lk, float sm_scale) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * H;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / H;
+    const int h = static_cast<int>(r % H);
+    const long long oh = (tok * H + h) * Dv;
+    float d = 0.f;
+    for (int v = lane; v < Dv; v += 32)
+      d += bf16_bits_to_float(dout[oh + v]) * bf16_bits_to_float(out[oh + v]);
+    d = warp_sum(d);
+    const float l = lse[tok * H + h];
+    const float* srow = S + r * k;
+    const float* prow = dP + r * k;
+    uint16_t* p_out = P16 + r * k;
+    uint16_t* z_out = dz16 + r * k;
+    for (int j = lane; j < k; j += 32) {
+      float p = 0.f, z = 0.f;
+      if (selected_key(idx, tok, j, k, Lk) >= 0) {
+        p = expf(srow[j] * sm_scale - l);
+        z = sm_scale * p * (prow[j] - d);
+      }
+      p_out[j] = float_to_bf16_bits(p);
+      z_out[j] = float_to_bf16_bits(z);
+    }
+  }
+}
+
+// dst[b][idx[tok][j]][:] += src[tt][j][:] over rows of V float4 vectors (atomic:
+// tokens of one sequence share keys).
+__global__ void scatter_add_rows_kernel(const float4* __restrict__ src,
+                                        const int32_t* __restrict__ idx, float4* __restrict__ dst,
+                                        long long tok0, int T, int Lq, int Lk, int k, int V) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * k;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / k;
+    const int j = static_cast<int>(r % k);
+    const int s = selected_key(idx, tok, j, k, Lk);
+    if (s < 0) continue;
+    const long long b = tok / Lq;
+    float4* d = dst + (b * Lk + s) * V;
+    const float4* x = src + r * V;
+    for (int v = lane; v < V; v += 32) atomicAdd(d + v, x[v]);
+  }
+}
+
+// out[tt][j][:] = khat[b][idx[tok][j]][:] as float64 for e4m3 rows of d_I bytes
+// (the unscaled codes), zeros for a slot without a valid key.
+__global__ void gather_e4m3_rows_kernel(const uint8_t* __restrict__ kI,
+                                        const int32_t* __restrict__ idx, double* __restrict__ out,
+                                        long long tok0, int T, int Lq, int Lk, int k, int d_I) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * k;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / k;
+    const int j = static_cast<int>(r % k);
+    const int s = selected_key(idx, tok, j, k, Lk);
+    const long long b = tok / Lq;
+    double* dst = out + r * d_I;
+    for (int c = lane; c < d_I; c += 32)
+      dst[c] = s < 0 ? 0.0 : static_cast<double>(e4m3_to_float(kI[(b * Lk + s) * d_I + c]));
+  }
+}
+
+// out[i] = codes[i] as float64 for n e4m3 codes.
+__global__ void decode_e4m3_kernel(const uint8_t* __restrict__ codes, double* __restrict__ out,
+                                   long long n) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    out[i] = static_cast<double>(e4m3_to_float(codes[i]));
+}
+
+// out[i] = (float)in[i].
+__global__ void f64_to_f32_kernel(const double* __restrict__ in, float* __restrict__ out,
+                                  long long n) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    out[i] = static_cast<float>(in[i]);
+}
+
+// dst[b][idx[tok][j]][:] += (float)src[tt][j][:] for float64 rows of D values
+// (D % 4 == 0), four at a time (atomic).
+__global__ void scatter_add_rows_f64_kernel(const double* __restrict__ src,
+                                            const int32_t* __restrict__ idx,
+                                            float4* __restrict__ dst, long long tok0, int T,
+                                            int Lq, int Lk, int k, int V) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * k;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / k;
+    const int j = static_cast<int>(r % k);
+    const int s = selected_key(idx, tok, j, k, Lk);
+    if (s < 0) continue;
+    const long long b = tok / Lq;
+    float4* d = dst + (b * Lk + s) * V;
+    const double* x = src + r * V * 4;
+    for (int v = lane; v < V; v += 32) {
+      const float4 f = make_float4(static_cast<float>(x[4 * v]), static_cast<float>(x[4 * v + 1]),
+                                   static_cast<float>(x[4 * v + 2]),
+                                   static_cast<float>(x[4 * v + 3]));
+      atomicAdd(d + v, f);
+    }
+  }
+}
+
+// ReLU gradient of one (token, indexer head j) row over its k slots. X holds the
+// dots qhat_j . khat_s of the codes (exact in float64); with the dequantised dot
+// x = s^q_j s^k_s X:
+//   dw_j    = sum_s dI_s max(x, 0)
+//   g_s     = dI_s w_j [X > 0]
+//   G1[j,s] = g_s s^k_s   (dq^I_j = sum_s G1[j,s] khat_s)
+//   G2[j,s] = g_s s^q_j   (dk^I_s = sum_j G2[j,s] qhat_j)
+__global__ void indexer_bwd_relu_kernel(const double* __restrict__ X,
+                                        const int32_t* __restrict__ idx,
+                                        const float* __restrict__ dI,
+                                        const float* __restrict__ qI_scale,
+                                        const float* __restrict__ kI_scale,
+                                        const void* __restrict__ w, int w_bf16,
+                                        double* __restrict__ G1, double* __restrict__ G2,
+                                        float* __restrict__ dw, long long tok0, int T, int Lq,
+                                        int Lk, int H_I, int k) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * H_I;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / H_I;
+    const int jh = static_cast<int>(r % H_I);
+    const long long b = tok / Lq;
+    const long long qrow = tok * H_I + jh;
+    const double sq = qI_scale[qrow];
+    const double wj = w_bf16 ? bf16_bits_to_float(static_cast<const uint16_t*>(w)[qrow])
+                             : static_cast<const float*>(w)[qrow];
+    const double* xrow = X + r * k;
+    double* g1 = G1 + r * k;
+    double* g2 = G2 + r * k;
+    double acc = 0.0;
+    for (int j = lane; j < k; j += 32) {
+      const int s = selected_key(idx, tok, j, k, Lk);
+      double a = 0.0, c = 0.0;
+      if (s >= 0) {
+        const double xh = xrow[j];
+        const double sk = kI_scale[b * Lk + s];
+        const double d = dI[tok * k + j];
+        acc += d * fmax(xh * sq * sk, 0.0);
+        const double g = xh > 0.0 ? d * wj : 0.0;
+        a = g * sk;
+        c = g * sq;
+      }
+      g1[j] = a;
+      g2[j] = c;
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) dw[qrow] = static_cast<float>(acc);
+  }
+}
+
+// dI = loss_scale (softmax(sel over the set) - p) per row of k slots; 0 outside
+// the set (and everywhere for a row with an empty set).
+__global__ void kl_score_grad_kernel(const float* __restrict__ sel, const float* __restrict__ p,
+                                     const int32_t* __restrict__ idx, float* __restrict__ dI,
+                                     long long rows, int k, int Lk, float loss_scale) {
+  const int lane = threadIdx.x & 31;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const float* srow = sel + r * k;
+    float m = -INFINITY;
+    for (int j = lane; j < k; j += 32)
+      if (selected_key(idx, r, j, k, Lk) >= 0) m = fmaxf(m, srow[j]);
+    m = warp_max(m);
+    float sum = 0.f;
+    if (m != -INFINITY)
+      for (int j = lane; j < k; j += 32)
+        if (selected_key(idx, r, j, k, Lk) >= 0) sum += expf(srow[j] - m);
+    sum = warp_sum(sum);
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    for (int j = lane; j < k; j += 32) {
+      float g = 0.f;
+      if (selected_key(idx, r, j, k, Lk) >= 0)
+        g = loss_scale * (expf(srow[j] - m) * inv - p[r * k + j]);
+      dI[r * k + j] = g;
+    }
+  }
+}
+
+// Blocks for a warp-per-row loop: enough to fill the GPU, never more than rows.
+int row_blocks(long long rows, int num_sms) {
+  const long long per_block = kRowThreads / 32;
+  long long want = (rows + per_block - 1) / per_block;
+  const long long cap = static_cast<long long>(num_sms > 0 ? num_sms : 148) * 16;
+  if (want > cap) want = cap;
+  return static_cast<int>(want < 1 ? 1 : want);
+}
+
+// Blocks for a flat element loop.
+int flat_blocks(long long n, int num_sms) {
+  long long blocks = (n + kRowThreads - 1) / kRowThreads;
+  const long long cap = static_cast<long long>(num_sms > 0 ? num_sms : 148) * 16;
+  if (blocks > cap) blocks = cap;
+  return static_cast<int>(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows_bf16(const uint16_t* kv, const int32_t* idx, uint16_t* out,
+                                    long long tok0, int T, int Lq, int Lk, int k, int D,
+                                    int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * k;
+  gather_rows_bf16_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(kv), idx, reinterpret_cast<uint4*>(out), tok0, T, Lq, Lk, k,
+      D / 8);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mla_bwd_softmax(const float* S, const float* dP, const uint16_t* out,
+                                   const uint16_t* dout, const float* lse, const int32_t* idx,
+                                   uint16_t* P16, uint16_t* dz16, long long tok0, int T, int H,
+                                   int Dv, int k, int Lk, float sm_scale, int num_sms,
+                                   cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * H;
+  mla_bwd_softmax_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      S, dP, out, dout, lse, idx, P16, dz16, tok0, T, H, Dv, k, Lk, sm_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float* dst,
+                                    long long tok0, int T, int Lq, int Lk, int k, int D,
+                                    int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * k;
+  scatter_add_rows_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      reinterpret_cast<const float4*>(src), idx, reinterpret_cast<float4*>(dst), tok0, T, Lq, Lk,
+      k, D / 4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_e4m3_rows(const uint8_t* kI, const int32_t* idx, double* out,
+                                    long long tok0, int T, int Lq, int Lk, int k, int d_I,
+                                    int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * k;
+  gather_e4m3_rows_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      kI, idx, out, tok0, T, Lq, Lk, k, d_I);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_e4m3(const uint8_t* codes, double* out, long long n, int num_sms,
+                               cudaStream_t stream) {
+  decode_e4m3_kernel<<<flat_blocks(n, num_sms), kRowThreads, 0, stream>>>(codes, out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f64_to_f32(const double* in, float* out, long long n, int num_sms,
+                              cudaStream_t stream) {
+  f64_to_f32_kernel<<<flat_blocks(n, num_sms), kRowThreads, 0, stream>>>(in, out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_add_rows_f64(const double* src, const int32_t* idx, float* dst,
+                                        long long tok0, int T, int Lq, int Lk, int k, int D,
+                                        int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * k;
+  scatter_add_rows_f64_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      src, idx, reinterpret_cast<float4*>(dst), tok0, T, Lq, Lk, k, D / 4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_indexer_bwd_relu(const double* X, const int32_t* idx, const float* dI,
+                                    const float* qI_scale, const float* kI_scale, const void* w,
+                                    int w_bf16, double* G1, double* G2, float* dw,
+                                    long long tok0, int T, int Lq, int Lk, int H_I, int k,
+                                    int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * H_I;
+  indexer_bwd_relu_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      X, idx, dI, qI_scale, kI_scale, w, w_bf16, G1, G2, dw, tok0, T, Lq, Lk, H_I, k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kl_score_grad(const float* sel, const float* p, const int32_t* idx, float* dI,
+                                 long long rows, int k, int Lk, float loss_scale, int num_sms,
+                                 cudaStream_t stream) {
+  kl_score_grad_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      sel, p, idx, dI, rows, k, Lk, loss_scale);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -3,6 +3,7 @@
 // forward path (indexer -> top-k -> sparse MLA; "DeepSeek-V3.2: Pushing the
 // Frontier of Open Large Language Models", bud-325 paper digest, "Key claims",
 // section 2.1 Eq. 1-2, and "Method").
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -983,6 +984,330 @@ int dsa_debug_wait_timeout(void* stream) {
   int sms = 0;
   DSA_TRY(device_ctl(ctl, sms));
   DSA_TRY_CUDA(dsa::launch_debug_wait(ctl, static_cast<cudaStream_t>(stream)), "debug launch");
+  return DSA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Sparse-stage gradients (bud-325 digest, "Method": the main model learns
+// through attention over the selected entries; the indexer through its own
+// detached inputs with the KL on the selected tokens).
+//
+// Per chunk of T tokens the selected rows are gathered into a dense [T, k, D]
+// block, the per-token contractions run as strided-batched GEMMs in cuBLAS
+// (bf16 operands with fp32 accumulation for the attention, fp64 for the
+// indexer), and the per-token key gradients are scatter-added into the shared
+// rows. The cuBLAS handle of each device is created on first use and keeps a
+// small device allocation of cuBLAS's own until the process exits; GEMM scratch
+// comes from the caller's workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kBlasWorkspace = size_t(32) << 20;   // cuBLAS scratch per call
+constexpr int kBwdChunkTokens = 64;                   // tokens per gathered block
+
+struct Blas {
+  std::mutex mu;
+  cublasHandle_t h = nullptr;
+};
+Blas g_blas[kMaxDevices];
+
+int blas_fail(cublasStatus_t st, const char* what) {
+  return fail(DSA_ERR_CUDA, "%s: cuBLAS status %d", what, static_cast<int>(st));
+}
+
+#define DSA_TRY_BLAS(expr, what)                                   \
+  do {                                                             \
+    cublasStatus_t b_ = (expr);                                    \
+    if (b_ != CUBLAS_STATUS_SUCCESS) return blas_fail(b_, what);   \
+  } while (0)
+
+int blas_for_device(Blas** out) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_CUDA, "device ordinal %d out of range", dev);
+  Blas& b = g_blas[dev];
+  std::lock_guard<std::mutex> lk(b.mu);
+  if (b.h == nullptr) DSA_TRY_BLAS(cublasCreate(&b.h), "cublasCreate");
+  *out = &b;
+  return DSA_OK;
+}
+
+// Row-major strided-batched GEMM: C[M x N] = op(A)[M x K] op(B)[K x N] + beta C.
+// A is stored row-major as [M x K] (tA false) or [K x M] (tA true) with leading
+// dimension lda, B as [K x N] or [N x K] with ldb. Operands of `type`: bf16 or
+// fp32 accumulate and write fp32; fp64 accumulates and writes fp64. cuBLAS is
+// column-major and a row-major X is the column-major X^T, so this is the
+// column-major product C^T = op(B)^T op(A)^T.
+int gemm_rm(cublasHandle_t h, bool tA, bool tB, int M, int N, int K, const void* A, int lda,
+            long long sA, const void* B, int ldb, long long sB, double beta, void* C, int ldc,
+            long long sC, int batch, cudaDataType_t type, const char* what) {
+  const cublasOperation_t opB = tB ? CUBLAS_OP_T : CUBLAS_OP_N;
+  const cublasOperation_t opA = tA ? CUBLAS_OP_T : CUBLAS_OP_N;
+  if (type == CUDA_R_64F) {
+    const double alpha = 1.0;
+    DSA_TRY_BLAS(cublasGemmStridedBatchedEx(h, opB, opA, N, M, K, &alpha, B, type, ldb, sB, A,
+                                            type, lda, sA, &beta, C, CUDA_R_64F, ldc, sC, batch,
+                                            CUBLAS_COMPUTE_64F, CUBLAS_GEMM_DEFAULT),
+                 what);
+  } else {
+    const float alpha = 1.f, beta32 = static_cast<float>(beta);
+    DSA_TRY_BLAS(cublasGemmStridedBatchedEx(h, opB, opA, N, M, K, &alpha, B, type, ldb, sB, A,
+                                            type, lda, sA, &beta32, C, CUDA_R_32F, ldc, sC, batch,
+                                            CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT),
+                 what);
+  }
+  return DSA_OK;
+}
+
+char* align256(void* p) {
+  return reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(p) + 255) & ~uintptr_t(255));
+}
+
+// Workspace of the attention backward for T tokens (offsets from a 256-byte
+// aligned base; total includes the alignment slack).
+struct MlaBwdLayout {
+  size_t cg, s, dp, p16, dz16, dc, blas, total;
+};
+MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
+  MlaBwdLayout L{};
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t tk = (size_t)T * k, thk = (size_t)T * H * k;
+  L.cg = take(tk * Dqk * sizeof(uint16_t));     // gathered latent rows, bf16
+  L.s = take(thk * sizeof(float));              // q . c
+  L.dp = take(thk * sizeof(float));             // dout . c[:Dv]
+  L.p16 = take(thk * sizeof(uint16_t));         // probabilities, bf16
+  L.dz16 = take(thk * sizeof(uint16_t));        // logit gradients, bf16
+  L.dc = take(tk * Dqk * sizeof(float));        // per-token row gradients
+  L.blas = take(kBlasWorkspace);
+  L.total = off + 256;
+  return L;
+}
+
+// The indexer backward works in fp64: the dots of the e4m3 codes are then exact
+// (each product needs at most 8 significant bits and every partial sum is a
+// multiple of 2^-18 below 2^25), so the ReLU mask is decided exactly.
+struct IdxBwdLayout {
+  size_t kd, qd, x, g1, g2, dk, dq, blas, total;
+};
+IdxBwdLayout idx_bwd_layout(int T, int H_I, int d_I, int k) {
+  IdxBwdLayout L{};
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t tk = (size_t)T * k, thk = (size_t)T * H_I * k, thd = (size_t)T * H_I * d_I;
+  L.kd = take(tk * d_I * sizeof(double));     // gathered key codes, decoded
+  L.qd = take(thd * sizeof(double));          // query codes, decoded
+  L.x = take(thk * sizeof(double));           // code dots
+  L.g1 = take(thk * sizeof(double));
+  L.g2 = take(thk * sizeof(double));
+  L.dk = take(tk * d_I * sizeof(double));     // per-token key gradients
+  L.dq = take(thd * sizeof(double));          // query gradients before the fp32 store
+  L.blas = take(kBlasWorkspace);
+  L.total = off + 256;
+  return L;
+}
+
+int bwd_chunk(long long tokens) {
+  return tokens < kBwdChunkTokens ? static_cast<int>(tokens) : kBwdChunkTokens;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_sparse_mla_bwd_workspace_size(int B, int Lq, int H, int Dqk, int Dv, int k) {
+  if (B < 1 || Lq < 1 || H < 1 || Dqk < 1 || Dv < 1 || k < 1) return 0;
+  return mla_bwd_layout(bwd_chunk((long long)B * Lq), H, Dqk, k).total;
+}
+
+int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                       const uint16_t* out, const float* lse, const uint16_t* dout, float* dq,
+                       float* dkv, int accumulate_dkv, int B, int Lq, int Lk, int H, int Dqk,
+                       int Dv, int k, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(check_ptr(q, "q"));
+  DSA_TRY(check_ptr(kv, "kv"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(out, "out"));
+  DSA_TRY(check_ptr(lse, "lse"));
+  DSA_TRY(check_ptr(dout, "dout"));
+  DSA_TRY(check_ptr(dq, "dq"));
+  DSA_TRY(check_ptr(dkv, "dkv"));
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1");
+  if ((long long)B * Lk > (1LL << 30)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lk must be <= 2^30");
+  DSA_TRY(check_mla_shape(H, Dqk, Dv, B, Lq));
+  DSA_TRY(check_k(k, 4096));
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
+    return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+  const long long n = (long long)B * Lq;
+  int T = bwd_chunk(n);
+  while (T > 1 && mla_bwd_layout(T, H, Dqk, k).total > ws_bytes) --T;
+  const MlaBwdLayout L = mla_bwd_layout(T, H, Dqk, k);
+  if (L.total > ws_bytes)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "sparse MLA backward workspace: need at least %zu bytes (recommended %zu), got %zu",
+                L.total, dsa_sparse_mla_bwd_workspace_size(B, Lq, H, Dqk, Dv, k), ws_bytes);
+  DSA_TRY(check_ptr(ws, "ws"));
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  Blas* bl = nullptr;
+  DSA_TRY(blas_for_device(&bl));
+  std::lock_guard<std::mutex> lk(bl->mu);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = align256(ws);
+  uint16_t* cg = reinterpret_cast<uint16_t*>(base + L.cg);
+  float* S = reinterpret_cast<float*>(base + L.s);
+  float* dP = reinterpret_cast<float*>(base + L.dp);
+  uint16_t* P16 = reinterpret_cast<uint16_t*>(base + L.p16);
+  uint16_t* dz16 = reinterpret_cast<uint16_t*>(base + L.dz16);
+  float* dC = reinterpret_cast<float*>(base + L.dc);
+  // setting the stream resets the workspace, so the workspace comes second
+  DSA_TRY_BLAS(cublasSetStream(bl->h, s), "cublasSetStream");
+  DSA_TRY_BLAS(cublasSetWorkspace(bl->h, base + L.blas, kBlasWorkspace), "cublasSetWorkspace");
+  int launched = 0;
+  if (!accumulate_dkv)
+    DSA_TRY_CUDA(cudaMemsetAsync(dkv, 0, (size_t)B * Lk * Dqk * sizeof(float), s), "dkv clear");
+  const long long qs = (long long)H * Dqk, os = (long long)H * Dv, hk = (long long)H * k,
+                  cs = (long long)k * Dqk;
+  for (long long tok0 = 0; tok0 < n; tok0 += T) {
+    const int Tc = (int)(n - tok0 < T ? n - tok0 : T);
+    const uint16_t* Qc = q + tok0 * qs;
+    const uint16_t* dOc = dout + tok0 * os;
+    DSA_TRY_CUDA(dsa::launch_gather_rows_bf16(kv, idx, cg, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
+                 "latent row gather launch");
+    // S[H x k] = Q[H x Dqk] C^T, dP[H x k] = dout[H x Dv] C[:, :Dv]^T
+    DSA_TRY(gemm_rm(bl->h, false, true, H, k, Dqk, Qc, Dqk, qs, cg, Dqk, cs, 0.f, S, k, hk, Tc,
+                    CUDA_R_16BF, "S = Q C^T"));
+    DSA_TRY(gemm_rm(bl->h, false, true, H, k, Dv, dOc, Dv, os, cg, Dqk, cs, 0.f, dP, k, hk, Tc,
+                    CUDA_R_16BF, "dP = dout V^T"));
+    DSA_TRY_CUDA(dsa::launch_mla_bwd_softmax(S, dP, out, dout, lse, idx, P16, dz16, tok0, Tc, H,
+                                             Dv, k, Lk, sm_scale, sms, s),
+                 "softmax gradient launch");
+    // dq[H x Dqk] = dz[H x k] C[k x Dqk]
+    DSA_TRY(gemm_rm(bl->h, false, false, H, Dqk, k, dz16, k, hk, cg, Dqk, cs, 0.f, dq + tok0 * qs,
+                    Dqk, qs, Tc, CUDA_R_16BF, "dq = dz C"));
+    // dC[k x Dqk] = dz^T Q, then dC[:, :Dv] += P^T dout
+    DSA_TRY(gemm_rm(bl->h, true, false, k, Dqk, H, dz16, k, hk, Qc, Dqk, qs, 0.f, dC, Dqk, cs, Tc,
+                    CUDA_R_16BF, "dC = dz^T Q"));
+    DSA_TRY(gemm_rm(bl->h, true, false, k, Dv, H, P16, k, hk, dOc, Dv, os, 1.f, dC, Dqk, cs, Tc,
+                    CUDA_R_16BF, "dC += P^T dout"));
+    DSA_TRY_CUDA(dsa::launch_scatter_add_rows(dC, idx, dkv, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
+                 "row gradient scatter launch");
+    launched += 3;
+  }
+  g_last_launches = launched;
+  return DSA_OK;
+}
+
+size_t dsa_indexer_bwd_workspace_size(int B, int Lq, int H_I, int d_I, int k) {
+  if (B < 1 || Lq < 1 || H_I < 1 || d_I < 1 || k < 1) return 0;
+  return idx_bwd_layout(bwd_chunk((long long)B * Lq), H_I, d_I, k).total;
+}
+
+int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
+                    const float* kI_scale, const void* w, int w_dtype, const int32_t* idx,
+                    const float* dI, float* dqI, float* dkI, float* dw, int accumulate_dkI, int B,
+                    int Lq, int Lk, int H_I, int d_I, int k, void* ws, size_t ws_bytes,
+                    void* stream) {
+  DSA_TRY(check_ptr(qI, "qI"));
+  DSA_TRY(check_ptr(qI_scale, "qI_scale"));
+  DSA_TRY(check_ptr(kI, "kI"));
+  DSA_TRY(check_ptr(kI_scale, "kI_scale"));
+  DSA_TRY(check_ptr(w, "w"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(dI, "dI"));
+  DSA_TRY(check_ptr(dqI, "dqI"));
+  DSA_TRY(check_ptr(dkI, "dkI"));
+  DSA_TRY(check_ptr(dw, "dw"));
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1");
+  if ((long long)B * Lk > (1LL << 30)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lk must be <= 2^30");
+  DSA_TRY(check_indexer_shape(H_I, d_I, B, Lq));
+  DSA_TRY(check_k(k, 4096));
+  if (w_dtype != DSA_DTYPE_F32 && w_dtype != DSA_DTYPE_BF16)
+    return fail(DSA_ERR_INVALID_ARG, "w_dtype must be DSA_DTYPE_F32 or DSA_DTYPE_BF16");
+  const long long n = (long long)B * Lq;
+  int T = bwd_chunk(n);
+  while (T > 1 && idx_bwd_layout(T, H_I, d_I, k).total > ws_bytes) --T;
+  const IdxBwdLayout L = idx_bwd_layout(T, H_I, d_I, k);
+  if (L.total > ws_bytes)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "indexer backward workspace: need at least %zu bytes (recommended %zu), got %zu",
+                L.total, dsa_indexer_bwd_workspace_size(B, Lq, H_I, d_I, k), ws_bytes);
+  DSA_TRY(check_ptr(ws, "ws"));
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  Blas* bl = nullptr;
+  DSA_TRY(blas_for_device(&bl));
+  std::lock_guard<std::mutex> lk(bl->mu);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = align256(ws);
+  double* Kd = reinterpret_cast<double*>(base + L.kd);
+  double* Qd = reinterpret_cast<double*>(base + L.qd);
+  double* X = reinterpret_cast<double*>(base + L.x);
+  double* G1 = reinterpret_cast<double*>(base + L.g1);
+  double* G2 = reinterpret_cast<double*>(base + L.g2);
+  double* dK = reinterpret_cast<double*>(base + L.dk);
+  double* dQ = reinterpret_cast<double*>(base + L.dq);
+  DSA_TRY_BLAS(cublasSetStream(bl->h, s), "cublasSetStream");
+  DSA_TRY_BLAS(cublasSetWorkspace(bl->h, base + L.blas, kBlasWorkspace), "cublasSetWorkspace");
+  int launched = 0;
+  if (!accumulate_dkI)
+    DSA_TRY_CUDA(cudaMemsetAsync(dkI, 0, (size_t)B * Lk * d_I * sizeof(float), s), "dkI clear");
+  const long long qs = (long long)H_I * d_I, hk = (long long)H_I * k, ks = (long long)k * d_I;
+  for (long long tok0 = 0; tok0 < n; tok0 += T) {
+    const int Tc = (int)(n - tok0 < T ? n - tok0 : T);
+    DSA_TRY_CUDA(dsa::launch_decode_e4m3(qI + tok0 * qs, Qd, (long long)Tc * qs, sms, s),
+                 "query decode launch");
+    DSA_TRY_CUDA(dsa::launch_gather_e4m3_rows(kI, idx, Kd, tok0, Tc, Lq, Lk, k, d_I, sms, s),
+                 "indexer key gather launch");
+    // X[H_I x k] = qhat[H_I x d_I] khat^T (exact)
+    DSA_TRY(gemm_rm(bl->h, false, true, H_I, k, d_I, Qd, d_I, qs, Kd, d_I, ks, 0.0, X, k, hk, Tc,
+                    CUDA_R_64F, "X = qhat khat^T"));
+    DSA_TRY_CUDA(dsa::launch_indexer_bwd_relu(X, idx, dI, qI_scale, kI_scale, w,
+                                              w_dtype == DSA_DTYPE_BF16 ? 1 : 0, G1, G2, dw, tok0,
+                                              Tc, Lq, Lk, H_I, k, sms, s),
+                 "ReLU gradient launch");
+    // dq^I[H_I x d_I] = G1[H_I x k] khat[k x d_I];  dK[k x d_I] = G2^T qhat
+    DSA_TRY(gemm_rm(bl->h, false, false, H_I, d_I, k, G1, k, hk, Kd, d_I, ks, 0.0, dQ, d_I, qs,
+                    Tc, CUDA_R_64F, "dqI = G1 khat"));
+    DSA_TRY_CUDA(dsa::launch_f64_to_f32(dQ, dqI + tok0 * qs, (long long)Tc * qs, sms, s),
+                 "query gradient store launch");
+    DSA_TRY(gemm_rm(bl->h, true, false, k, d_I, H_I, G2, k, hk, Qd, d_I, qs, 0.0, dK, d_I, ks, Tc,
+                    CUDA_R_64F, "dK = G2^T qhat"));
+    DSA_TRY_CUDA(dsa::launch_scatter_add_rows_f64(dK, idx, dkI, tok0, Tc, Lq, Lk, k, d_I, sms, s),
+                 "key gradient scatter launch");
+    launched += 5;
+  }
+  g_last_launches = launched;
+  return DSA_OK;
+}
+
+int dsa_indexer_kl_grad(const float* sel_scores, const float* p, const int32_t* idx, float* dI,
+                        int B, int Lq, int Lk, int k, float loss_scale, void* stream) {
+  DSA_TRY(check_ptr(sel_scores, "sel_scores"));
+  DSA_TRY(check_ptr(p, "p"));
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(dI, "dI"));
+  if (B < 1 || Lq < 1 || Lk < 1) return fail(DSA_ERR_INVALID_ARG, "B, Lq, Lk must be >= 1");
+  if ((long long)B * Lq > (1LL << 30)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B*Lq must be <= 2^30");
+  DSA_TRY(check_k(k, 4096));
+  if (!std::isfinite(loss_scale)) return fail(DSA_ERR_INVALID_ARG, "loss_scale must be finite");
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  DSA_TRY_CUDA(dsa::launch_kl_score_grad(sel_scores, p, idx, dI, (long long)B * Lq, k, Lk,
+                                         loss_scale, sms, static_cast<cudaStream_t>(stream)),
+               "KL score gradient launch");
+  g_last_launches = 1;
   return DSA_OK;
 }
 

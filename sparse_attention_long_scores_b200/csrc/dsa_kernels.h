@@ -96,6 +96,50 @@ struct KlArgs {
 // (H, Dqk) in {(8, 80), (128, 576)}.
 cudaError_t launch_indexer_kl(const uint16_t* kv, const KlArgs& a, cudaStream_t stream);
 
+// ---------------- sparse-stage gradients (backward.cu) ----------------
+// Chunk of T tokens starting at flattened token tok0 (sequence tok / Lq); slot j
+// of token tok is key idx[tok * k + j], skipped outside [0, Lk).
+// out [T, k, D] bf16 = the selected rows of kv [B, Lk, D] (zeros for skipped
+// slots); D % 8 == 0.
+cudaError_t launch_gather_rows_bf16(const uint16_t* kv, const int32_t* idx, uint16_t* out,
+                                    long long tok0, int T, int Lq, int Lk, int k, int D,
+                                    int num_sms, cudaStream_t stream);
+// P16 / dz16 [T, H, k] bf16 from S / dP [T, H, k] fp32 (raw q.c and dout.c[:Dv]),
+// out / dout [B*Lq, H, Dv] bf16 and lse [B*Lq, H].
+cudaError_t launch_mla_bwd_softmax(const float* S, const float* dP, const uint16_t* out,
+                                   const uint16_t* dout, const float* lse, const int32_t* idx,
+                                   uint16_t* P16, uint16_t* dz16, long long tok0, int T, int H,
+                                   int Dv, int k, int Lk, float sm_scale, int num_sms,
+                                   cudaStream_t stream);
+// dst [B, Lk, D] fp32 += src [T, k, D] fp32 row by row (atomic); D % 4 == 0.
+cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float* dst,
+                                    long long tok0, int T, int Lq, int Lk, int k, int D,
+                                    int num_sms, cudaStream_t stream);
+// out [T, k, d_I] fp64 = the selected e4m3 rows of kI [B, Lk, d_I], decoded.
+cudaError_t launch_gather_e4m3_rows(const uint8_t* kI, const int32_t* idx, double* out,
+                                    long long tok0, int T, int Lq, int Lk, int k, int d_I,
+                                    int num_sms, cudaStream_t stream);
+// out [n] fp64 = decoded e4m3 codes [n].
+cudaError_t launch_decode_e4m3(const uint8_t* codes, double* out, long long n, int num_sms,
+                               cudaStream_t stream);
+// out [n] fp32 = in [n] fp64.
+cudaError_t launch_f64_to_f32(const double* in, float* out, long long n, int num_sms,
+                              cudaStream_t stream);
+// dst [B, Lk, D] fp32 += src [T, k, D] fp64 row by row (atomic); D % 4 == 0.
+cudaError_t launch_scatter_add_rows_f64(const double* src, const int32_t* idx, float* dst,
+                                        long long tok0, int T, int Lq, int Lk, int k, int D,
+                                        int num_sms, cudaStream_t stream);
+// G1 / G2 [T, H_I, k] fp64 and dw [B*Lq, H_I] fp32 from the code dots X [T, H_I, k].
+cudaError_t launch_indexer_bwd_relu(const double* X, const int32_t* idx, const float* dI,
+                                    const float* qI_scale, const float* kI_scale, const void* w,
+                                    int w_bf16, double* G1, double* G2, float* dw,
+                                    long long tok0, int T, int Lq, int Lk, int H_I, int k,
+                                    int num_sms, cudaStream_t stream);
+// dI [rows, k] = loss_scale (softmax over the set of sel - p).
+cudaError_t launch_kl_score_grad(const float* sel, const float* p, const int32_t* idx, float* dI,
+                                 long long rows, int k, int Lk, float loss_scale, int num_sms,
+                                 cudaStream_t stream);
+
 // ---------------- debug ----------------
 cudaError_t launch_debug_wait(DevCtl ctl, cudaStream_t stream);
 

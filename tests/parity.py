@@ -111,3 +111,47 @@ def check_kl(gpu_kl, gpu_p, ref_kl, ref_p, sel, idx, where=""):
         bound = 1e-12
     assert abs(gk - ref_kl) <= bound, f"{where}: kl {gk} vs {ref_kl} (bound {bound})"
     return abs(gk - ref_kl)
+
+
+# ---------------------------------------------------------------------------
+# Sparse-stage gradients
+# ---------------------------------------------------------------------------
+# Attention backward: P and dz enter their GEMMs rounded to bf16 (relative error at
+# most 2^-9 each, independent from slot to slot) and D = dout . out uses the
+# forward's bf16 output. Each gradient is a sum over up to 2048 slots in which
+# these errors do not line up, so its relative error is of order 2^-9 ~ 2e-3.
+# Bound: 1e-2 per row (a row under a tenth of the RMS row norm is held to 1e-2 of
+# that tenth) and 5e-3 over the whole tensor.
+GRAD_ATT_ROW = 1e-2
+GRAD_ATT_ALL = 5e-3
+# Indexer backward: fp64 contractions on exact code dots; fp32 only in the stored
+# results and in the atomic sums of key gradients (2^-24 relative per addition, so
+# about 2^-24 sqrt(n / 2) after n additions of random sign: 1e-6 at 2000 tokens).
+GRAD_IDX_ROW = 1e-5
+GRAD_IDX_ALL = 1e-5
+# KL score gradient r - p: fp32 softmax of at most 4096 scores.
+KL_GRAD_RTOL = 1e-4
+KL_GRAD_ATOL = 1e-6
+
+
+def check_grad(gpu, ref, row_tol, all_tol, where, floor=0.1):
+    """Row-wise relative L2 error of a gradient (rows = the last axis), with rows
+    under floor * the RMS row norm held to row_tol of that floor, plus the relative
+    Frobenius error of the whole tensor. Returns the worst row ratio."""
+    g = np.asarray(gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    g = g.reshape(-1, g.shape[-1])
+    r = r.reshape(-1, r.shape[-1])
+    assert g.shape == r.shape, where
+    rn = np.linalg.norm(r, axis=1)
+    en = np.linalg.norm(g - r, axis=1)
+    rms = float(np.sqrt(np.mean(rn ** 2)))
+    assert rms > 0, f"{where}: reference gradient is zero"
+    den = np.maximum(rn, floor * rms)
+    ratio = en / den
+    bad = np.flatnonzero(ratio > row_tol)
+    assert bad.size == 0, (f"{where}: {bad.size} of {rn.size} rows off, worst relative error "
+                           f"{ratio.max():.3g} at row {int(np.argmax(ratio))}")
+    tot = float(np.linalg.norm(g - r) / np.linalg.norm(r))
+    assert tot <= all_tol, f"{where}: relative Frobenius error {tot:.3g}"
+    return float(ratio.max())

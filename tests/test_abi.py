@@ -101,6 +101,60 @@ def test_indexer_kl_rejects_bad_args(L):
     assert rc == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_backward_entry_points_reject_bad_args(L):
+    """The sparse-stage gradient calls validate everything before any device work."""
+    p = ctypes.c_void_p(FAKE)
+    odd = ctypes.c_void_p(FAKE + 8)
+    big = 1 << 40
+
+    def mla(**kw):
+        a = dict(q=p, kv=p, idx=p, out=p, lse=p, dout=p, dq=p, dkv=p, acc=0, B=1, Lq=4, Lk=8, H=8,
+                 Dqk=80, Dv=64, k=32, scale=0.1, ws=p, ws_bytes=big)
+        a.update(kw)
+        return L.dsa_sparse_mla_bwd(*a.values(), None)
+
+    for kw, code, text in ((dict(lse=None), dsa.DSA_ERR_INVALID_ARG, "lse"),
+                           (dict(dq=odd), dsa.DSA_ERR_INVALID_ARG, "aligned"),
+                           (dict(H=16), dsa.DSA_ERR_UNSUPPORTED_SHAPE, ""),
+                           (dict(k=40), dsa.DSA_ERR_UNSUPPORTED_SHAPE, ""),
+                           (dict(scale=0.0), dsa.DSA_ERR_INVALID_ARG, "sm_scale"),
+                           (dict(Lq=0), dsa.DSA_ERR_INVALID_ARG, ""),
+                           (dict(ws_bytes=4096), dsa.DSA_ERR_WORKSPACE_TOO_SMALL, "workspace")):
+        rc = mla(**kw)
+        assert rc == code and text in L.dsa_last_error().decode(), (kw, L.dsa_last_error())
+
+    def idx_bwd(**kw):
+        a = dict(qI=p, qs=p, kI=p, ks=p, w=p, wd=dsa.DSA_DTYPE_BF16, idx=p, dI=p, dqI=p, dkI=p, dw=p,
+                 acc=0, B=1, Lq=4, Lk=8, H_I=4, d_I=32, k=32, ws=p, ws_bytes=big)
+        a.update(kw)
+        return L.dsa_indexer_bwd(*a.values(), None)
+
+    for kw, code, text in ((dict(dw=None), dsa.DSA_ERR_INVALID_ARG, "dw"),
+                           (dict(H_I=8), dsa.DSA_ERR_UNSUPPORTED_SHAPE, ""),
+                           (dict(wd=7), dsa.DSA_ERR_INVALID_ARG, "w_dtype"),
+                           (dict(k=0), dsa.DSA_ERR_UNSUPPORTED_SHAPE, ""),
+                           (dict(ws_bytes=4096), dsa.DSA_ERR_WORKSPACE_TOO_SMALL, "workspace")):
+        rc = idx_bwd(**kw)
+        assert rc == code and text in L.dsa_last_error().decode(), (kw, L.dsa_last_error())
+
+    assert L.dsa_indexer_kl_grad(p, None, p, p, 1, 4, 8, 32, 1.0, None) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_indexer_kl_grad(p, p, p, p, 1, 4, 8, 33, 1.0, None) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert L.dsa_indexer_kl_grad(p, p, p, p, 1, 4, 8, 32, math.nan, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_backward_workspace_sizes(L):
+    """Chunks of at most 64 tokens: the recommended workspace grows with the token
+    count up to 64 and then stays flat; about 10 MB per token at the full shapes."""
+    f = L.dsa_sparse_mla_bwd_workspace_size
+    sizes = [f(1, n, 128, 576, 512, 2048) for n in (1, 2, 64, 65, 65536)]
+    assert sizes[0] < sizes[1] < sizes[2] == sizes[3] == sizes[4]
+    per_token = (sizes[2] - sizes[0]) / 63
+    assert 9e6 < per_token < 11e6, per_token
+    g = L.dsa_indexer_bwd_workspace_size
+    assert 0 < g(1, 1, 64, 128, 2048) < g(2, 32768, 64, 128, 2048) == g(1, 64, 64, 128, 2048)
+    assert f(0, 1, 8, 80, 64, 32) == 0 and g(1, 0, 4, 32, 32) == 0
+
+
 def test_forward_paged_rejects_bad_cache(L):
     from dsa_inputs import CONFIGS
     p = dsa.Problem.from_config(CONFIGS["tiny"].with_(Lq=1, Lk=512, q_pos0=511))
