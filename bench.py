@@ -391,7 +391,7 @@ def time_backward(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     launches = {}
 
     def attention():
-        dsa.sparse_mla_bwd(inp["q"], inp["kv"], idx, out, lse, dout, cfg.sm_scale, dq=dq, dkv=dkv,
+        dsa.sparse_mla_bwd(inp["q"], inp["kv"], idx, lse, dout, cfg.sm_scale, dq=dq, dkv=dkv,
                            ws=ws)
         launches["attention"] = dsa.last_launch_count()
 

@@ -198,15 +198,17 @@ int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, co
  *
  * dsa_sparse_mla_bwd - gradients of the sparse attention (dsa_sparse_mla_fwd)
  * with respect to q and the latent rows, given dout = dL/d(out). With
- * z[h,s] = sm_scale q[h].c_s over the valid slots s of idx[t,:] and
- * P = exp(z - lse):
- *     D[h]    = dout[h] . out[h]
- *     dz[h,s] = sm_scale P[h,s] (dout[h] . c_s[:Dv] - D[h])
+ * z[h,s] = sm_scale q[h].c_s over the valid slots s of idx[t,:], P = exp(z - lse)
+ * and dP[h,s] = dout[h] . c_s[:Dv]:
+ *     D[h]    = sum_s P[h,s] dP[h,s] / sum_s P[h,s]    (= dout[h] . out[h])
+ *     dz[h,s] = sm_scale P[h,s] (dP[h,s] - D[h])
  *     dq[h]   = sum_s dz[h,s] c_s                      (all Dqk columns)
  *     dkv[s] += sum_h dz[h,s] q[h]   and, on columns < Dv, sum_h P[h,s] dout[h]
- *   q [B, Lq, H, Dqk], kv [B, Lk, Dqk], out and dout [B, Lq, H, Dv]: bf16;
- *   idx [B, Lq, k] int32 (slots < 0 or >= Lk skipped); lse [B, Lq, H] fp32 as
- *   the forward returned it; dq [B, Lq, H, Dqk] fp32 (overwritten);
+ *   D is formed from the recomputed fp32 P and dP rather than from the forward's
+ *   bf16 output, so a set of one key gets dq = 0 exactly.
+ *   q [B, Lq, H, Dqk], kv [B, Lk, Dqk], dout [B, Lq, H, Dv]: bf16; idx [B, Lq, k]
+ *   int32 (slots < 0 or >= Lk skipped); lse [B, Lq, H] fp32 as the forward
+ *   returned it; dq [B, Lq, H, Dqk] fp32 (overwritten);
  *   dkv [B, Lk, Dqk] fp32, zeroed first unless accumulate_dkv != 0.
  *   (H, Dqk, Dv) in {(8, 80, 64), (128, 576, 512)}; k a multiple of 32 in
  *   [32, 4096]. P and dz enter their GEMMs rounded to bf16.
@@ -215,9 +217,9 @@ int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, co
  */
 size_t dsa_sparse_mla_bwd_workspace_size(int B, int Lq, int H, int Dqk, int Dv, int k);
 int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
-                       const uint16_t* out, const float* lse, const uint16_t* dout, float* dq,
-                       float* dkv, int accumulate_dkv, int B, int Lq, int Lk, int H, int Dqk,
-                       int Dv, int k, float sm_scale, void* ws, size_t ws_bytes, void* stream);
+                       const float* lse, const uint16_t* dout, float* dq, float* dkv,
+                       int accumulate_dkv, int B, int Lq, int Lk, int H, int Dqk, int Dv, int k,
+                       float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * dsa_indexer_kl_grad - dI = loss_scale * (r - p): the gradient of

@@ -110,7 +110,7 @@ def lib() -> ctypes.CDLL:
                                        ctypes.POINTER(ctypes.c_int), i, ctypes.POINTER(ctypes.c_int)]
     L.dsa_sparse_mla_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
     L.dsa_sparse_mla_bwd_workspace_size.restype = sz
-    L.dsa_sparse_mla_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+    L.dsa_sparse_mla_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
                                      ctypes.c_float, vp, sz, vp]
     L.dsa_indexer_kl_grad.argtypes = [vp, vp, vp, vp, i, i, i, i, ctypes.c_float, vp]
     L.dsa_indexer_bwd_workspace_size.argtypes = [i, i, i, i, i]
@@ -260,11 +260,11 @@ def _workspace(nbytes: int, device):
     return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
 
 
-def sparse_mla_bwd(q, kv, idx, out, lse, dout, sm_scale: float, dq=None, dkv=None,
+def sparse_mla_bwd(q, kv, idx, lse, dout, sm_scale: float, dq=None, dkv=None,
                    accumulate_dkv: bool = False, ws=None, stream=None):
     """Sparse-stage attention gradients: dq [B, Lq, H, Dqk] fp32 and dkv [B, Lk, Dqk]
-    fp32 from dout = dL/d(out) [B, Lq, H, Dv] bf16, given the forward's idx, out and
-    lse. dkv is overwritten unless accumulate_dkv. Returns (dq, dkv)."""
+    fp32 from dout = dL/d(out) [B, Lq, H, Dv] bf16, given the forward's idx and lse.
+    dkv is overwritten unless accumulate_dkv. Returns (dq, dkv)."""
     B, Lq, H, Dqk = q.shape
     Lk = kv.shape[1]
     k = idx.shape[2]
@@ -272,7 +272,6 @@ def sparse_mla_bwd(q, kv, idx, out, lse, dout, sm_scale: float, dq=None, dkv=Non
     _need(q, "q", torch.bfloat16)
     _need(kv, "kv", torch.bfloat16, (B, Lk, Dqk))
     _need(idx, "idx", torch.int32, (B, Lq, k))
-    _need(out, "out", torch.bfloat16, (B, Lq, H, Dv))
     _need(lse, "lse", torch.float32, (B, Lq, H))
     _need(dout, "dout", torch.bfloat16, (B, Lq, H, Dv))
     if dq is None:
@@ -283,7 +282,7 @@ def sparse_mla_bwd(q, kv, idx, out, lse, dout, sm_scale: float, dq=None, dkv=Non
     _need(dkv, "dkv", torch.float32, (B, Lk, Dqk))
     if ws is None:
         ws = _workspace(lib().dsa_sparse_mla_bwd_workspace_size(B, Lq, H, Dqk, Dv, k), q.device)
-    _check(lib().dsa_sparse_mla_bwd(_ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(lse),
+    _check(lib().dsa_sparse_mla_bwd(_ptr(q), _ptr(kv), _ptr(idx), _ptr(lse),
                                     _ptr(dout), _ptr(dq), _ptr(dkv), int(bool(accumulate_dkv)),
                                     B, Lq, Lk, H, Dqk, Dv, k, float(sm_scale), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(stream)))

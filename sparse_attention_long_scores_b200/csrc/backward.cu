@@ -84,30 +84,39 @@ __global__ void gather_rows_bf16_kernel(const uint4* __restrict__ kv,
   }
 }
 
-// Softmax gradient of one (token, head) row over its k slots:
-//   D = dout . out,  P_s = exp(sm_scale S_s - lse),  dz_s = sm_scale P_s (dP_s - D)
-// with S and dP the raw q.c_s and dout.c_s[:Dv] of the batched GEMMs. P and dz are
-// written as bf16 for the GEMMs that follow; slots without a valid key get 0.
+// Softmax gradient of one (token, head) row over its k slots, with S and dP the
+// raw q.c_s and dout.c_s[:Dv] of the batched GEMMs:
+//   P_s  = exp(sm_scale S_s - lse)
+//   D    = sum_s P_s dP_s / sum_s P_s       (= dout . out; from the fp32 P and dP,
+//                                             so that sum_s dz_s = 0 and a single
+//                                             key gives dz = 0 exactly)
+//   dz_s = sm_scale P_s (dP_s - D)
+// P and dz are written as bf16 for the GEMMs that follow; slots without a valid key
+// get 0.
 __global__ void mla_bwd_softmax_kernel(const float* __restrict__ S, const float* __restrict__ dP,
-                                       const uint16_t* __restrict__ out,
-                                       const uint16_t* __restrict__ dout,
                                        const float* __restrict__ lse,
                                        const int32_t* __restrict__ idx, uint16_t* __restrict__ P16,
                                        uint16_t* __restrict__ dz16, long long tok0, int T, int H,
-                                       int Dv, int k, int Lk, float sm_scale) {
+                                       int k, int Lk, float sm_scale) {
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(T) * H;
   for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
     const long long tok = tok0 + r / H;
     const int h = static_cast<int>(r % H);
-    const long long oh = (tok * H + h) * Dv;
-    float d = 0.f;
-    for (int v = lane; v < Dv; v += 32)
-      d += bf16_bits_to_float(dout[oh + v]) * bf16_bits_to_float(out[oh + v]);
-    d = warp_sum(d);
     const float l = lse[tok * H + h];
     const float* srow = S + r * k;
     const float* prow = dP + r * k;
+    float sp = 0.f, spd = 0.f;
+    for (int j = lane; j < k; j += 32) {
+      if (selected_key(idx, tok, j, k, Lk) >= 0) {
+        const float p = expf(srow[j] * sm_scale - l);
+        sp += p;
+        spd += p * prow[j];
+      }
+    }
+    sp = warp_sum(sp);
+    spd = warp_sum(spd);
+    const float d = sp > 0.f ? spd / sp : 0.f;
     uint16_t* p_out = P16 + r * k;
     uint16_t* z_out = dz16 + r * k;
     for (int j = lane; j < k; j += 32) {
@@ -306,14 +315,13 @@ cudaError_t launch_gather_rows_bf16(const uint16_t* kv, const int32_t* idx, uint
   return cudaGetLastError();
 }
 
-cudaError_t launch_mla_bwd_softmax(const float* S, const float* dP, const uint16_t* out,
-                                   const uint16_t* dout, const float* lse, const int32_t* idx,
-                                   uint16_t* P16, uint16_t* dz16, long long tok0, int T, int H,
-                                   int Dv, int k, int Lk, float sm_scale, int num_sms,
-                                   cudaStream_t stream) {
+cudaError_t launch_mla_bwd_softmax(const float* S, const float* dP, const float* lse,
+                                   const int32_t* idx, uint16_t* P16, uint16_t* dz16,
+                                   long long tok0, int T, int H, int k, int Lk, float sm_scale,
+                                   int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(T) * H;
   mla_bwd_softmax_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
-      S, dP, out, dout, lse, idx, P16, dz16, tok0, T, H, Dv, k, Lk, sm_scale);
+      S, dP, lse, idx, P16, dz16, tok0, T, H, k, Lk, sm_scale);
   return cudaGetLastError();
 }
 

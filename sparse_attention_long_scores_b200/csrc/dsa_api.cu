@@ -1131,13 +1131,12 @@ size_t dsa_sparse_mla_bwd_workspace_size(int B, int Lq, int H, int Dqk, int Dv, 
 }
 
 int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
-                       const uint16_t* out, const float* lse, const uint16_t* dout, float* dq,
-                       float* dkv, int accumulate_dkv, int B, int Lq, int Lk, int H, int Dqk,
-                       int Dv, int k, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+                       const float* lse, const uint16_t* dout, float* dq, float* dkv,
+                       int accumulate_dkv, int B, int Lq, int Lk, int H, int Dqk, int Dv, int k,
+                       float sm_scale, void* ws, size_t ws_bytes, void* stream) {
   DSA_TRY(check_ptr(q, "q"));
   DSA_TRY(check_ptr(kv, "kv"));
   DSA_TRY(check_ptr(idx, "idx"));
-  DSA_TRY(check_ptr(out, "out"));
   DSA_TRY(check_ptr(lse, "lse"));
   DSA_TRY(check_ptr(dout, "dout"));
   DSA_TRY(check_ptr(dq, "dq"));
@@ -1189,8 +1188,8 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
                     CUDA_R_16BF, "S = Q C^T"));
     DSA_TRY(gemm_rm(bl->h, false, true, H, k, Dv, dOc, Dv, os, cg, Dqk, cs, 0.f, dP, k, hk, Tc,
                     CUDA_R_16BF, "dP = dout V^T"));
-    DSA_TRY_CUDA(dsa::launch_mla_bwd_softmax(S, dP, out, dout, lse, idx, P16, dz16, tok0, Tc, H,
-                                             Dv, k, Lk, sm_scale, sms, s),
+    DSA_TRY_CUDA(dsa::launch_mla_bwd_softmax(S, dP, lse, idx, P16, dz16, tok0, Tc, H, k, Lk,
+                                             sm_scale, sms, s),
                  "softmax gradient launch");
     // dq[H x Dqk] = dz[H x k] C[k x Dqk]
     DSA_TRY(gemm_rm(bl->h, false, false, H, Dqk, k, dz16, k, hk, cg, Dqk, cs, 0.f, dq + tok0 * qs,

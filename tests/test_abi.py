@@ -108,7 +108,7 @@ def test_backward_entry_points_reject_bad_args(L):
     big = 1 << 40
 
     def mla(**kw):
-        a = dict(q=p, kv=p, idx=p, out=p, lse=p, dout=p, dq=p, dkv=p, acc=0, B=1, Lq=4, Lk=8, H=8,
+        a = dict(q=p, kv=p, idx=p, lse=p, dout=p, dq=p, dkv=p, acc=0, B=1, Lq=4, Lk=8, H=8,
                  Dqk=80, Dv=64, k=32, scale=0.1, ws=p, ws_bytes=big)
         a.update(kw)
         return L.dsa_sparse_mla_bwd(*a.values(), None)

@@ -9,9 +9,9 @@ input detached (``dsa_indexer_kl_grad`` then ``dsa_indexer_bwd``).
 Inputs are seeded: queries, latent rows and indexer tensors from the workload
 generator, key sets from ``dsa_inputs.random_key_sets`` (or the CUDA forward's own
 selection at full size), output gradients from ``dsa_inputs.output_gradient`` and
-index-score gradients from ``dsa_inputs.random_scores``. The forward's out and lse,
-which the attention backward consumes, come from the CUDA forward; the oracle
-recomputes everything from the definitions.
+index-score gradients from ``dsa_inputs.random_scores``. The forward's lse, which
+the attention backward consumes, comes from the CUDA forward; the oracle recomputes
+everything from the definitions.
 """
 import numpy as np
 import pytest
@@ -40,12 +40,12 @@ def _u16(t):
 
 
 def _attention_grads(cfg, inp, idx, dout, accumulate_twice=False):
-    """CUDA path: forward over idx (out, lse), then the backward."""
+    """CUDA path: forward over idx (for lse), then the backward."""
     q, kv, idxd, doutd = inp["q"].cuda(), inp["kv"].cuda(), idx.cuda(), dout.cuda()
-    out, lse = dsa.sparse_mla_fwd(q, kv, idxd, cfg.sm_scale, cfg.Dv)
-    dq, dkv = dsa.sparse_mla_bwd(q, kv, idxd, out, lse, doutd, cfg.sm_scale)
+    _, lse = dsa.sparse_mla_fwd(q, kv, idxd, cfg.sm_scale, cfg.Dv)
+    dq, dkv = dsa.sparse_mla_bwd(q, kv, idxd, lse, doutd, cfg.sm_scale)
     if accumulate_twice:
-        dq2, dkv2 = dsa.sparse_mla_bwd(q, kv, idxd, out, lse, doutd, cfg.sm_scale, dkv=dkv.clone(),
+        dq2, dkv2 = dsa.sparse_mla_bwd(q, kv, idxd, lse, doutd, cfg.sm_scale, dkv=dkv.clone(),
                                        accumulate_dkv=True)
     torch.cuda.synchronize()
     dsa.check_status()
@@ -148,7 +148,7 @@ def test_mla_backward_prefill_32k_sampled_rows():
     idx = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.int32, device="cuda")
     dsa.forward(p, inp, out=out, lse=lse, idx_out=idx)
     dout = output_gradient((cfg.B, cfg.Lq, cfg.H, cfg.Dv), seed=74, device="cuda")
-    dq, dkv = dsa.sparse_mla_bwd(inp["q"], inp["kv"], idx, out, lse, dout, cfg.sm_scale)
+    dq, dkv = dsa.sparse_mla_bwd(inp["q"], inp["kv"], idx, lse, dout, cfg.sm_scale)
     torch.cuda.synchronize()
     dsa.check_status()
     rope = dkv[:, :, cfg.Dv:].double()
