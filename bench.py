@@ -533,12 +533,15 @@ PROFILE_CASES = {
     "decode_small": ("decode_128k", dict(B=16)),
     # the indexer KL target over the forward's top-k sets of the prefill chunk above
     "kl_chunk": ("prefill_8k", dict(Lq=2048, q_pos0=6144)),
+    # the sparse-stage gradients of the last 256 rows of the 8K workload (4 chunks of
+    # 64 tokens): attention backward, KL score gradient, indexer backward
+    "bwd_chunk": ("prefill_8k", dict(Lq=256, q_pos0=7936)),
 }
 
 
 def profile_case(name: str) -> None:
-    """Two untimed forwards of a small case, for an ncu capture of its kernels
-    (the second forward's launches are the ones to capture)."""
+    """Two untimed passes of a small case, for an ncu capture of its kernels (the
+    second pass's launches are the ones to capture)."""
     import sparse_attention_long_scores_b200 as dsa
     from sparse_attention_long_scores_b200.build import build
 
@@ -556,6 +559,19 @@ def profile_case(name: str) -> None:
         sel = random_scores((cfg.B, cfg.Lq, cfg.k), seed=77).cuda()
         for _ in range(2):
             dsa.indexer_kl(inp["q"], inp["kv"], idx, lse, sel, cfg.sm_scale)
+    elif name == "bwd_chunk":
+        from dsa_inputs import output_gradient, random_scores
+        lse = torch.empty((cfg.B, cfg.Lq, cfg.H), dtype=torch.float32, device="cuda")
+        idx = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.int32, device="cuda")
+        dsa.forward(p, inp, lse=lse, idx_out=idx)
+        dout = output_gradient((cfg.B, cfg.Lq, cfg.H, cfg.Dv), seed=5, device="cuda")
+        sel = random_scores((cfg.B, cfg.Lq, cfg.k), seed=77).cuda()
+        _, pt = dsa.indexer_kl(inp["q"], inp["kv"], idx, lse, sel, cfg.sm_scale)
+        for _ in range(2):
+            dsa.sparse_mla_bwd(inp["q"], inp["kv"], idx, lse, dout, cfg.sm_scale)
+            dI = dsa.indexer_kl_grad(sel, pt, idx, cfg.Lk)
+            dsa.indexer_bwd(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"], idx,
+                            dI)
     else:
         for _ in range(2):
             dsa.forward(p, inp)
