@@ -84,28 +84,53 @@ __global__ void gather_rows_bf16_kernel(const uint4* __restrict__ kv,
   }
 }
 
+// QO[tt] = [q[tok] (H rows); dout[tok] padded with zeros to Dqk columns (H rows)],
+// bf16 rows of V 16-byte vectors (Vd of them hold dout).
+__global__ void pack_qo_kernel(const uint4* __restrict__ q, const uint4* __restrict__ dout,
+                               uint4* __restrict__ qo, long long tok0, int T, int H, int V,
+                               int Vd) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(T) * 2 * H;
+  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
+    const long long tok = tok0 + r / (2 * H);
+    const int hh = static_cast<int>(r % (2 * H));
+    uint4* dst = qo + r * V;
+    if (hh < H) {
+      const uint4* src = q + (tok * H + hh) * V;
+      for (int v = lane; v < V; v += 32) dst[v] = src[v];
+    } else {
+      const uint4* src = dout + (tok * H + (hh - H)) * Vd;
+      for (int v = lane; v < V; v += 32) dst[v] = v < Vd ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 // Softmax gradient of one (token, head) row over its k slots, with S and dP the
-// raw q.c_s and dout.c_s[:Dv] of the batched GEMMs:
+// raw q.c_s and dout.c_s[:Dv] of the batched GEMM (per token, SP holds the H rows
+// of S and then the H rows of dP):
 //   P_s  = exp(sm_scale S_s - lse)
 //   D    = sum_s P_s dP_s / sum_s P_s       (= dout . out; from the fp32 P and dP,
 //                                             so that sum_s dz_s = 0 and a single
 //                                             key gives dz = 0 exactly)
 //   dz_s = sm_scale P_s (dP_s - D)
-// P and dz are written as bf16 for the GEMMs that follow; slots without a valid key
-// get 0.
-__global__ void mla_bwd_softmax_kernel(const float* __restrict__ S, const float* __restrict__ dP,
+// dz and P are written as bf16 for the GEMMs that follow, per token the H rows of dz
+// and then the H rows of P (PZ); slots without a valid key get 0.
+__global__ void mla_bwd_softmax_kernel(const float* __restrict__ SP,
                                        const float* __restrict__ lse,
-                                       const int32_t* __restrict__ idx, uint16_t* __restrict__ P16,
-                                       uint16_t* __restrict__ dz16, long long tok0, int T, int H,
-                                       int k, int Lk, float sm_scale) {
+                                       const int32_t* __restrict__ idx, uint16_t* __restrict__ PZ,
+                                       long long tok0, int T, int H, int k, int Lk,
+                                       float sm_scale) {
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(T) * H;
   for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
-    const long long tok = tok0 + r / H;
+    const long long tt = r / H;
+    const long long tok = tok0 + tt;
     const int h = static_cast<int>(r % H);
     const float l = lse[tok * H + h];
-    const float* srow = S + r * k;
-    const float* prow = dP + r * k;
+    const long long zrow = (tt * 2 * H + h) * k;        // row h of the token's block
+    const long long prow_off = zrow + static_cast<long long>(H) * k;   // row H + h
+    const float* srow = SP + zrow;
+    const float* prow = SP + prow_off;
     float sp = 0.f, spd = 0.f;
     for (int j = lane; j < k; j += 32) {
       if (selected_key(idx, tok, j, k, Lk) >= 0) {
@@ -117,8 +142,8 @@ __global__ void mla_bwd_softmax_kernel(const float* __restrict__ S, const float*
     sp = warp_sum(sp);
     spd = warp_sum(spd);
     const float d = sp > 0.f ? spd / sp : 0.f;
-    uint16_t* p_out = P16 + r * k;
-    uint16_t* z_out = dz16 + r * k;
+    uint16_t* z_out = PZ + zrow;
+    uint16_t* p_out = PZ + prow_off;
     for (int j = lane; j < k; j += 32) {
       float p = 0.f, z = 0.f;
       if (selected_key(idx, tok, j, k, Lk) >= 0) {
@@ -315,13 +340,21 @@ cudaError_t launch_gather_rows_bf16(const uint16_t* kv, const int32_t* idx, uint
   return cudaGetLastError();
 }
 
-cudaError_t launch_mla_bwd_softmax(const float* S, const float* dP, const float* lse,
-                                   const int32_t* idx, uint16_t* P16, uint16_t* dz16,
-                                   long long tok0, int T, int H, int k, int Lk, float sm_scale,
-                                   int num_sms, cudaStream_t stream) {
+cudaError_t launch_pack_qo(const uint16_t* q, const uint16_t* dout, uint16_t* qo, long long tok0,
+                           int T, int H, int Dqk, int Dv, int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(T) * 2 * H;
+  pack_qo_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(dout),
+      reinterpret_cast<uint4*>(qo), tok0, T, H, Dqk / 8, Dv / 8);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mla_bwd_softmax(const float* SP, const float* lse, const int32_t* idx,
+                                   uint16_t* PZ, long long tok0, int T, int H, int k, int Lk,
+                                   float sm_scale, int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(T) * H;
   mla_bwd_softmax_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
-      S, dP, lse, idx, P16, dz16, tok0, T, H, k, Lk, sm_scale);
+      SP, lse, idx, PZ, tok0, T, H, k, Lk, sm_scale);
   return cudaGetLastError();
 }
 

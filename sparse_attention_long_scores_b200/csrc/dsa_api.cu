@@ -1068,7 +1068,7 @@ char* align256(void* p) {
 // Workspace of the attention backward for T tokens (offsets from a 256-byte
 // aligned base; total includes the alignment slack).
 struct MlaBwdLayout {
-  size_t cg, s, dp, p16, dz16, dc, blas, total;
+  size_t cg, qo, sp, pz, dc, blas, total;
 };
 MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
   MlaBwdLayout L{};
@@ -1078,13 +1078,12 @@ MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
     off += align_up(bytes, 256);
     return o;
   };
-  const size_t tk = (size_t)T * k, thk = (size_t)T * H * k;
-  L.cg = take(tk * Dqk * sizeof(uint16_t));     // gathered latent rows, bf16
-  L.s = take(thk * sizeof(float));              // q . c
-  L.dp = take(thk * sizeof(float));             // dout . c[:Dv]
-  L.p16 = take(thk * sizeof(uint16_t));         // probabilities, bf16
-  L.dz16 = take(thk * sizeof(uint16_t));        // logit gradients, bf16
-  L.dc = take(tk * Dqk * sizeof(float));        // per-token row gradients
+  const size_t tk = (size_t)T * k, t2hk = (size_t)T * 2 * H * k;
+  L.cg = take(tk * Dqk * sizeof(uint16_t));              // gathered latent rows, bf16
+  L.qo = take((size_t)T * 2 * H * Dqk * sizeof(uint16_t));  // [q; dout padded], bf16
+  L.sp = take(t2hk * sizeof(float));                     // [q . c; dout . c[:Dv]]
+  L.pz = take(t2hk * sizeof(uint16_t));                  // [dz; P], bf16
+  L.dc = take(tk * Dqk * sizeof(float));                 // per-token row gradients
   L.blas = take(kBlasWorkspace);
   L.total = off + 256;
   return L;
@@ -1164,10 +1163,9 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = align256(ws);
   uint16_t* cg = reinterpret_cast<uint16_t*>(base + L.cg);
-  float* S = reinterpret_cast<float*>(base + L.s);
-  float* dP = reinterpret_cast<float*>(base + L.dp);
-  uint16_t* P16 = reinterpret_cast<uint16_t*>(base + L.p16);
-  uint16_t* dz16 = reinterpret_cast<uint16_t*>(base + L.dz16);
+  uint16_t* QO = reinterpret_cast<uint16_t*>(base + L.qo);
+  float* SP = reinterpret_cast<float*>(base + L.sp);
+  uint16_t* PZ = reinterpret_cast<uint16_t*>(base + L.pz);
   float* dC = reinterpret_cast<float*>(base + L.dc);
   // setting the stream resets the workspace, so the workspace comes second
   DSA_TRY_BLAS(cublasSetStream(bl->h, s), "cublasSetStream");
@@ -1175,33 +1173,29 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
   int launched = 0;
   if (!accumulate_dkv)
     DSA_TRY_CUDA(cudaMemsetAsync(dkv, 0, (size_t)B * Lk * Dqk * sizeof(float), s), "dkv clear");
-  const long long qs = (long long)H * Dqk, os = (long long)H * Dv, hk = (long long)H * k,
+  // Per token, with QO = [q; dout padded to Dqk] (2H x Dqk) and the gathered rows C
+  // (k x Dqk): [S; dP] = QO C^T, dq = dz C, dC = [dz; P]^T QO (the padded columns of
+  // dout make the second half of each product act on the value columns only).
+  const long long qs = (long long)H * Dqk, q2s = 2LL * H * Dqk, h2k = 2LL * H * k,
                   cs = (long long)k * Dqk;
   for (long long tok0 = 0; tok0 < n; tok0 += T) {
     const int Tc = (int)(n - tok0 < T ? n - tok0 : T);
-    const uint16_t* Qc = q + tok0 * qs;
-    const uint16_t* dOc = dout + tok0 * os;
     DSA_TRY_CUDA(dsa::launch_gather_rows_bf16(kv, idx, cg, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
                  "latent row gather launch");
-    // S[H x k] = Q[H x Dqk] C^T, dP[H x k] = dout[H x Dv] C[:, :Dv]^T
-    DSA_TRY(gemm_rm(bl->h, false, true, H, k, Dqk, Qc, Dqk, qs, cg, Dqk, cs, 0.f, S, k, hk, Tc,
-                    CUDA_R_16BF, "S = Q C^T"));
-    DSA_TRY(gemm_rm(bl->h, false, true, H, k, Dv, dOc, Dv, os, cg, Dqk, cs, 0.f, dP, k, hk, Tc,
-                    CUDA_R_16BF, "dP = dout V^T"));
-    DSA_TRY_CUDA(dsa::launch_mla_bwd_softmax(S, dP, lse, idx, P16, dz16, tok0, Tc, H, k, Lk,
-                                             sm_scale, sms, s),
+    DSA_TRY_CUDA(dsa::launch_pack_qo(q, dout, QO, tok0, Tc, H, Dqk, Dv, sms, s),
+                 "query / output-gradient pack launch");
+    DSA_TRY(gemm_rm(bl->h, false, true, 2 * H, k, Dqk, QO, Dqk, q2s, cg, Dqk, cs, 0.0, SP, k, h2k,
+                    Tc, CUDA_R_16BF, "[S; dP] = QO C^T"));
+    DSA_TRY_CUDA(dsa::launch_mla_bwd_softmax(SP, lse, idx, PZ, tok0, Tc, H, k, Lk, sm_scale, sms,
+                                             s),
                  "softmax gradient launch");
-    // dq[H x Dqk] = dz[H x k] C[k x Dqk]
-    DSA_TRY(gemm_rm(bl->h, false, false, H, Dqk, k, dz16, k, hk, cg, Dqk, cs, 0.f, dq + tok0 * qs,
+    DSA_TRY(gemm_rm(bl->h, false, false, H, Dqk, k, PZ, k, h2k, cg, Dqk, cs, 0.0, dq + tok0 * qs,
                     Dqk, qs, Tc, CUDA_R_16BF, "dq = dz C"));
-    // dC[k x Dqk] = dz^T Q, then dC[:, :Dv] += P^T dout
-    DSA_TRY(gemm_rm(bl->h, true, false, k, Dqk, H, dz16, k, hk, Qc, Dqk, qs, 0.f, dC, Dqk, cs, Tc,
-                    CUDA_R_16BF, "dC = dz^T Q"));
-    DSA_TRY(gemm_rm(bl->h, true, false, k, Dv, H, P16, k, hk, dOc, Dv, os, 1.f, dC, Dqk, cs, Tc,
-                    CUDA_R_16BF, "dC += P^T dout"));
+    DSA_TRY(gemm_rm(bl->h, true, false, k, Dqk, 2 * H, PZ, k, h2k, QO, Dqk, q2s, 0.0, dC, Dqk, cs,
+                    Tc, CUDA_R_16BF, "dC = [dz; P]^T QO"));
     DSA_TRY_CUDA(dsa::launch_scatter_add_rows(dC, idx, dkv, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
                  "row gradient scatter launch");
-    launched += 3;
+    launched += 4;
   }
   g_last_launches = launched;
   return DSA_OK;

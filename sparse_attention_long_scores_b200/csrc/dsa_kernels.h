@@ -104,12 +104,15 @@ cudaError_t launch_indexer_kl(const uint16_t* kv, const KlArgs& a, cudaStream_t 
 cudaError_t launch_gather_rows_bf16(const uint16_t* kv, const int32_t* idx, uint16_t* out,
                                     long long tok0, int T, int Lq, int Lk, int k, int D,
                                     int num_sms, cudaStream_t stream);
-// P16 / dz16 [T, H, k] bf16 from S / dP [T, H, k] fp32 (raw q.c and dout.c[:Dv])
-// and lse [B*Lq, H].
-cudaError_t launch_mla_bwd_softmax(const float* S, const float* dP, const float* lse,
-                                   const int32_t* idx, uint16_t* P16, uint16_t* dz16,
-                                   long long tok0, int T, int H, int k, int Lk, float sm_scale,
-                                   int num_sms, cudaStream_t stream);
+// qo [T, 2H, Dqk] bf16 = per token the H rows of q [B*Lq, H, Dqk] and the H rows of
+// dout [B*Lq, H, Dv] padded with zeros to Dqk columns; Dqk % 8 == 0, Dv % 8 == 0.
+cudaError_t launch_pack_qo(const uint16_t* q, const uint16_t* dout, uint16_t* qo, long long tok0,
+                           int T, int H, int Dqk, int Dv, int num_sms, cudaStream_t stream);
+// PZ [T, 2H, k] bf16 (rows of dz, then rows of P) from SP [T, 2H, k] fp32 (rows of
+// raw q.c, then rows of dout.c[:Dv]) and lse [B*Lq, H].
+cudaError_t launch_mla_bwd_softmax(const float* SP, const float* lse, const int32_t* idx,
+                                   uint16_t* PZ, long long tok0, int T, int H, int k, int Lk,
+                                   float sm_scale, int num_sms, cudaStream_t stream);
 // dst [B, Lk, D] fp32 += src [T, k, D] fp32 row by row (atomic); D % 4 == 0.
 cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float* dst,
                                     long long tok0, int T, int Lq, int Lk, int k, int D,
