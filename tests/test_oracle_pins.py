@@ -372,6 +372,40 @@ def pin_indexer_backward_finite_differences(orc):
     assert not dq.any() and not dk.any() and not dw.any()
 
 
+def pin_gradients_golden(orc):
+    """Hand-worked gradients (tests/golden/sparse_stage_gradients.json): the attention
+    backward on two keys, the indexer backward on the three-token example's last
+    row, and the KL score gradient."""
+    g = json.load(open(os.path.join(GOLDEN, "sparse_stage_gradients.json")))
+    a = g["attention"]
+    kv = np.array([[_golden_value(x) for x in row] for row in a["keys"]])
+    for case in a["cases"]:
+        q = np.array([[_golden_value(x) for x in row] for row in case["q"]])
+        dout = np.array([[_golden_value(x) for x in row] for row in case["dout"]])
+        dq, dkv = orc.sparse_mla_backward(q, kv, np.array(a["idx"]), dout, a["sm_scale"], case["Dv"])
+        want_q = np.array([[_golden_value(x) for x in row] for row in case["dq"]])
+        want_kv = np.array([[_golden_value(x) for x in row] for row in case["dkv"]])
+        assert np.allclose(dq, want_q, rtol=0, atol=1e-14), case["note"]
+        assert np.allclose(dkv, want_kv, rtol=0, atol=1e-14), case["note"]
+    ix = g["indexer"]
+    keys = e4m3_codes(ix["keys"])
+    q = e4m3_codes(ix["q"])
+    one_q = np.ones(len(ix["q"]), np.float32)
+    one_k = np.ones(len(ix["keys"]), np.float32)
+    for case in ix["cases"]:
+        dq, dk, dw = orc.indexer_backward(q, one_q, np.asarray(ix["w"], np.float32), keys, one_k,
+                                          np.array(ix["idx"]), np.asarray(case["dI"], np.float64))
+        assert dw.tolist() == case["dw"], (case, dw)
+        assert dq.tolist() == case["dq"], (case, dq)
+        assert dk.tolist() == case["dk"], (case, dk)
+    for case in g["kl_score_grad"]:
+        idx = np.array(case.get("idx", list(range(len(case["p"])))))
+        grad = orc.indexer_kl_score_grad(np.array([_golden_value(x) for x in case["p"]]),
+                                         np.array([_golden_value(x) for x in case["scores"]]), idx, 2)
+        assert np.allclose(grad, [_golden_value(x) for x in case["grad"]], rtol=0, atol=1e-15), \
+            case["note"]
+
+
 def pin_code_dots_exact(orc):
     """The indexer backward decides its ReLU mask on dots of e4m3 codes in float64,
     which must be exact: every e4m3 value times 2^9 is an integer, so the dot times
@@ -417,7 +451,7 @@ PINS = [pin_three_token, pin_e4m3_table, pin_indexer_closed_forms, pin_indexer_m
         pin_topk_bruteforce, pin_topk_properties, pin_attention_special_cases,
         pin_dense_equivalence, pin_invariances, pin_kl_golden, pin_kl_properties,
         pin_mla_backward_finite_differences, pin_mla_backward_closed_forms,
-        pin_indexer_backward_finite_differences, pin_code_dots_exact,
+        pin_indexer_backward_finite_differences, pin_code_dots_exact, pin_gradients_golden,
         pin_kl_score_grad_finite_differences]
 
 
