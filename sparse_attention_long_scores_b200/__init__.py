@@ -153,6 +153,8 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None, cuda=True):
         raise ValueError(f"{name} must be contiguous")
     if cuda and not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device")
+    if not cuda and t.is_cuda:
+        raise ValueError(f"{name} must be in host memory")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
@@ -384,6 +386,18 @@ def _tensors(inp: dict, out, lse, idx_out) -> DsaTensors:
         out, lse, idx_out)])
 
 
+def _need_inputs(p: "Problem", inp: dict, prefix: str = "", cuda: bool = True) -> None:
+    """Dtype, shape and contiguity of the seven input tensors of problem p."""
+    _need(inp["qI"], prefix + "qI", torch.uint8, (p.B, p.Lq, p.H_I, p.d_I), cuda)
+    _need(inp["qI_scale"], prefix + "qI_scale", torch.float32, (p.B, p.Lq, p.H_I), cuda)
+    _need(inp["kI"], prefix + "kI", torch.uint8, (p.B, p.Lk, p.d_I), cuda)
+    _need(inp["kI_scale"], prefix + "kI_scale", torch.float32, (p.B, p.Lk), cuda)
+    _need(inp["w"], prefix + "w", torch.float32 if p.w_dtype == DSA_DTYPE_F32 else torch.bfloat16,
+          (p.B, p.Lq, p.H_I), cuda)
+    _need(inp["q"], prefix + "q", torch.bfloat16, (p.B, p.Lq, p.H, p.Dqk), cuda)
+    _need(inp["kv"], prefix + "kv", torch.bfloat16, (p.B, p.Lk, p.Dqk), cuda)
+
+
 def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, stream=None):
     """Whole DSA forward (indexer -> top-k -> sparse MLA) on device tensors.
 
@@ -391,14 +405,7 @@ def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, st
     Returns out [B, Lq, H, Dv] bf16 (lse / idx_out are filled when given).
     """
     dev = inp["q"].device
-    _need(inp["qI"], "qI", torch.uint8, (p.B, p.Lq, p.H_I, p.d_I))
-    _need(inp["qI_scale"], "qI_scale", torch.float32, (p.B, p.Lq, p.H_I))
-    _need(inp["kI"], "kI", torch.uint8, (p.B, p.Lk, p.d_I))
-    _need(inp["kI_scale"], "kI_scale", torch.float32, (p.B, p.Lk))
-    _need(inp["w"], "w", torch.float32 if p.w_dtype == DSA_DTYPE_F32 else torch.bfloat16,
-          (p.B, p.Lq, p.H_I))
-    _need(inp["q"], "q", torch.bfloat16, (p.B, p.Lq, p.H, p.Dqk))
-    _need(inp["kv"], "kv", torch.bfloat16, (p.B, p.Lk, p.Dqk))
+    _need_inputs(p, inp)
     if out is None:
         out = torch.empty((p.B, p.Lq, p.H, p.Dv), dtype=torch.bfloat16, device=dev)
     _need(out, "out", torch.bfloat16, (p.B, p.Lq, p.H, p.Dv))
@@ -487,7 +494,23 @@ def forward_host(p: Problem, host: dict, dev: dict, host_out, dev_out, ws, strea
                  host_lse=None, dev_lse=None, host_idx=None, dev_idx=None):
     """dsa_forward on host tensors: H2D copies, forward, D2H copies of out (and of lse
     / idx_out when both their host and device tensors are given), synchronise. With
-    Lq >= 1024 the library pipelines the copies with the compute by blocks of rows."""
+    Lq >= 1024 the library pipelines the copies with the compute by blocks of rows.
+    Host and device tensors are checked for dtype, shape and contiguity first (the
+    copies trust those sizes)."""
+    extra = ((host_lse, dev_lse, "lse", torch.float32, (p.B, p.Lq, p.H)),
+             (host_idx, dev_idx, "idx", torch.int32, (p.B, p.Lq, p.k)))
+    _need_inputs(p, host, "host ", cuda=False)
+    _need(host_out, "host out", torch.bfloat16, (p.B, p.Lq, p.H, p.Dv), cuda=False)
+    for h, _, name, dt, shp in extra:
+        if h is not None:
+            _need(h, "host " + name, dt, shp, cuda=False)
+    _need_inputs(p, dev, "device ")
+    _need(dev_out, "device out", torch.bfloat16, (p.B, p.Lq, p.H, p.Dv))
+    for _, d, name, dt, shp in extra:
+        if d is not None:
+            _need(d, "device " + name, dt, shp)
+    if not ws.is_cuda:
+        raise ValueError("ws must be on a CUDA device")
     cp = p.c()
     ch = _tensors(host, host_out, host_lse, host_idx)
     cd = _tensors(dev, dev_out, dev_lse, dev_idx)

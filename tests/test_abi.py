@@ -142,6 +142,34 @@ def test_backward_entry_points_reject_bad_args(L):
     assert L.dsa_indexer_kl_grad(p, p, p, p, 1, 4, 8, 32, math.nan, None) == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_forward_host_checks_host_tensors_before_any_copy():
+    """dsa_forward_host's copies trust the tensor sizes, so the binding checks the
+    host tensors' dtype, shape and contiguity before the call (no GPU needed: with
+    valid host tensors the next check to fail is the device one)."""
+    import torch
+    from dsa_inputs import CONFIGS, gen_inputs
+    cfg = CONFIGS["tiny"].with_(Lq=8, Lk=8)
+    p = dsa.Problem.from_config(cfg)
+    host = gen_inputs(cfg, "cpu", seed=3)
+    out = torch.empty((1, 8, cfg.H, cfg.Dv), dtype=torch.bfloat16)
+    ws = torch.empty(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="must be on a CUDA device"):
+        dsa.forward_host(p, host, host, out, out, ws)
+    bad = dict(host, q=host["q"][:, :4].contiguous())
+    with pytest.raises(ValueError, match="host q has shape"):
+        dsa.forward_host(p, bad, host, out, out, ws)
+    bad = dict(host, kv=host["kv"].transpose(1, 2))
+    with pytest.raises(ValueError, match="host kv must be contiguous"):
+        dsa.forward_host(p, bad, host, out, out, ws)
+    bad = dict(host, kI_scale=host["kI_scale"].double())
+    with pytest.raises(TypeError, match="host kI_scale must be"):
+        dsa.forward_host(p, bad, host, out, out, ws)
+    with pytest.raises(ValueError, match="host out has shape"):
+        dsa.forward_host(p, host, host, out[:, :4], out, ws)
+    with pytest.raises(ValueError, match="host lse has shape"):
+        dsa.forward_host(p, host, host, out, out, ws, host_lse=torch.empty(3))
+
+
 def test_backward_workspace_sizes(L):
     """Chunks of at most 64 tokens: the recommended workspace grows with the token
     count up to 64 and then stays flat; about 10 MB per token at the full shapes."""
