@@ -205,7 +205,7 @@ int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, co
  *     dq[h]   = sum_s dz[h,s] c_s                      (all Dqk columns)
  *     dkv[s] += sum_h dz[h,s] q[h]   and, on columns < Dv, sum_h P[h,s] dout[h]
  *   D is formed from the recomputed fp32 P and dP rather than from the forward's
- *   bf16 output, so a set of one key gets dq = 0 exactly.
+ *   bf16 output, whose bf16-rounded P would dominate dP - D on short sets.
  *   q [B, Lq, H, Dqk], kv [B, Lk, Dqk], dout [B, Lq, H, Dv]: bf16; idx [B, Lq, k]
  *   int32 (slots < 0 or >= Lk skipped); lse [B, Lq, H] fp32 as the forward
  *   returned it; dq [B, Lq, H, Dqk] fp32 (overwritten);

@@ -110,8 +110,8 @@ __global__ void pack_qo_kernel(const uint4* __restrict__ q, const uint4* __restr
 // of S and then the H rows of dP):
 //   P_s  = exp(sm_scale S_s - lse)
 //   D    = sum_s P_s dP_s / sum_s P_s       (= dout . out; from the fp32 P and dP,
-//                                             so that sum_s dz_s = 0 and a single
-//                                             key gives dz = 0 exactly)
+//                                             so that sum_s dz_s vanishes up to fp32
+//                                             rounding, also for short sets)
 //   dz_s = sm_scale P_s (dP_s - D)
 // dz and P are written as bf16 for the GEMMs that follow, per token the H rows of dz
 // and then the H rows of P (PZ); slots without a valid key get 0.
