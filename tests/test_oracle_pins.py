@@ -486,6 +486,17 @@ def test_generator_is_seeded_and_shaped():
     assert torch.all(vals == 448.0)
 
 
+def test_output_gradient_is_seeded_bf16_normal():
+    from dsa_inputs import output_gradient
+    a = output_gradient((2, 3, 8, 64), seed=5)
+    b = output_gradient((2, 3, 8, 64), seed=5)
+    c = output_gradient((2, 3, 8, 64), seed=6)
+    assert a.dtype == torch.bfloat16 and a.shape == (2, 3, 8, 64)
+    assert torch.equal(a, b) and not torch.equal(a, c)
+    x = output_gradient((1 << 16,), seed=7, std=2.0).double()
+    assert abs(x.mean().item()) < 0.05 and abs(x.std().item() - 2.0) < 0.05
+
+
 def test_random_key_sets_look_like_selections():
     from dsa_inputs import random_key_sets, random_scores
     idx = random_key_sets(2, 40, 16, 5, seed=3)
