@@ -170,6 +170,48 @@ def test_forward_host_checks_host_tensors_before_any_copy():
         dsa.forward_host(p, host, host, out, out, ws, host_lse=torch.empty(3))
 
 
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "dsa.h"
+int main(void) {
+  /* host-only calls: version, sizes and argument validation (no device needed) */
+  dsa_problem p;
+  memset(&p, 0, sizeof p);
+  p.mode = DSA_MODE_PREFILL; p.B = 1; p.Lq = 256; p.Lk = 256; p.H_I = 4; p.d_I = 32;
+  p.H = 8; p.Dqk = 80; p.Dv = 64; p.k = 32; p.sm_scale = 0.1f; p.w_dtype = DSA_DTYPE_F32;
+  if (dsa_forward_workspace_size(&p) == 0) return 1;
+  if (dsa_sparse_mla_bwd_workspace_size(1, 256, 8, 80, 64, 32) == 0) return 2;
+  int rc = dsa_sparse_mla_bwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 1, 256, 256, 8, 80,
+                              64, 32, 0.1f, NULL, 0, NULL);
+  if (rc != DSA_ERR_INVALID_ARG || strstr(dsa_last_error(), "q") == NULL) return 3;
+  if (dsa_last_launch_count() != 0) return 4;
+  printf("%s\n", dsa_version());
+  return 0;
+}
+"""
+
+
+def test_plain_c_program_uses_the_abi(L, tmp_path):
+    """The boundary is plain C: a C99 program compiles against include/dsa.h, links
+    to libdsa.so and makes host-only calls through it."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "abi.c"
+    exe = tmp_path / "abi"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(dsa.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir,
+                    "-ldsa", "-Wl,-rpath," + libdir], check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("dsa-b200")
+
+
 def test_backward_workspace_sizes(L):
     """Chunks of at most 64 tokens: the recommended workspace grows with the token
     count up to 64 and then stays flat; about 10 MB per token at the full shapes."""
