@@ -492,6 +492,50 @@ def cpu_baseline(cfg, budget_s: float = 20.0) -> dict:
                       f"positions, {dt:.1f} s), numpy fp64 with BLAS on {cores} host threads"}
 
 
+def oracle_backward_sample(cfg, rows: int, seed: int = 4243):
+    """A bounded sample of the sparse-stage gradients for the fp64 oracle: `rows`
+    query rows at evenly spread positions of one sequence, each with a seeded set of
+    min(k, p + 1) causal keys standing in for its top-k set, a seeded output gradient
+    and a seeded index-score gradient. One unit is the attention and indexer
+    gradients of one row."""
+    import oracle as ORC
+    from dsa_inputs import output_gradient, random_key_sets, random_scores
+
+    c1 = cfg.with_(B=1, Lq=rows, q_pos0=0)
+    inp = ORC.numpy_inputs(gen_inputs(c1, "cpu", seed=seed))
+    pos = [min(cfg.Lk - 1, int((i + 0.5) * cfg.Lk / rows)) for i in range(rows)]
+    sets = [random_key_sets(1, 1, cfg.k, p, seed=seed + 3 + i)[0, 0].numpy()
+            for i, p in enumerate(pos)]
+    dout = ORC.numpy_inputs({"d": output_gradient((1, rows, cfg.H, cfg.Dv), seed=seed + 1)})["d"]
+    dI = random_scores((1, rows, cfg.k), seed=seed + 2).numpy()
+
+    def run(i):
+        ORC.sparse_mla_backward(inp["q"][0, i], inp["kv"][0], sets[i], dout[0, i], cfg.sm_scale,
+                                cfg.Dv)
+        ORC.indexer_backward(inp["qI"][0, i], inp["qI_scale"][0, i], inp["w"][0, i], inp["kI"][0],
+                             inp["kI_scale"][0], sets[i], dI[0, i])
+
+    return run, pos
+
+
+def cpu_baseline_backward(cfg, budget_s: float = 10.0, rows: int = 64) -> dict:
+    run, pos = oracle_backward_sample(cfg, rows)
+    t0 = time.perf_counter()
+    done = 0
+    for i in range(len(pos)):
+        run(i)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"attention and indexer gradients of {done} query rows of {cfg.name} "
+                      f"(one sequence, rows at evenly spread positions, seeded key sets of "
+                      f"min(k, p + 1) keys, {dt:.1f} s), numpy fp64 with BLAS on {cores} host "
+                      f"threads"}
+
+
 def reference_arm(args):
     cfg = CONFIGS[args.workload]
     rows_per_step = 8
@@ -674,6 +718,8 @@ def main():
         if kl is not None:
             line["indexer_kl"] = kl
         if bwd is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                bwd["cpu_baseline"] = cpu_baseline_backward(CONFIGS[bwd["workload"]])
             line["backward"] = bwd
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)

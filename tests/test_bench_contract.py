@@ -29,3 +29,15 @@ def test_reference_arm_prints_one_contract_line():
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_backward_cpu_baseline_reports_a_bounded_oracle_sample():
+    """The fp64 oracle timing that bench.py attaches to its gradients line (run here on
+    the tiny workload, the same function the bench calls on the 2 x 32K one)."""
+    import sys as _sys
+    _sys.path.insert(0, ROOT)
+    import bench
+    from dsa_inputs import CONFIGS
+    r = bench.cpu_baseline_backward(CONFIGS["tiny"], budget_s=2.0, rows=8)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
+    assert r["cores"] >= 1 and "gradients of" in r["sample"]
