@@ -66,21 +66,33 @@ def work(cfg) -> dict:
 
     indexer  flops = 2 * H_I * d_I per (query row, causal key) of rows that need
              scoring (p + 1 > k); rows with p + 1 <= k select every key unscored.
+             bytes = key codes + scales once per sequence, query codes, scales and
+             weights, and 4 per score written (the decode roofline: one query row
+             per sequence makes it bandwidth-bound).
     topk     bytes = 4 per candidate score read + 4 * k per selected row written.
     mla      flops = 2 * H * (Dqk + Dv) per (query row, selected key).
+             bytes = 2 * Dqk per selected key + q, idx and out per row (decode).
     decode   bytes = indexer keys + scales + gathered latent rows + q, qI, w, out.
     """
+    w_bytes = 4 if cfg.w_dtype == "f32" else 2
     p = cfg.q_pos0 + np.arange(cfg.Lq, dtype=np.int64)
     n = np.minimum(p + 1, cfg.Lk)
     scored = n > cfg.k
     pairs_idx = int(n[scored].sum()) * cfg.B
     sel = int(np.minimum(n, cfg.k).sum()) * cfg.B
     rows_scored = int(scored.sum()) * cfg.B
-    w_bytes = 4 if cfg.w_dtype == "f32" else 2
+    tokens = cfg.B * cfg.Lq
     return {
         "indexer_flops": 2.0 * cfg.H_I * cfg.d_I * pairs_idx,
+        # indexer bytes: the key codes and scales of every causal key of each
+        # sequence, read once, plus the query rows, weights and scores written
+        "indexer_bytes": float(cfg.B * min(cfg.Lk, cfg.q_pos0 + cfg.Lq) * (cfg.d_I + 4)
+                               + tokens * cfg.H_I * (cfg.d_I + 4 + w_bytes) + 4.0 * pairs_idx),
         "topk_bytes": 4.0 * pairs_idx + 4.0 * cfg.k * rows_scored,
         "mla_flops": 2.0 * cfg.H * (cfg.Dqk + cfg.Dv) * sel,
+        # attention bytes: each selected latent row once, q and idx in, out written
+        "mla_bytes": float(sel * cfg.Dqk * 2 + tokens * (cfg.H * cfg.Dqk * 2 + 4 * cfg.k
+                                                         + cfg.H * cfg.Dv * 2)),
         "hbm_bytes": float(cfg.B * cfg.Lk * (cfg.d_I + 4)            # indexer keys + scales
                            + sel * cfg.Dqk * 2                      # gathered latent rows
                            + cfg.B * cfg.Lq * (cfg.H * cfg.Dqk * 2 + cfg.H_I * (cfg.d_I + 4 + w_bytes)
@@ -247,11 +259,17 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     w = work(cfg)
     fp8_peak = 2.0 * pk["bf16_sustained"]   # FP8 dense = 2 x bf16 dense (nominal ratio)
     roof = {}
+    decode = cfg.mode == "decode"
     if "indexer" in kernels:
         t = kernels["indexer"]["ms_per_step"] * 1e-3
-        a = w["indexer_flops"] / t / 1e12
-        roof["indexer"] = {"bound": "tensor", "achieved": a, "peak": fp8_peak, "unit": "TFLOP/s",
-                           "frac": a / fp8_peak, "peak_note": "fp8 = 2 x measured bf16 sustained"}
+        if decode:   # one query row per sequence: every key is read for 16 KFLOP
+            a = w["indexer_bytes"] / t / 1e9
+            roof["indexer"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s",
+                               "frac": a / pk["hbm"]}
+        else:
+            a = w["indexer_flops"] / t / 1e12
+            roof["indexer"] = {"bound": "tensor", "achieved": a, "peak": fp8_peak, "unit": "TFLOP/s",
+                               "frac": a / fp8_peak, "peak_note": "fp8 = 2 x measured bf16 sustained"}
     if "topk" in kernels:
         t = kernels["topk"]["ms_per_step"] * 1e-3
         a = w["topk_bytes"] / t / 1e9
@@ -259,10 +277,15 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
                         "frac": a / pk["hbm"]}
     if "sparse_mla" in kernels:
         t = kernels["sparse_mla"]["ms_per_step"] * 1e-3
-        a = w["mla_flops"] / t / 1e12
-        roof["sparse_mla"] = {"bound": "tensor", "achieved": a, "peak": pk["bf16_sustained"],
-                              "unit": "TFLOP/s", "frac": a / pk["bf16_sustained"],
-                              "peak_note": "measured bf16 sustained"}
+        if decode:   # 64 query rows: each gathered latent row serves one token
+            a = w["mla_bytes"] / t / 1e9
+            roof["sparse_mla"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s",
+                                  "frac": a / pk["hbm"]}
+        else:
+            a = w["mla_flops"] / t / 1e12
+            roof["sparse_mla"] = {"bound": "tensor", "achieved": a, "peak": pk["bf16_sustained"],
+                                  "unit": "TFLOP/s", "frac": a / pk["bf16_sustained"],
+                                  "peak_note": "measured bf16 sustained"}
     for k, r in roof.items():
         r["traffic"] = traffic_per_launch(k, cfg.mode, cfg.B * cfg.Lq / kernels[k]["launches_per_step"])
     res = {"cfg": cfg, "ms": ms, "tokens_per_s": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, ms),

@@ -131,6 +131,9 @@ int dsa_sparse_mla_fwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
  *     needs none), so every shape dsa_sparse_mla_fwd accepts is accepted.
  *   - The first call on a device looks up the array's device address with the
  *     device current; make that first call before any stream capture.
+ *   - That address is kept for the life of the process. cudaDeviceReset
+ *     unloads the library's device code, so after a reset the kept address is
+ *     stale: do not call this entry point again in that process.
  *   - All calls share the one array and every call fully overwrites the part it
  *     uses (nothing needs clearing), so calls that overlap on the GPU (other
  *     streams, other host threads) race with each other: serialise them.

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -22,6 +23,16 @@
 namespace {
 
 thread_local std::string g_err;
+
+// NVTX range around the enqueue of one kernel launch (or one entry point): a
+// profiler attached to the process shows each stage of the path by name; with
+// no tool attached a push/pop costs a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Bound on device-side waits; DSA_WAIT_LIMIT_NS overrides the 2 s default.
 unsigned long long initial_wait_ns() {
@@ -231,8 +242,11 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
             size_t ws_bytes, const dsa::DevCtl& ctl, int num_sms, cudaStream_t stream,
             Recorder& rec = g_no_rec, bool fit_splits = false,
             const dsa_paged_cache* pc = nullptr) {
-  (void)num_sms;
-  int splits = mla_splits(B, Lq, Dv, k, assumed_sms());
+  // Key splits for this device's SM count. Workspaces are sized for assumed_sms()
+  // (no device needed), and fewer SMs never need more splits, so a device with
+  // more SMs than that is scheduled as if it had assumed_sms().
+  const int sched_sms = (num_sms > 0 && num_sms < assumed_sms()) ? num_sms : assumed_sms();
+  int splits = mla_splits(B, Lq, Dv, k, sched_sms);
   // fit_splits: use fewer key splits rather than fail when the partials of the
   // recommended count do not fit (one split needs none)
   while (fit_splits && splits > 1 && mla_ws_bytes(B, Lq, H, Dv, splits) > ws_bytes) --splits;
@@ -265,9 +279,13 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
     a.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                          align_up(tok * splits * H * Dv * sizeof(float), 256));
   }
-  DSA_TRY_CUDA(dsa::launch_sparse_mla(tq, kv, a, stream), "sparse MLA launch");
+  {
+    NvtxRange r("dsa:sparse_mla");
+    DSA_TRY_CUDA(dsa::launch_sparse_mla(tq, kv, a, stream), "sparse MLA launch");
+  }
   DSA_TRY(rec.mark(DSA_KIND_SPARSE_MLA, stream));
   if (splits > 1) {
+    NvtxRange r("dsa:mla_combine");
     DSA_TRY_CUDA(dsa::launch_mla_combine(a, stream), "split combine launch");
     DSA_TRY(rec.mark(DSA_KIND_COMBINE, stream));
   }
@@ -393,7 +411,10 @@ int launch_indexer_rows(const uint8_t* qI, const float* qI_scale, const uint8_t*
   int keys_max = q_pos0 + t_hi < Lk ? q_pos0 + t_hi : Lk;
   a.piece_keys = indexer_piece_keys(B, t_hi - t_lo, n_tok, keys_max, num_sms);
   a.ctl = ctl;
-  DSA_TRY_CUDA(dsa::launch_indexer(tq, tk, a, H_I, d_I, num_sms, stream), "indexer launch");
+  {
+    NvtxRange r("dsa:indexer");
+    DSA_TRY_CUDA(dsa::launch_indexer(tq, tk, a, H_I, d_I, num_sms, stream), "indexer launch");
+  }
   DSA_TRY(rec.mark(DSA_KIND_INDEXER, stream));
   return DSA_OK;
 }
@@ -665,6 +686,7 @@ dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld,
 
 int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
                  void* stream, Recorder& rec, const dsa_paged_cache* pc = nullptr) {
+  NvtxRange whole("dsa_forward");
   DSA_TRY(validate_problem(p));
   DSA_TRY(validate_tensors(t));
   DSA_TRY(check_ptr(ws, "ws", true));
@@ -718,8 +740,11 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
       }
       DSA_TRY_CUDA(cudaEventRecord(r->scored[b], s), "cudaEventRecord");
       DSA_TRY_CUDA(cudaStreamWaitEvent(r->side, r->scored[b], 0), "cudaStreamWaitEvent");
-      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl, pc), sms, r->side),
-                   "top-k launch");
+      {
+        NvtxRange nr("dsa:topk");
+        DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl, pc), sms, r->side),
+                     "top-k launch");
+      }
       DSA_TRY(rec.mark(DSA_KIND_TOPK, r->side));   // counts it (no events on this path)
       DSA_TRY_CUDA(cudaEventRecord(r->selected[b], r->side), "cudaEventRecord");
     }
@@ -734,8 +759,11 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
                                     f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
                                     t1, ctl, sms, s, rec, pc));
       }
-      DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl, pc), sms, s),
-                   "top-k launch");
+      {
+        NvtxRange nr("dsa:topk");
+        DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl, pc), sms, s),
+                     "top-k launch");
+      }
       DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
     }
   }
