@@ -134,6 +134,45 @@ def test_mla_backward_full_shapes(holes):
     _check_attention(cfg, inp, idx, dout, f"full holes={holes}")
 
 
+def test_mla_backward_small_workspace_uses_short_chunks():
+    """A workspace sized for 7 tokens (the recommended size of a 7-token call) makes
+    dsa_sparse_mla_bwd and dsa_indexer_bwd work through 70 tokens in chunks of 7:
+    the results must match the oracle, and the full-workspace call."""
+    cfg = CONFIGS["prefill_8k"].with_(B=1, Lq=70, Lk=2100, q_pos0=2030, **FULL)
+    inp = gen_inputs(cfg, "cpu", seed=75)
+    idx = random_key_sets(1, cfg.Lq, cfg.k, cfg.q_pos0, seed=76, holes=0.1)
+    dout = output_gradient((1, cfg.Lq, cfg.H, cfg.Dv), seed=77)
+    q, kv, idxd, doutd = inp["q"].cuda(), inp["kv"].cuda(), idx.cuda(), dout.cuda()
+    _, lse = dsa.sparse_mla_fwd(q, kv, idxd, cfg.sm_scale, cfg.Dv)
+    small = lambda n: torch.empty(int(n), dtype=torch.uint8, device="cuda")
+    ws7 = small(dsa.lib().dsa_sparse_mla_bwd_workspace_size(1, 7, cfg.H, cfg.Dqk, cfg.Dv, cfg.k))
+    assert ws7.numel() < dsa.lib().dsa_sparse_mla_bwd_workspace_size(1, cfg.Lq, cfg.H, cfg.Dqk,
+                                                                       cfg.Dv, cfg.k)
+    dq7, dkv7 = dsa.sparse_mla_bwd(q, kv, idxd, lse, doutd, cfg.sm_scale, ws=ws7)
+    dq, dkv = dsa.sparse_mla_bwd(q, kv, idxd, lse, doutd, cfg.sm_scale)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    rq, rkv = _oracle_attention_grads(cfg, inp, idx, dout)
+    check_grad(dq7.cpu().numpy(), rq, GRAD_ATT_ROW, GRAD_ATT_ALL, "7-token chunks dq")
+    check_grad(dkv7.cpu().numpy(), rkv, GRAD_ATT_ROW, GRAD_ATT_ALL, "7-token chunks dkv")
+    # the chunking changes only summation orders
+    check_grad(dq7.cpu().numpy(), dq.cpu().numpy().astype(np.float64), GRAD_ATT_ROW, GRAD_ATT_ALL,
+               "7-token chunks dq vs full workspace")
+    check_grad(dkv7.cpu().numpy(), dkv.cpu().numpy().astype(np.float64), GRAD_ATT_ROW, GRAD_ATT_ALL,
+               "7-token chunks dkv vs full workspace")
+    # the indexer backward with a 7-token workspace
+    iinp, iidx, dI = _indexer_case(cfg, 78)
+    wsi = small(dsa.lib().dsa_indexer_bwd_workspace_size(1, 7, cfg.H_I, cfg.d_I, cfg.k))
+    args = [iinp[n].cuda() for n in ("qI", "qI_scale", "kI", "kI_scale", "w")]
+    a7 = dsa.indexer_bwd(*args, iidx.cuda(), dI.cuda(), ws=wsi)
+    af = dsa.indexer_bwd(*args, iidx.cuda(), dI.cuda())
+    torch.cuda.synchronize()
+    dsa.check_status()
+    for j, name in enumerate(("dqI", "dkI", "dw")):
+        check_grad(a7[j].cpu().numpy(), af[j].cpu().numpy().astype(np.float64), GRAD_IDX_ROW,
+                   GRAD_IDX_ALL, f"7-token chunks {name} vs full workspace")
+
+
 def test_mla_backward_prefill_32k_sampled_rows():
     """The bench workload (2 x 32K, the forward's own top-k sets): dq rows of sampled
     tokens against the oracle one by one, and for dkv a property that holds at any

@@ -193,23 +193,45 @@ def test_topk_exact_ties_and_long_rows(Lk, k, levels):
 # ---------------------------------------------------------------------------
 
 
-def _check_big(cfg, n_rows, score_blocks=2):
+def _check_big(cfg, n_rows, score_blocks=2, all_rows=False):
+    """Sampled rows of a full-size workload, run in the benchmark's launch
+    configuration: selection and attention of ``n_rows`` rows per sequence, and
+    the indexer scores of ``score_blocks`` blocks of 8 rows per sequence through
+    the public score entry point. With ``all_rows`` every row's scores (the whole
+    causal score matrix, one launch) and every row's selection are checked too."""
     inp = gen_inputs(cfg, "cuda")
     out, lse, idx = _forward(cfg, inp)
     rows = Rows(cfg, inp)
     samples = sample_rows(cfg, n_rows)
     n_band = 0
+    if all_rows:
+        sc_all = dsa.indexer_scores(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"],
+                                    q_pos0=cfg.q_pos0)
+        dsa.check_status()
+        idx_all = idx.cpu().numpy()
+        for b in range(cfg.B):
+            sc_h = sc_all[b].cpu().numpy()
+            for t in range(cfg.Lq):
+                p = cfg.q_pos0 + t
+                ref_sc = rows.scores(b, t)
+                check_scores(sc_h[t, :p + 1], ref_sc, f"{cfg.name} all-row scores b={b} t={t}")
+                n_band += check_selection(idx_all[b, t], ref_sc, ORC.topk_select(ref_sc, cfg.k), cfg.k, p,
+                                          f"{cfg.name} all-row selection b={b} t={t}")
+            del sc_h
+        del sc_all
+        torch.cuda.empty_cache()
     for b in range(cfg.B):
         ro, rl, go, gl = [], [], [], []
         for t in samples:
             p = cfg.q_pos0 + t
             gidx = idx[b, t].cpu().numpy()
-            if p + 1 > cfg.k:
-                sc = rows.scores(b, t)
-                ref_idx = ORC.topk_select(sc, cfg.k)
-            else:
-                sc, ref_idx = None, ORC.topk_select(np.zeros(p + 1), cfg.k)
-            n_band += check_selection(gidx, sc, ref_idx, cfg.k, p, f"{cfg.name} b={b} t={t}")
+            if not all_rows:
+                if p + 1 > cfg.k:
+                    sc = rows.scores(b, t)
+                    ref_idx = ORC.topk_select(sc, cfg.k)
+                else:
+                    sc, ref_idx = None, ORC.topk_select(np.zeros(p + 1), cfg.k)
+                n_band += check_selection(gidx, sc, ref_idx, cfg.k, p, f"{cfg.name} b={b} t={t}")
             o, l = rows.attention(b, t, gidx)
             ro.append(o)
             rl.append(l)
@@ -238,15 +260,16 @@ def _check_big(cfg, n_rows, score_blocks=2):
 
 
 def test_prefill_8k():
-    _check_big(CONFIGS["prefill_8k"], 48)
+    """Every row's scores and selection; attention on 512 rows."""
+    _check_big(CONFIGS["prefill_8k"], 512, all_rows=True)
 
 
 def test_prefill_32k_batch2():
-    _check_big(CONFIGS["prefill_32k"], 24)
+    _check_big(CONFIGS["prefill_32k"], 64)
 
 
 def test_prefill_128k():
-    _check_big(CONFIGS["prefill_128k"], 16)
+    _check_big(CONFIGS["prefill_128k"], 64)
 
 
 def test_decode_128k():
@@ -254,10 +277,18 @@ def test_decode_128k():
     inp = gen_inputs(cfg, "cuda")
     out, lse, idx = _forward(cfg, inp)
     rows = Rows(cfg, inp)
+    # the single-token indexer variant that decode runs, score for score: one query
+    # row per sequence at position Lk - 1 against all 131072 cached keys
+    sc_gpu = dsa.indexer_scores(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"],
+                                q_pos0=cfg.q_pos0)
+    dsa.check_status()
+    assert tuple(sc_gpu.shape) == (cfg.B, 1, cfg.Lk)
+    sc_gpu = sc_gpu.cpu().numpy()
     go, gl, ro, rl = [], [], [], []
     for b in range(cfg.B):
         gidx = idx[b, 0].cpu().numpy()
         sc = rows.scores(b, 0)
+        check_scores(sc_gpu[b, 0], sc, f"decode scores b={b}")
         check_selection(gidx, sc, ORC.topk_select(sc, cfg.k), cfg.k, cfg.q_pos0, f"decode b={b}")
         o, l = rows.attention(b, 0, gidx)
         ro.append(o)
