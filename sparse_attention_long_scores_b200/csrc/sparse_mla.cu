@@ -11,17 +11,22 @@
 //     O[h, chunk] += P[h,s] . c_s[chunk]    (tcgen05, M = 128, N = DVC, K = 64 keys)
 // Layout of the work:
 //   warp 0      tcgen05 issuer: Q's shared-memory part once (TMA tiles), then for
-//               each 64-key tile S_i = Q K_i^T into one of two TMEM buffers and
-//               O += P_i V_i with P read from TMEM;
-//   warps 5..12 gather producers: the selected latent rows of each tile, 16 bytes
-//               per thread per cp.async, stored straight into the 128-byte-
-//               swizzled K-major layout the tensor core reads, into a 2-stage
-//               ring. A TMA gather4 costs about as much issue time per 512 bytes
-//               as these warps need for a whole tile, so threads gather the rows;
-//   warps 1..4  softmax: one head (TMEM lane) per thread. Reads S_i, writes P_i
-//               (bf16) over the first half of S_i's own TMEM buffer, rescales O
-//               in TMEM only when the running max grew by more than 2^8, and
-//               normalises at the end.
+//               each 64-key tile, in a fixed order, S_i = Q K_i^T into one of two
+//               TMEM buffers (part A of the columns, then part B) and, between the
+//               two parts as soon as P_{i-1} is ready, O += P_{i-1} V_{i-1} with P
+//               read from TMEM;
+//   warps 1..8  softmax, two warps per TMEM lane quadrant: a thread owns one head
+//               (TMEM lane) and 32 of the tile's 64 keys. The two threads of a head
+//               exchange their maxima through shared memory, write P_i (bf16) over
+//               the first half of S_i's own TMEM buffer, rescale their half of O in
+//               TMEM only when the running max grew by more than 2^8, and
+//               normalise at the end;
+//   warps 9..16 gather producers: each warp owns 8 rows of every tile, loads their
+//               indices once and copies the rows 16 bytes per thread per cp.async,
+//               straight into the 128-byte-swizzled K-major layout the tensor core
+//               reads, into a 2-stage ring. A TMA gather4 costs about as much issue
+//               time per 512 bytes as these warps need for a whole tile, so
+//               threads gather the rows.
 // O for 128 heads x 512 values in fp32 would fill all of TMEM, so the value
 // columns are split over CTAs (DVC = 256): each CTA recomputes S for its token.
 // With several key splits (decode) each CTA writes an unnormalised partial
@@ -34,13 +39,13 @@ namespace dsa {
 namespace {
 
 constexpr int KEYS = 64;                       // keys per tile (N of the S MMA)
+constexpr int SMX_WARPS = 8;                   // softmax warps (two per lane quadrant)
 constexpr int PROD_WARPS = 8;                  // gather warps
-constexpr int MLA_THREADS = 32 + 128 + PROD_WARPS * 32;
-constexpr int PROD_T0 = 160;                   // first producer thread
-
-// How long the MMA thread may sleep on one barrier while it polls the inputs of
-// S and PV in turn: short, so that whichever becomes ready first is issued.
-constexpr uint32_t kMmaPollNs = 40;
+constexpr int ROWS_PER_PROD = KEYS / PROD_WARPS;
+constexpr int MLA_THREADS = 32 + SMX_WARPS * 32 + PROD_WARPS * 32;
+constexpr int SMX_T0 = 32;                     // first softmax thread
+constexpr int PROD_T0 = SMX_T0 + SMX_WARPS * 32;   // first producer thread
+static_assert(KEYS % PROD_WARPS == 0 && ROWS_PER_PROD <= 32, "rows per producer warp");
 
 template <int NKB, int DVC>
 struct MlaTraits {
@@ -55,8 +60,10 @@ struct MlaTraits {
   static constexpr int NB_B = DVC / 64;
   static constexpr int NB_A = NKB - NB_B;
   static constexpr int NP = PROD_WARPS * 32;
-  static constexpr int CPT_A = (KEYS * NB_A * 8 + NP - 1) / NP;   // chunks per thread, part A
-  static constexpr int CPT_B = (KEYS * NB_B * 8 + NP - 1) / NP;   // chunks per thread, part B
+  // 16-byte chunks per producer lane and part: 8 rows x NB blocks x 8 chunks / 32
+  static constexpr int CPL_A = ROWS_PER_PROD * NB_A * 8 / 32;
+  static constexpr int CPL_B = ROWS_PER_PROD * NB_B * 8 / 32;
+  static_assert(ROWS_PER_PROD * NB_A * 8 % 32 == 0 && ROWS_PER_PROD * NB_B * 8 % 32 == 0, "chunks");
   static_assert(NB_A >= 1 && NB_B >= 1, "both parts must be non-empty");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + QS_KB * QBLK;
@@ -69,9 +76,14 @@ struct MlaTraits {
   static constexpr int BAR_S_FULL = BAR_KV_EMPTY + 2 * STAGES;   // [2] S buffer computed
   static constexpr int BAR_P_FULL = BAR_S_FULL + 2;   // [2] P written over its S buffer
   static constexpr int BAR_PV_DONE = BAR_P_FULL + 2;  // [2] PV of a tile of that parity done
-  static constexpr int BAR_DONE = BAR_PV_DONE + 2;
+  static constexpr int BAR_XMAX = BAR_PV_DONE + 2;    // [2] both halves' tile maxima written
+  static constexpr int BAR_XL = BAR_XMAX + 2;         // both halves' sums written (end)
+  static constexpr int BAR_DONE = BAR_XL + 1;
   static constexpr int NUM_BARS = BAR_DONE + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  // exchange area of the two softmax halves: tile maxima as bf16 [2 tiles][2 halves]
+  // [128 heads], and at the end the row sums as fp32 [2 halves][128 heads]
+  static constexpr int OFF_XMAX = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_MISC = OFF_XMAX + 2 * 2 * 128 * 2;
   static constexpr int SMEM_BYTES = OFF_MISC + 48 + 1024;
   // TMEM columns: O [0, DVC), two S buffers [DVC, DVC + 2 KEYS) (P_i, bf16, is
   // written over the first KEYS / 2 columns of S_i's buffer), Q part after them
@@ -84,6 +96,7 @@ struct MlaTraits {
   // PV: A = P from TMEM, B = values MN-major
   static constexpr uint32_t IDESC_PV = make_idesc(1, 1, 0, 1, DVC, 128);
   static_assert(DVC % 64 == 0 && DVC <= 256, "DVC");
+  static_assert(QT_KB % 2 == 0 || QT_KB == 1, "Q blocks in TMEM split over the two halves");
   static_assert(COLS_USED <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -95,8 +108,7 @@ struct MlaTraits {
 // constants: Q's first QT_KB column blocks are read from TMEM, the rest from
 // shared memory. Issue from a fully unrolled sequence costs about as much as
 // the MMAs take to run; the same sequence built from a runtime block index
-// costs up to twice as much per MMA, and so does a part split into shorter
-// sequences with other work between them.
+// costs up to twice as much per MMA.
 template <int NKB, int DVC, int DVCI, int PART>
 __device__ __forceinline__ void issue_s_part(uint32_t s_tmem, uint32_t qt_tmem, uint64_t qd0, uint64_t kd0) {
   using Tr = MlaTraits<NKB, DVC>;
@@ -117,6 +129,103 @@ __device__ __forceinline__ void issue_s_part(uint32_t s_tmem, uint32_t qt_tmem, 
                    Tr::IDESC_S, acc);
     }
   }
+}
+
+// PV for one tile: O += P V, P = the bf16 probabilities over the first KEYS / 2
+// columns of the tile's S buffer, V = this CTA's value blocks of the stage (bd0).
+template <int NKB, int DVC>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t pt, uint64_t bd0, bool first) {
+  using Tr = MlaTraits<NKB, DVC>;
+#pragma unroll
+  for (int kk = 0; kk < KEYS / 16; ++kk)
+    mma_f16_ts(o_tmem, pt + kk * 8, bd0 + (uint64_t)(kk * 16 * 128 >> 4), Tr::IDESC_PV,
+               (!first || kk > 0) ? 1u : 0u);
+}
+
+// The issuer's loop over the CTA's tiles, for output-column slice DVCI. Per tile
+// i, in this order: part A of S_i (its stage's part-A blocks have landed; its S
+// buffer was last read by PV_{i-2}, issued before), then PV_{i-1} if P_{i-1} is
+// already written, part B of S_i once the value blocks have landed, and PV_{i-1}
+// if it was not issued yet. The tensor pipe runs MMAs in issue order, which
+// orders every buffer reuse. Returns false if a wait gave up.
+template <int NKB, int DVC, int DVCI>
+__device__ __noinline__ bool mla_issue_tiles(int ntiles, uint32_t tbase, uint32_t kv_base, uint64_t qd0,
+                                             uint64_t* bars, const DevCtl& ctl, volatile int* abort_flag) {
+  using Tr = MlaTraits<NKB, DVC>;
+  uint64_t* kvA_full = bars + Tr::BAR_KV_FULL;
+  uint64_t* kvB_full = bars + Tr::BAR_KV_FULL + Tr::STAGES;
+  uint64_t* kvA_empty = bars + Tr::BAR_KV_EMPTY;
+  uint64_t* kvB_empty = bars + Tr::BAR_KV_EMPTY + Tr::STAGES;
+  uint64_t* s_full = bars + Tr::BAR_S_FULL;
+  uint64_t* p_full = bars + Tr::BAR_P_FULL;
+  uint64_t* pv_done = bars + Tr::BAR_PV_DONE;
+  const uint32_t o_tmem = tbase, s_tmem = tbase + Tr::COL_S, qt_tmem = tbase + Tr::COL_Q;
+  // stage descriptors: K-major for S, and this slice's value blocks MN-major for PV
+  const uint64_t kd[2] = {make_sdesc(kv_base, 16, 1024, 2),
+                          make_sdesc(kv_base + NKB * Tr::KVBLK, 16, 1024, 2)};
+  constexpr uint32_t v_off = (uint32_t)(DVCI * Tr::NB_B) * Tr::KVBLK;
+  const uint64_t bd[2] = {make_sdesc(kv_base + v_off, Tr::KVBLK, 1024, 2),
+                          make_sdesc(kv_base + NKB * Tr::KVBLK + v_off, Tr::KVBLK, 1024, 2)};
+  auto pv = [&](int j) {
+    issue_pv<NKB, DVC>(o_tmem, s_tmem + (uint32_t)((j & 1) * KEYS), bd[j & 1], j == 0);
+    mma_commit(&kvB_empty[j & 1]);
+    mma_commit(&pv_done[j & 1]);
+  };
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i & 1;   // STAGES == 2
+    const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+    const uint32_t sb = s_tmem + (uint32_t)(st * KEYS);
+    if (!mbar_wait(&kvA_full[st], ph, ctl, abort_flag, kSiteMla, 3)) return false;
+    tc_fence_after();
+    issue_s_part<NKB, DVC, DVCI, 0>(sb, qt_tmem, qd0, kd[st]);
+    mma_commit(&kvA_empty[st]);
+    bool pv_pending = i > 0;
+    if (pv_pending && mbar_test_wait(smem_u32(&p_full[(i - 1) & 1]), (uint32_t)((i - 1) >> 1) & 1u)) {
+      tc_fence_after();
+      pv(i - 1);
+      pv_pending = false;
+    }
+    if (!mbar_wait(&kvB_full[st], ph, ctl, abort_flag, kSiteMla, 4)) return false;
+    tc_fence_after();
+    issue_s_part<NKB, DVC, DVCI, 1>(sb, qt_tmem, qd0, kd[st]);
+    mma_commit(&s_full[st]);
+    if (pv_pending) {
+      if (!mbar_wait(&p_full[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, ctl, abort_flag, kSiteMla, 5))
+        return false;
+      tc_fence_after();
+      pv(i - 1);
+    }
+  }
+  if (ntiles > 0) {
+    const int j = ntiles - 1;
+    if (!mbar_wait(&p_full[j & 1], (uint32_t)(j >> 1) & 1u, ctl, abort_flag, kSiteMla, 6)) return false;
+    tc_fence_after();
+    pv(j);
+  }
+  return true;
+}
+
+// The smallest bf16 value >= x (x not NaN), as its bit pattern. Both softmax
+// halves of a head derive the running max from the same two such values, so they
+// agree on it exactly; an upper bound of the tile max serves the online softmax as
+// well as the max itself (P and the row sum use the same reference).
+__device__ __forceinline__ uint16_t bf16_at_least(float x) {
+  const uint32_t u = __float_as_uint(x);
+  uint32_t hi = u >> 16;
+  if ((u & 0xffffu) != 0u && (u & 0x80000000u) == 0u) ++hi;   // positive: round up
+  return (uint16_t)hi;                                         // negative: truncation rounds up
+}
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+
+// 16 consecutive 32-bit TMEM columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
 }
 
 // PAGED: latent rows are gathered through the block table (pool rows); the
@@ -141,12 +250,18 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   uint64_t* s_full = bars + Tr::BAR_S_FULL;     // [2] S_i computed (buffer i % 2)
   uint64_t* p_full = bars + Tr::BAR_P_FULL;     // [2] P_i written over S_i
   uint64_t* pv_done = bars + Tr::BAR_PV_DONE;   // [2] PV_i done (tile parity)
+  uint64_t* xmax_bar = bars + Tr::BAR_XMAX;     // [2] tile maxima of both halves written
+  uint64_t* xl_bar = bars + Tr::BAR_XL;         // row sums of both halves written
   uint64_t* done_bar = bars + Tr::BAR_DONE;
+  uint16_t* xmax = reinterpret_cast<uint16_t*>(smem + Tr::OFF_XMAX);   // [tile parity][half][head]
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Tr::OFF_MISC);
   uint32_t* tmem_slot = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* ntiles_slot = reinterpret_cast<volatile int*>(misc + 2);   // [2]
-  volatile uint32_t* masks = misc + 4;   // [STAGES][2]: valid-key bits of the tile in each stage
+  // valid-key bits of the tile in each stage: [STAGES][8 producer warps] bytes, read
+  // as [STAGES][2] 32-key words
+  volatile uint8_t* mask8 = reinterpret_cast<volatile uint8_t*>(misc + 4);
+  const volatile uint32_t* masks = misc + 4;
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -160,7 +275,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
 
   // Warm L2 for the Q and index rows of the CTA that will probably run next on
   // this SM (one wave of block indices further on): its prologue waits on them.
-  if (warp == 5 && lane == 0) {
+  if (warp == PROD_T0 / 32 && lane == 0) {
     const long long nb = (long long)blockIdx.x + a.wave;
     if (nb < (long long)gridDim.x) {
       const long long ntok = nb / per_token;
@@ -174,7 +289,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(qt_full, 128);
+    mbar_init(qt_full, SMX_WARPS * 32);
     for (int i = 0; i < Tr::STAGES; ++i) {
       mbar_init(&kvA_full[i], Tr::NP);
       mbar_init(&kvB_full[i], Tr::NP);
@@ -183,9 +298,11 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], SMX_WARPS * 32);
       mbar_init(&pv_done[i], 1);
+      mbar_init(&xmax_bar[i], SMX_WARPS * 32);
     }
+    mbar_init(xl_bar, SMX_WARPS * 32);
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -228,7 +345,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         for (int kb = 0; kb < Tr::QS_KB; ++kb)
           tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, (Tr::QT_KB + kb) * 64, (int)(token * a.H),
                       q_full);
-        ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 3);
+        ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 1);
         if (!ok) {
           DevCtl drain = a.ctl;
           volatile int never = 0;
@@ -239,91 +356,13 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       // Descriptors are built once; per MMA only the start-address field moves
       // (byte offset / 16 added to the low bits, which never carry: smem < 256 KB).
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
-      const uint32_t v_off = (uint32_t)(dvc * (DVC / 64)) * Tr::KVBLK;
-      // Part `part` of S for tile i into buffer i % 2: the slice index selects
-      // one of the compile-time block orders (output columns are split in at
-      // most two slices). Part A ends by releasing its blocks, part B by handing
-      // S over.
-      auto issue_s = [&](int i, int part) {
-        const uint64_t kd0 = make_sdesc(smem_u32(kv_smem + (i % Tr::STAGES) * NKB * Tr::KVBLK), 16, 1024, 2);
-        const uint32_t sb = s_tmem + (uint32_t)((i & 1) * KEYS);
-        if (dvc == 0) {
-          if (part == 0) issue_s_part<NKB, DVC, 0, 0>(sb, qt_tmem, qd0, kd0);
-          else issue_s_part<NKB, DVC, 0, 1>(sb, qt_tmem, qd0, kd0);
-        } else {
-          if (part == 0) issue_s_part<NKB, DVC, 1, 0>(sb, qt_tmem, qd0, kd0);
-          else issue_s_part<NKB, DVC, 1, 1>(sb, qt_tmem, qd0, kd0);
-        }
-        mma_commit(part == 0 ? &kvA_empty[i % Tr::STAGES] : &s_full[i & 1]);
-      };
-      auto issue_pv = [&](int j) {
-        const int stj = j % Tr::STAGES;
-        const uint64_t bd0 = make_sdesc(smem_u32(kv_smem + stj * NKB * Tr::KVBLK) + v_off,
-                                        Tr::KVBLK, 1024, 2);
-        const uint32_t pt = s_tmem + (uint32_t)((j & 1) * KEYS);   // P_j: 16 keys per 8 columns
-#pragma unroll
-        for (int kk = 0; kk < KEYS / 16; ++kk)
-          mma_f16_ts(o_tmem, pt + kk * 8, bd0 + (uint64_t)(kk * 16 * 128 >> 4), Tr::IDESC_PV,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kvB_empty[stj]);
-        mma_commit(&pv_done[j & 1]);
-      };
-      // Issue S_i and PV_j in whichever order their inputs become ready, a ready
-      // PV first: S_i needs part A of tile i in shared memory and its TMEM buffer
-      // free, which it is once PV_{i-2} (the reader of P_{i-2}, written over the
-      // same buffer) has been issued: the tensor pipe runs the MMAs in order.
-      // Then part B. PV_j needs P_j. The barriers are tested without blocking;
-      // only when nothing is ready does the thread sleep briefly. Bounded like
-      // every other wait.
-      int ns = 0, npv = 0, spart = 0;
-      uint64_t t_mark = globaltimer_ns();
-      uint32_t spins = 0;
-      while (ok && npv < ntiles) {
-        bool did = false;
-        if (npv < ns && mbar_test_wait(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1)) {
-          tc_fence_after();
-          issue_pv(npv);
-          ++npv;
-          did = true;
-        }
-        if (ns < ntiles) {
-          const int st = ns % Tr::STAGES;
-          const uint32_t ph = (ns / Tr::STAGES) & 1;
-          const bool ready = spart == 0 ? npv >= ns - 1 && mbar_test_wait(smem_u32(&kvA_full[st]), ph)
-                                        : mbar_test_wait(smem_u32(&kvB_full[st]), ph);
-          if (ready) {
-            tc_fence_after();
-            issue_s(ns, spart);
-            if (spart) ++ns;
-            spart ^= 1;
-            did = true;
-          }
-        }
-        if (did) {
-          spins = 0;
-          t_mark = globaltimer_ns();
-          continue;
-        }
-        // nothing ready: sleep briefly on the barrier S waits for (else P's)
-        const int st_n = ns % Tr::STAGES;
-        const uint32_t ph_n = (ns / Tr::STAGES) & 1;
-        if (ns < ntiles && spart == 1)
-          mbar_try_wait_for(smem_u32(&kvB_full[st_n]), ph_n, kMmaPollNs);
-        else if (ns < ntiles && npv >= ns - 1)
-          mbar_try_wait_for(smem_u32(&kvA_full[st_n]), ph_n, kMmaPollNs);
+      if (ok && ntiles > 0) {
+        if (Tr::NB_B * 2 <= NKB && dvc != 0)
+          ok = mla_issue_tiles<NKB, DVC, 1>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
         else
-          mbar_try_wait_for(smem_u32(&p_full[npv & 1]), (npv >> 1) & 1, kMmaPollNs);
-        if ((++spins & 63u) == 0) {
-          if (*abort_flag || *reinterpret_cast<volatile int*>(a.ctl.status) != 0) {
-            *abort_flag = 1;
-            ok = false;
-          } else if (globaltimer_ns() - t_mark > a.ctl.wait_ns) {
-            report_timeout(a.ctl, kSiteMla, 4);
-            *abort_flag = 1;
-            ok = false;
-          }
-        }
+          ok = mla_issue_tiles<NKB, DVC, 0>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
       }
+      if (!ok) *abort_flag = 1;
       mma_commit(done_bar);
       DevCtl drain = a.ctl;
       volatile int never = 0;
@@ -331,94 +370,95 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     }
   } else if (warp >= PROD_T0 / 32) {
     // ------------------------------------------------ gather producers
-    // Chunk c of a part is 16 bytes: row r = c / (8 NB), then column block j and
-    // 16-byte chunk q8 within it. It lands in the 128-byte-swizzled K-major layout
-    // the tensor core reads: column block kb, row r, 16-byte slot q8 ^ (r % 8).
-    // Chunks past the end of a row (padding up to the 64-column block) are zeros.
-    // Once its copies of a part have landed, a thread makes them visible to the
-    // tensor core (proxy fence) and arrives on that part's full barrier.
-    const int ptid = threadIdx.x - PROD_T0;
+    // Producer warp pw owns rows 8 pw .. 8 pw + 7 of every tile. Lanes 0..7 load
+    // the rows' indices once per tile; the row offsets are broadcast by shuffle.
+    // A part's chunks are 16 bytes: chunk q of the warp = row q / (8 NB), column
+    // block q / 8 % NB of the part, 16-byte slot q % 8; consecutive lanes copy
+    // consecutive 16 bytes of a row. A chunk lands in the 128-byte-swizzled
+    // K-major layout the tensor core reads: column block kb, row r, 16-byte slot
+    // q8 ^ (r % 8). Chunks past the end of a row (padding up to the 64-column
+    // block) are zeros. Once its copies of a part have landed, a thread makes them
+    // visible to the tensor core (proxy fence) and arrives on that part's full
+    // barrier.
+    const int pw = warp - PROD_T0 / 32;
     const int row_bytes = a.Dqk * 2;
     const uint8_t* kv_g = reinterpret_cast<const uint8_t*>(kv);
     const uint8_t* kv_b = kv_g + (size_t)b * a.Lk * row_bytes;   // unpaged: sequence b's rows
     const uint32_t kv_base = smem_u32(kv_smem);
     const int vb0 = dvc * Tr::NB_B;
-    // copy this thread's chunks of one part of tile i into its stage
-    auto gather_part = [&](int i, auto part_c) {
+    auto gather_part = [&](int i, const uint8_t* src_row, auto part_c) {
       constexpr int PART = decltype(part_c)::value;
       constexpr int NB = PART ? Tr::NB_B : Tr::NB_A;
-      constexpr int CPT = PART ? Tr::CPT_B : Tr::CPT_A;
+      constexpr int CPL = PART ? Tr::CPL_B : Tr::CPL_A;
       const uint32_t stage = kv_base + (i % Tr::STAGES) * NKB * Tr::KVBLK;
 #pragma unroll
-      for (int jj = 0; jj < CPT; ++jj) {
-        const int c = ptid + jj * Tr::NP;
-        if (c < KEYS * NB * 8) {
-          const int r = c / (NB * 8);
-          const int rem = c - r * NB * 8;
-          const int j = rem >> 3, q8 = rem & 7;
-          const int kb = PART ? vb0 + j : (j < vb0 ? j : j + Tr::NB_B);
-          const int q = kb * 8 + q8;                  // 16-byte chunk within the row
-          const int pos = (tile0 + i) * KEYS + r;
-          const int v = pos < a.k ? __ldg(idx_row + pos) : -1;
-          // invalid keys read row 0 and are masked later; paged: the key's pool row,
-          // and a page outside the pool reads pool row 0
-          const uint8_t* src;
-          if constexpr (PAGED) {
-            long long prow = (v >= 0 && v < a.Lk)
-                                 ? key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, b, a.Lk, v)
-                                 : 0;
-            if (prow < 0) prow = 0;
-            src = kv_g + (size_t)prow * row_bytes;
-          } else {
-            const int row = (v >= 0 && v < a.Lk) ? v : 0;
-            src = kv_b + (size_t)row * row_bytes;
-          }
-          const bool in_row = q * 16 < row_bytes;
-          cp_async16(stage + kb * Tr::KVBLK + r * 128 + ((q8 ^ (r & 7)) << 4),
-                     src + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
-        }
+      for (int jj = 0; jj < CPL; ++jj) {
+        const int q = lane + jj * 32;
+        const int rr = q / (NB * 8);             // row within the warp's 8
+        const int rem = q - rr * NB * 8;
+        const int j = rem >> 3, q8 = rem & 7;
+        const int kb = PART ? vb0 + j : (j < vb0 ? j : j + Tr::NB_B);
+        const int qc = kb * 8 + q8;               // 16-byte chunk within the row
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(src_row), rr));
+        const int r = pw * ROWS_PER_PROD + rr;
+        const bool in_row = qc * 16 < row_bytes;
+        cp_async16(stage + kb * Tr::KVBLK + r * 128 + ((q8 ^ (r & 7)) << 4), src + (in_row ? qc * 16 : 0),
+                   in_row ? 16u : 0u);
       }
       cp_async_commit();
     };
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
       const uint32_t ph = ((i / Tr::STAGES) & 1) ^ 1;
+      // this warp's rows: index, validity and source row (invalid keys read row 0
+      // and are masked later; paged: the key's pool row, a page outside the pool
+      // reads pool row 0)
+      const int pos = (tile0 + i) * KEYS + pw * ROWS_PER_PROD + lane;
+      int v = -1;
+      if (lane < ROWS_PER_PROD && pos < a.k) v = __ldg(idx_row + pos);
+      const bool valid = lane < ROWS_PER_PROD && v >= 0 && v < a.Lk;
+      const uint8_t* src_row;
+      if constexpr (PAGED) {
+        long long prow = valid ? key_row(a.block_table, a.max_blocks, a.page_size, a.num_pages, b, a.Lk, v) : 0;
+        if (prow < 0) prow = 0;
+        src_row = kv_g + (size_t)prow * row_bytes;
+      } else {
+        src_row = kv_b + (size_t)(valid ? v : 0) * row_bytes;
+      }
+      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
       // part A is free once S of the tile that last used this stage is done ...
-      if (!mbar_wait(&kvA_empty[st], ph, a.ctl, abort_flag, kSiteMla, 1)) break;
-      gather_part(i, std::integral_constant<int, 0>{});
+      if (!mbar_wait(&kvA_empty[st], ph, a.ctl, abort_flag, kSiteMla, 8)) break;
+      gather_part(i, src_row, std::integral_constant<int, 0>{});
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(&kvA_full[st]);
       // ... part B (the values) once PV of that tile is done
-      if (!mbar_wait(&kvB_empty[st], ph, a.ctl, abort_flag, kSiteMla, 14)) break;
-      gather_part(i, std::integral_constant<int, 1>{});
-      if (ptid < 32) {
-#pragma unroll
-        for (int hw = 0; hw < KEYS / 32; ++hw) {
-          const int pos = (tile0 + i) * KEYS + hw * 32 + lane;
-          const int vi = pos < a.k ? __ldg(idx_row + pos) : -1;
-          const unsigned m = __ballot_sync(0xffffffffu, vi >= 0 && vi < a.Lk);
-          if (ptid == 0) masks[st * 2 + hw] = m;   // slot free: PV of its previous tile is done
-        }
-      }
+      if (!mbar_wait(&kvB_empty[st], ph, a.ctl, abort_flag, kSiteMla, 9)) break;
+      gather_part(i, src_row, std::integral_constant<int, 1>{});
+      if (lane == 0) mask8[st * PROD_WARPS + pw] = (uint8_t)(vmask & ((1u << ROWS_PER_PROD) - 1u));
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(&kvB_full[st]);
     }
     cp_async_wait_all();
   } else {
-    // ------------------------------------------------ softmax / epilogue (warps 1..4)
-    const int quad = warp & 3;
-    const int h = quad * 32 + lane;  // head = TMEM lane
+    // ------------------------------------------------ softmax / epilogue (warps 1..8)
+    const int sw = warp - SMX_T0 / 32;       // 0 .. 7
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+    const int hf = sw / 4;                   // which 32 keys of each tile, which half of O
+    const int h = quad * 32 + lane;          // head = TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    constexpr int OCOLS = DVC / 2;           // O columns this thread rescales and writes
     // this head's first QT_KB * 64 query columns go to TMEM (the MMA's A operand:
-    // lane = head, 32-bit column = two consecutive bf16 of the row)
+    // lane = head, 32-bit column = two consecutive bf16 of the row); each half
+    // writes its share of the blocks
     if (ntiles > 0) {
       const long long qrow = token * a.H + h;
       const bool have = qrow < (long long)a.B * a.Lq * a.H;
       const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) + (have ? qrow : 0) * (long long)a.Dqk * 2;
 #pragma unroll 1
-      for (int kb = 0; kb < Tr::QT_KB; ++kb) {
+      for (int kb = hf; kb < Tr::QT_KB; kb += 2) {
         uint32_t qv[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -432,38 +472,43 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       mbar_arrive(qt_full);
     }
     float m_used = -INFINITY;  // running max (log2 domain) that P is relative to
-    float l = 0.f;
+    float l = 0.f;             // this thread's 32-key share of the row sum
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
-      if (!mbar_wait(&s_full[i & 1], (i >> 1) & 1, a.ctl, abort_flag, kSiteMla, 8)) { ok = false; break; }
-      if (!mbar_wait(&kvB_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 9)) { ok = false; break; }
+      if (!mbar_wait(&s_full[i & 1], (i >> 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
+      if (!mbar_wait(&kvB_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 11)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sbuf = s_tmem + (uint32_t)((i & 1) * KEYS) + lane_off;   // this head's S_i
-      float x[KEYS];
+      uint32_t r[32];
+      tmem_ld32(sbuf + hf * 32, r);
+      tmem_wait_ld();
+      const uint32_t m = masks[st * 2 + hf];
+      float x[32];
       float tmax = -INFINITY;
 #pragma unroll
-      for (int hw = 0; hw < KEYS / 32; ++hw) {
-        uint32_t r[32];
-        tmem_ld32(sbuf + hw * 32, r);
-        tmem_wait_ld();
-        const uint32_t m = masks[st * 2 + hw];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          x[hw * 32 + j] = ((m >> j) & 1u) ? __uint_as_float(r[j]) * a.scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, x[hw * 32 + j]);
-        }
+      for (int j = 0; j < 32; ++j) {
+        x[j] = ((m >> j) & 1u) ? __uint_as_float(r[j]) * a.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, x[j]);
       }
+      // both halves' maxima: S_i has been read into registers by both threads of
+      // the head once this barrier completes, so P may be written over it
+      volatile uint16_t* xm = xmax + (i & 1) * 256;
+      const uint16_t mine = bf16_at_least(tmax);
+      xm[hf * 128 + h] = mine;
+      mbar_arrive(&xmax_bar[i & 1]);
+      if (!mbar_wait(&xmax_bar[i & 1], (i >> 1) & 1, a.ctl, abort_flag, kSiteMla, 13)) { ok = false; break; }
+      tmax = fmaxf(bf16_bits_to_float(mine), bf16_bits_to_float(xm[(hf ^ 1) * 128 + h]));
       const bool grow = tmax > m_used + 8.0f;
       const float m_new = grow ? tmax : m_used;
       const bool need_o = grow && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
         // O is rescaled in place: PV_{i-1} (the last one issued) must be done
-        if (!mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
+        if (!mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 14)) { ok = false; break; }
         tc_fence_after();
         const float alpha = need_o ? ex2(m_used - m_new) : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < DVC; c0 += 32) {
+        for (int c0 = hf * OCOLS; c0 < (hf + 1) * OCOLS; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(o_tmem + lane_off + c0, o);
           tmem_wait_ld();
@@ -475,10 +520,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         l *= alpha;
       }
       m_used = m_new;
-      uint32_t pk[KEYS / 2];
+      uint32_t pk[16];
       float psum0 = 0.f, psum1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < KEYS / 2; ++j) {
+      for (int j = 0; j < 16; ++j) {
         float p0 = ex2(x[2 * j] - m_used);
         float p1 = ex2(x[2 * j + 1] - m_used);
         if (m_used == -INFINITY) { p0 = 0.f; p1 = 0.f; }
@@ -487,16 +532,23 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         pk[j] = pack_bf16x2(p0, p1);
       }
       l += psum0 + psum1;
-      // P_i over the first half of S_i's buffer (S_i is in registers already;
-      // PV_{i-2}, the last reader of this buffer, finished before S_i did)
-      tmem_st32(sbuf, pk);
+      // P_i for this thread's 32 keys over columns 16 hf .. 16 hf + 15 of S_i's buffer
+      tmem_st16(sbuf + hf * 16, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[i & 1]);
     }
     if (ok && ntiles > 0) {
-      ok = mbar_wait(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 11);
+      ok = mbar_wait(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, a.ctl, abort_flag, kSiteMla, 15);
       tc_fence_after();
+    }
+    if (ok) {
+      // the head's row sum over both halves of every tile
+      volatile float* xl = reinterpret_cast<volatile float*>(xmax);   // the maxima are no longer read
+      xl[hf * 128 + h] = l;
+      mbar_arrive(xl_bar);
+      ok = mbar_wait(xl_bar, 0, a.ctl, abort_flag, kSiteMla, 16);
+      if (ok) l += xl[(hf ^ 1) * 128 + h];
     }
     if (ok) {
       const bool row_ok = h < a.H;
@@ -505,7 +557,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
         const float inv = empty ? 0.f : 1.f / l;
         uint16_t* orow = a.out + (token * a.H + h) * (long long)a.Dv + dvc * DVC;
 #pragma unroll 1
-        for (int c0 = 0; c0 < DVC; c0 += 32) {
+        for (int c0 = hf * OCOLS; c0 < (hf + 1) * OCOLS; c0 += 32) {
           uint32_t o[32];
           if (ntiles > 0) {
             tmem_ld32(o_tmem + lane_off + c0, o);
@@ -524,13 +576,13 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
             for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
           }
         }
-        if (row_ok && dvc == 0 && a.lse != nullptr)
+        if (row_ok && hf == 0 && dvc == 0 && a.lse != nullptr)
           a.lse[token * a.H + h] = empty ? -INFINITY : (m_used + __log2f(l)) * 0.69314718055994531f;
       } else {
         const long long prow_i = (token * a.splits + split) * a.H + h;
         float* po = a.part_o + prow_i * a.Dv + dvc * DVC;
 #pragma unroll 1
-        for (int c0 = 0; c0 < DVC; c0 += 32) {
+        for (int c0 = hf * OCOLS; c0 < (hf + 1) * OCOLS; c0 += 32) {
           uint32_t o[32];
           if (ntiles > 0) {
             tmem_ld32(o_tmem + lane_off + c0, o);
@@ -547,7 +599,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
                                   __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
           }
         }
-        if (row_ok && dvc == 0) {
+        if (row_ok && hf == 0 && dvc == 0) {
           a.part_ml[prow_i * 2 + 0] = empty ? -INFINITY : m_used;
           a.part_ml[prow_i * 2 + 1] = empty ? 0.f : l;
         }
