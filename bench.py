@@ -70,6 +70,8 @@ def work(cfg) -> dict:
              weights, and 4 per score written (the decode roofline: one query row
              per sequence makes it bandwidth-bound).
     topk     bytes = 4 per candidate score read + 4 * k per selected row written.
+    fused    indexer + top-k in one kernel: the indexer's flops (prefill); bytes =
+             key codes and scales once, queries and weights, 4 * k per row written.
     mla      flops = 2 * H * (Dqk + Dv) per (query row, selected key).
              bytes = 2 * Dqk per selected key + q, idx and out per row (decode).
     decode   bytes = indexer keys + scales + gathered latent rows + q, qI, w, out.
@@ -89,6 +91,10 @@ def work(cfg) -> dict:
         "indexer_bytes": float(cfg.B * min(cfg.Lk, cfg.q_pos0 + cfg.Lq) * (cfg.d_I + 4)
                                + tokens * cfg.H_I * (cfg.d_I + 4 + w_bytes) + 4.0 * pairs_idx),
         "topk_bytes": 4.0 * pairs_idx + 4.0 * cfg.k * rows_scored,
+        # fused indexer + top-k: its inputs once and the selected keys out (the scores
+        # stay in the L2-resident chunk between scoring and selection)
+        "fused_bytes": float(cfg.B * min(cfg.Lk, cfg.q_pos0 + cfg.Lq) * (cfg.d_I + 4)
+                             + tokens * cfg.H_I * (cfg.d_I + 4 + w_bytes) + 4.0 * cfg.k * tokens),
         "mla_flops": 2.0 * cfg.H * (cfg.Dqk + cfg.Dv) * sel,
         # attention bytes: each selected latent row once, q and idx in, out written
         "mla_bytes": float(sel * cfg.Dqk * 2 + tokens * (cfg.H * cfg.Dqk * 2 + 4 * cfg.k
@@ -239,6 +245,17 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     dsa.check_status()
     ms_local = e0.elapsed_time(e1) / steps
     ms = dist_max(ms_local, world)
+    # the fused indexer + top-k schedule (dsa_forward_fused), for comparison
+    ef0 = torch.cuda.Event(enable_timing=True)
+    ef1 = torch.cuda.Event(enable_timing=True)
+    dsa.forward(p, inp, out=out, ws=ws, fused=True)
+    ef0.record(stream)
+    for i in range(steps):
+        dsa.forward(p, inp, out=out, ws=ws, fused=True)
+    ef1.record(stream)
+    torch.cuda.synchronize()
+    dsa.check_status()
+    fused_ms = dist_max(ef0.elapsed_time(ef1) / steps, world)
     # per-kernel device time: the same steps again through dsa_forward_profiled,
     # which keeps every launch on the caller's stream (no top-k / indexer overlap)
     # so that the events around a launch time that launch alone
@@ -260,6 +277,19 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     fp8_peak = 2.0 * pk["bf16_sustained"]   # FP8 dense = 2 x bf16 dense (nominal ratio)
     roof = {}
     decode = cfg.mode == "decode"
+    if "indexer_topk" in kernels:
+        # fused indexer + top-k: the indexer's FP8 work (prefill), or its algorithmic
+        # bytes (decode: key codes and scales once, queries, selected keys written)
+        t = kernels["indexer_topk"]["ms_per_step"] * 1e-3
+        if decode:
+            a = w["fused_bytes"] / t / 1e9
+            roof["indexer_topk"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s",
+                                    "frac": a / pk["hbm"]}
+        else:
+            a = w["indexer_flops"] / t / 1e12
+            roof["indexer_topk"] = {"bound": "tensor", "achieved": a, "peak": fp8_peak,
+                                    "unit": "TFLOP/s", "frac": a / fp8_peak,
+                                    "peak_note": "fp8 = 2 x measured bf16 sustained"}
     if "indexer" in kernels:
         t = kernels["indexer"]["ms_per_step"] * 1e-3
         if decode:   # one query row per sequence: every key is read for 16 KFLOP
@@ -289,6 +319,8 @@ def time_workload(name: str, steps: int, warmup: int, world: int, rank: int, pk:
     for k, r in roof.items():
         r["traffic"] = traffic_per_launch(k, cfg.mode, cfg.B * cfg.Lq / kernels[k]["launches_per_step"])
     res = {"cfg": cfg, "ms": ms, "tokens_per_s": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, ms),
+           "fused": {"entry": "dsa_forward_fused", "ms_per_step": fused_ms,
+                     "value": aggregate_tokens_per_s(cfg.B * cfg.Lq, world, fused_ms)},
            "kernels": kernels,
            "roof": roof, "launches": timed_launches, "clocks": clocks, "work": w}
     if cfg.mode == "decode":
@@ -725,6 +757,7 @@ def main():
                         for k, v in pre["kernels"].items()},
             "gpu_launches": pre["launches"],
             "clocks": pre["clocks"],
+            "fused_schedule": pre["fused"],
         }
         if "e2e" in pre:
             line["e2e"] = pre["e2e"]
@@ -736,6 +769,7 @@ def main():
                 "kernels": {k: {**v, **({"roofline": dec["roof"][k]} if k in dec["roof"] else {})}
                             for k, v in dec["kernels"].items()},
                 "gpu_launches": dec["launches"],
+                "fused_schedule": dec["fused"],
                 "config": {"batch": dc.B, "cached_tokens": dc.Lk, "topk": dc.k},
             }
         if kl is not None:

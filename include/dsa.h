@@ -293,6 +293,10 @@ typedef struct dsa_tensors {
   uint16_t* out;    /* [B, Lq, H, Dv] bf16 */
   float* lse;       /* [B, Lq, H] fp32, optional (NULL) */
   int32_t* idx_out; /* [B, Lq, k] int32, optional: the selected set */
+  float* sel_scores_out; /* [B, Lq, k] fp32, optional: the index score I[t, idx_out[t, j]]
+                            of every selected key, aligned with idx_out (0 at the -1
+                            padding); what dsa_indexer_kl takes as sel_scores. When
+                            given, rows with p + 1 <= k are scored too. Needs idx_out. */
 } dsa_tensors;
 
 /* Bytes of workspace dsa_forward needs for problem p (scores are streamed in
@@ -300,15 +304,30 @@ typedef struct dsa_tensors {
 size_t dsa_forward_workspace_size(const dsa_problem* p);
 
 /*
- * dsa_forward - the fused hot path: indexer -> top-k -> sparse MLA, for prefill
+ * dsa_forward - the hot path: indexer -> top-k -> sparse MLA, for prefill
  * (q_pos0 = 0) and decode (q_pos0 = Lk - Lq). Query rows with p + 1 <= k select
  * every causal key without scoring (the top-k of at most k candidates is all of
  * them). The score matrix is produced and consumed one query chunk at a time in
- * the workspace. Results equal dsa_indexer_scores + dsa_topk_select +
- * dsa_sparse_mla_fwd.
+ * the workspace (a chunk stays in L2): the indexer scores a half-chunk while the
+ * top-k of the previous one runs on a library-owned stream. Results equal
+ * dsa_indexer_scores + dsa_topk_select + dsa_sparse_mla_fwd.
  */
 int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
                 void* stream);
+
+/*
+ * dsa_forward_fused - dsa_forward with the top-k selection inside the indexer
+ * kernel: selector warps of each persistent indexer CTA pick a row's top-k from
+ * the score chunk (in L2) as soon as every piece of the row is scored, while the
+ * CTA's other warps score further rows. One cooperative launch per chunk (every
+ * CTA resident at once, so the waits between CTAs always end; they are bounded
+ * as well). Same arguments, workspace (dsa_forward_workspace_size) and results,
+ * bit for bit, as dsa_forward; sel_scores_out is supported. On B200 it is slower
+ * than dsa_forward: the few selector threads that fit beside the indexer's warps
+ * take longer to select than the separate top-k kernel needs.
+ */
+int dsa_forward_fused(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                      void* stream);
 
 /*
  * Paged, variable-length caches (a serving layout; the pages describe the method
@@ -369,6 +388,7 @@ int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_te
 #define DSA_KIND_TOPK 2
 #define DSA_KIND_SPARSE_MLA 3
 #define DSA_KIND_COMBINE 4
+#define DSA_KIND_INDEXER_TOPK 5   /* the fused indexer + top-k launch */
 
 /*
  * dsa_forward_profiled - dsa_forward that also records a CUDA event around each

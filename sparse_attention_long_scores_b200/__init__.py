@@ -40,10 +40,10 @@ EXPORTED = [
     "dsa_forward", "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status",
     "dsa_set_wait_limit_ns", "dsa_debug_wait_timeout", "dsa_sparse_mla_fwd_noalloc",
     "dsa_indexer_kl", "dsa_last_launch_count", "dsa_forward_paged_workspace_size",
-    "dsa_forward_paged", "dsa_sparse_mla_bwd_workspace_size", "dsa_sparse_mla_bwd",
+    "dsa_forward_paged", "dsa_forward_fused", "dsa_sparse_mla_bwd_workspace_size", "dsa_sparse_mla_bwd",
     "dsa_indexer_kl_grad", "dsa_indexer_bwd_workspace_size", "dsa_indexer_bwd",
 ]
-KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine"}
+KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine", 5: "indexer_topk"}
 
 
 class DsaError(RuntimeError):
@@ -62,7 +62,8 @@ class DsaProblem(ctypes.Structure):
 
 class DsaTensors(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("qI", "qI_scale", "kI", "kI_scale", "w", "q", "kv", "out", "lse", "idx_out")]
+                ("qI", "qI_scale", "kI", "kI_scale", "w", "q", "kv", "out", "lse", "idx_out",
+                 "sel_scores_out")]
 
 
 class DsaPagedCache(ctypes.Structure):
@@ -99,6 +100,7 @@ def lib() -> ctypes.CDLL:
     L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
     L.dsa_forward_workspace_size.restype = sz
     L.dsa_forward.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp, sz, vp]
+    L.dsa_forward_fused.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors), vp, sz, vp]
     L.dsa_forward_paged_workspace_size.argtypes = [ctypes.POINTER(DsaProblem)]
     L.dsa_forward_paged_workspace_size.restype = sz
     L.dsa_forward_paged.argtypes = [ctypes.POINTER(DsaProblem), ctypes.POINTER(DsaTensors),
@@ -380,10 +382,10 @@ def forward_workspace_size(p: Problem) -> int:
     return n
 
 
-def _tensors(inp: dict, out, lse, idx_out) -> DsaTensors:
+def _tensors(inp: dict, out, lse, idx_out, sel_scores=None) -> DsaTensors:
     return DsaTensors(*[None if x is None else x.data_ptr() for x in (
         inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"], inp["q"], inp["kv"],
-        out, lse, idx_out)])
+        out, lse, idx_out, sel_scores)])
 
 
 def _need_inputs(p: "Problem", inp: dict, prefix: str = "", cuda: bool = True) -> None:
@@ -398,11 +400,14 @@ def _need_inputs(p: "Problem", inp: dict, prefix: str = "", cuda: bool = True) -
     _need(inp["kv"], prefix + "kv", torch.bfloat16, (p.B, p.Lk, p.Dqk), cuda)
 
 
-def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, stream=None):
+def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, stream=None,
+            sel_scores=None, fused: bool = False):
     """Whole DSA forward (indexer -> top-k -> sparse MLA) on device tensors.
 
     inp: dict with qI, qI_scale, kI, kI_scale, w, q, kv (see ``dsa_inputs.gen_inputs``).
-    Returns out [B, Lq, H, Dv] bf16 (lse / idx_out are filled when given).
+    Returns out [B, Lq, H, Dv] bf16 (lse / idx_out are filled when given; sel_scores
+    [B, Lq, k] fp32 receives the index score of every selected key and needs idx_out).
+    fused: run dsa_forward_fused (top-k selection inside the indexer kernel).
     """
     dev = inp["q"].device
     _need_inputs(p, inp)
@@ -413,12 +418,15 @@ def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, st
         _need(lse, "lse", torch.float32, (p.B, p.Lq, p.H))
     if idx_out is not None:
         _need(idx_out, "idx_out", torch.int32, (p.B, p.Lq, p.k))
+    if sel_scores is not None:
+        _need(sel_scores, "sel_scores", torch.float32, (p.B, p.Lq, p.k))
     if ws is None:
         ws = torch.empty(forward_workspace_size(p), dtype=torch.uint8, device=dev)
     cp = p.c()
-    ct = _tensors(inp, out, lse, idx_out)
-    _check(lib().dsa_forward(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws),
-                             ws.numel() * ws.element_size(), _stream(stream)))
+    ct = _tensors(inp, out, lse, idx_out, sel_scores)
+    entry = lib().dsa_forward_fused if fused else lib().dsa_forward
+    _check(entry(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws), ws.numel() * ws.element_size(),
+                 _stream(stream)))
     return out
 
 
@@ -428,7 +436,7 @@ def forward_paged_workspace_size(p: Problem) -> int:
 
 
 def forward_paged(p: Problem, inp: dict, block_table, seq_lens, page_size: int, out=None,
-                  lse=None, idx_out=None, ws=None, stream=None):
+                  lse=None, idx_out=None, ws=None, stream=None, sel_scores=None):
     """dsa_forward over a paged cache with per-sequence lengths.
 
     inp: qI, qI_scale, w, q as for ``forward`` ([B, Lq, ...]); kv, kI, kI_scale are
@@ -447,7 +455,7 @@ def forward_paged(p: Problem, inp: dict, block_table, seq_lens, page_size: int, 
     if ws is None:
         ws = torch.empty(forward_paged_workspace_size(p), dtype=torch.uint8, device=dev)
     cp = p.c()
-    ct = _tensors(inp, out, lse, idx_out)
+    ct = _tensors(inp, out, lse, idx_out, sel_scores)
     cc = DsaPagedCache(block_table.data_ptr(), seq_lens.data_ptr(), max_blocks, page_size,
                        rows // page_size)
     _check(lib().dsa_forward_paged(ctypes.byref(cp), ctypes.byref(ct), ctypes.byref(cc), _ptr(ws),

@@ -295,52 +295,66 @@ int run_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, uint16_t*
 struct ForwardPlan {
   int chunk;         // query rows per chunk
   long long ld;      // score row stride (floats)
-  size_t scores_bytes, idx_bytes, mla_bytes, total;
+  size_t scores_bytes, idx_bytes, cnt_bytes, mla_bytes, total;
 };
 
-ForwardPlan plan_forward(const dsa_problem* p, bool need_idx, size_t ws_bytes_or_zero) {
+// Rows of problem p that are scored: those with p + 1 > k, or every row when the
+// selected scores are returned.
+int first_scored_row(const dsa_problem* p, bool score_all) {
+  if (score_all) return 0;
+  const int f = p->k - p->q_pos0;
+  return f < 0 ? 0 : f;
+}
+
+// Workspace, in order: a score chunk of B x chunk x round4(Lk) fp32, the selected
+// keys (when the caller does not want them back), one counter per row of a chunk
+// (pieces scored, for the fused selection), and the attention's split partials.
+ForwardPlan plan_forward(const dsa_problem* p, bool need_idx, size_t ws_bytes_or_zero,
+                         bool score_all = false) {
   ForwardPlan f{};
   f.ld = (long long)align_up((size_t)p->Lk, 4);
   const size_t row_bytes = (size_t)p->B * f.ld * sizeof(float);
   f.idx_bytes = need_idx ? align_up((size_t)p->B * p->Lq * p->k * sizeof(int32_t), 256) : 0;
   f.mla_bytes = align_up(mla_ws_bytes(p->B, p->Lq, p->H, p->Dv,
                                       mla_splits(p->B, p->Lq, p->Dv, p->k, assumed_sms())), 256);
-  // Rows that need scores are those with q_pos0 + t + 1 > k.
-  int first_scored = p->k - p->q_pos0;
-  if (first_scored < 0) first_scored = 0;
-  int scored_rows = p->Lq - first_scored;
+  const int scored_rows = p->Lq - first_scored_row(p, score_all);
   if (scored_rows <= 0) {
     f.chunk = p->Lq;
     f.scores_bytes = 0;
   } else {
     // default: about 64 MB of scores per chunk so one chunk stays in L2
     long long c = (64ll << 20) / (long long)row_bytes;
-    if (ws_bytes_or_zero) {
-      size_t fixed = f.idx_bytes + f.mla_bytes;
-      long long avail = ws_bytes_or_zero > fixed + 256
-                            ? (long long)((ws_bytes_or_zero - fixed - 256) / row_bytes) : 0;
-      c = avail;
-    }
     if (c > scored_rows) c = scored_rows;
     if (c >= 4) c &= ~3ll;
-    if (c < 1) c = 0;
-    if (!ws_bytes_or_zero && c < 4) c = scored_rows < 4 ? scored_rows : 4;
+    if (c < 4) c = scored_rows < 4 ? scored_rows : 4;
+    if (ws_bytes_or_zero) {
+      // as many rows as the given workspace holds (scores and counters), down to 1
+      auto total_for = [&](long long rows) {
+        return f.idx_bytes + f.mla_bytes + align_up((size_t)rows * row_bytes, 256) +
+               align_up((size_t)p->B * rows * sizeof(int), 256) + 256;
+      };
+      const size_t fixed = f.idx_bytes + f.mla_bytes;
+      c = ws_bytes_or_zero > fixed ? (long long)((ws_bytes_or_zero - fixed) / row_bytes) : 0;
+      if (c > scored_rows) c = scored_rows;
+      while (c > 0 && total_for(c) > ws_bytes_or_zero) --c;
+      if (c >= 4) c &= ~3ll;
+    }
     f.chunk = (int)c;
     f.scores_bytes = align_up((size_t)c * row_bytes, 256);
   }
-  f.total = f.scores_bytes + f.idx_bytes + f.mla_bytes + (f.scores_bytes ? 256 : 0);
+  f.cnt_bytes = align_up((size_t)p->B * (f.chunk > 0 ? f.chunk : 1) * sizeof(int), 256);
+  f.total = f.scores_bytes + f.idx_bytes + f.cnt_bytes + f.mla_bytes + (f.scores_bytes ? 256 : 0);
   return f;
 }
 
-// Smallest workspace dsa_forward accepts: the fixed parts plus score rows for
-// one chunk of min(4, scored rows) query rows.
-size_t min_forward_bytes(const dsa_problem* p, const ForwardPlan& f) {
-  int first_scored = p->k - p->q_pos0;
-  if (first_scored < 0) first_scored = 0;
-  int scored_rows = p->Lq - first_scored;
-  size_t rows = scored_rows <= 0 ? 0 : (size_t)(scored_rows < 4 ? scored_rows : 4);
-  if (rows == 0) return f.idx_bytes + f.mla_bytes;
-  return f.idx_bytes + f.mla_bytes + rows * (size_t)p->B * f.ld * sizeof(float) + 256;
+// Smallest workspace dsa_forward accepts: the fixed parts plus score rows and
+// counters for one chunk of min(4, scored rows) query rows.
+size_t min_forward_bytes(const dsa_problem* p, const ForwardPlan& f, bool score_all = false) {
+  const int scored_rows = p->Lq - first_scored_row(p, score_all);
+  const size_t rows = scored_rows <= 0 ? 0 : (size_t)(scored_rows < 4 ? scored_rows : 4);
+  if (rows == 0) return f.idx_bytes + f.mla_bytes + f.cnt_bytes;
+  return f.idx_bytes + f.mla_bytes + align_up(rows * (size_t)p->B * f.ld * sizeof(float), 256) +
+         align_up(rows * (size_t)p->B * sizeof(int), 256) + 256;
 }
 
 int validate_problem(const dsa_problem* p) {
@@ -373,13 +387,23 @@ int validate_tensors(const dsa_tensors* t) {
   return DSA_OK;
 }
 
+// Fused top-k selection of rows [t0, t1) of every sequence by the indexer launch.
+struct FusedSelect {
+  int k = 0;
+  int t0 = 0, t1 = 0;
+  int32_t* idx = nullptr;
+  float* sel_scores = nullptr;
+  int* row_cnt = nullptr;
+};
+
 int launch_indexer_rows(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
                         const float* kI_scale, const void* w, int w_dtype, float* scores,
                         long long sc_ld, long long sc_bstride, int sc_t0, int B, int Lq, int Lk,
                         int q_pos0, int H_I, int d_I, int t_lo, int t_hi, const dsa::DevCtl& ctl,
                         int num_sms, cudaStream_t stream, Recorder& rec = g_no_rec,
-                        const dsa_paged_cache* pc = nullptr) {
-  if (t_hi <= t_lo) return DSA_OK;
+                        const dsa_paged_cache* pc = nullptr, const FusedSelect* fs = nullptr) {
+  if (fs == nullptr && t_hi <= t_lo) return DSA_OK;
+  if (t_hi < t_lo) t_hi = t_lo;
   const int n_tok = (H_I == 64) ? ((t_hi - t_lo == 1) ? 1 : 4) : 64;
   CUtensorMap tq, tk;
   DSA_TRY(make_map_2d(&tq, qI, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)d_I,
@@ -409,13 +433,23 @@ int launch_indexer_rows(const uint8_t* qI, const float* qI_scale, const uint8_t*
     a.num_pages = pc->num_pages;
   }
   int keys_max = q_pos0 + t_hi < Lk ? q_pos0 + t_hi : Lk;
-  a.piece_keys = indexer_piece_keys(B, t_hi - t_lo, n_tok, keys_max, num_sms);
+  a.piece_keys = t_hi > t_lo ? indexer_piece_keys(B, t_hi - t_lo, n_tok, keys_max, num_sms) : 128;
   a.ctl = ctl;
-  {
-    NvtxRange r("dsa:indexer");
-    DSA_TRY_CUDA(dsa::launch_indexer(tq, tk, a, H_I, d_I, num_sms, stream), "indexer launch");
+  if (fs != nullptr) {
+    a.select = 1;
+    a.k = fs->k;
+    a.sel_t0 = fs->t0;
+    a.sel_t1 = fs->t1;
+    a.idx = fs->idx;
+    a.sel_scores = fs->sel_scores;
+    a.row_cnt = fs->row_cnt;
   }
-  DSA_TRY(rec.mark(DSA_KIND_INDEXER, stream));
+  {
+    NvtxRange r(fs != nullptr ? "dsa:indexer_topk" : "dsa:indexer");
+    DSA_TRY_CUDA(dsa::launch_indexer(tq, tk, a, H_I, d_I, num_sms, stream),
+                 fs != nullptr ? "indexer + top-k launch" : "indexer launch");
+  }
+  DSA_TRY(rec.mark(fs != nullptr ? DSA_KIND_INDEXER_TOPK : DSA_KIND_INDEXER, stream));
   return DSA_OK;
 }
 
@@ -596,7 +630,9 @@ int dsa_sparse_mla_fwd_noalloc(const uint16_t* q, const uint16_t* kv, const int3
 
 size_t dsa_forward_workspace_size(const dsa_problem* p) {
   if (validate_problem(p) != DSA_OK) return 0;
-  return plan_forward(p, true, 0).total;
+  // enough for either schedule: with sel_scores_out every row is scored
+  const size_t a = plan_forward(p, true, 0, false).total, b = plan_forward(p, true, 0, true).total;
+  return a > b ? a : b;
 }
 
 }  // extern "C"
@@ -669,13 +705,14 @@ int host_pipe(HostPipe** out) {
 
 dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld, int bstride,
                         int t0, int t1, int32_t* idx, const dsa::DevCtl& ctl,
-                        const dsa_paged_cache* pc) {
+                        const dsa_paged_cache* pc, float* sel_scores = nullptr) {
   dsa::TopkArgs ta{};
   ta.scores = scores;
   ta.sc_ld = ld;
   ta.sc_bstride = bstride;
   ta.sc_t0 = t0;
   ta.idx = idx;
+  ta.sel = sel_scores;
   ta.B = p->B; ta.Lq = p->Lq; ta.Lk = p->Lk; ta.q_pos0 = p->q_pos0; ta.k = p->k;
   ta.t_lo = t0; ta.t_hi = t1;
   ta.vec4 = 1;
@@ -684,88 +721,137 @@ dsa::TopkArgs topk_args(const dsa_problem* p, const float* scores, long long ld,
   return ta;
 }
 
+// fused: one cooperative indexer + top-k launch per score chunk (dsa_forward_fused);
+// otherwise the indexer scores a chunk and a separate top-k kernel selects it
+// (overlapped on a side stream: the indexer scores the next half-chunk meanwhile).
 int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
-                 void* stream, Recorder& rec, const dsa_paged_cache* pc = nullptr) {
+                 void* stream, Recorder& rec, const dsa_paged_cache* pc = nullptr,
+                 bool fused = false) {
   NvtxRange whole("dsa_forward");
   DSA_TRY(validate_problem(p));
   DSA_TRY(validate_tensors(t));
   DSA_TRY(check_ptr(ws, "ws", true));
   const bool need_idx = t->idx_out == nullptr;
-  ForwardPlan rec_plan = plan_forward(p, need_idx, 0);
-  const size_t min_bytes = min_forward_bytes(p, rec_plan);
+  const bool score_all = t->sel_scores_out != nullptr;
+  if (score_all && need_idx)
+    return fail(DSA_ERR_INVALID_ARG, "sel_scores_out needs idx_out (the scores are aligned with it)");
+  ForwardPlan rec_plan = plan_forward(p, need_idx, 0, score_all);
+  const size_t min_bytes = min_forward_bytes(p, rec_plan, score_all);
   if (ws_bytes < min_bytes)
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL,
                 "dsa_forward workspace: need at least %zu bytes (recommended %zu), got %zu",
                 min_bytes, rec_plan.total, ws_bytes);
   if (ws == nullptr) return fail(DSA_ERR_INVALID_ARG, "ws is NULL");
-  ForwardPlan f = plan_forward(p, need_idx, ws_bytes);
+  ForwardPlan f = plan_forward(p, need_idx, ws_bytes, score_all);
   dsa::DevCtl ctl;
   int sms = 0;
   DSA_TRY(device_ctl(ctl, sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   char* wsb = static_cast<char*>(ws);
-  float* scores = reinterpret_cast<float*>(wsb);
+  float* scores = f.scores_bytes ? reinterpret_cast<float*>(wsb) : nullptr;
   int32_t* idx = need_idx ? reinterpret_cast<int32_t*>(wsb + f.scores_bytes) : t->idx_out;
-  void* mla_ws = wsb + f.scores_bytes + f.idx_bytes;
+  int* row_cnt = reinterpret_cast<int*>(wsb + f.scores_bytes + f.idx_bytes);
+  void* mla_ws = wsb + f.scores_bytes + f.idx_bytes + f.cnt_bytes;
 
-  int first_scored = p->k - p->q_pos0;
-  if (first_scored < 0) first_scored = 0;
-  if (f.scores_bytes > 0 && (f.chunk < 1 || f.total > ws_bytes))
+  const int first_scored = first_scored_row(p, score_all);
+  if (first_scored < p->Lq && (f.chunk < 1 || f.scores_bytes == 0 || f.total > ws_bytes))
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "dsa_forward workspace: no room for one score row");
   const int C = f.chunk > 0 ? f.chunk : p->Lq;
-  // Overlapped schedule: the score area holds two half-size chunk buffers; the
-  // top-k of a chunk runs on the side stream while the indexer scores the next
-  // chunk into the other buffer (their CTAs fit on one SM together). The
-  // profiling entry point keeps the serial schedule so that each launch's events
-  // time that launch alone.
-  const int C2 = (C / 2) & ~3;
-  if (rec.events == nullptr && f.scores_bytes > 0 && C2 >= 4) {
-    SideStream* r = nullptr;
-    DSA_TRY(side_stream(&r));
-    std::lock_guard<std::mutex> lk(r->mu);
-    const size_t half = (size_t)p->B * C2 * (size_t)f.ld;   // floats per buffer
-    int c = 0;
-    for (int t0 = 0; t0 < p->Lq; t0 += C2, ++c) {
-      const int t1 = t0 + C2 < p->Lq ? t0 + C2 : p->Lq;
-      const int ts = t0 > first_scored ? t0 : first_scored;
-      const int b = c & 1;
-      float* sb = scores + b * half;
-      // the buffer's previous chunk must have been selected before it is rewritten
-      if (c >= 2) DSA_TRY_CUDA(cudaStreamWaitEvent(s, r->selected[b], 0), "cudaStreamWaitEvent");
-      if (ts < t1) {
-        DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, sb,
-                                    f.ld, C2, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
-                                    t1, ctl, sms, s, rec, pc));
-      }
-      DSA_TRY_CUDA(cudaEventRecord(r->scored[b], s), "cudaEventRecord");
-      DSA_TRY_CUDA(cudaStreamWaitEvent(r->side, r->scored[b], 0), "cudaStreamWaitEvent");
-      {
-        NvtxRange nr("dsa:topk");
-        DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl, pc), sms, r->side),
-                     "top-k launch");
-      }
-      DSA_TRY(rec.mark(DSA_KIND_TOPK, r->side));   // counts it (no events on this path)
-      DSA_TRY_CUDA(cudaEventRecord(r->selected[b], r->side), "cudaEventRecord");
+  // One fused indexer + top-k launch per chunk of C query rows: the chunk's scored
+  // rows are scored into the workspace and every row of the chunk is selected by
+  // the same kernel as soon as it is complete. The per-row piece counters start at
+  // zero and each launch leaves them at zero.
+  if (first_scored >= p->Lq) {
+    // Short context: every row has at most k candidates and selects all of them, so
+    // nothing is scored; one selection launch fills the index rows.
+    dsa::TopkArgs ta{};
+    ta.idx = idx;
+    ta.B = p->B; ta.Lq = p->Lq; ta.Lk = p->Lk; ta.q_pos0 = p->q_pos0; ta.k = p->k;
+    ta.t_lo = 0; ta.t_hi = p->Lq;
+    ta.seq_lens = pc != nullptr ? pc->seq_lens : nullptr;
+    ta.ctl = ctl;
+    {
+      NvtxRange nr("dsa:topk");
+      DSA_TRY_CUDA(dsa::launch_topk(ta, sms, s), "top-k launch");
     }
-    // top-k launches run in order on the side stream: the last one covers all
-    if (c >= 1) DSA_TRY_CUDA(cudaStreamWaitEvent(s, r->selected[(c - 1) & 1], 0), "cudaStreamWaitEvent");
-  } else {
-    for (int t0 = 0; t0 < p->Lq; t0 += C) {
-      const int t1 = t0 + C < p->Lq ? t0 + C : p->Lq;
-      const int ts = t0 > first_scored ? t0 : first_scored;
-      if (ts < t1) {
-        DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
-                                    f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
-                                    t1, ctl, sms, s, rec, pc));
+    DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
+    return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
+                   p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+  }
+  if (!fused) {
+    // Overlapped schedule: the score area holds two half-size chunk buffers; the
+    // top-k of a chunk runs on the side stream while the indexer scores the next
+    // chunk into the other buffer (their CTAs fit on one SM together). The
+    // profiling entry point keeps the serial schedule so that each launch's events
+    // time that launch alone.
+    const int C2 = (C / 2) & ~3;
+    if (rec.events == nullptr && f.scores_bytes > 0 && C2 >= 4) {
+      SideStream* r = nullptr;
+      DSA_TRY(side_stream(&r));
+      std::lock_guard<std::mutex> lk(r->mu);
+      const size_t half = (size_t)p->B * C2 * (size_t)f.ld;   // floats per buffer
+      int c = 0;
+      for (int t0 = 0; t0 < p->Lq; t0 += C2, ++c) {
+        const int t1 = t0 + C2 < p->Lq ? t0 + C2 : p->Lq;
+        const int ts = t0 > first_scored ? t0 : first_scored;
+        const int b = c & 1;
+        float* sb = scores + b * half;
+        // the buffer's previous chunk must have been selected before it is rewritten
+        if (c >= 2) DSA_TRY_CUDA(cudaStreamWaitEvent(s, r->selected[b], 0), "cudaStreamWaitEvent");
+        if (ts < t1) {
+          DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, sb,
+                                      f.ld, C2, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
+                                      t1, ctl, sms, s, rec, pc));
+        }
+        DSA_TRY_CUDA(cudaEventRecord(r->scored[b], s), "cudaEventRecord");
+        DSA_TRY_CUDA(cudaStreamWaitEvent(r->side, r->scored[b], 0), "cudaStreamWaitEvent");
+        {
+          NvtxRange nr("dsa:topk");
+          DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, sb, f.ld, C2, t0, t1, idx, ctl, pc, t->sel_scores_out),
+                                        sms, r->side),
+                       "top-k launch");
+        }
+        DSA_TRY(rec.mark(DSA_KIND_TOPK, r->side));   // counts it (no events on this path)
+        DSA_TRY_CUDA(cudaEventRecord(r->selected[b], r->side), "cudaEventRecord");
       }
-      {
-        NvtxRange nr("dsa:topk");
-        DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl, pc), sms, s),
-                     "top-k launch");
+      // top-k launches run in order on the side stream: the last one covers all
+      if (c >= 1) DSA_TRY_CUDA(cudaStreamWaitEvent(s, r->selected[(c - 1) & 1], 0), "cudaStreamWaitEvent");
+    } else {
+      for (int t0 = 0; t0 < p->Lq; t0 += C) {
+        const int t1 = t0 + C < p->Lq ? t0 + C : p->Lq;
+        const int ts = t0 > first_scored ? t0 : first_scored;
+        if (ts < t1) {
+          DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
+                                      f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
+                                      t1, ctl, sms, s, rec, pc));
+        }
+        {
+          NvtxRange nr("dsa:topk");
+          DSA_TRY_CUDA(dsa::launch_topk(topk_args(p, scores, f.ld, C, t0, t1, idx, ctl, pc, t->sel_scores_out),
+                                        sms, s),
+                       "top-k launch");
+        }
+        DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
       }
-      DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
     }
+    return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
+                   p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+  }
+  DSA_TRY_CUDA(cudaMemsetAsync(row_cnt, 0, f.cnt_bytes, s), "row counter clear");
+  FusedSelect fs;
+  fs.k = p->k;
+  fs.idx = idx;
+  fs.sel_scores = t->sel_scores_out;
+  fs.row_cnt = row_cnt;
+  for (int t0 = 0; t0 < p->Lq; t0 += C) {
+    const int t1 = t0 + C < p->Lq ? t0 + C : p->Lq;
+    const int ts = t0 > first_scored ? t0 : first_scored;
+    fs.t0 = t0;
+    fs.t1 = t1;
+    DSA_TRY(launch_indexer_rows(t->qI, t->qI_scale, t->kI, t->kI_scale, t->w, p->w_dtype, scores,
+                                f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
+                                ts < t1 ? t1 : ts, ctl, sms, s, rec, pc, &fs));
   }
   return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
                  p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
@@ -803,6 +889,14 @@ int dsa_forward(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_
                 void* stream) {
   Recorder none;
   const int rc = forward_impl(p, t, ws, ws_bytes, stream, none);
+  g_last_launches = none.launched;
+  return rc;
+}
+
+int dsa_forward_fused(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws_bytes,
+                      void* stream) {
+  Recorder none;
+  const int rc = forward_impl(p, t, ws, ws_bytes, stream, none, nullptr, /*fused=*/true);
   g_last_launches = none.launched;
   return rc;
 }
@@ -893,6 +987,8 @@ int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_te
     DSA_TRY(d2h(host->out, dev->out, 0, B * Lq * r_out, s));
     if (host->lse && dev->lse) DSA_TRY(d2h(host->lse, dev->lse, 0, B * Lq * r_lse, s));
     if (host->idx_out && dev->idx_out) DSA_TRY(d2h(host->idx_out, dev->idx_out, 0, B * Lq * r_idx, s));
+    if (host->sel_scores_out && dev->sel_scores_out)
+      DSA_TRY(d2h(host->sel_scores_out, dev->sel_scores_out, 0, B * Lq * r_idx, s));
     DSA_TRY_CUDA(cudaStreamSynchronize(s), "stream synchronize");
     g_last_launches = launched;
     return DSA_OK;
@@ -953,6 +1049,7 @@ int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_te
         st.out = dev->out + row0 * (size_t)p->H * p->Dv;
         st.lse = dev->lse ? dev->lse + row0 * p->H : nullptr;
         st.idx_out = dev->idx_out ? dev->idx_out + row0 * p->k : nullptr;
+        st.sel_scores_out = dev->sel_scores_out ? dev->sel_scores_out + row0 * p->k : nullptr;
         // at most the block's recommended workspace, so that its score chunks keep
         // the default size (a larger area would only make them spill out of L2)
         const size_t sub_rec = dsa_forward_workspace_size(&sp);
@@ -964,6 +1061,8 @@ int dsa_forward_host(const dsa_problem* p, const dsa_tensors* host, const dsa_te
         if (host->lse && dev->lse) DSA_TRY(d2h(host->lse, dev->lse, row0 * r_lse, nrow * r_lse, hpipe->out));
         if (host->idx_out && dev->idx_out)
           DSA_TRY(d2h(host->idx_out, dev->idx_out, row0 * r_idx, nrow * r_idx, hpipe->out));
+        if (host->sel_scores_out && dev->sel_scores_out)
+          DSA_TRY(d2h(host->sel_scores_out, dev->sel_scores_out, row0 * r_idx, nrow * r_idx, hpipe->out));
       }
     }
     return DSA_OK;

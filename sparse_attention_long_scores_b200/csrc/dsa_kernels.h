@@ -28,10 +28,21 @@ struct IndexerArgs {
   const int32_t* seq_lens;
   const int32_t* block_table;
   int max_blocks, page_size, num_pages;
+  // Fused top-k selection (select != 0): selector warps of the same kernel pick the
+  // k largest scores of every row of rows [sel_t0, sel_t1) of each sequence once all
+  // pieces of the row are scored (rows of at most k candidates select every key);
+  // the scored rows [t_lo, t_hi) lie inside that range.
+  int select;
+  int k;
+  int sel_t0, sel_t1;
+  int32_t* idx;          // [B, Lq, k] selected keys, ascending, -1 padded
+  float* sel_scores;     // [B, Lq, k] or null: the index score of each selected key (0 at padding)
+  int* row_cnt;          // [B * (sel_t1 - sel_t0)] pieces scored per row; zero on entry, left zero
   DevCtl ctl;
 };
 
-// Launch the tcgen05 FP8 indexer for (H_I, d_I) in {(4,32), (64,128)}.
+// Launch the tcgen05 FP8 indexer for (H_I, d_I) in {(4,32), (64,128)}. With
+// a.select set the launch is cooperative (every CTA resident at once).
 // `decode_like` selects the one-token-per-block variant (Lq == 1).
 cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                            const IndexerArgs& a, int H_I, int d_I, int num_sms,
@@ -52,6 +63,8 @@ struct TopkArgs {
   int t_lo, t_hi;  // rows [t_lo, t_hi) of every sequence
   int vec4;        // rows are 16-byte aligned (sc_ld % 4 == 0, aligned base)
   const int32_t* seq_lens;   // [B] or null: per-sequence lengths (row t at seq_lens[b] - Lq + t)
+  float* sel;      // [B, Lq, k] or null: score of each selected key (0 at padding); rows with
+                   // at most k candidates then read their scores too
   DevCtl ctl;
 };
 cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream);

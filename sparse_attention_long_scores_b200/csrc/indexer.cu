@@ -25,7 +25,191 @@
 namespace dsa {
 namespace {
 
-template <int D_I, int H_I, int N>
+// ---------------------------------------------------------------------------
+// Fused top-k: exact selection of the k largest scores of a row by a group of NT
+// selector threads (bar.sync 1 among them), reading the row from L2 where the
+// epilogue left it. Scores map to order-preserving 32-bit keys (-0.0 folded onto
+// +0.0); a three-digit radix select (11 + 11 + 10 bits, most significant first)
+// finds the exact k-th largest key T, each pass histogramming the keys that match
+// the prefix chosen so far; a final pass in index order writes every key > T and
+// the first (k - #{key > T}) keys == T, so ties go to the lowest index and the
+// output is ascending ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language
+// Models", bud-325 paper digest, "Key claims", section 2.1: attention reads the
+// top-k entries of I[t,:]; "Method": k = 2048).
+// ---------------------------------------------------------------------------
+struct SelShared {
+  uint32_t hist[2048];
+  uint32_t tmp[32];
+  uint32_t sel[2];
+  uint32_t ucnt[4];   // epilogue threads done with the CTA's recent units (ring of 4)
+  int go;             // the row's scores are complete (set by selector thread 0)
+};
+
+template <int NT>
+__device__ __forceinline__ void sel_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
+__device__ __forceinline__ uint32_t sel_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;   // -0.0 == +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const int* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Exclusive scan of one value per selector thread; also returns the total.
+template <int NT>
+__device__ __forceinline__ uint32_t sel_scan(uint32_t v, SelShared& sh, int tid, uint32_t& total) {
+  const int lane = tid & 31, wid = tid >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) sh.tmp[wid] = incl;
+  sel_bar<NT>();
+  uint32_t off = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const uint32_t x = sh.tmp[w];
+    off += w < wid ? x : 0u;
+    tot += x;
+  }
+  sel_bar<NT>();
+  total = tot;
+  return off + incl - v;
+}
+
+// From the histogram of the current digit, the digit holding the need-th largest
+// key: extends prefix by it and makes need the rank within that digit.
+template <int NT, int BITS>
+__device__ __forceinline__ void sel_find(SelShared& sh, int tid, bool first, uint32_t& prefix,
+                                         uint32_t& need) {
+  constexpr int BPT = (1 << BITS) / NT;
+  static_assert(BPT >= 1, "bins per thread");
+  const int b0 = tid * BPT;
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) local += sh.hist[b0 + j];
+  uint32_t total;
+  const uint32_t before = sel_scan<NT>(local, sh, tid, total);
+  uint32_t above = total - before - local;   // keys in the bins of higher-numbered threads
+#pragma unroll
+  for (int j = BPT - 1; j >= 0; --j) {
+    const uint32_t h = sh.hist[b0 + j];
+    if (above < need && need <= above + h) {
+      sh.sel[0] = (uint32_t)(b0 + j);
+      sh.sel[1] = need - above;
+    }
+    above += h;
+  }
+  sel_bar<NT>();
+  prefix = first ? sh.sel[0] : ((prefix << BITS) | sh.sel[0]);
+  need = sh.sel[1];
+  sel_bar<NT>();
+}
+
+// One radix pass over the row: histogram of digit (key >> shift) of the keys whose
+// higher bits equal prefix, then the digit that holds the need-th largest key.
+template <int NT, int BITS>
+__device__ __forceinline__ void sel_pass(const float* src, int n, int shift, bool first,
+                                         uint32_t& prefix, uint32_t& need, SelShared& sh, int tid) {
+  constexpr int NB = 1 << BITS;
+  for (int i = tid; i < NB; i += NT) sh.hist[i] = 0u;
+  sel_bar<NT>();
+  const int hi = shift + BITS;
+  auto count = [&](float x) {
+    const uint32_t key = sel_key(x);
+    if (first || (key >> hi) == prefix) atomicAdd(&sh.hist[(key >> shift) & (NB - 1)], 1u);
+  };
+  const int n4 = n & ~3;
+  for (int i = tid * 4; i < n4; i += NT * 4) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(src + i));
+    count(v.x);
+    count(v.y);
+    count(v.z);
+    count(v.w);
+  }
+  for (int i = n4 + tid; i < n; i += NT) count(__ldcg(src + i));
+  sel_bar<NT>();
+  sel_find<NT, BITS>(sh, tid, first, prefix, need);
+}
+
+// The top-k of the n scores at src (16-byte aligned): indices ascending into dst
+// [k] (-1 padded when n < k) and, if dsc is not null, their scores into dsc.
+template <int NT>
+__device__ void select_row(const float* src, int n, int k, int32_t* dst, float* dsc, SelShared& sh,
+                           int tid) {
+  if (n <= k) {
+    for (int i = tid; i < k; i += NT) {
+      dst[i] = i < n ? i : -1;
+      if (dsc != nullptr) dsc[i] = i < n ? __ldcg(src + i) : 0.f;
+    }
+    return;
+  }
+  uint32_t prefix = 0, need = (uint32_t)k;
+  sel_pass<NT, 11>(src, n, 21, true, prefix, need, sh, tid);
+  sel_pass<NT, 11>(src, n, 10, false, prefix, need, sh, tid);
+  sel_pass<NT, 10>(src, n, 0, false, prefix, need, sh, tid);
+  const uint32_t T = prefix;
+  const uint32_t need_eq = need;   // keys equal to T that are selected, lowest indices first
+  constexpr int ITEMS = 8;
+  uint32_t g_run = 0, e_run = 0;
+  for (int base = 0; base < n; base += NT * ITEMS) {
+    const int i0 = base + tid * ITEMS;
+    float x[ITEMS];
+    if (i0 + ITEMS <= n) {
+      const float4 v0 = __ldcg(reinterpret_cast<const float4*>(src + i0));
+      const float4 v1 = __ldcg(reinterpret_cast<const float4*>(src + i0 + 4));
+      x[0] = v0.x; x[1] = v0.y; x[2] = v0.z; x[3] = v0.w;
+      x[4] = v1.x; x[5] = v1.y; x[6] = v1.z; x[7] = v1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) x[j] = i0 + j < n ? __ldcg(src + i0 + j) : 0.f;
+    }
+    uint32_t g = 0, e = 0;
+#pragma unroll
+    for (int j = 0; j < ITEMS; ++j) {
+      const uint32_t key = sel_key(x[j]);
+      if (i0 + j < n) {
+        g += key > T;
+        e += key == T;
+      }
+    }
+    uint32_t total;
+    const uint32_t excl = sel_scan<NT>((e << 16) | g, sh, tid, total);
+    uint32_t G = g_run + (excl & 0xFFFFu);
+    uint32_t E = e_run + (excl >> 16);
+#pragma unroll
+    for (int j = 0; j < ITEMS; ++j) {
+      if (i0 + j < n) {
+        const uint32_t key = sel_key(x[j]);
+        if (key > T) {
+          const uint32_t pos = G + min(E, need_eq);
+          dst[pos] = i0 + j;
+          if (dsc != nullptr) dsc[pos] = x[j];
+          ++G;
+        } else if (key == T) {
+          if (E < need_eq) {
+            dst[G + E] = i0 + j;
+            if (dsc != nullptr) dsc[G + E] = x[j];
+          }
+          ++E;
+        }
+      }
+    }
+    g_run += total & 0xFFFFu;
+    e_run += total >> 16;
+  }
+}
+
+template <int D_I, int H_I, int N, bool SEL = false>
 struct IdxTraits {
   static constexpr int T_BLK = N / H_I;
   static constexpr int KT = 128;
@@ -39,7 +223,11 @@ struct IdxTraits {
   static constexpr int EPI_WARPS = (T_BLK >= 2) ? 8 : 4;
   static constexpr int MIN_CTAS = (N == 64) ? 2 : 1;        // CTAs per SM the registers must allow
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
-  static constexpr int THREADS = 64 + EPI_THREADS;
+  // selector warps of the fused top-k (two beside the single-token epilogue, so two
+  // CTAs still share an SM)
+  static constexpr int SEL_WARPS = SEL ? (N == 64 ? 2 : 4) : 0;
+  static constexpr int SEL_THREADS = SEL_WARPS * 32;
+  static constexpr int THREADS = 64 + EPI_THREADS + SEL_THREADS;
   static constexpr uint32_t SWZ = (D_I == 128) ? 2u : 6u;   // 128B / 32B swizzle
   static constexpr uint32_t SBO = 8u * D_I;                  // bytes per 8-row group
   static constexpr uint32_t IDESC = make_idesc(0, 0, 0, 0, N, 128);
@@ -50,7 +238,8 @@ struct IdxTraits {
   static constexpr int OFF_BAR = OFF_W + 4 * N * 4;  // EPI_WARPS x (N / HALVES) floats
   static constexpr int NUM_BARS = 2 + 2 + 2 * STAGES + 2 * ACC + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int OFF_SEL = OFF_MISC + 16;             // selector state (fused top-k)
+  static constexpr int SMEM_BYTES = OFF_SEL + (SEL ? (int)sizeof(SelShared) : 0) + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N <= 256, "N");
   static_assert(ACC * N <= 512, "TMEM");
   static_assert(H_I == 64 || (H_I < 32 && 32 % H_I == 0), "heads per chunk");
@@ -87,11 +276,13 @@ __device__ __forceinline__ bool get_unit(const IndexerArgs& a, int u, int nblk, 
 
 // PAGED: keys, key scales and causal bounds come through the paged-cache fields
 // (block table, per-sequence lengths); the unpaged instantiation has none of it.
-template <int D_I, int H_I, int N, bool PAGED>
-__global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I, H_I, N>::MIN_CTAS)
+// SEL: fused top-k; selector warps (after the epilogue warps) select rows once the
+// pieces of every unit of the row have been scored, from the same score chunk.
+template <int D_I, int H_I, int N, bool PAGED, bool SEL>
+__global__ void __launch_bounds__(IdxTraits<D_I, H_I, N, SEL>::THREADS, IdxTraits<D_I, H_I, N, SEL>::MIN_CTAS)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs a) {
-  using Tr = IdxTraits<D_I, H_I, N>;
+  using Tr = IdxTraits<D_I, H_I, N, SEL>;
   constexpr int T_BLK = Tr::T_BLK;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -129,6 +320,10 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
+    if constexpr (SEL) {
+      SelShared* sh = reinterpret_cast<SelShared*>(smem + Tr::OFF_SEL);
+      for (int i = 0; i < 4; ++i) sh->ucnt[i] = 0u;
+    }
     fence_barrier_init();
     tma_prefetch_map(&tmap_q);
     tma_prefetch_map(&tmap_k);
@@ -222,7 +417,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
       volatile int never = 0;
       mbar_wait(done_bar, 0, drain, &never, kSiteIndexer, 7);
     }
-  } else {
+  } else if (warp < 2 + Tr::EPI_WARPS) {
     // ------------------------------------------------ epilogue
     const int ew = warp - 2;                 // 0 .. EPI_WARPS-1
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
@@ -235,6 +430,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
     const uint32_t t_lane = tbase + ((uint32_t)(quad * 32) << 16);
     int ac = 0, aph = 0;
     bool ok = true;
+    uint32_t ul = 0;   // units of this CTA done so far
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       Unit un;
       if (!get_unit<T_BLK, PAGED>(a, u, nblk, maxp, un)) continue;
@@ -335,6 +531,77 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
         mbar_arrive(&acc_empty[ac]);
         if (++ac == Tr::ACC) { ac = 0; aph ^= 1; }
       }
+      if constexpr (SEL) {
+        // The unit's scores are written. The last epilogue thread of the CTA to get
+        // here counts the unit as one scored piece of each of its rows: every
+        // thread fences its own score stores before its count, and the last one
+        // fences again before publishing, so a selector that reads the row's
+        // count with acquire semantics sees every score of the row.
+        if (ok) {
+          SelShared* sh = reinterpret_cast<SelShared*>(smem + Tr::OFF_SEL);
+          __threadfence();
+          const uint32_t old = atomicAdd(&sh->ucnt[ul & 3u], 1u);
+          if (old + 1u == (uint32_t)Tr::EPI_THREADS * ((ul >> 2) + 1u)) {
+            __threadfence();
+            const int rows = a.sel_t1 - a.sel_t0;
+            for (int t = un.t_a; t < un.t_b; ++t)
+              atomicAdd(a.row_cnt + (long long)un.b * rows + (t - a.sel_t0), 1);
+          }
+          ++ul;
+        }
+      }
+    }
+  } else if constexpr (SEL) {
+    // ------------------------------------------------ selectors (fused top-k)
+    // Row r of the launch (sequence b, query row t in [sel_t0, sel_t1)) belongs to
+    // CTA r % gridDim.x. Scored rows wait until all pieces of their unit are
+    // counted; rows with at most k candidates select every key.
+    SelShared& sh = *reinterpret_cast<SelShared*>(smem + Tr::OFF_SEL);
+    constexpr int NT = Tr::SEL_THREADS;
+    const int tid = threadIdx.x - (64 + Tr::EPI_THREADS);
+    const int rows_per_b = a.sel_t1 - a.sel_t0;
+    const long long nrows = (long long)a.B * rows_per_b;
+    for (long long r = blockIdx.x; r < nrows; r += gridDim.x) {
+      const int b = (int)(r / rows_per_b);
+      const int t = a.sel_t0 + (int)(r % rows_per_b);
+      const int qp = PAGED ? seq_pos0(a.seq_lens, a.q_pos0, a.Lq, b) : a.q_pos0;
+      const int n = min(a.Lk, qp + t + 1);
+      const bool scored = t >= a.t_lo && t < a.t_hi;
+      if (tid == 0) {
+        int go = 1;
+        if (scored) {
+          // pieces of the row's unit: as many as get_unit gives its token block
+          const int blk = (t - a.t_lo) / T_BLK;
+          const int t_b = min(a.t_lo + (blk + 1) * T_BLK, a.t_hi);
+          const int keys = min(a.Lk, qp + t_b);
+          const uint32_t pieces = (uint32_t)((keys + a.piece_keys - 1) / a.piece_keys);
+          const int* cnt = a.row_cnt + r;
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_u32(cnt) < pieces) {
+            if (*abort_flag || *reinterpret_cast<volatile int*>(a.ctl.status) != 0) { go = 0; break; }
+            if (globaltimer_ns() - t0 > a.ctl.wait_ns) {
+              report_timeout(a.ctl, kSiteIndexer, 20);
+              go = 0;
+              break;
+            }
+            __nanosleep(256);
+          }
+          if (go) a.row_cnt[r] = 0;   // counted out: zero again for the next launch
+        }
+        sh.go = go;
+      }
+      sel_bar<NT>();
+      const int go = sh.go;
+      sel_bar<NT>();
+      if (!go) {
+        if (tid == 0) *abort_flag = 1;
+        break;
+      }
+      const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld;
+      const long long orow = ((long long)b * a.Lq + t) * a.k;
+      select_row<NT>(src, scored ? n : min(n, a.k), a.k, a.idx + orow,
+                     a.sel_scores != nullptr && scored ? a.sel_scores + orow : nullptr, sh, tid);
+      sel_bar<NT>();
     }
   }
 
@@ -345,26 +612,53 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N>::THREADS, IdxTraits<D_I
   }
 }
 
-template <int D_I, int H_I, int N>
+template <int D_I, int H_I, int N, bool SEL>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                            int num_sms, cudaStream_t stream) {
-  using Tr = IdxTraits<D_I, H_I, N>;
+  using Tr = IdxTraits<D_I, H_I, N, SEL>;
   const bool paged = a.block_table != nullptr || a.seq_lens != nullptr;
-  auto kern = paged ? indexer_kernel<D_I, H_I, N, true> : indexer_kernel<D_I, H_I, N, false>;
+  auto kern = paged ? indexer_kernel<D_I, H_I, N, true, SEL> : indexer_kernel<D_I, H_I, N, false, SEL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   int nblk = (a.t_hi - a.t_lo + Tr::T_BLK - 1) / Tr::T_BLK;
+  if (nblk < 0) nblk = 0;
   int keys_max = a.seq_lens != nullptr ? a.Lk : (a.q_pos0 + a.t_hi < a.Lk ? a.q_pos0 + a.t_hi : a.Lk);
   long long maxp = (keys_max + a.piece_keys - 1) / a.piece_keys;
   long long units = (long long)a.B * nblk * maxp;
-  if (units <= 0) return cudaSuccess;
+  // fused top-k: CTAs without units still select rows
+  const long long work = SEL ? (units > (long long)a.B * (a.sel_t1 - a.sel_t0) ? units
+                                                                             : (long long)a.B * (a.sel_t1 - a.sel_t0))
+                             : units;
+  if (work <= 0) return cudaSuccess;
   // persistent CTAs: as many as fit on the SMs at once (smem and TMEM allow two
   // of the single-token variant per SM)
-  const int per_sm = (2 * Tr::SMEM_BYTES <= 227 * 1024 && 2 * Tr::TMEM_COLS <= 512) ? 2 : 1;
-  int grid = (int)(units < (long long)per_sm * num_sms ? units : (long long)per_sm * num_sms);
-  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, stream>>>(tq, tk, a);
-  return cudaGetLastError();
+  int per_sm = (2 * Tr::SMEM_BYTES <= 227 * 1024 && 2 * Tr::TMEM_COLS <= 512) ? 2 : 1;
+  if (SEL) {
+    // the selectors wait on rows other CTAs score: every CTA must be resident at
+    // once, which the cooperative launch guarantees for a grid within occupancy
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Tr::THREADS, Tr::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (occ < per_sm) per_sm = occ;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  }
+  const int grid = (int)(work < (long long)per_sm * num_sms ? work : (long long)per_sm * num_sms);
+  if (!SEL) {
+    kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, stream>>>(tq, tk, a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(Tr::THREADS);
+  cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, a);
 }
 
 __global__ void fill_noncausal_kernel(float* scores, int B, int Lq, int Lk, int q_pos0) {
@@ -375,19 +669,32 @@ __global__ void fill_noncausal_kernel(float* scores, int B, int Lq, int Lk, int 
   for (int s = first + (int)threadIdx.x; s < Lk; s += blockDim.x) dst[s] = -__int_as_float(0x7f800000);
 }
 
+
+template <bool SEL>
+cudaError_t launch_indexer_sel(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                               const IndexerArgs& a, int H_I, int d_I, int num_sms,
+                               cudaStream_t stream) {
+  if (H_I == 64 && d_I == 128) {
+    if (a.t_hi - a.t_lo <= 1) return launch_variant<128, 64, 64, SEL>(tmap_q, tmap_k, a, num_sms, stream);
+    return launch_variant<128, 64, 256, SEL>(tmap_q, tmap_k, a, num_sms, stream);
+  }
+  if (H_I == 4 && d_I == 32) return launch_variant<32, 4, 256, SEL>(tmap_q, tmap_k, a, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                            const IndexerArgs& a, int H_I, int d_I, int num_sms,
                            cudaStream_t stream) {
-  if (a.t_hi <= a.t_lo) return cudaSuccess;
-  if (H_I == 64 && d_I == 128) {
-    if (a.t_hi - a.t_lo == 1) return launch_variant<128, 64, 64>(tmap_q, tmap_k, a, num_sms, stream);
-    return launch_variant<128, 64, 256>(tmap_q, tmap_k, a, num_sms, stream);
+  if (a.select) {
+    if (a.sel_t1 <= a.sel_t0) return cudaSuccess;
+    return launch_indexer_sel<true>(tmap_q, tmap_k, a, H_I, d_I, num_sms, stream);
   }
-  if (H_I == 4 && d_I == 32) return launch_variant<32, 4, 256>(tmap_q, tmap_k, a, num_sms, stream);
-  return cudaErrorInvalidValue;
+  if (a.t_hi <= a.t_lo) return cudaSuccess;
+  return launch_indexer_sel<false>(tmap_q, tmap_k, a, H_I, d_I, num_sms, stream);
 }
+
 
 cudaError_t launch_fill_noncausal(float* scores, int B, int Lq, int Lk, int q_pos0,
                                   cudaStream_t stream) {

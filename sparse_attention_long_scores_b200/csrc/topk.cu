@@ -33,6 +33,11 @@ __device__ __forceinline__ uint32_t score_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The score of an order-preserving key (-0.0 comes back as +0.0).
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // Exclusive block scan of one int per thread; also returns the block total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t& total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -162,11 +167,15 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
     const int t = a.t_lo + (int)(r % rows_per_b);
     const int n = min(a.Lk, seq_pos0(a.seq_lens, a.q_pos0, a.Lq, b) + t + 1);
     int32_t* dst = a.idx + ((long long)b * a.Lq + t) * a.k;
+    float* dsc = a.sel != nullptr ? a.sel + ((long long)b * a.Lq + t) * a.k : nullptr;
+    const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld;
     if (n <= a.k) {
-      for (int i = threadIdx.x; i < a.k; i += TK_THREADS) dst[i] = i < n ? i : -1;
+      for (int i = threadIdx.x; i < a.k; i += TK_THREADS) {
+        dst[i] = i < n ? i : -1;
+        if (dsc != nullptr) dsc[i] = i < n ? src[i] : 0.f;
+      }
       continue;
     }
-    const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld;
     if constexpr (SMEM_ROW) {
       if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
         const int n4 = n >> 2;
@@ -228,9 +237,13 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
         if (i0 + j < n) {
           if (keys[j] > T) {
             dst[G + min(E, need_eq)] = i0 + j;
+            if (dsc != nullptr) dsc[G + min(E, need_eq)] = key_score(keys[j]);
             ++G;
           } else if (keys[j] == T) {
-            if (E < need_eq) dst[G + E] = i0 + j;
+            if (E < need_eq) {
+              dst[G + E] = i0 + j;
+              if (dsc != nullptr) dsc[G + E] = key_score(keys[j]);
+            }
             ++E;
           }
         }
@@ -290,9 +303,15 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   const int t = a.t_lo + (int)(r % rows_per_b);
   const int n = min(a.Lk, seq_pos0(a.seq_lens, a.q_pos0, a.Lq, b) + t + 1);
   int32_t* dst = a.idx + ((long long)b * a.Lq + t) * a.k;
+  float* dsc = a.sel != nullptr ? a.sel + ((long long)b * a.Lq + t) * a.k : nullptr;
   if (n <= a.k) {   // the same decision in every CTA of the cluster: no shared traffic below
-    if (rank == 0)
-      for (int i = threadIdx.x; i < a.k; i += TK_THREADS) dst[i] = i < n ? i : -1;
+    if (rank == 0) {
+      const float* row = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld;
+      for (int i = threadIdx.x; i < a.k; i += TK_THREADS) {
+        dst[i] = i < n ? i : -1;
+        if (dsc != nullptr) dsc[i] = i < n ? row[i] : 0.f;
+      }
+    }
     return;
   }
   const int seg = (((n + TKC - 1) / TKC) + 3) & ~3;
@@ -359,9 +378,13 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
       if (i0 + j < m) {
         if (keys[j] > T) {
           dst[G + min(E, need_eq)] = lo + i0 + j;
+          if (dsc != nullptr) dsc[G + min(E, need_eq)] = key_score(keys[j]);
           ++G;
         } else if (keys[j] == T) {
-          if (E < need_eq) dst[G + E] = lo + i0 + j;
+          if (E < need_eq) {
+            dst[G + E] = lo + i0 + j;
+            if (dsc != nullptr) dsc[G + E] = key_score(keys[j]);
+          }
           ++E;
         }
       }

@@ -344,6 +344,58 @@ def test_overlapped_schedule_matches_serial(name, kw):
     assert launches > prof.n and dsa.last_launch_count() == prof.n
 
 
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("tiny", dict(B=3, Lq=37, Lk=301, q_pos0=264)),
+                                     ("prefill_8k", dict(Lq=1000, q_pos0=7192)),
+                                     ("decode_128k", dict(B=5))])
+def test_fused_forward_matches_forward(name, kw):
+    """dsa_forward_fused selects inside the indexer kernel (selector warps, one
+    cooperative launch per score chunk); it computes every score and applies the
+    selection rule exactly as dsa_forward does, so idx, out and lse are identical."""
+    cfg = CONFIGS[name].with_(**kw)
+    inp = gen_inputs(cfg, "cuda", seed=31)
+    out1, lse1, idx1 = _forward(cfg, inp)
+    p = dsa.Problem.from_config(cfg)
+    out2 = torch.empty_like(out1)
+    lse2 = torch.empty_like(lse1)
+    idx2 = torch.empty_like(idx1)
+    dsa.forward(p, inp, out=out2, lse=lse2, idx_out=idx2, fused=True)
+    dsa.check_status()
+    assert dsa.last_launch_count() >= 2
+    assert torch.equal(idx1, idx2) and torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("prefill_8k", dict(Lq=600, q_pos0=7592)),
+                                     ("decode_128k", dict(B=4))])
+def test_forward_returns_selected_scores(name, kw, fused):
+    """sel_scores_out: the index score of every selected key, aligned with idx_out,
+    written by the kernel that selects (every row is scored, short rows included).
+    It must equal the materialised score matrix gathered at idx bit for bit, match
+    the oracle on sampled rows, and leave the selection unchanged."""
+    cfg = CONFIGS[name].with_(**kw)
+    inp = gen_inputs(cfg, "cuda", seed=29)
+    p = dsa.Problem.from_config(cfg)
+    idx = torch.empty((cfg.B, cfg.Lq, cfg.k), dtype=torch.int32, device="cuda")
+    sel = torch.full((cfg.B, cfg.Lq, cfg.k), float("nan"), dtype=torch.float32, device="cuda")
+    out = dsa.forward(p, inp, idx_out=idx, sel_scores=sel, fused=fused)
+    dsa.check_status()
+    out2, _, idx2 = _forward(cfg, inp)
+    assert torch.equal(idx, idx2) and torch.equal(out, out2)
+    sc = dsa.indexer_scores(inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"],
+                            q_pos0=cfg.q_pos0)
+    dsa.check_status()
+    valid = idx >= 0
+    gathered = torch.where(valid, torch.gather(sc, 2, idx.clamp(min=0).long()), torch.zeros_like(sel))
+    assert torch.equal(sel, gathered)
+    rows = Rows(cfg, inp)
+    idx_h, sel_h = idx.cpu().numpy(), sel.cpu().numpy()
+    for b in range(cfg.B):
+        for t in sorted({0, cfg.Lq // 2, cfg.Lq - 1}):
+            v = idx_h[b, t][idx_h[b, t] >= 0]
+            ref = rows.scores(b, t)
+            check_scores(sel_h[b, t][: v.size], ref[v], f"{name} sel_scores b={b} t={t}")
+
+
 @pytest.mark.parametrize("name,L,rows", [("tiny", 32, None), ("prefill_8k", 2048, (0, 1, 700, 2047))])
 def test_short_context_is_dense_attention_without_indexer(name, L, rows):
     """L <= k: every row selects all of its causal keys without scores (the top-k of at
