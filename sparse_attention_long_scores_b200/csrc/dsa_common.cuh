@@ -357,6 +357,16 @@ DSA_DEVICE_INLINE uint32_t ld_cluster_u32(uint32_t addr) {
   return v;
 }
 
+// Four consecutive words of (distributed) shared memory; addr 16-byte aligned.
+DSA_DEVICE_INLINE uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 DSA_DEVICE_INLINE void st_cluster_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)

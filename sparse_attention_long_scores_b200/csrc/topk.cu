@@ -7,16 +7,21 @@
 // (-0.0 folded onto +0.0) and the exact k-th largest key T is found by a
 // three-digit radix select (11 + 11 + 10 bits, most significant first): each
 // pass histograms the keys that still match the selected prefix in shared
-// memory and a block scan picks the digit where the running count from the top
-// crosses k. A final ordered pass writes every key > T and the first
-// (k - #{key > T}) keys == T, in ascending index order: one block-wide scan of
-// packed (greater, equal) counts per 4096 candidates gives every element its
-// output slot. Ties therefore go to the lowest index and the output is sorted.
+// memory (the first while the row is staged) and a block scan picks the digit
+// where the running count from the top crosses k. A final ordered pass writes
+// every key > T and the first (k - #{key > T}) keys == T, in ascending index
+// order: each warp owns a contiguous run of the row, counts its (greater,
+// equal) keys, and after one block-wide exchange of those counts writes its run
+// with warp scans of 128 keys at a time. Ties therefore go to the lowest index
+// and the output is sorted. Shared-memory sweeps read four keys per thread per
+// load.
 // Rows of up to 48K candidates are staged once in shared memory as keys. Longer
 // rows, or launches with fewer rows than SMs, spread each row over a cluster of
 // 8 CTAs (topk_cluster_kernel); rows beyond 8 x 48K are re-read from global
 // memory (L2) on each pass.
 // Rows with at most k candidates select all of them and pad with -1.
+#include <type_traits>
+
 #include "dsa_kernels.h"
 
 namespace dsa {
@@ -24,8 +29,8 @@ namespace {
 
 constexpr int TK_THREADS = 512;
 constexpr int TK_WARPS = TK_THREADS / 32;
-constexpr int TK_ITEMS = 8;                       // contiguous elements per thread, output pass
 constexpr int TK_SMEM_MAX = 48 * 1024;            // candidates staged in shared memory
+constexpr int TK_STEP = 128;                      // keys per warp step of the output pass
 
 __device__ __forceinline__ uint32_t score_key(float x) {
   uint32_t u = __float_as_uint(x);
@@ -36,6 +41,12 @@ __device__ __forceinline__ uint32_t score_key(float x) {
 // The score of an order-preserving key (-0.0 comes back as +0.0).
 __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // Exclusive block scan of one int per thread; also returns the block total.
@@ -94,72 +105,218 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, bool first, uint3
   __syncthreads();
 }
 
-template <bool SMEM_ROW>
-struct RowSrc {
-  const uint32_t* keys;  // shared-memory keys (SMEM_ROW)
-  const float* src;      // global scores
-  __device__ __forceinline__ uint32_t operator()(int i) const {
-    if constexpr (SMEM_ROW) return keys[i];
-    else return score_key(__ldg(src + i));
+// Keys staged in shared memory. The staging buffer holds a multiple of four
+// words, so a 16-byte load at any i % 4 == 0 with i < m stays inside it; the
+// words past m are never counted (callers pass validity separately).
+struct SmemKeys {
+  const uint32_t* keys;
+  __device__ __forceinline__ uint4 load4(int i, int) const {
+    return *reinterpret_cast<const uint4*>(keys + i);
   }
 };
 
-// One radix pass: histogram digit (key >> shift) & (nbins-1) of keys whose bits
-// above `shift + bits` equal `prefix`; then find the digit holding the `need`-th
-// largest key. Updates prefix/need in place (uniform across the block).
-template <bool SMEM_ROW, int BITS>
-__device__ __forceinline__ void radix_pass(const RowSrc<SMEM_ROW>& row, int n, int shift,
-                                           bool first, uint32_t& prefix, uint32_t& need,
-                                           uint32_t* hist, uint32_t* tmp, uint32_t* sel) {
+// Keys computed from global (L2-resident) scores on every read.
+struct GlobalKeys {
+  const float* src;
+  bool vec;   // 16-byte aligned row
+  __device__ __forceinline__ uint4 load4(int i, int m) const {
+    if (vec && i + 3 < m) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src + i));
+      return make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+    }
+    uint4 r;
+    r.x = i < m ? score_key(__ldg(src + i)) : 0u;
+    r.y = i + 1 < m ? score_key(__ldg(src + i + 1)) : 0u;
+    r.z = i + 2 < m ? score_key(__ldg(src + i + 2)) : 0u;
+    r.w = i + 3 < m ? score_key(__ldg(src + i + 3)) : 0u;
+    return r;
+  }
+};
+
+// Histogram (into `hist`, already cleared) the digit (key >> shift) of the keys
+// of [0, m) whose bits above `shift + BITS` equal `prefix`.
+template <int BITS, class Keys>
+__device__ __forceinline__ void histogram_digit(const Keys& keys, int m, int shift, bool first,
+                                                uint32_t prefix, uint32_t* hist) {
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  const int hi_shift = shift + BITS;
+  auto count = [&](uint32_t key, bool valid) {
+    if (valid && (first || (key >> hi_shift) == prefix)) atomicAdd(&hist[(key >> shift) & MASK], 1u);
+  };
+  const int groups = (m + 3) >> 2;
+#pragma unroll 4
+  for (int g = threadIdx.x; g < groups; g += TK_THREADS) {
+    const int i = g << 2;
+    const uint4 v = keys.load4(i, m);
+    count(v.x, true);
+    count(v.y, i + 1 < m);
+    count(v.z, i + 2 < m);
+    count(v.w, i + 3 < m);
+  }
+}
+
+// One radix pass of the single-CTA kernel: histogram, then find the digit
+// holding the `need`-th largest key. Updates prefix/need in place.
+template <int BITS, class Keys>
+__device__ __forceinline__ void radix_pass(const Keys& keys, int n, int shift, bool first,
+                                           uint32_t& prefix, uint32_t& need, uint32_t* hist,
+                                           uint32_t* tmp, uint32_t* sel) {
   constexpr int NB = 1 << BITS;
-  constexpr int BPT = NB / TK_THREADS;  // bins per thread
-  static_assert(BPT >= 1, "bins");
+  static_assert(NB / TK_THREADS >= 1, "bins");
   for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
   __syncthreads();
-  const int hi_shift = shift + BITS;
-  const int lane = threadIdx.x & 31;
-  auto count = [&](uint32_t key, bool valid) {
-    if (valid && (first || (key >> hi_shift) == prefix))
-      atomicAdd(&hist[(key >> shift) & (NB - 1)], 1u);
-  };
-  if constexpr (SMEM_ROW) {
-    for (int i = threadIdx.x; i < n; i += TK_THREADS) count(row.keys[i], true);
-  } else {
-    // eight consecutive scores per thread per step (two 16-byte loads in flight)
-    const bool vec = (reinterpret_cast<uintptr_t>(row.src) & 15u) == 0;
-    for (int base = (threadIdx.x & ~31) * 8; base < n; base += TK_THREADS * 8) {
-      const int i0 = base + lane * 8;
-      float4 v0, v1;
-      if (vec && i0 + 7 < n) {
-        v0 = __ldg(reinterpret_cast<const float4*>(row.src + i0));
-        v1 = __ldg(reinterpret_cast<const float4*>(row.src + i0 + 4));
-      } else {
-        float t[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) t[j] = i0 + j < n ? __ldg(row.src + i0 + j) : 0.f;
-        v0 = make_float4(t[0], t[1], t[2], t[3]);
-        v1 = make_float4(t[4], t[5], t[6], t[7]);
-      }
-      count(score_key(v0.x), i0 < n);
-      count(score_key(v0.y), i0 + 1 < n);
-      count(score_key(v0.z), i0 + 2 < n);
-      count(score_key(v0.w), i0 + 3 < n);
-      count(score_key(v1.x), i0 + 4 < n);
-      count(score_key(v1.y), i0 + 5 < n);
-      count(score_key(v1.z), i0 + 6 < n);
-      count(score_key(v1.w), i0 + 7 < n);
-    }
-  }
+  histogram_digit<BITS>(keys, n, shift, first, prefix, hist);
   __syncthreads();
   find_bin<BITS>(hist, first, prefix, need, tmp, sel);
 }
 
+// ---------------------------------------------------------------------------
+// The ordered output pass. Warp w owns the 128-key steps [s0, s1) of [0, m).
+// ---------------------------------------------------------------------------
+struct Run {
+  int s0, s1;
+};
+
+__device__ __forceinline__ Run warp_run(int m) {
+  const int steps = (m + TK_STEP - 1) / TK_STEP;
+  const int per = (steps + TK_WARPS - 1) / TK_WARPS;
+  const int s0 = min(steps, (int)(threadIdx.x >> 5) * per);
+  return Run{s0, min(steps, s0 + per)};
+}
+
+// (greater, equal) of one key against T, packed as equal << 16 | greater.
+__device__ __forceinline__ uint32_t ge_bits(uint32_t key, bool valid, uint32_t T) {
+  return (uint32_t)(valid && key > T) | ((uint32_t)(valid && key == T) << 16);
+}
+
+// Counts of keys > T and == T in this warp's run (warp-uniform results).
+template <class Keys>
+__device__ __forceinline__ void run_counts(const Keys& keys, int m, uint32_t T, Run run,
+                                           uint32_t& g, uint32_t& e) {
+  const int lane = threadIdx.x & 31;
+  uint32_t gl = 0, el = 0;
+  for (int s = run.s0; s < run.s1; ++s) {
+    const int i = s * TK_STEP + lane * 4;
+    if (i < m) {
+      const uint4 v = keys.load4(i, m);
+      const uint32_t c = ge_bits(v.x, true, T) + ge_bits(v.y, i + 1 < m, T) +
+                         ge_bits(v.z, i + 2 < m, T) + ge_bits(v.w, i + 3 < m, T);
+      gl += c & 0xFFFFu;
+      el += c >> 16;
+    }
+  }
+  g = warp_sum_u32(gl);
+  e = warp_sum_u32(el);
+}
+
+// Write the selected keys of this warp's run. G and E are the numbers of keys
+// > T and == T before the run (in index order, over the whole row); the output
+// index of key i is base + i.
+template <class Keys>
+__device__ __forceinline__ void write_run(const Keys& keys, int m, uint32_t T, uint32_t need_eq,
+                                          uint32_t G, uint32_t E, int base, Run run,
+                                          int32_t* dst, float* dsc) {
+  const int lane = threadIdx.x & 31;
+  for (int s = run.s0; s < run.s1; ++s) {
+    const int i = s * TK_STEP + lane * 4;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (i < m) v = keys.load4(i, m);
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+    uint32_t own = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) own += ge_bits(kk[j], i + j < m, T);
+    uint32_t incl = own;   // a step holds at most 128 keys: the packed halves cannot carry
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    const uint32_t ex = incl - own;
+    uint32_t Gl = G + (ex & 0xFFFFu), El = E + (ex >> 16);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool valid = i + j < m;
+      const bool gt = valid && kk[j] > T, eq = valid && kk[j] == T;
+      // a key > T goes after the selected equal keys before it; an equal key is
+      // selected while fewer than need_eq equal keys precede it
+      const uint32_t slot = Gl + (gt ? min(El, need_eq) : El);
+      if (gt || (eq && El < need_eq)) {
+        dst[slot] = base + i + j;
+        if (dsc != nullptr) dsc[slot] = key_score(kk[j]);
+      }
+      Gl += gt;
+      El += eq;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+    G += tot & 0xFFFFu;
+    E += tot >> 16;
+  }
+}
+
+// Per-warp counts of the run into tmp[wid] / tmp[TK_WARPS + wid], then this
+// warp's (G, E) offsets within the block and the block totals.
+template <class Keys>
+__device__ __forceinline__ void block_run_offsets(const Keys& keys, int m, uint32_t T, Run run,
+                                                  uint32_t* tmp, uint32_t& G, uint32_t& E,
+                                                  uint32_t& g_tot, uint32_t& e_tot) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint32_t g, e;
+  run_counts(keys, m, T, run, g, e);
+  if (lane == 0) {
+    tmp[wid] = g;
+    tmp[TK_WARPS + wid] = e;
+  }
+  __syncthreads();
+  G = 0;
+  E = 0;
+  g_tot = 0;
+  e_tot = 0;
+#pragma unroll
+  for (int w = 0; w < TK_WARPS; ++w) {
+    const uint32_t gw = tmp[w], ew = tmp[TK_WARPS + w];
+    if (w < wid) {
+      G += gw;
+      E += ew;
+    }
+    g_tot += gw;
+    e_tot += ew;
+  }
+}
+
+// Stage scores [0, m) as keys in shared memory and histogram their top 11 bits
+// (hist already cleared). The caller synchronises.
+__device__ __forceinline__ void stage_keys(const float* src, int m, uint32_t* keys, uint32_t* hist) {
+  auto put = [&](int i, uint32_t key) {
+    keys[i] = key;
+    atomicAdd(&hist[key >> 21], 1u);
+  };
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+    const int m4 = m >> 2;
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    uint4* k4 = reinterpret_cast<uint4*>(keys);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < m4; i += TK_THREADS) {
+      const float4 v = __ldg(s4 + i);
+      const uint4 kk = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+      k4[i] = kk;
+      atomicAdd(&hist[kk.x >> 21], 1u);
+      atomicAdd(&hist[kk.y >> 21], 1u);
+      atomicAdd(&hist[kk.z >> 21], 1u);
+      atomicAdd(&hist[kk.w >> 21], 1u);
+    }
+    for (int i = (m4 << 2) + threadIdx.x; i < m; i += TK_THREADS) put(i, score_key(__ldg(src + i)));
+  } else {
+    for (int i = threadIdx.x; i < m; i += TK_THREADS) put(i, score_key(__ldg(src + i)));
+  }
+}
+
 template <bool SMEM_ROW>
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
-  extern __shared__ uint32_t row_keys[];
+  extern __shared__ __align__(16) uint32_t row_keys[];
   __shared__ uint32_t hist[2048];
-  __shared__ uint32_t tmp[32];
+  __shared__ uint32_t tmp[2 * TK_WARPS];
   __shared__ uint32_t sel[2];
+  using Keys = typename std::conditional<SMEM_ROW, SmemKeys, GlobalKeys>::type;
   const int rows_per_b = a.t_hi - a.t_lo;
   const long long nrows = (long long)a.B * rows_per_b;
   for (long long r = blockIdx.x; r < nrows; r += gridDim.x) {
@@ -176,82 +333,30 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
       }
       continue;
     }
-    if constexpr (SMEM_ROW) {
-      if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-        const int n4 = n >> 2;
-        const float4* s4 = reinterpret_cast<const float4*>(src);
-        uint4* k4 = reinterpret_cast<uint4*>(row_keys);
-        for (int i = threadIdx.x; i < n4; i += TK_THREADS) {
-          const float4 v = __ldg(s4 + i);
-          k4[i] = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
-        }
-        for (int i = (n4 << 2) + threadIdx.x; i < n; i += TK_THREADS) row_keys[i] = score_key(__ldg(src + i));
-      } else {
-        for (int i = threadIdx.x; i < n; i += TK_THREADS) row_keys[i] = score_key(__ldg(src + i));
-      }
-      __syncthreads();
-    }
-    RowSrc<SMEM_ROW> row{row_keys, src};
+    Keys keys;
     uint32_t prefix = 0, need = (uint32_t)a.k;
-    radix_pass<SMEM_ROW, 11>(row, n, 21, true, prefix, need, hist, tmp, sel);
-    radix_pass<SMEM_ROW, 11>(row, n, 10, false, prefix, need, hist, tmp, sel);
-    radix_pass<SMEM_ROW, 10>(row, n, 0, false, prefix, need, hist, tmp, sel);
+    if constexpr (SMEM_ROW) {
+      // staging builds the first digit's histogram on the way
+      for (int i = threadIdx.x; i < 2048; i += TK_THREADS) hist[i] = 0u;
+      __syncthreads();
+      stage_keys(src, n, row_keys, hist);
+      __syncthreads();
+      find_bin<11>(hist, true, prefix, need, tmp, sel);
+      keys = SmemKeys{row_keys};
+    } else {
+      keys = GlobalKeys{src, a.vec4 != 0};
+      radix_pass<11>(keys, n, 21, true, prefix, need, hist, tmp, sel);
+    }
+    radix_pass<11>(keys, n, 10, false, prefix, need, hist, tmp, sel);
+    radix_pass<10>(keys, n, 0, false, prefix, need, hist, tmp, sel);
     const uint32_t T = prefix;
     const uint32_t need_eq = need;  // keys equal to T that are selected (lowest indices first)
 
-    uint32_t g_run = 0, e_run = 0;
-    for (int base = 0; base < n; base += TK_THREADS * TK_ITEMS) {
-      const int i0 = base + threadIdx.x * TK_ITEMS;
-      uint32_t keys[TK_ITEMS];
-      bool full = i0 + TK_ITEMS <= n;
-      if constexpr (!SMEM_ROW) {
-        if (full && a.vec4) {
-          float4 v0 = __ldg(reinterpret_cast<const float4*>(src + i0));
-          float4 v1 = __ldg(reinterpret_cast<const float4*>(src + i0 + 4));
-          keys[0] = score_key(v0.x); keys[1] = score_key(v0.y);
-          keys[2] = score_key(v0.z); keys[3] = score_key(v0.w);
-          keys[4] = score_key(v1.x); keys[5] = score_key(v1.y);
-          keys[6] = score_key(v1.z); keys[7] = score_key(v1.w);
-        } else {
-#pragma unroll
-          for (int j = 0; j < TK_ITEMS; ++j) keys[j] = (i0 + j < n) ? row(i0 + j) : 0u;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < TK_ITEMS; ++j) keys[j] = (i0 + j < n) ? row_keys[i0 + j] : 0u;
-      }
-      uint32_t g = 0, e = 0;
-#pragma unroll
-      for (int j = 0; j < TK_ITEMS; ++j) {
-        if (i0 + j < n) {
-          g += keys[j] > T;
-          e += keys[j] == T;
-        }
-      }
-      uint32_t total;
-      uint32_t excl = block_excl_scan((e << 16) | g, tmp, total);
-      uint32_t G = g_run + (excl & 0xFFFFu);
-      uint32_t E = e_run + (excl >> 16);
-#pragma unroll
-      for (int j = 0; j < TK_ITEMS; ++j) {
-        if (i0 + j < n) {
-          if (keys[j] > T) {
-            dst[G + min(E, need_eq)] = i0 + j;
-            if (dsc != nullptr) dsc[G + min(E, need_eq)] = key_score(keys[j]);
-            ++G;
-          } else if (keys[j] == T) {
-            if (E < need_eq) {
-              dst[G + E] = i0 + j;
-              if (dsc != nullptr) dsc[G + E] = key_score(keys[j]);
-            }
-            ++E;
-          }
-        }
-      }
-      g_run += total & 0xFFFFu;
-      e_run += total >> 16;
-    }
-    __syncthreads();
+    const Run run = warp_run(n);
+    uint32_t G, E, g_tot, e_tot;
+    block_run_offsets(keys, n, T, run, tmp, G, E, g_tot, e_tot);
+    write_run(keys, n, T, need_eq, G, E, 0, run, dst, dsc);
+    __syncthreads();   // tmp, hist and the staged row are reused by the next row
   }
 }
 
@@ -264,36 +369,50 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
 // ---------------------------------------------------------------------------
 constexpr int TKC = 8;
 
+// Sum the CTAs' histograms of one digit over the cluster and pick the digit.
 template <int BITS>
-__device__ __forceinline__ void cluster_pass(const uint32_t* keys, int m, int shift, bool first,
-                                             uint32_t& prefix, uint32_t& need, uint32_t* hist,
-                                             uint32_t* ghist, uint32_t* tmp, uint32_t* sel) {
+__device__ __forceinline__ void cluster_find(bool first, uint32_t& prefix, uint32_t& need,
+                                             uint32_t* hist, uint32_t* ghist, uint32_t* tmp,
+                                             uint32_t* sel) {
   constexpr int NB = 1 << BITS;
-  for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
-  __syncthreads();
-  const int hi_shift = shift + BITS;
-  for (int i = threadIdx.x; i < m; i += TK_THREADS) {
-    const uint32_t key = keys[i];
-    if (first || (key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (NB - 1)], 1u);
-  }
   cluster_sync();   // every CTA's histogram is complete and visible
+  // cluster sum, four bins per load with all TKC loads of a thread in flight
   const uint32_t h0 = smem_u32(hist);
-  for (int i = threadIdx.x; i < NB; i += TK_THREADS) {
-    uint32_t sum = 0;
+  for (int i = threadIdx.x; i < NB / 4; i += TK_THREADS) {
+    uint4 v[TKC];
 #pragma unroll
-    for (int p = 0; p < TKC; ++p) sum += ld_cluster_u32(mapa_shared(h0 + 4u * i, p));
-    ghist[i] = sum;
+    for (int p = 0; p < TKC; ++p) v[p] = ld_cluster_v4(mapa_shared(h0 + 16u * i, p));
+    uint4 acc = v[0];
+#pragma unroll
+    for (int p = 1; p < TKC; ++p) {
+      acc.x += v[p].x;
+      acc.y += v[p].y;
+      acc.z += v[p].z;
+      acc.w += v[p].w;
+    }
+    reinterpret_cast<uint4*>(ghist)[i] = acc;
   }
   cluster_sync();   // peers are done reading `hist` before it is cleared again
   find_bin<BITS>(ghist, first, prefix, need, tmp, sel);
 }
 
+template <int BITS>
+__device__ __forceinline__ void cluster_pass(const SmemKeys& keys, int m, int shift,
+                                             uint32_t& prefix, uint32_t& need, uint32_t* hist,
+                                             uint32_t* ghist, uint32_t* tmp, uint32_t* sel) {
+  constexpr int NB = 1 << BITS;
+  for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
+  __syncthreads();
+  histogram_digit<BITS>(keys, m, shift, false, prefix, hist);
+  cluster_find<BITS>(false, prefix, need, hist, ghist, tmp, sel);
+}
+
 __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
     topk_cluster_kernel(const TopkArgs a) {
-  extern __shared__ uint32_t seg_keys[];
-  __shared__ uint32_t hist[2048];
-  __shared__ uint32_t ghist[2048];
-  __shared__ uint32_t tmp[32];
+  extern __shared__ __align__(16) uint32_t seg_keys[];
+  __shared__ __align__(16) uint32_t hist[2048];
+  __shared__ __align__(16) uint32_t ghist[2048];
+  __shared__ uint32_t tmp[2 * TK_WARPS];
   __shared__ uint32_t sel[2];
   __shared__ uint32_t counts[2];
   const uint32_t rank = cluster_ctarank();
@@ -318,80 +437,32 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   const int lo = (int)rank * seg;
   const int m = max(0, min(n - lo, seg));
   const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + lo;
-  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-    const int m4 = m >> 2;
-    for (int i = threadIdx.x; i < m4; i += TK_THREADS) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
-      reinterpret_cast<uint4*>(seg_keys)[i] =
-          make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
-    }
-    for (int i = (m4 << 2) + threadIdx.x; i < m; i += TK_THREADS) seg_keys[i] = score_key(__ldg(src + i));
-  } else {
-    for (int i = threadIdx.x; i < m; i += TK_THREADS) seg_keys[i] = score_key(__ldg(src + i));
-  }
+  for (int i = threadIdx.x; i < 2048; i += TK_THREADS) hist[i] = 0u;
   __syncthreads();
+  stage_keys(src, m, seg_keys, hist);   // with the first digit's histogram
+  const SmemKeys keys{seg_keys};
   uint32_t prefix = 0, need = (uint32_t)a.k;
-  cluster_pass<11>(seg_keys, m, 21, true, prefix, need, hist, ghist, tmp, sel);
-  cluster_pass<11>(seg_keys, m, 10, false, prefix, need, hist, ghist, tmp, sel);
-  cluster_pass<10>(seg_keys, m, 0, false, prefix, need, hist, ghist, tmp, sel);
+  cluster_find<11>(true, prefix, need, hist, ghist, tmp, sel);   // its cluster barrier publishes the keys
+  cluster_pass<11>(keys, m, 10, prefix, need, hist, ghist, tmp, sel);
+  cluster_pass<10>(keys, m, 0, prefix, need, hist, ghist, tmp, sel);
   const uint32_t T = prefix;
   const uint32_t need_eq = need;
 
-  // counts of this segment, then the counts of the segments before it
-  uint32_t g = 0, e = 0;
-  for (int i = threadIdx.x; i < m; i += TK_THREADS) {
-    g += seg_keys[i] > T;
-    e += seg_keys[i] == T;
-  }
-  uint32_t total;
-  block_excl_scan((e << 16) | g, tmp, total);   // segment of <= 48K keys: counts fit 16 bits
+  // this CTA's counts, then the counts of the segments before it
+  const Run run = warp_run(m);
+  uint32_t G, E, g_tot, e_tot;
+  block_run_offsets(keys, m, T, run, tmp, G, E, g_tot, e_tot);
   if (threadIdx.x == 0) {
-    counts[0] = total & 0xFFFFu;
-    counts[1] = total >> 16;
+    counts[0] = g_tot;
+    counts[1] = e_tot;
   }
   cluster_sync();
-  uint32_t g_run = 0, e_run = 0;
   const uint32_t c0 = smem_u32(counts);
   for (uint32_t p = 0; p < rank; ++p) {
-    g_run += ld_cluster_u32(mapa_shared(c0, p));
-    e_run += ld_cluster_u32(mapa_shared(c0 + 4u, p));
+    G += ld_cluster_u32(mapa_shared(c0, p));
+    E += ld_cluster_u32(mapa_shared(c0 + 4u, p));
   }
-  for (int base = 0; base < m; base += TK_THREADS * TK_ITEMS) {
-    const int i0 = base + threadIdx.x * TK_ITEMS;
-    uint32_t keys[TK_ITEMS];
-#pragma unroll
-    for (int j = 0; j < TK_ITEMS; ++j) keys[j] = (i0 + j < m) ? seg_keys[i0 + j] : 0u;
-    uint32_t gl = 0, el = 0;
-#pragma unroll
-    for (int j = 0; j < TK_ITEMS; ++j) {
-      if (i0 + j < m) {
-        gl += keys[j] > T;
-        el += keys[j] == T;
-      }
-    }
-    uint32_t tot;
-    const uint32_t excl = block_excl_scan((el << 16) | gl, tmp, tot);
-    uint32_t G = g_run + (excl & 0xFFFFu);
-    uint32_t E = e_run + (excl >> 16);
-#pragma unroll
-    for (int j = 0; j < TK_ITEMS; ++j) {
-      if (i0 + j < m) {
-        if (keys[j] > T) {
-          dst[G + min(E, need_eq)] = lo + i0 + j;
-          if (dsc != nullptr) dsc[G + min(E, need_eq)] = key_score(keys[j]);
-          ++G;
-        } else if (keys[j] == T) {
-          if (E < need_eq) {
-            dst[G + E] = lo + i0 + j;
-            if (dsc != nullptr) dsc[G + E] = key_score(keys[j]);
-          }
-          ++E;
-        }
-      }
-    }
-    g_run += tot & 0xFFFFu;
-    e_run += tot >> 16;
-  }
+  write_run(keys, m, T, need_eq, G, E, lo, run, dst, dsc);
   cluster_sync();   // peers are done reading `counts` before this CTA exits
 }
 
