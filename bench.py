@@ -409,9 +409,6 @@ def time_indexer_kl(name: str, steps: int, warmup: int, world: int, rank: int, p
     return res
 
 
-FP64_NOMINAL_TFLOPS = 37.0   # B200 datasheet fp64, for context (no measured fp64 peak)
-
-
 def time_backward(name: str, steps: int, warmup: int, world: int, rank: int, pk: dict):
     """The sparse-stage gradients on the workload's own selected sets, each timed with
     CUDA events on the launching stream: the attention backward (dsa_sparse_mla_bwd,
@@ -491,15 +488,16 @@ def time_backward(name: str, steps: int, warmup: int, world: int, rank: int, pk:
                                       "peak_note": "measured bf16 sustained; work = "
                                                    "2 H (3 Dqk + 2 Dv) per selected pair"}},
            "indexer": {"ms_per_step": ms_idx, "launches_per_step": launches.get("indexer"),
-                       "roofline": {"bound": "fp64", "achieved": idx_tf,
-                                    "peak": FP64_NOMINAL_TFLOPS, "unit": "TFLOP/s",
-                                    "frac": idx_tf / FP64_NOMINAL_TFLOPS, "traffic": None,
-                                    "peak_note": "nominal B200 fp64 (not measured); work = "
-                                                 "6 H_I d_I per selected pair"}},
-           "note": "gradients of the sparse training stage: cuBLAS strided-batched GEMMs over "
-                   "gathered rows (bf16 for attention, fp64 for the indexer) with this library's "
-                   "gather, softmax/ReLU-gradient and scatter-add kernels; launches count this "
-                   "library's kernels only"}
+                       "roofline": {"bound": "tensor", "achieved": idx_tf,
+                                    "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                                    "frac": idx_tf / pk["bf16_sustained"], "traffic": None,
+                                    "peak_note": "measured bf16 sustained; work = 6 H_I d_I per "
+                                                 "selected pair (the three-term bf16 split of the "
+                                                 "gradient factors executes 14 H_I d_I)"}},
+           "note": "gradients of the sparse training stage: this library's batched tcgen05 bf16 "
+                   "GEMMs (fp32 accumulation) over gathered rows, with its gather, "
+                   "softmax/ReLU-gradient and scatter-add kernels; the indexer's ReLU mask is "
+                   "re-decided exactly in fp64 near zero"}
     del inp, out, lse, idx, dout, sel, pt, dq, dkv, ws, dI, dqI, dkI, dw, wsi
     torch.cuda.empty_cache()
     return res

@@ -187,17 +187,16 @@ int dsa_indexer_kl(const uint16_t* q, const uint16_t* kv, const int32_t* idx, co
  * stage the main model is trained through attention over the top-k selected
  * entries, and the indexer keeps training on the KL over the selected tokens with
  * its input detached from the main model's graph.) The contractions run as
- * strided-batched cuBLAS GEMMs (bf16 operands with fp32 accumulation for the
- * attention, fp64 for the indexer) over the selected rows, gathered per chunk of
- * up to 64 tokens into the workspace; the gathers, the softmax / ReLU gradients and
- * the scatter-add of key gradients are this library's kernels. The first call on
- * a device creates a cuBLAS handle, which keeps a small device allocation of
- * cuBLAS's own until the process exits; GEMM scratch comes from `ws`. Key
- * gradients are accumulated with atomics, so their last bits may differ from
- * run to run. All pointers are caller-owned device memory, 16-byte aligned.
+ * batched bf16 GEMMs on the tensor cores (tcgen05, fp32 accumulation) over the
+ * selected rows, gathered per chunk of up to 64 tokens into the workspace; the
+ * gathers, the softmax / ReLU gradients and the scatter-add of key gradients are
+ * kernels of this library too, and nothing is allocated. Key gradients are
+ * accumulated with atomics, so their last bits may differ from run to run. All
+ * pointers are caller-owned device memory, 16-byte aligned.
  * Errors: DSA_ERR_INVALID_ARG (null or misaligned pointer, bad scalar),
  * DSA_ERR_UNSUPPORTED_SHAPE, DSA_ERR_WORKSPACE_TOO_SMALL (below one token's
- * share), DSA_ERR_CUDA (a launch or cuBLAS call failed).
+ * share), DSA_ERR_CUDA (a launch failed); a device wait that ran out is reported
+ * by dsa_check_status.
  *
  * dsa_sparse_mla_bwd - gradients of the sparse attention (dsa_sparse_mla_fwd)
  * with respect to q and the latent rows, given dout = dL/d(out). With
@@ -248,8 +247,12 @@ int dsa_indexer_kl_grad(const float* sel_scores, const float* p, const int32_t* 
  *   kI_scale [B, Lk], w [B, Lq, H_I] (w_dtype) as for dsa_indexer_scores;
  *   idx, dI [B, Lq, k] aligned (slots < 0 or >= Lk skipped); dqI
  *   [B, Lq, H_I, d_I], dw [B, Lq, H_I] fp32 (overwritten); dkI [B, Lk, d_I] fp32,
- *   zeroed first unless accumulate_dkI != 0. The contractions run in fp64, where
- *   the dots of the e4m3 codes are exact, so the ReLU mask is decided exactly.
+ *   zeroed first unless accumulate_dkI != 0. The code dots qhat . khat run on
+ *   the tensor cores with fp32 accumulation (every product of two e4m3 codes is
+ *   exact); wherever their rounding could flip the sign (|X| within 2^-12
+ *   |qhat| |khat| of zero) the dot is recomputed exactly in fp64, so the ReLU mask
+ *   is the exact code dot's. The gradient factors g enter the two remaining
+ *   products as three bf16 terms each (24 significant bits).
  *   ws: dsa_indexer_bwd_workspace_size(...) bytes; less makes smaller chunks.
  */
 size_t dsa_indexer_bwd_workspace_size(int B, int Lq, int H_I, int d_I, int k);
@@ -263,8 +266,8 @@ int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
  * dsa_last_launch_count - number of kernel launches that the calling thread's
  * last dsa_forward, dsa_forward_host, dsa_forward_profiled, dsa_sparse_mla_bwd,
  * dsa_indexer_bwd or dsa_indexer_kl_grad call enqueued (all of this library's
- * kernels, on the caller's stream and on the library's internal side stream;
- * not cuBLAS's). 0 before the first call. For benchmarks that report how many
+ * kernels, on the caller's stream and on the library's internal side stream).
+ * 0 before the first call. For benchmarks that report how many
  * of the library's kernels ran in a timed region.
  */
 int dsa_last_launch_count(void);

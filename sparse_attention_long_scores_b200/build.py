@@ -18,13 +18,14 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libdsa.so")
-SOURCES = ["dsa_api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "indexer_kl.cu", "backward.cu"]
+SOURCES = ["dsa_api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "indexer_kl.cu", "backward.cu",
+           "bgemm.cu"]
 HEADERS = ["dsa_common.cuh", "dsa_kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-# cuBLAS runs the batched GEMMs of the sparse-stage gradients.
-CUDA_LIB = "/usr/local/cuda/lib64"
-LINK = ["-L" + CUDA_LIB, "-lcublas", "-Xlinker", "-rpath=" + CUDA_LIB]
+# The driver API (tensor-map encoding) is reached through the runtime entry-point
+# query, so nothing beyond the CUDA runtime is linked.
+LINK: list = []
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 

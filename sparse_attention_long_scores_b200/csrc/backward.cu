@@ -4,11 +4,12 @@
 // learns through attention over the selected entries, and the indexer through
 // its own detached inputs with the KL on the selected tokens).
 //
-// The contractions of both gradients run as batched GEMMs (dsa_api.cu) over
-// the selected rows gathered here into a dense per-token block; these kernels
-// do the gathers, the softmax / ReLU gradient in between and the scatter-add of
-// the per-token key gradients back into the shared rows. Every kernel is a
-// grid-stride loop over rows with one warp per row, so any grid size is correct.
+// The contractions of both gradients run as batched tensor-core GEMMs
+// (bgemm.cu) over the selected rows gathered here into a dense per-token block;
+// these kernels do the gathers, the softmax / ReLU gradient in between and the
+// scatter-add of the per-token key gradients back into the shared rows. The
+// row kernels are grid-stride loops with one warp per row, so any grid size is
+// correct.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -175,11 +176,12 @@ __global__ void scatter_add_rows_kernel(const float4* __restrict__ src,
   }
 }
 
-// out[tt][j][:] = khat[b][idx[tok][j]][:] as float64 for e4m3 rows of d_I bytes
-// (the unscaled codes), zeros for a slot without a valid key.
-__global__ void gather_e4m3_rows_kernel(const uint8_t* __restrict__ kI,
-                                        const int32_t* __restrict__ idx, double* __restrict__ out,
-                                        long long tok0, int T, int Lq, int Lk, int k, int d_I) {
+// out[tt][j][:] = khat[b][idx[tok][j]][:] as bf16 for e4m3 rows of d_I bytes (the
+// unscaled codes, which bf16 holds exactly), zeros for a slot without a valid key.
+__global__ void gather_e4m3_rows_bf16_kernel(const uint8_t* __restrict__ kI,
+                                             const int32_t* __restrict__ idx,
+                                             uint16_t* __restrict__ out, long long tok0, int T,
+                                             int Lq, int Lk, int k, int d_I) {
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(T) * k;
   for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
@@ -187,101 +189,145 @@ __global__ void gather_e4m3_rows_kernel(const uint8_t* __restrict__ kI,
     const int j = static_cast<int>(r % k);
     const int s = selected_key(idx, tok, j, k, Lk);
     const long long b = tok / Lq;
-    double* dst = out + r * d_I;
+    uint16_t* dst = out + r * d_I;
     for (int c = lane; c < d_I; c += 32)
-      dst[c] = s < 0 ? 0.0 : static_cast<double>(e4m3_to_float(kI[(b * Lk + s) * d_I + c]));
+      dst[c] = s < 0 ? uint16_t(0) : float_to_bf16_bits(e4m3_to_float(kI[(b * Lk + s) * d_I + c]));
   }
 }
 
-// out[i] = codes[i] as float64 for n e4m3 codes.
-__global__ void decode_e4m3_kernel(const uint8_t* __restrict__ codes, double* __restrict__ out,
-                                   long long n) {
+// out[i] = codes[i] as bf16 (exact) for n e4m3 codes.
+__global__ void decode_e4m3_bf16_kernel(const uint8_t* __restrict__ codes,
+                                        uint16_t* __restrict__ out, long long n) {
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x)
-    out[i] = static_cast<double>(e4m3_to_float(codes[i]));
+    out[i] = float_to_bf16_bits(e4m3_to_float(codes[i]));
 }
 
-// out[i] = (float)in[i].
-__global__ void f64_to_f32_kernel(const double* __restrict__ in, float* __restrict__ out,
-                                  long long n) {
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    out[i] = static_cast<float>(in[i]);
+// Three bf16 terms whose sum is v to 24 significant bits: each residual
+// v - hi is exact in fp32, so the terms carry 8 + 8 + 8 bits.
+__device__ __forceinline__ void split3(float v, uint16_t& a, uint16_t& b, uint16_t& c) {
+  a = float_to_bf16_bits(v);
+  const float r1 = v - bf16_bits_to_float(a);
+  b = float_to_bf16_bits(r1);
+  const float r2 = r1 - bf16_bits_to_float(b);
+  c = float_to_bf16_bits(r2);
 }
 
-// dst[b][idx[tok][j]][:] += (float)src[tt][j][:] for float64 rows of D values
-// (D % 4 == 0), four at a time (atomic).
-__global__ void scatter_add_rows_f64_kernel(const double* __restrict__ src,
-                                            const int32_t* __restrict__ idx,
-                                            float4* __restrict__ dst, long long tok0, int T,
-                                            int Lq, int Lk, int k, int V) {
-  const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(T) * k;
-  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
-    const long long tok = tok0 + r / k;
-    const int j = static_cast<int>(r % k);
-    const int s = selected_key(idx, tok, j, k, Lk);
-    if (s < 0) continue;
-    const long long b = tok / Lq;
-    float4* d = dst + (b * Lk + s) * V;
-    const double* x = src + r * V * 4;
-    for (int v = lane; v < V; v += 32) {
-      const float4 f = make_float4(static_cast<float>(x[4 * v]), static_cast<float>(x[4 * v + 1]),
-                                   static_cast<float>(x[4 * v + 2]),
-                                   static_cast<float>(x[4 * v + 3]));
-      atomicAdd(d + v, f);
-    }
+// The code dots X = qhat_j . khat_s come from a tensor-core product with fp32
+// accumulation; an fp32 sum of d_I <= 128 exact products is within
+// d_I 2^-23 sum_i |qhat_ji khat_si| <= 2^-16 |qhat_j| |khat_s| of the exact dot.
+// Where |X| is within kDotBand |qhat_j| |khat_s| of zero (sixteen times that bound)
+// the dot is recomputed exactly in fp64, so the ReLU mask is the exact code
+// dot's sign.
+constexpr float kDotBand = 1.0f / 4096.0f;
+constexpr int kReluThreads = 256;
+constexpr int kReluMaxHeads = 64;
+constexpr int kReluMaxDim = 128;
+
+// ReLU gradient for token tt of the chunk and 256 of its slots (one thread per
+// slot), from XT [T][k][H_I] (fp32 code dots), the gathered key codes Kb
+// [T][k][d_I] and the query codes Qb [T][H_I][d_I] (bf16). With the dequantised
+// dot x = s^q_j s^k_s X:
+//   dw_j    += sum_s dI_s max(x, 0)                     (dw zeroed by the caller)
+//   g       = dI_s w_j [X > 0]
+//   G1[j,s] = g s^k_s   -> G1s [T][H_I][3 kp]: part p at columns p kp + s
+//   G2[j,s] = g s^q_j   -> G2s [T][3 hp][k]:  part p at rows p hp + j
+// (three bf16 parts each, see split3), so that dq^I_j = sum_s G1[j,s] khat_s and
+// dk^I_s = sum_j G2[j,s] qhat_j run as bf16 tensor-core products with fp32-level
+// accuracy. Columns k..kp-1 of G1s and rows H_I..hp-1 of G2s are written as zeros.
+__global__ void __launch_bounds__(kReluThreads) indexer_bwd_relu_tc_kernel(
+    const float* __restrict__ XT, const uint16_t* __restrict__ Kb,
+    const uint16_t* __restrict__ Qb, const int32_t* __restrict__ idx,
+    const float* __restrict__ dI, const float* __restrict__ qI_scale,
+    const float* __restrict__ kI_scale, const void* __restrict__ w, int w_bf16,
+    uint16_t* __restrict__ G1s, uint16_t* __restrict__ G2s, float* __restrict__ dw,
+    long long tok0, int Lq, int Lk, int H_I, int d_I, int k, int kp, int hp) {
+  __shared__ float s_q[kReluMaxHeads * kReluMaxDim];
+  __shared__ float s_sq[kReluMaxHeads], s_w[kReluMaxHeads], s_qn[kReluMaxHeads];
+  __shared__ float s_dw[kReluMaxHeads];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tt = blockIdx.y;
+  const long long tok = tok0 + tt;
+  const long long b = tok / Lq;
+  for (int i = threadIdx.x; i < H_I * d_I; i += kReluThreads)
+    s_q[i] = bf16_bits_to_float(Qb[static_cast<long long>(tt) * H_I * d_I + i]);
+  for (int j = threadIdx.x; j < H_I; j += kReluThreads) {
+    const long long qrow = tok * H_I + j;
+    s_sq[j] = qI_scale[qrow];
+    s_w[j] = w_bf16 ? bf16_bits_to_float(static_cast<const uint16_t*>(w)[qrow])
+                    : static_cast<const float*>(w)[qrow];
+    s_dw[j] = 0.f;
   }
-}
+  __syncthreads();
+  for (int j = warp; j < H_I; j += kReluThreads / 32) {
+    float acc = 0.f;
+    for (int c = lane; c < d_I; c += 32) acc += s_q[j * d_I + c] * s_q[j * d_I + c];
+    acc = warp_sum(acc);
+    if (lane == 0) s_qn[j] = sqrtf(acc);
+  }
+  __syncthreads();
 
-// ReLU gradient of one (token, indexer head j) row over its k slots. X holds the
-// dots qhat_j . khat_s of the codes (exact in float64); with the dequantised dot
-// x = s^q_j s^k_s X:
-//   dw_j    = sum_s dI_s max(x, 0)
-//   g_s     = dI_s w_j [X > 0]
-//   G1[j,s] = g_s s^k_s   (dq^I_j = sum_s G1[j,s] khat_s)
-//   G2[j,s] = g_s s^q_j   (dk^I_s = sum_j G2[j,s] qhat_j)
-__global__ void indexer_bwd_relu_kernel(const double* __restrict__ X,
-                                        const int32_t* __restrict__ idx,
-                                        const float* __restrict__ dI,
-                                        const float* __restrict__ qI_scale,
-                                        const float* __restrict__ kI_scale,
-                                        const void* __restrict__ w, int w_bf16,
-                                        double* __restrict__ G1, double* __restrict__ G2,
-                                        float* __restrict__ dw, long long tok0, int T, int Lq,
-                                        int Lk, int H_I, int k) {
-  const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(T) * H_I;
-  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
-    const long long tok = tok0 + r / H_I;
-    const int jh = static_cast<int>(r % H_I);
-    const long long b = tok / Lq;
-    const long long qrow = tok * H_I + jh;
-    const double sq = qI_scale[qrow];
-    const double wj = w_bf16 ? bf16_bits_to_float(static_cast<const uint16_t*>(w)[qrow])
-                             : static_cast<const float*>(w)[qrow];
-    const double* xrow = X + r * k;
-    double* g1 = G1 + r * k;
-    double* g2 = G2 + r * k;
-    double acc = 0.0;
-    for (int j = lane; j < k; j += 32) {
-      const int s = selected_key(idx, tok, j, k, Lk);
-      double a = 0.0, c = 0.0;
-      if (s >= 0) {
-        const double xh = xrow[j];
-        const double sk = kI_scale[b * Lk + s];
-        const double d = dI[tok * k + j];
-        acc += d * fmax(xh * sq * sk, 0.0);
-        const double g = xh > 0.0 ? d * wj : 0.0;
-        a = g * sk;
-        c = g * sq;
+  const int slot = blockIdx.x * kReluThreads + threadIdx.x;
+  const bool in_row = slot < k;
+  const uint16_t* krow = Kb + (static_cast<long long>(tt) * k + slot) * d_I;
+  int s = -1;
+  float d = 0.f, sk = 0.f, kn = 0.f;
+  if (in_row) {
+    s = selected_key(idx, tok, slot, k, Lk);
+    if (s >= 0) {
+      d = dI[tok * k + slot];
+      sk = kI_scale[b * Lk + s];
+      float acc = 0.f;
+      for (int c = 0; c < d_I; ++c) {
+        const float v = bf16_bits_to_float(krow[c]);
+        acc += v * v;
       }
-      g1[j] = a;
-      g2[j] = c;
+      kn = sqrtf(acc);
     }
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) dw[qrow] = static_cast<float>(acc);
   }
+  const float* xrow = XT + (static_cast<long long>(tt) * k + slot) * H_I;
+  uint16_t* g1row = G1s + static_cast<long long>(tt) * H_I * 3 * kp + slot;
+  uint16_t* g2col = G2s + static_cast<long long>(tt) * 3 * hp * k + slot;
+  for (int j = 0; j < hp; ++j) {
+    float g1 = 0.f, g2 = 0.f, contrib = 0.f;
+    if (s >= 0 && j < H_I) {
+      const float x = xrow[j];
+      double xe = x;
+      if (fabsf(x) <= kDotBand * kn * s_qn[j]) {
+        double e = 0.0;   // exact: products of codes need <= 8 bits, sums stay on a 2^-18 grid below 2^25
+        for (int c = 0; c < d_I; ++c)
+          e += static_cast<double>(s_q[j * d_I + c]) * static_cast<double>(bf16_bits_to_float(krow[c]));
+        xe = e;
+      }
+      if (xe > 0.0) {
+        const float g = d * s_w[j];
+        g1 = g * sk;
+        g2 = g * s_sq[j];
+        contrib = static_cast<float>(static_cast<double>(d) *
+                                     (static_cast<double>(s_sq[j]) * static_cast<double>(sk) * xe));
+      }
+    }
+    const float wsum = warp_sum(contrib);
+    if (lane == 0 && j < H_I && wsum != 0.f) atomicAdd(&s_dw[j], wsum);
+    if (j < H_I && slot < kp) {
+      uint16_t a0, a1, a2;
+      split3(g1, a0, a1, a2);
+      uint16_t* g1p = g1row + static_cast<long long>(j) * 3 * kp;
+      g1p[0] = a0;
+      g1p[kp] = a1;
+      g1p[2 * kp] = a2;
+    }
+    if (in_row) {
+      uint16_t c0, c1, c2;
+      split3(g2, c0, c1, c2);
+      g2col[static_cast<long long>(j) * k] = c0;
+      g2col[static_cast<long long>(hp + j) * k] = c1;
+      g2col[static_cast<long long>(2 * hp + j) * k] = c2;
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < H_I; j += kReluThreads)
+    if (s_dw[j] != 0.f) atomicAdd(&dw[tok * H_I + j], s_dw[j]);
 }
 
 // dI = loss_scale (softmax(sel over the set) - p) per row of k slots; 0 outside
@@ -368,44 +414,33 @@ cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float*
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_e4m3_rows(const uint8_t* kI, const int32_t* idx, double* out,
-                                    long long tok0, int T, int Lq, int Lk, int k, int d_I,
-                                    int num_sms, cudaStream_t stream) {
+cudaError_t launch_gather_e4m3_rows_bf16(const uint8_t* kI, const int32_t* idx, uint16_t* out,
+                                         long long tok0, int T, int Lq, int Lk, int k, int d_I,
+                                         int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(T) * k;
-  gather_e4m3_rows_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
+  gather_e4m3_rows_bf16_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
       kI, idx, out, tok0, T, Lq, Lk, k, d_I);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_e4m3(const uint8_t* codes, double* out, long long n, int num_sms,
-                               cudaStream_t stream) {
-  decode_e4m3_kernel<<<flat_blocks(n, num_sms), kRowThreads, 0, stream>>>(codes, out, n);
+cudaError_t launch_decode_e4m3_bf16(const uint8_t* codes, uint16_t* out, long long n, int num_sms,
+                                    cudaStream_t stream) {
+  decode_e4m3_bf16_kernel<<<flat_blocks(n, num_sms), kRowThreads, 0, stream>>>(codes, out, n);
   return cudaGetLastError();
 }
 
-cudaError_t launch_f64_to_f32(const double* in, float* out, long long n, int num_sms,
-                              cudaStream_t stream) {
-  f64_to_f32_kernel<<<flat_blocks(n, num_sms), kRowThreads, 0, stream>>>(in, out, n);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_scatter_add_rows_f64(const double* src, const int32_t* idx, float* dst,
-                                        long long tok0, int T, int Lq, int Lk, int k, int D,
-                                        int num_sms, cudaStream_t stream) {
-  const long long rows = static_cast<long long>(T) * k;
-  scatter_add_rows_f64_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
-      src, idx, reinterpret_cast<float4*>(dst), tok0, T, Lq, Lk, k, D / 4);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_indexer_bwd_relu(const double* X, const int32_t* idx, const float* dI,
-                                    const float* qI_scale, const float* kI_scale, const void* w,
-                                    int w_bf16, double* G1, double* G2, float* dw,
-                                    long long tok0, int T, int Lq, int Lk, int H_I, int k,
-                                    int num_sms, cudaStream_t stream) {
-  const long long rows = static_cast<long long>(T) * H_I;
-  indexer_bwd_relu_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
-      X, idx, dI, qI_scale, kI_scale, w, w_bf16, G1, G2, dw, tok0, T, Lq, Lk, H_I, k);
+cudaError_t launch_indexer_bwd_relu_tc(const float* XT, const uint16_t* Kb, const uint16_t* Qb,
+                                       const int32_t* idx, const float* dI,
+                                       const float* qI_scale, const float* kI_scale,
+                                       const void* w, int w_bf16, uint16_t* G1s, uint16_t* G2s,
+                                       float* dw, long long tok0, int T, int Lq, int Lk, int H_I,
+                                       int d_I, int k, int kp, int hp, cudaStream_t stream) {
+  if (H_I > kReluMaxHeads || d_I > kReluMaxDim || T > 65535) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>((kp + kReluThreads - 1) / kReluThreads),
+                  static_cast<unsigned>(T));
+  indexer_bwd_relu_tc_kernel<<<grid, kReluThreads, 0, stream>>>(
+      XT, Kb, Qb, idx, dI, qI_scale, kI_scale, w, w_bf16, G1s, G2s, dw, tok0, Lq, Lk, H_I, d_I,
+      k, kp, hp);
   return cudaGetLastError();
 }
 

@@ -3,7 +3,6 @@
 // forward path (indexer -> top-k -> sparse MLA; "DeepSeek-V3.2: Pushing the
 // Frontier of Open Large Language Models", bud-325 paper digest, "Key claims",
 // section 2.1 Eq. 1-2, and "Method").
-#include <cublas_v2.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -126,6 +125,25 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int el
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DSA_OK;
+}
+
+// 3-D tiled tensor map over [depth][rows][inner] elements with row stride
+// `row_stride` and depth stride `depth_stride` (in elements).
+int make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                uint64_t inner, uint64_t rows, uint64_t depth, uint64_t row_stride,
+                uint64_t depth_stride, uint32_t box_inner, uint32_t box_rows,
+                CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (driver too old?)");
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {row_stride * (uint64_t)elem_bytes, depth_stride * (uint64_t)elem_bytes};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
   return DSA_OK;
 }
 
@@ -1122,69 +1140,52 @@ int dsa_debug_wait_timeout(void* stream) {
 // detached inputs with the KL on the selected tokens).
 //
 // Per chunk of T tokens the selected rows are gathered into a dense [T, k, D]
-// block, the per-token contractions run as strided-batched GEMMs in cuBLAS
-// (bf16 operands with fp32 accumulation for the attention, fp64 for the
-// indexer), and the per-token key gradients are scatter-added into the shared
-// rows. The cuBLAS handle of each device is created on first use and keeps a
-// small device allocation of cuBLAS's own until the process exits; GEMM scratch
-// comes from the caller's workspace.
+// block, the per-token contractions run as batched bf16 tensor-core GEMMs with
+// fp32 accumulation (bgemm.cu), and the per-token key gradients are
+// scatter-added into the shared rows. The indexer's code dots are exact up to
+// fp32 rounding and the ReLU mask is re-decided exactly in fp64 wherever that
+// rounding could change its sign; its real-valued gradient operands enter the
+// products as three bf16 terms (24 significant bits).
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kBlasWorkspace = size_t(32) << 20;   // cuBLAS scratch per call
 constexpr int kBwdChunkTokens = 64;                   // tokens per gathered block
 
-struct Blas {
-  std::mutex mu;
-  cublasHandle_t h = nullptr;
+// One operand of a batched product: `depth` blocks of `rows` rows of `inner`
+// contiguous bf16 elements; mn says whether the contiguous dimension is M / N
+// (else K). period: K tiles of 64 after which the operand repeats (0: none).
+struct GemmOperand {
+  const void* base;
+  bool mn;
+  uint64_t inner, rows, depth, row_stride, depth_stride;
+  int period;
 };
-Blas g_blas[kMaxDevices];
 
-int blas_fail(cublasStatus_t st, const char* what) {
-  return fail(DSA_ERR_CUDA, "%s: cuBLAS status %d", what, static_cast<int>(st));
-}
-
-#define DSA_TRY_BLAS(expr, what)                                   \
-  do {                                                             \
-    cublasStatus_t b_ = (expr);                                    \
-    if (b_ != CUBLAS_STATUS_SUCCESS) return blas_fail(b_, what);   \
-  } while (0)
-
-int blas_for_device(Blas** out) {
-  int dev = 0;
-  DSA_TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_CUDA, "device ordinal %d out of range", dev);
-  Blas& b = g_blas[dev];
-  std::lock_guard<std::mutex> lk(b.mu);
-  if (b.h == nullptr) DSA_TRY_BLAS(cublasCreate(&b.h), "cublasCreate");
-  *out = &b;
-  return DSA_OK;
-}
-
-// Row-major strided-batched GEMM: C[M x N] = op(A)[M x K] op(B)[K x N] + beta C.
-// A is stored row-major as [M x K] (tA false) or [K x M] (tA true) with leading
-// dimension lda, B as [K x N] or [N x K] with ldb. Operands of `type`: bf16 or
-// fp32 accumulate and write fp32; fp64 accumulates and writes fp64. cuBLAS is
-// column-major and a row-major X is the column-major X^T, so this is the
-// column-major product C^T = op(B)^T op(A)^T.
-int gemm_rm(cublasHandle_t h, bool tA, bool tB, int M, int N, int K, const void* A, int lda,
-            long long sA, const void* B, int ldb, long long sB, double beta, void* C, int ldc,
-            long long sC, int batch, cudaDataType_t type, const char* what) {
-  const cublasOperation_t opB = tB ? CUBLAS_OP_T : CUBLAS_OP_N;
-  const cublasOperation_t opA = tA ? CUBLAS_OP_T : CUBLAS_OP_N;
-  if (type == CUDA_R_64F) {
-    const double alpha = 1.0;
-    DSA_TRY_BLAS(cublasGemmStridedBatchedEx(h, opB, opA, N, M, K, &alpha, B, type, ldb, sB, A,
-                                            type, lda, sA, &beta, C, CUDA_R_64F, ldc, sC, batch,
-                                            CUBLAS_COMPUTE_64F, CUBLAS_GEMM_DEFAULT),
-                 what);
-  } else {
-    const float alpha = 1.f, beta32 = static_cast<float>(beta);
-    DSA_TRY_BLAS(cublasGemmStridedBatchedEx(h, opB, opA, N, M, K, &alpha, B, type, ldb, sB, A,
-                                            type, lda, sA, &beta32, C, CUDA_R_32F, ldc, sC, batch,
-                                            CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT),
-                 what);
-  }
+// C[z] (fp32, element (z, m, n) at C + z sC + m c_sm + n c_sn) = A[z] B[z]^T.
+int tc_gemm(const GemmOperand& A, const GemmOperand& B, int M, int N, int K, float* C,
+            long long c_sm, long long c_sn, long long sC, int batch, const dsa::DevCtl& ctl,
+            cudaStream_t s, const char* what) {
+  const int bn = dsa::bgemm_tile_n(N);
+  CUtensorMap ta, tb;
+  DSA_TRY(make_map_3d(&ta, A.base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A.inner, A.rows, A.depth,
+                      A.row_stride, A.depth_stride, 64, A.mn ? 64 : 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
+  DSA_TRY(make_map_3d(&tb, B.base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B.inner, B.rows, B.depth,
+                      B.row_stride, B.depth_stride, 64, B.mn ? 64 : (uint32_t)bn,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
+  const int kt = (K + 63) / 64;
+  dsa::BgemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.a_kt = A.period > 0 ? A.period : kt;
+  a.b_kt = B.period > 0 ? B.period : kt;
+  a.C = C;
+  a.c_sm = c_sm;
+  a.c_sn = c_sn;
+  a.sC = sC;
+  a.ctl = ctl;
+  DSA_TRY_CUDA(dsa::launch_bgemm(ta, tb, a, batch, A.mn, B.mn, bn, s), what);
   return DSA_OK;
 }
 
@@ -1195,7 +1196,7 @@ char* align256(void* p) {
 // Workspace of the attention backward for T tokens (offsets from a 256-byte
 // aligned base; total includes the alignment slack).
 struct MlaBwdLayout {
-  size_t cg, qo, sp, pz, dc, blas, total;
+  size_t cg, qo, sp, pz, dc, total;
 };
 MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
   MlaBwdLayout L{};
@@ -1211,16 +1212,15 @@ MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
   L.sp = take(t2hk * sizeof(float));                     // [q . c; dout . c[:Dv]]
   L.pz = take(t2hk * sizeof(uint16_t));                  // [dz; P], bf16
   L.dc = take(tk * Dqk * sizeof(float));                 // per-token row gradients
-  L.blas = take(kBlasWorkspace);
   L.total = off + 256;
   return L;
 }
 
-// The indexer backward works in fp64: the dots of the e4m3 codes are then exact
-// (each product needs at most 8 significant bits and every partial sum is a
-// multiple of 2^-18 below 2^25), so the ReLU mask is decided exactly.
+// Workspace of the indexer backward for T tokens; kp = k rounded up to 64,
+// hp = H_I rounded up to 64 (the K tiles of the split products).
 struct IdxBwdLayout {
-  size_t kd, qd, x, g1, g2, dk, dq, blas, total;
+  size_t kb, qb, xt, g1, g2, dk, total;
+  int kp, hp;
 };
 IdxBwdLayout idx_bwd_layout(int T, int H_I, int d_I, int k) {
   IdxBwdLayout L{};
@@ -1230,15 +1230,15 @@ IdxBwdLayout idx_bwd_layout(int T, int H_I, int d_I, int k) {
     off += align_up(bytes, 256);
     return o;
   };
-  const size_t tk = (size_t)T * k, thk = (size_t)T * H_I * k, thd = (size_t)T * H_I * d_I;
-  L.kd = take(tk * d_I * sizeof(double));     // gathered key codes, decoded
-  L.qd = take(thd * sizeof(double));          // query codes, decoded
-  L.x = take(thk * sizeof(double));           // code dots
-  L.g1 = take(thk * sizeof(double));
-  L.g2 = take(thk * sizeof(double));
-  L.dk = take(tk * d_I * sizeof(double));     // per-token key gradients
-  L.dq = take(thd * sizeof(double));          // query gradients before the fp32 store
-  L.blas = take(kBlasWorkspace);
+  L.kp = (k + 63) / 64 * 64;
+  L.hp = (H_I + 63) / 64 * 64;
+  const size_t tk = (size_t)T * k;
+  L.kb = take(tk * d_I * sizeof(uint16_t));                        // gathered key codes
+  L.qb = take((size_t)T * H_I * d_I * sizeof(uint16_t));           // query codes
+  L.xt = take(tk * H_I * sizeof(float));                           // code dots [T][k][H_I]
+  L.g1 = take((size_t)T * H_I * 3 * L.kp * sizeof(uint16_t));      // G1 in three parts
+  L.g2 = take((size_t)T * 3 * L.hp * k * sizeof(uint16_t));        // G2 in three parts
+  L.dk = take(tk * d_I * sizeof(float));                           // per-token key gradients
   L.total = off + 256;
   return L;
 }
@@ -1284,9 +1284,6 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
   dsa::DevCtl ctl;
   int sms = 0;
   DSA_TRY(device_ctl(ctl, sms));
-  Blas* bl = nullptr;
-  DSA_TRY(blas_for_device(&bl));
-  std::lock_guard<std::mutex> lk(bl->mu);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = align256(ws);
   uint16_t* cg = reinterpret_cast<uint16_t*>(base + L.cg);
@@ -1294,35 +1291,39 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
   float* SP = reinterpret_cast<float*>(base + L.sp);
   uint16_t* PZ = reinterpret_cast<uint16_t*>(base + L.pz);
   float* dC = reinterpret_cast<float*>(base + L.dc);
-  // setting the stream resets the workspace, so the workspace comes second
-  DSA_TRY_BLAS(cublasSetStream(bl->h, s), "cublasSetStream");
-  DSA_TRY_BLAS(cublasSetWorkspace(bl->h, base + L.blas, kBlasWorkspace), "cublasSetWorkspace");
   int launched = 0;
   if (!accumulate_dkv)
     DSA_TRY_CUDA(cudaMemsetAsync(dkv, 0, (size_t)B * Lk * Dqk * sizeof(float), s), "dkv clear");
   // Per token, with QO = [q; dout padded to Dqk] (2H x Dqk) and the gathered rows C
   // (k x Dqk): [S; dP] = QO C^T, dq = dz C, dC = [dz; P]^T QO (the padded columns of
   // dout make the second half of each product act on the value columns only).
-  const long long qs = (long long)H * Dqk, q2s = 2LL * H * Dqk, h2k = 2LL * H * k,
-                  cs = (long long)k * Dqk;
+  const uint64_t h2 = 2ull * H, uk = (uint64_t)k, ud = (uint64_t)Dqk, uT = (uint64_t)T;
+  // operands, as blocks of the chunk's buffers (the maps span T tokens; a shorter
+  // last chunk launches fewer blocks)
+  const GemmOperand qo_k{QO, false, ud, h2, uT, ud, h2 * ud, 0};      // [2H][Dqk], K = Dqk
+  const GemmOperand qo_mn{QO, true, ud, h2, uT, ud, h2 * ud, 0};      // K = 2H rows, N = Dqk
+  const GemmOperand c_k{cg, false, ud, uk, uT, ud, uk * ud, 0};       // [k][Dqk], K = Dqk
+  const GemmOperand c_mn{cg, true, ud, uk, uT, ud, uk * ud, 0};       // K = k rows, N = Dqk
+  const GemmOperand dz_k{PZ, false, uk, (uint64_t)H, uT, uk, h2 * uk, 0};   // rows 0..H-1, K = k
+  const GemmOperand pz_mn{PZ, true, uk, h2, uT, uk, h2 * uk, 0};      // K = 2H rows, M = k
   for (long long tok0 = 0; tok0 < n; tok0 += T) {
     const int Tc = (int)(n - tok0 < T ? n - tok0 : T);
     DSA_TRY_CUDA(dsa::launch_gather_rows_bf16(kv, idx, cg, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
                  "latent row gather launch");
     DSA_TRY_CUDA(dsa::launch_pack_qo(q, dout, QO, tok0, Tc, H, Dqk, Dv, sms, s),
                  "query / output-gradient pack launch");
-    DSA_TRY(gemm_rm(bl->h, false, true, 2 * H, k, Dqk, QO, Dqk, q2s, cg, Dqk, cs, 0.0, SP, k, h2k,
-                    Tc, CUDA_R_16BF, "[S; dP] = QO C^T"));
+    DSA_TRY(tc_gemm(qo_k, c_k, 2 * H, k, Dqk, SP, k, 1, 2LL * H * k, Tc, ctl, s,
+                    "[S; dP] = QO C^T"));
     DSA_TRY_CUDA(dsa::launch_mla_bwd_softmax(SP, lse, idx, PZ, tok0, Tc, H, k, Lk, sm_scale, sms,
                                              s),
                  "softmax gradient launch");
-    DSA_TRY(gemm_rm(bl->h, false, false, H, Dqk, k, PZ, k, h2k, cg, Dqk, cs, 0.0, dq + tok0 * qs,
-                    Dqk, qs, Tc, CUDA_R_16BF, "dq = dz C"));
-    DSA_TRY(gemm_rm(bl->h, true, false, k, Dqk, 2 * H, PZ, k, h2k, QO, Dqk, q2s, 0.0, dC, Dqk, cs,
-                    Tc, CUDA_R_16BF, "dC = [dz; P]^T QO"));
+    DSA_TRY(tc_gemm(dz_k, c_mn, H, Dqk, k, dq + tok0 * H * Dqk, Dqk, 1, (long long)H * Dqk, Tc,
+                    ctl, s, "dq = dz C"));
+    DSA_TRY(tc_gemm(pz_mn, qo_mn, k, Dqk, 2 * H, dC, Dqk, 1, (long long)k * Dqk, Tc, ctl, s,
+                    "dC = [dz; P]^T QO"));
     DSA_TRY_CUDA(dsa::launch_scatter_add_rows(dC, idx, dkv, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
                  "row gradient scatter launch");
-    launched += 4;
+    launched += 7;
   }
   g_last_launches = launched;
   return DSA_OK;
@@ -1365,47 +1366,49 @@ int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
   dsa::DevCtl ctl;
   int sms = 0;
   DSA_TRY(device_ctl(ctl, sms));
-  Blas* bl = nullptr;
-  DSA_TRY(blas_for_device(&bl));
-  std::lock_guard<std::mutex> lk(bl->mu);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = align256(ws);
-  double* Kd = reinterpret_cast<double*>(base + L.kd);
-  double* Qd = reinterpret_cast<double*>(base + L.qd);
-  double* X = reinterpret_cast<double*>(base + L.x);
-  double* G1 = reinterpret_cast<double*>(base + L.g1);
-  double* G2 = reinterpret_cast<double*>(base + L.g2);
-  double* dK = reinterpret_cast<double*>(base + L.dk);
-  double* dQ = reinterpret_cast<double*>(base + L.dq);
-  DSA_TRY_BLAS(cublasSetStream(bl->h, s), "cublasSetStream");
-  DSA_TRY_BLAS(cublasSetWorkspace(bl->h, base + L.blas, kBlasWorkspace), "cublasSetWorkspace");
+  uint16_t* Kb = reinterpret_cast<uint16_t*>(base + L.kb);
+  uint16_t* Qb = reinterpret_cast<uint16_t*>(base + L.qb);
+  float* XT = reinterpret_cast<float*>(base + L.xt);
+  uint16_t* G1s = reinterpret_cast<uint16_t*>(base + L.g1);
+  uint16_t* G2s = reinterpret_cast<uint16_t*>(base + L.g2);
+  float* dK = reinterpret_cast<float*>(base + L.dk);
   int launched = 0;
   if (!accumulate_dkI)
     DSA_TRY_CUDA(cudaMemsetAsync(dkI, 0, (size_t)B * Lk * d_I * sizeof(float), s), "dkI clear");
-  const long long qs = (long long)H_I * d_I, hk = (long long)H_I * k, ks = (long long)k * d_I;
+  DSA_TRY_CUDA(cudaMemsetAsync(dw, 0, (size_t)n * H_I * sizeof(float), s), "dw clear");
+  const long long qs = (long long)H_I * d_I;
+  const uint64_t uk = (uint64_t)k, ud = (uint64_t)d_I, uh = (uint64_t)H_I, uT = (uint64_t)T;
+  const uint64_t kp3 = 3ull * L.kp, hp3 = 3ull * L.hp;
+  const GemmOperand kb_k{Kb, false, ud, uk, uT, ud, uk * ud, 0};            // [k][d_I], K = d_I
+  const GemmOperand qb_k{Qb, false, ud, uh, uT, ud, uh * ud, 0};            // [H_I][d_I], K = d_I
+  const GemmOperand kb_mn{Kb, true, ud, uk, uT, ud, uk * ud, L.kp / 64};    // K = slots, M = d_I
+  const GemmOperand g1_k{G1s, false, kp3, uh, uT, kp3, uh * kp3, 0};        // [H_I][3 kp], K = 3 kp
+  const GemmOperand g2_mn{G2s, true, uk, hp3, uT, uk, hp3 * uk, 0};         // K = 3 hp rows, M = k
+  const GemmOperand qb_mn{Qb, true, ud, uh, uT, ud, uh * ud, L.hp / 64};    // K = heads, N = d_I
   for (long long tok0 = 0; tok0 < n; tok0 += T) {
     const int Tc = (int)(n - tok0 < T ? n - tok0 : T);
-    DSA_TRY_CUDA(dsa::launch_decode_e4m3(qI + tok0 * qs, Qd, (long long)Tc * qs, sms, s),
-                 "query decode launch");
-    DSA_TRY_CUDA(dsa::launch_gather_e4m3_rows(kI, idx, Kd, tok0, Tc, Lq, Lk, k, d_I, sms, s),
+    DSA_TRY_CUDA(dsa::launch_decode_e4m3_bf16(qI + tok0 * qs, Qb, (long long)Tc * qs, sms, s),
+                 "query code launch");
+    DSA_TRY_CUDA(dsa::launch_gather_e4m3_rows_bf16(kI, idx, Kb, tok0, Tc, Lq, Lk, k, d_I, sms, s),
                  "indexer key gather launch");
-    // X[H_I x k] = qhat[H_I x d_I] khat^T (exact)
-    DSA_TRY(gemm_rm(bl->h, false, true, H_I, k, d_I, Qd, d_I, qs, Kd, d_I, ks, 0.0, X, k, hk, Tc,
-                    CUDA_R_64F, "X = qhat khat^T"));
-    DSA_TRY_CUDA(dsa::launch_indexer_bwd_relu(X, idx, dI, qI_scale, kI_scale, w,
-                                              w_dtype == DSA_DTYPE_BF16 ? 1 : 0, G1, G2, dw, tok0,
-                                              Tc, Lq, Lk, H_I, k, sms, s),
+    // X^T [k x H_I] = khat qhat^T (code dots, fp32 accumulation)
+    DSA_TRY(tc_gemm(kb_k, qb_k, k, H_I, d_I, XT, H_I, 1, (long long)k * H_I, Tc, ctl, s,
+                    "X^T = khat qhat^T"));
+    DSA_TRY_CUDA(dsa::launch_indexer_bwd_relu_tc(XT, Kb, Qb, idx, dI, qI_scale, kI_scale, w,
+                                                 w_dtype == DSA_DTYPE_BF16 ? 1 : 0, G1s, G2s, dw,
+                                                 tok0, Tc, Lq, Lk, H_I, d_I, k, L.kp, L.hp, s),
                  "ReLU gradient launch");
-    // dq^I[H_I x d_I] = G1[H_I x k] khat[k x d_I];  dK[k x d_I] = G2^T qhat
-    DSA_TRY(gemm_rm(bl->h, false, false, H_I, d_I, k, G1, k, hk, Kd, d_I, ks, 0.0, dQ, d_I, qs,
-                    Tc, CUDA_R_64F, "dqI = G1 khat"));
-    DSA_TRY_CUDA(dsa::launch_f64_to_f32(dQ, dqI + tok0 * qs, (long long)Tc * qs, sms, s),
-                 "query gradient store launch");
-    DSA_TRY(gemm_rm(bl->h, true, false, k, d_I, H_I, G2, k, hk, Qd, d_I, qs, 0.0, dK, d_I, ks, Tc,
-                    CUDA_R_64F, "dK = G2^T qhat"));
-    DSA_TRY_CUDA(dsa::launch_scatter_add_rows_f64(dK, idx, dkI, tok0, Tc, Lq, Lk, k, d_I, sms, s),
+    // dq^I [H_I x d_I], written transposed from (dq^I)^T = khat^T G1^T over K = 3 kp
+    DSA_TRY(tc_gemm(kb_mn, g1_k, d_I, H_I, 3 * L.kp, dqI + tok0 * qs, 1, d_I, qs, Tc, ctl, s,
+                    "dqI = G1 khat"));
+    // dK [k x d_I] = G2^T qhat over K = 3 hp
+    DSA_TRY(tc_gemm(g2_mn, qb_mn, k, d_I, 3 * L.hp, dK, d_I, 1, (long long)k * d_I, Tc, ctl, s,
+                    "dK = G2^T qhat"));
+    DSA_TRY_CUDA(dsa::launch_scatter_add_rows(dK, idx, dkI, tok0, Tc, Lq, Lk, k, d_I, sms, s),
                  "key gradient scatter launch");
-    launched += 5;
+    launched += 7;
   }
   g_last_launches = launched;
   return DSA_OK;

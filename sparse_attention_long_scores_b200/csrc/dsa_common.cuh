@@ -21,6 +21,7 @@ enum : int {
   kSiteTopk = 2,
   kSiteMla = 3,
   kSiteKl = 4,
+  kSiteGemm = 5,
   kSiteDebug = 9,
 };
 
@@ -153,6 +154,15 @@ DSA_DEVICE_INLINE void tma_load_2d(void* dst, const void* tmap, int x, int y, ui
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// One box of a 3-D tensor map at (x, y, z) (x innermost).
+DSA_DEVICE_INLINE void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -130,30 +130,45 @@ cudaError_t launch_mla_bwd_softmax(const float* SP, const float* lse, const int3
 cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float* dst,
                                     long long tok0, int T, int Lq, int Lk, int k, int D,
                                     int num_sms, cudaStream_t stream);
-// out [T, k, d_I] fp64 = the selected e4m3 rows of kI [B, Lk, d_I], decoded.
-cudaError_t launch_gather_e4m3_rows(const uint8_t* kI, const int32_t* idx, double* out,
-                                    long long tok0, int T, int Lq, int Lk, int k, int d_I,
-                                    int num_sms, cudaStream_t stream);
-// out [n] fp64 = decoded e4m3 codes [n].
-cudaError_t launch_decode_e4m3(const uint8_t* codes, double* out, long long n, int num_sms,
-                               cudaStream_t stream);
-// out [n] fp32 = in [n] fp64.
-cudaError_t launch_f64_to_f32(const double* in, float* out, long long n, int num_sms,
-                              cudaStream_t stream);
-// dst [B, Lk, D] fp32 += src [T, k, D] fp64 row by row (atomic); D % 4 == 0.
-cudaError_t launch_scatter_add_rows_f64(const double* src, const int32_t* idx, float* dst,
-                                        long long tok0, int T, int Lq, int Lk, int k, int D,
-                                        int num_sms, cudaStream_t stream);
-// G1 / G2 [T, H_I, k] fp64 and dw [B*Lq, H_I] fp32 from the code dots X [T, H_I, k].
-cudaError_t launch_indexer_bwd_relu(const double* X, const int32_t* idx, const float* dI,
-                                    const float* qI_scale, const float* kI_scale, const void* w,
-                                    int w_bf16, double* G1, double* G2, float* dw,
-                                    long long tok0, int T, int Lq, int Lk, int H_I, int k,
-                                    int num_sms, cudaStream_t stream);
+// out [T, k, d_I] bf16 = the selected e4m3 rows of kI [B, Lk, d_I] (codes, exact).
+cudaError_t launch_gather_e4m3_rows_bf16(const uint8_t* kI, const int32_t* idx, uint16_t* out,
+                                         long long tok0, int T, int Lq, int Lk, int k, int d_I,
+                                         int num_sms, cudaStream_t stream);
+// out [n] bf16 = e4m3 codes [n] (exact).
+cudaError_t launch_decode_e4m3_bf16(const uint8_t* codes, uint16_t* out, long long n, int num_sms,
+                                    cudaStream_t stream);
+// ReLU gradient of the indexer from the tensor-core code dots XT [T, k, H_I] fp32:
+// G1s [T, H_I, 3 kp] and G2s [T, 3 hp, k] bf16 (three-term splits of G1 / G2, zero
+// padded), dw [B*Lq, H_I] += the weight gradient (zeroed by the caller). The ReLU
+// mask is the sign of the exact code dot. H_I <= 64, d_I <= 128.
+cudaError_t launch_indexer_bwd_relu_tc(const float* XT, const uint16_t* Kb, const uint16_t* Qb,
+                                       const int32_t* idx, const float* dI,
+                                       const float* qI_scale, const float* kI_scale,
+                                       const void* w, int w_bf16, uint16_t* G1s, uint16_t* G2s,
+                                       float* dw, long long tok0, int T, int Lq, int Lk, int H_I,
+                                       int d_I, int k, int kp, int hp, cudaStream_t stream);
 // dI [rows, k] = loss_scale (softmax over the set of sel - p).
 cudaError_t launch_kl_score_grad(const float* sel, const float* p, const int32_t* idx, float* dI,
                                  long long rows, int k, int Lk, float loss_scale, int num_sms,
                                  cudaStream_t stream);
+
+// ---------------- batched tensor-core GEMM (sparse-stage gradients) ----------------
+// C[z] (fp32) = A[z] B[z]^T for z < batch: A is M x K, B is N x K, bf16, each
+// K-major (stored [M][K] / [N][K]) or MN-major (stored [K][M] / [K][N]) as given
+// by a_mn / b_mn; the tensor maps (built by the caller) are 3-D {inner, rows, z}
+// with 128-byte swizzle and boxes {64, 128} (A, K-major), {64, bn} (B, K-major)
+// or {64, 64} (MN-major). K tile kt of A reads A's tile kt % a_kt (B likewise).
+struct BgemmArgs {
+  int M, N, K;
+  int a_kt, b_kt;
+  float* C;                  // element (z, m, n) at C + z * sC + m * c_sm + n * c_sn
+  long long c_sm, c_sn, sC;
+  DevCtl ctl;
+};
+// Tile width (N) used for an N-column product: 64, 128, 192 or 256.
+int bgemm_tile_n(int N);
+cudaError_t launch_bgemm(const CUtensorMap& ta, const CUtensorMap& tb, const BgemmArgs& a,
+                         int batch, bool a_mn, bool b_mn, int bn, cudaStream_t stream);
 
 // ---------------- debug ----------------
 cudaError_t launch_debug_wait(DevCtl ctl, cudaStream_t stream);
