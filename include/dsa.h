@@ -263,6 +263,54 @@ int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
                     void* stream);
 
 /*
+ * Decode with one sequence's key cache split over G devices ("Key claims",
+ * section 2.1: the top-k over I[t,:] and attention over the selected entries).
+ * Shard g holds keys [shard_lo[g], shard_lo[g] + len_g) of every sequence, the
+ * shards in key order. Per step:
+ *   1. each device selects the top-k of its shard: dsa_forward on its shard as a
+ *      decode problem (Lk = len_g, q_pos0 = len_g - 1) with out = NULL, idx_out
+ *      and sel_scores_out;
+ *   2. the candidates (sel_scores_out, idx_out) of all shards are all-gathered
+ *      (a collective of the caller's) and merged: dsa_topk_merge;
+ *   3. each device takes its view of the merged selection (dsa_index_localize)
+ *      and attends over it with dsa_sparse_mla_fwd on its shard, giving out_g
+ *      and lse_g (zeros and -inf where the shard holds none of the keys);
+ *   4. the pairs (out_g, lse_g) are all-gathered and combined: dsa_attn_combine.
+ * The merged selection equals the unsplit one bit for bit: a key among the k
+ * largest overall is among the k largest of its shard under the same tie rule,
+ * and the merge keeps (score descending, lower global index first). The output
+ * is the lse-weighted mean of the partial outputs, each rounded to bf16 once.
+ *
+ * dsa_topk_merge - the top-k of G shards' candidate lists.
+ *   cand_scores [G, R, k] fp32 and cand_idx [G, R, k] int32 (shard-local key
+ *   indices, ascending, < 0 for no candidate), device; shard_lo [G] int64, host:
+ *   first key of each shard, increasing; G in [1, 16]; k a multiple of 32 in
+ *   [32, 4096]. idx_out [R, k] int32: the k best candidates by (score
+ *   descending, global index ascending), as global indices in ascending order,
+ *   -1 padded when fewer than k candidates exist; sel_out [R, k] fp32 or NULL:
+ *   their scores (0 at padding). ws: dsa_topk_merge_workspace_size(G, R, k)
+ *   bytes, caller-owned device memory.
+ * dsa_index_localize - idx_local[i] = idx[i] - lo for lo <= idx[i] < lo + len,
+ *   else -1 (n int32 entries, device).
+ * dsa_attn_combine - out[r, h, :] = sum_g exp(lse_g - L) out_g[r, h, :] with
+ *   L = ln sum_g exp(lse_g) (lse_out, optional): part_out [G, R, H, Dv] bf16 and
+ *   part_lse [G, R, H] fp32 as dsa_sparse_mla_fwd returns them; out [R, H, Dv]
+ *   bf16 (round to nearest even). A row with every lse_g = -inf gives zeros and
+ *   L = -inf.
+ * All pointers 16-byte aligned; nothing is allocated. Errors as for the other
+ * calls (DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED_SHAPE,
+ * DSA_ERR_WORKSPACE_TOO_SMALL, DSA_ERR_CUDA).
+ */
+size_t dsa_topk_merge_workspace_size(int G, int R, int k);
+int dsa_topk_merge(const float* cand_scores, const int32_t* cand_idx, const long long* shard_lo,
+                   int G, int R, int k, int32_t* idx_out, float* sel_out, void* ws,
+                   size_t ws_bytes, void* stream);
+int dsa_index_localize(const int32_t* idx, int32_t* idx_local, long long n, int lo, int len,
+                       void* stream);
+int dsa_attn_combine(const uint16_t* part_out, const float* part_lse, int G, int R, int H, int Dv,
+                     uint16_t* out, float* lse_out, void* stream);
+
+/*
  * dsa_last_launch_count - number of kernel launches that the calling thread's
  * last dsa_forward, dsa_forward_host, dsa_forward_profiled, dsa_sparse_mla_bwd,
  * dsa_indexer_bwd or dsa_indexer_kl_grad call enqueued (all of this library's
@@ -293,7 +341,9 @@ typedef struct dsa_tensors {
   const void* w;
   const uint16_t* q;
   const uint16_t* kv;
-  uint16_t* out;    /* [B, Lq, H, Dv] bf16 */
+  uint16_t* out;    /* [B, Lq, H, Dv] bf16; NULL for a selection-only call, which
+                       stops after the top-k (idx_out then required; q, kv and lse
+                       are not read) */
   float* lse;       /* [B, Lq, H] fp32, optional (NULL) */
   int32_t* idx_out; /* [B, Lq, k] int32, optional: the selected set */
   float* sel_scores_out; /* [B, Lq, k] fp32, optional: the index score I[t, idx_out[t, j]]

@@ -42,6 +42,7 @@ EXPORTED = [
     "dsa_indexer_kl", "dsa_last_launch_count", "dsa_forward_paged_workspace_size",
     "dsa_forward_paged", "dsa_forward_fused", "dsa_sparse_mla_bwd_workspace_size", "dsa_sparse_mla_bwd",
     "dsa_indexer_kl_grad", "dsa_indexer_bwd_workspace_size", "dsa_indexer_bwd",
+    "dsa_topk_merge_workspace_size", "dsa_topk_merge", "dsa_index_localize", "dsa_attn_combine",
 ]
 KIND_NAMES = {1: "indexer", 2: "topk", 3: "sparse_mla", 4: "combine", 5: "indexer_topk"}
 
@@ -119,13 +120,19 @@ def lib() -> ctypes.CDLL:
     L.dsa_indexer_bwd_workspace_size.restype = sz
     L.dsa_indexer_bwd.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
                                   vp, sz, vp]
+    L.dsa_topk_merge_workspace_size.argtypes = [i, i, i]
+    L.dsa_topk_merge_workspace_size.restype = sz
+    L.dsa_topk_merge.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_longlong), i, i, i, vp, vp, vp,
+                                 sz, vp]
+    L.dsa_index_localize.argtypes = [vp, vp, ctypes.c_longlong, i, i, vp]
+    L.dsa_attn_combine.argtypes = [vp, vp, i, i, i, i, vp, vp, vp]
     L.dsa_check_status.argtypes = [vp]
     L.dsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     L.dsa_debug_wait_timeout.argtypes = [vp]
     for name in ("dsa_indexer_scores", "dsa_topk_select", "dsa_sparse_mla_fwd", "dsa_forward",
                  "dsa_forward_host", "dsa_forward_profiled", "dsa_check_status", "dsa_set_wait_limit_ns",
                  "dsa_debug_wait_timeout", "dsa_sparse_mla_bwd", "dsa_indexer_kl_grad",
-                 "dsa_indexer_bwd"):
+                 "dsa_indexer_bwd", "dsa_topk_merge", "dsa_index_localize", "dsa_attn_combine"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -428,6 +435,154 @@ def forward(p: Problem, inp: dict, out=None, lse=None, idx_out=None, ws=None, st
     _check(entry(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws), ws.numel() * ws.element_size(),
                  _stream(stream)))
     return out
+
+
+def select(p: Problem, inp: dict, idx_out, sel_scores=None, ws=None, stream=None):
+    """Selection only: dsa_forward with out = NULL (indexer and top-k; q and kv are not
+    read). Fills idx_out [B, Lq, k] and, when given, sel_scores [B, Lq, k]."""
+    dev = inp["qI"].device
+    for name, t, dt, shape in (("qI", inp["qI"], torch.uint8, (p.B, p.Lq, p.H_I, p.d_I)),
+                               ("qI_scale", inp["qI_scale"], torch.float32, (p.B, p.Lq, p.H_I)),
+                               ("kI", inp["kI"], torch.uint8, (p.B, p.Lk, p.d_I)),
+                               ("kI_scale", inp["kI_scale"], torch.float32, (p.B, p.Lk))):
+        _need(t, name, dt, shape)
+    _need(inp["w"], "w", torch.float32 if p.w_dtype == DSA_DTYPE_F32 else torch.bfloat16,
+          (p.B, p.Lq, p.H_I))
+    _need(idx_out, "idx_out", torch.int32, (p.B, p.Lq, p.k))
+    if sel_scores is not None:
+        _need(sel_scores, "sel_scores", torch.float32, (p.B, p.Lq, p.k))
+    if ws is None:
+        ws = torch.empty(forward_workspace_size(p), dtype=torch.uint8, device=dev)
+    cp = p.c()
+    ct = DsaTensors(*[None if x is None else x.data_ptr() for x in (
+        inp["qI"], inp["qI_scale"], inp["kI"], inp["kI_scale"], inp["w"], None, None,
+        None, None, idx_out, sel_scores)])
+    _check(lib().dsa_forward(ctypes.byref(cp), ctypes.byref(ct), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)))
+    return idx_out
+
+
+def topk_merge(cand_scores, cand_idx, shard_lo, idx_out=None, sel_out=None, ws=None, stream=None):
+    """The top-k of G shards' candidates (dsa_topk_merge): cand_scores [G, *rows, k] fp32,
+    cand_idx [G, *rows, k] int32 shard-local (ascending, < 0 none), shard_lo: the first
+    key of each shard. Returns (idx_out [*rows, k] global, sel_out [*rows, k])."""
+    G = cand_scores.shape[0]
+    rows_shape = tuple(cand_scores.shape[1:-1])
+    k = cand_scores.shape[-1]
+    R = 1
+    for d in rows_shape:
+        R *= d
+    _need(cand_scores, "cand_scores", torch.float32)
+    _need(cand_idx, "cand_idx", torch.int32, tuple(cand_scores.shape))
+    if len(shard_lo) != G:
+        raise ValueError("shard_lo needs one entry per shard")
+    dev = cand_scores.device
+    if idx_out is None:
+        idx_out = torch.empty(rows_shape + (k,), dtype=torch.int32, device=dev)
+    _need(idx_out, "idx_out", torch.int32, rows_shape + (k,))
+    if sel_out is None:
+        sel_out = torch.empty(rows_shape + (k,), dtype=torch.float32, device=dev)
+    _need(sel_out, "sel_out", torch.float32, rows_shape + (k,))
+    need = int(lib().dsa_topk_merge_workspace_size(G, R, k))
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    lo = (ctypes.c_longlong * G)(*[int(x) for x in shard_lo])
+    _check(lib().dsa_topk_merge(_ptr(cand_scores), _ptr(cand_idx), lo, G, R, k, _ptr(idx_out),
+                                _ptr(sel_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)))
+    return idx_out, sel_out
+
+
+def index_localize(idx, lo: int, length: int, out=None, stream=None):
+    """A shard's view of a selection: idx - lo where lo <= idx < lo + length, else -1."""
+    _need(idx, "idx", torch.int32)
+    if out is None:
+        out = torch.empty_like(idx)
+    _need(out, "out", torch.int32, tuple(idx.shape))
+    _check(lib().dsa_index_localize(_ptr(idx), _ptr(out), idx.numel(), int(lo), int(length),
+                                    _stream(stream)))
+    return out
+
+
+def attn_combine(part_out, part_lse, out=None, lse=None, stream=None):
+    """lse-weighted combine of G partial attentions (dsa_attn_combine): part_out
+    [G, *rows, H, Dv] bf16, part_lse [G, *rows, H] fp32 -> (out [*rows, H, Dv], lse)."""
+    G, H, Dv = part_out.shape[0], part_out.shape[-2], part_out.shape[-1]
+    rows_shape = tuple(part_out.shape[1:-2])
+    R = 1
+    for d in rows_shape:
+        R *= d
+    _need(part_out, "part_out", torch.bfloat16)
+    _need(part_lse, "part_lse", torch.float32, (G,) + rows_shape + (H,))
+    dev = part_out.device
+    if out is None:
+        out = torch.empty(rows_shape + (H, Dv), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, rows_shape + (H, Dv))
+    if lse is None:
+        lse = torch.empty(rows_shape + (H,), dtype=torch.float32, device=dev)
+    _need(lse, "lse", torch.float32, rows_shape + (H,))
+    _check(lib().dsa_attn_combine(_ptr(part_out), _ptr(part_lse), G, R, H, Dv, _ptr(out), _ptr(lse),
+                                  _stream(stream)))
+    return out, lse
+
+
+def _all_gather(t: torch.Tensor) -> torch.Tensor:
+    """[G, *t.shape]: t from every rank of the default process group, in rank order."""
+    import torch.distributed as dist
+    parts = [torch.empty_like(t) for _ in range(dist.get_world_size())]
+    dist.all_gather(parts, t.contiguous())
+    return torch.stack(parts)
+
+
+class _CudaSplitOps:
+    """The per-device steps of decode_split_cache, on this library's kernels."""
+
+    @staticmethod
+    def select(p, inp, idx, sel):
+        return select(p, inp, idx, sel)
+
+    @staticmethod
+    def merge(cand_scores, cand_idx, shard_lo):
+        return topk_merge(cand_scores, cand_idx, shard_lo)[0]
+
+    @staticmethod
+    def localize(idx, lo, length):
+        return index_localize(idx, lo, length)
+
+    @staticmethod
+    def attend(q, kv, idx_local, sm_scale, Dv):
+        return sparse_mla_fwd(q, kv, idx_local, sm_scale, Dv)
+
+    @staticmethod
+    def combine(part_out, part_lse):
+        return attn_combine(part_out, part_lse)
+
+
+def decode_split_cache(p: Problem, inp: dict, shard_lo, rank=None, gather=None, ops=None):
+    """Decode over key caches split across devices, one shard per rank.
+
+    p: this rank's shard as a decode problem (Lq = 1, Lk = the shard's key count,
+    q_pos0 = Lk - 1); inp: kI, kI_scale, kv of the shard and qI, qI_scale, w, q of the
+    query rows (the same on every rank). shard_lo: the first key of every rank's shard,
+    in rank order, the shards tiling the key range in that order. rank: this rank
+    (default: torch.distributed's). gather(t) returns [G, *t.shape] from all ranks in
+    rank order (default: torch.distributed all_gather). Every rank returns the same
+    (out [B, 1, H, Dv] bf16, lse [B, 1, H] fp32, idx [B, 1, k] global key indices).
+    """
+    gather = gather or _all_gather
+    ops = ops or _CudaSplitOps
+    if rank is None:
+        import torch.distributed as dist
+        rank = dist.get_rank()
+    dev = inp["q"].device
+    cand_idx = torch.empty((p.B, p.Lq, p.k), dtype=torch.int32, device=dev)
+    cand_sc = torch.empty((p.B, p.Lq, p.k), dtype=torch.float32, device=dev)
+    ops.select(p, inp, cand_idx, cand_sc)
+    idx = ops.merge(gather(cand_sc), gather(cand_idx), shard_lo)
+    idx_local = ops.localize(idx, int(shard_lo[rank]), p.Lk)
+    o, l = ops.attend(inp["q"], inp["kv"], idx_local, p.sm_scale, p.Dv)
+    out, lse = ops.combine(gather(o), gather(l))
+    return out, lse, idx
 
 
 def forward_paged_workspace_size(p: Problem) -> int:

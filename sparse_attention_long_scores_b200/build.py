@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libdsa.so")
 SOURCES = ["dsa_api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "indexer_kl.cu", "backward.cu",
-           "bgemm.cu"]
+           "bgemm.cu", "context_parallel.cu"]
 HEADERS = ["dsa_common.cuh", "dsa_kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -132,12 +132,22 @@ __global__ void mla_bwd_softmax_kernel(const float* __restrict__ SP,
     const long long prow_off = zrow + static_cast<long long>(H) * k;   // row H + h
     const float* srow = SP + zrow;
     const float* prow = SP + prow_off;
+    // four consecutive slots per lane per step (k % 32 == 0: rows are 16-byte aligned)
+    const int4* irow = reinterpret_cast<const int4*>(idx + tok * k);
     float sp = 0.f, spd = 0.f;
-    for (int j = lane; j < k; j += 32) {
-      if (selected_key(idx, tok, j, k, Lk) >= 0) {
-        const float p = expf(srow[j] * sm_scale - l);
-        sp += p;
-        spd += p * prow[j];
+    for (int j = lane * 4; j < k; j += 128) {
+      const int4 iv = irow[j >> 2];
+      const float4 sv = *reinterpret_cast<const float4*>(srow + j);
+      const float4 dv = *reinterpret_cast<const float4*>(prow + j);
+      const int ii[4] = {iv.x, iv.y, iv.z, iv.w};
+      const float ss[4] = {sv.x, sv.y, sv.z, sv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (ii[q] >= 0 && ii[q] < Lk) {
+          const float p = expf(ss[q] * sm_scale - l);
+          sp += p;
+          spd += p * dd[q];
+        }
       }
     }
     sp = warp_sum(sp);
@@ -145,14 +155,25 @@ __global__ void mla_bwd_softmax_kernel(const float* __restrict__ SP,
     const float d = sp > 0.f ? spd / sp : 0.f;
     uint16_t* z_out = PZ + zrow;
     uint16_t* p_out = PZ + prow_off;
-    for (int j = lane; j < k; j += 32) {
-      float p = 0.f, z = 0.f;
-      if (selected_key(idx, tok, j, k, Lk) >= 0) {
-        p = expf(srow[j] * sm_scale - l);
-        z = sm_scale * p * (prow[j] - d);
+    for (int j = lane * 4; j < k; j += 128) {
+      const int4 iv = irow[j >> 2];
+      const float4 sv = *reinterpret_cast<const float4*>(srow + j);
+      const float4 dv = *reinterpret_cast<const float4*>(prow + j);
+      const int ii[4] = {iv.x, iv.y, iv.z, iv.w};
+      const float ss[4] = {sv.x, sv.y, sv.z, sv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
+      uint16_t pb[4], zb[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float p = 0.f, z = 0.f;
+        if (ii[q] >= 0 && ii[q] < Lk) {
+          p = expf(ss[q] * sm_scale - l);
+          z = sm_scale * p * (dd[q] - d);
+        }
+        pb[q] = float_to_bf16_bits(p);
+        zb[q] = float_to_bf16_bits(z);
       }
-      p_out[j] = float_to_bf16_bits(p);
-      z_out[j] = float_to_bf16_bits(z);
+      *reinterpret_cast<uint2*>(p_out + j) = make_uint2(pb[0] | (uint32_t(pb[1]) << 16), pb[2] | (uint32_t(pb[3]) << 16));
+      *reinterpret_cast<uint2*>(z_out + j) = make_uint2(zb[0] | (uint32_t(zb[1]) << 16), zb[2] | (uint32_t(zb[3]) << 16));
     }
   }
 }
@@ -214,12 +235,13 @@ __device__ __forceinline__ void split3(float v, uint16_t& a, uint16_t& b, uint16
 }
 
 // The code dots X = qhat_j . khat_s come from a tensor-core product with fp32
-// accumulation; an fp32 sum of d_I <= 128 exact products is within
+// accumulation; an fp32 sum of d_I <= 128 exact products, each addition off by
+// at most 2^-23 relative (rounded or truncated), is within
 // d_I 2^-23 sum_i |qhat_ji khat_si| <= 2^-16 |qhat_j| |khat_s| of the exact dot.
-// Where |X| is within kDotBand |qhat_j| |khat_s| of zero (sixteen times that bound)
+// Where |X| is within kDotBand |qhat_j| |khat_s| of zero (four times that bound)
 // the dot is recomputed exactly in fp64, so the ReLU mask is the exact code
 // dot's sign.
-constexpr float kDotBand = 1.0f / 4096.0f;
+constexpr float kDotBand = 1.0f / 16384.0f;
 constexpr int kReluThreads = 256;
 constexpr int kReluMaxHeads = 64;
 constexpr int kReluMaxDim = 128;
@@ -278,9 +300,15 @@ __global__ void __launch_bounds__(kReluThreads) indexer_bwd_relu_tc_kernel(
       d = dI[tok * k + slot];
       sk = kI_scale[b * Lk + s];
       float acc = 0.f;
-      for (int c = 0; c < d_I; ++c) {
-        const float v = bf16_bits_to_float(krow[c]);
-        acc += v * v;
+      const uint4* k8 = reinterpret_cast<const uint4*>(krow);
+      for (int c8 = 0; c8 < d_I / 8; ++c8) {
+        const uint4 v = k8[c8];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float lo = __uint_as_float(wv[h] << 16), hi = __uint_as_float(wv[h] & 0xFFFF0000u);
+          acc += lo * lo + hi * hi;
+        }
       }
       kn = sqrtf(acc);
     }
@@ -288,15 +316,28 @@ __global__ void __launch_bounds__(kReluThreads) indexer_bwd_relu_tc_kernel(
   const float* xrow = XT + (static_cast<long long>(tt) * k + slot) * H_I;
   uint16_t* g1row = G1s + static_cast<long long>(tt) * H_I * 3 * kp + slot;
   uint16_t* g2col = G2s + static_cast<long long>(tt) * 3 * hp * k + slot;
+  float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);   // four heads' dots per load (H_I % 4 == 0)
   for (int j = 0; j < hp; ++j) {
     float g1 = 0.f, g2 = 0.f, contrib = 0.f;
     if (s >= 0 && j < H_I) {
-      const float x = xrow[j];
+      if ((j & 3) == 0) x4 = *reinterpret_cast<const float4*>(xrow + j);
+      const float x = (j & 3) == 0 ? x4.x : (j & 3) == 1 ? x4.y : (j & 3) == 2 ? x4.z : x4.w;
       double xe = x;
       if (fabsf(x) <= kDotBand * kn * s_qn[j]) {
-        double e = 0.0;   // exact: products of codes need <= 8 bits, sums stay on a 2^-18 grid below 2^25
-        for (int c = 0; c < d_I; ++c)
-          e += static_cast<double>(s_q[j * d_I + c]) * static_cast<double>(bf16_bits_to_float(krow[c]));
+        // exact: products of codes need <= 8 bits, sums stay on a 2^-18 grid below 2^25
+        double e = 0.0;
+        const uint4* k8 = reinterpret_cast<const uint4*>(krow);
+        const float* qj = s_q + j * d_I;
+        for (int c8 = 0; c8 < d_I / 8; ++c8) {
+          const uint4 v = k8[c8];
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            e += static_cast<double>(qj[c8 * 8 + 2 * h]) * static_cast<double>(__uint_as_float(wv[h] << 16));
+            e += static_cast<double>(qj[c8 * 8 + 2 * h + 1]) *
+                 static_cast<double>(__uint_as_float(wv[h] & 0xFFFF0000u));
+          }
+        }
         xe = e;
       }
       if (xe > 0.0) {
@@ -398,6 +439,7 @@ cudaError_t launch_pack_qo(const uint16_t* q, const uint16_t* dout, uint16_t* qo
 cudaError_t launch_mla_bwd_softmax(const float* SP, const float* lse, const int32_t* idx,
                                    uint16_t* PZ, long long tok0, int T, int H, int k, int Lk,
                                    float sm_scale, int num_sms, cudaStream_t stream) {
+  if (k % 4 != 0) return cudaErrorInvalidValue;
   const long long rows = static_cast<long long>(T) * H;
   mla_bwd_softmax_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
       SP, lse, idx, PZ, tok0, T, H, k, Lk, sm_scale);
@@ -435,7 +477,8 @@ cudaError_t launch_indexer_bwd_relu_tc(const float* XT, const uint16_t* Kb, cons
                                        const void* w, int w_bf16, uint16_t* G1s, uint16_t* G2s,
                                        float* dw, long long tok0, int T, int Lq, int Lk, int H_I,
                                        int d_I, int k, int kp, int hp, cudaStream_t stream) {
-  if (H_I > kReluMaxHeads || d_I > kReluMaxDim || T > 65535) return cudaErrorInvalidValue;
+  if (H_I > kReluMaxHeads || H_I % 4 != 0 || d_I > kReluMaxDim || d_I % 8 != 0 || T > 65535)
+    return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((kp + kReluThreads - 1) / kReluThreads),
                   static_cast<unsigned>(T));
   indexer_bwd_relu_tc_kernel<<<grid, kReluThreads, 0, stream>>>(

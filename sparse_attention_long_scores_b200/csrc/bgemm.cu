@@ -15,10 +15,11 @@
 // transposed result needs no separate pass.
 //
 // One CTA computes one 128 x BN tile: thread 0 streams 64-deep K tiles of A and
-// B with TMA (128-byte swizzle) through a four-stage ring, thread 32 issues
+// B with TMA (128-byte swizzle) through a ring of 2 to 4 stages, thread 32 issues
 // tcgen05.mma (M = 128, N = BN, K = 16) into a TMEM accumulator, and the four
-// warps then read their 32 TMEM lanes each and store the rows. Every wait is
-// bounded (site kSiteGemm).
+// warps then read their 32 TMEM lanes each and store the rows; two CTAs share
+// an SM, so one's stores overlap the other's main loop. Every wait is bounded
+// (site kSiteGemm).
 #include <cuda_bf16.h>
 
 #include "dsa_kernels.h"
@@ -28,18 +29,21 @@ namespace {
 
 constexpr int BG_BM = 128;
 constexpr int BG_BK = 64;          // K elements per tile: 128 bytes of bf16
-constexpr int BG_STAGES = 4;
 constexpr int BG_THREADS = 128;
 
 template <int BN, bool A_MN, bool B_MN>
 struct BgTraits {
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  // as many stages as leave room for two CTAs per SM: one CTA's epilogue then
+  // overlaps the other's loads and MMAs
+  static constexpr int STAGES = BN >= 192 ? 2 : BN == 128 ? 3 : 4;
   static constexpr int A_BYTES = BG_BM * 128;   // K-major: 128 rows x 128 B; MN-major: 2 boxes of 64 x 64
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int OFF_BAR = BG_STAGES * STAGE_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
   // full[STAGES], empty[STAGES], done; then the TMEM base and the abort flag
-  static constexpr int SMEM_BYTES = OFF_BAR + (2 * BG_STAGES + 1) * 8 + 16 + 1024;
+  static constexpr int SMEM_BYTES = OFF_BAR + (2 * STAGES + 1) * 8 + 16 + 1024;
+  static_assert(2 * SMEM_BYTES <= 232448, "two CTAs per SM");
   static constexpr int TMEM_COLS = BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
   static constexpr uint32_t IDESC = make_idesc(1, 1, A_MN ? 1 : 0, B_MN ? 1 : 0, BN, 128);
   // MN-major operands: 64-element column blocks of BG_BK rows x 128 B each
@@ -47,7 +51,7 @@ struct BgTraits {
 };
 
 template <int BN, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(BG_THREADS, 1)
+__global__ void __launch_bounds__(BG_THREADS, 2)
     bgemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                  const __grid_constant__ CUtensorMap tmap_b, const BgemmArgs a) {
   using Tr = BgTraits<BN, A_MN, B_MN>;
@@ -55,8 +59,8 @@ __global__ void __launch_bounds__(BG_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
-  uint64_t* empty = full + BG_STAGES;
-  uint64_t* done = empty + BG_STAGES;
+  uint64_t* empty = full + Tr::STAGES;
+  uint64_t* done = empty + Tr::STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -64,7 +68,7 @@ __global__ void __launch_bounds__(BG_THREADS, 1)
   const int KT = (a.K + BG_BK - 1) / BG_BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < BG_STAGES; ++s) {
+    for (int s = 0; s < Tr::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -83,9 +87,9 @@ __global__ void __launch_bounds__(BG_THREADS, 1)
   if (threadIdx.x == 0) {
     // producer: K tile kt of A is tile kt % a_kt of its own K extent (likewise B)
     for (int kt = 0; kt < KT; ++kt) {
-      const int st = kt % BG_STAGES;
-      if (kt >= BG_STAGES &&
-          !mbar_wait(&empty[st], (uint32_t)((kt / BG_STAGES) - 1) & 1u, a.ctl, abort_flag, kSiteGemm, 1))
+      const int st = kt % Tr::STAGES;
+      if (kt >= Tr::STAGES &&
+          !mbar_wait(&empty[st], (uint32_t)((kt / Tr::STAGES) - 1) & 1u, a.ctl, abort_flag, kSiteGemm, 1))
         break;
       uint8_t* sa = smem + st * Tr::STAGE_BYTES;
       uint8_t* sb = sa + Tr::A_BYTES;
@@ -109,8 +113,8 @@ __global__ void __launch_bounds__(BG_THREADS, 1)
     // along the swizzled row, an MN-major step 16 rows of 128 bytes
     bool ok = true;
     for (int kt = 0; kt < KT && ok; ++kt) {
-      const int st = kt % BG_STAGES;
-      if (!mbar_wait(&full[st], (uint32_t)(kt / BG_STAGES) & 1u, a.ctl, abort_flag, kSiteGemm, 2)) {
+      const int st = kt % Tr::STAGES;
+      if (!mbar_wait(&full[st], (uint32_t)(kt / Tr::STAGES) & 1u, a.ctl, abort_flag, kSiteGemm, 2)) {
         ok = false;
         break;
       }

@@ -397,11 +397,16 @@ int validate_tensors(const dsa_tensors* t) {
   DSA_TRY(check_ptr(t->kI, "kI"));
   DSA_TRY(check_ptr(t->kI_scale, "kI_scale"));
   DSA_TRY(check_ptr(t->w, "w"));
+  DSA_TRY(check_ptr(t->out, "out", true));
+  DSA_TRY(check_ptr(t->idx_out, "idx_out", true));
+  if (t->out == nullptr) {   // selection only: q, kv and lse are not read
+    if (t->idx_out == nullptr)
+      return fail(DSA_ERR_INVALID_ARG, "out is NULL: a selection-only call needs idx_out");
+    return DSA_OK;
+  }
   DSA_TRY(check_ptr(t->q, "q"));
   DSA_TRY(check_ptr(t->kv, "kv"));
-  DSA_TRY(check_ptr(t->out, "out"));
   DSA_TRY(check_ptr(t->lse, "lse", true));
-  DSA_TRY(check_ptr(t->idx_out, "idx_out", true));
   return DSA_OK;
 }
 
@@ -772,6 +777,12 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
   int* row_cnt = reinterpret_cast<int*>(wsb + f.scores_bytes + f.idx_bytes);
   void* mla_ws = wsb + f.scores_bytes + f.idx_bytes + f.cnt_bytes;
 
+  // the attention step; a selection-only call (out == NULL) ends after the top-k
+  auto attend = [&]() -> int {
+    if (t->out == nullptr) return DSA_OK;
+    return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
+                   p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+  };
   const int first_scored = first_scored_row(p, score_all);
   if (first_scored < p->Lq && (f.chunk < 1 || f.scores_bytes == 0 || f.total > ws_bytes))
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "dsa_forward workspace: no room for one score row");
@@ -794,8 +805,7 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
       DSA_TRY_CUDA(dsa::launch_topk(ta, sms, s), "top-k launch");
     }
     DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
-    return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
-                   p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+    return attend();
   }
   if (!fused) {
     // Overlapped schedule: the score area holds two half-size chunk buffers; the
@@ -853,8 +863,7 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
         DSA_TRY(rec.mark(DSA_KIND_TOPK, s));
       }
     }
-    return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
-                   p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+    return attend();
   }
   DSA_TRY_CUDA(cudaMemsetAsync(row_cnt, 0, f.cnt_bytes, s), "row counter clear");
   FusedSelect fs;
@@ -871,8 +880,7 @@ int forward_impl(const dsa_problem* p, const dsa_tensors* t, void* ws, size_t ws
                                 f.ld, C, t0, p->B, p->Lq, p->Lk, p->q_pos0, p->H_I, p->d_I, ts,
                                 ts < t1 ? t1 : ts, ctl, sms, s, rec, pc, &fs));
   }
-  return run_mla(t->q, t->kv, idx, t->out, t->lse, p->B, p->Lq, p->Lk, p->H, p->Dqk, p->Dv, p->k,
-                 p->sm_scale, mla_ws, f.mla_bytes, ctl, sms, s, rec, false, pc);
+  return attend();
 }
 
 // A paged problem is scheduled as the uniform problem whose rows sit as late as
@@ -1430,6 +1438,138 @@ int dsa_indexer_kl_grad(const float* sel_scores, const float* p, const int32_t* 
   DSA_TRY_CUDA(dsa::launch_kl_score_grad(sel_scores, p, idx, dI, (long long)B * Lq, k, Lk,
                                          loss_scale, sms, static_cast<cudaStream_t>(stream)),
                "KL score gradient launch");
+  g_last_launches = 1;
+  return DSA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode with one sequence's key cache split over G devices (context_parallel.cu):
+// the merge of the shards' candidates, the shard-local view of the merged
+// selection, and the combine of the partial attentions.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct MergeLayout {
+  size_t scores, idx, pos, total;
+};
+MergeLayout merge_layout(int G, int R, int k) {
+  MergeLayout L{};
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t n = (size_t)R * G * k;
+  L.scores = take(n * sizeof(float));
+  L.idx = take(n * sizeof(int32_t));
+  L.pos = take((size_t)R * k * sizeof(int32_t));
+  L.total = off + 256;
+  return L;
+}
+
+constexpr int kMaxShards = 16;
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_topk_merge_workspace_size(int G, int R, int k) {
+  if (G < 1 || G > kMaxShards || R < 1 || k < 1) return 0;
+  return merge_layout(G, R, k).total;
+}
+
+int dsa_topk_merge(const float* cand_scores, const int32_t* cand_idx, const long long* shard_lo,
+                   int G, int R, int k, int32_t* idx_out, float* sel_out, void* ws,
+                   size_t ws_bytes, void* stream) {
+  NvtxRange nr("dsa_topk_merge");
+  DSA_TRY(check_ptr(cand_scores, "cand_scores"));
+  DSA_TRY(check_ptr(cand_idx, "cand_idx"));
+  DSA_TRY(check_ptr(idx_out, "idx_out"));
+  DSA_TRY(check_ptr(sel_out, "sel_out", true));
+  if (shard_lo == nullptr) return fail(DSA_ERR_INVALID_ARG, "shard_lo is NULL");
+  if (G < 1 || G > kMaxShards) return fail(DSA_ERR_INVALID_ARG, "G must be in [1, %d]", kMaxShards);
+  if (R < 1) return fail(DSA_ERR_INVALID_ARG, "R must be >= 1");
+  DSA_TRY(check_k(k, 4096));
+  if ((long long)R * G * k > (1LL << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "R * G * k must be <= 2^31");
+  dsa::ShardOffsets lo{};
+  for (int g = 0; g < G; ++g) {
+    if (shard_lo[g] < 0 || (g > 0 && shard_lo[g] <= shard_lo[g - 1]) || shard_lo[g] >= (1LL << 31))
+      return fail(DSA_ERR_INVALID_ARG, "shard_lo must be increasing, >= 0 and < 2^31");
+    lo.v[g] = shard_lo[g];
+  }
+  const MergeLayout L = merge_layout(G, R, k);
+  if (ws_bytes < L.total)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "dsa_topk_merge workspace: need %zu bytes, got %zu",
+                L.total, ws_bytes);
+  DSA_TRY(check_ptr(ws, "ws"));
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = align256(ws);
+  float* ext_scores = reinterpret_cast<float*>(base + L.scores);
+  int32_t* ext_idx = reinterpret_cast<int32_t*>(base + L.idx);
+  int32_t* pos = reinterpret_cast<int32_t*>(base + L.pos);
+  const int n = G * k;
+  DSA_TRY_CUDA(dsa::launch_cp_pack(cand_scores, cand_idx, lo, G, R, k, ext_scores, ext_idx, sms, s),
+               "candidate pack launch");
+  // every row has n = G k candidate positions: row r is "sequence" r, one query
+  // row at position n - 1
+  dsa::TopkArgs ta{};
+  ta.scores = ext_scores;
+  ta.sc_ld = n;
+  ta.sc_bstride = 1;
+  ta.sc_t0 = 0;
+  ta.idx = pos;
+  ta.B = R;
+  ta.Lq = 1;
+  ta.Lk = n;
+  ta.q_pos0 = n - 1;
+  ta.k = k;
+  ta.t_lo = 0;
+  ta.t_hi = 1;
+  ta.vec4 = (n % 4 == 0) ? 1 : 0;
+  ta.seq_lens = nullptr;
+  ta.sel = sel_out;
+  ta.ctl = ctl;
+  DSA_TRY_CUDA(dsa::launch_topk(ta, sms, s), "candidate top-k launch");
+  DSA_TRY_CUDA(dsa::launch_cp_map_compact(pos, ext_idx, R, n, k, idx_out, sel_out, sms, s),
+               "candidate map launch");
+  g_last_launches = 3;
+  return DSA_OK;
+}
+
+int dsa_index_localize(const int32_t* idx, int32_t* idx_local, long long n, int lo, int len,
+                       void* stream) {
+  DSA_TRY(check_ptr(idx, "idx"));
+  DSA_TRY(check_ptr(idx_local, "idx_local"));
+  if (n < 1 || lo < 0 || len < 1) return fail(DSA_ERR_INVALID_ARG, "need n >= 1, lo >= 0, len >= 1");
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  DSA_TRY_CUDA(dsa::launch_cp_localize(idx, idx_local, n, lo, len, sms, static_cast<cudaStream_t>(stream)),
+               "index localize launch");
+  g_last_launches = 1;
+  return DSA_OK;
+}
+
+int dsa_attn_combine(const uint16_t* part_out, const float* part_lse, int G, int R, int H, int Dv,
+                     uint16_t* out, float* lse_out, void* stream) {
+  DSA_TRY(check_ptr(part_out, "part_out"));
+  DSA_TRY(check_ptr(part_lse, "part_lse"));
+  DSA_TRY(check_ptr(out, "out"));
+  DSA_TRY(check_ptr(lse_out, "lse_out", true));
+  if (G < 1 || G > kMaxShards) return fail(DSA_ERR_INVALID_ARG, "G must be in [1, %d]", kMaxShards);
+  if (R < 1 || H < 1 || Dv < 1) return fail(DSA_ERR_INVALID_ARG, "R, H, Dv must be >= 1");
+  dsa::DevCtl ctl;
+  int sms = 0;
+  DSA_TRY(device_ctl(ctl, sms));
+  DSA_TRY_CUDA(dsa::launch_cp_combine(part_out, part_lse, G, (long long)R * H, Dv, out, lse_out, sms,
+                                      static_cast<cudaStream_t>(stream)),
+               "partial attention combine launch");
   g_last_launches = 1;
   return DSA_OK;
 }

@@ -170,6 +170,28 @@ int bgemm_tile_n(int N);
 cudaError_t launch_bgemm(const CUtensorMap& ta, const CUtensorMap& tb, const BgemmArgs& a,
                          int batch, bool a_mn, bool b_mn, int bn, cudaStream_t stream);
 
+// ---------------- split key cache (decode over G devices) ----------------
+struct ShardOffsets {
+  long long v[16];   // first key of shard g
+};
+// ext_scores / ext_idx [R][G k] from the shards' candidates [G][R][k] (score and
+// shard-local index, < 0 none): -inf and -1 where there is no candidate.
+cudaError_t launch_cp_pack(const float* cand_scores, const int32_t* cand_idx,
+                           const ShardOffsets& lo, int G, long long R, int k, float* ext_scores,
+                           int32_t* ext_idx, int num_sms, cudaStream_t stream);
+// idx_out [R][k] = global indices of the selected positions pos [R][k], keyless
+// ones dropped, ascending then -1; sel [R][k] (optional) compacted alongside.
+cudaError_t launch_cp_map_compact(const int32_t* pos, const int32_t* ext_idx, long long R, int n,
+                                  int k, int32_t* idx_out, float* sel, int num_sms,
+                                  cudaStream_t stream);
+cudaError_t launch_cp_localize(const int32_t* idx, int32_t* out, long long n, int lo, int len,
+                               int num_sms, cudaStream_t stream);
+// out [rows][Dv] bf16 (and lse_out [rows], optional) from G partial pairs
+// part_out [G][rows][Dv] bf16, part_lse [G][rows].
+cudaError_t launch_cp_combine(const uint16_t* part_out, const float* part_lse, int G,
+                              long long rows, int Dv, uint16_t* out, float* lse_out, int num_sms,
+                              cudaStream_t stream);
+
 // ---------------- debug ----------------
 cudaError_t launch_debug_wait(DevCtl ctl, cudaStream_t stream);
 
