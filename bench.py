@@ -626,6 +626,8 @@ def reference_arm(args):
 PROFILE_CASES = {
     # one 2048-row prefill chunk of the 8K workload (rows 6144..8191, all keys causal)
     "prefill_chunk": ("prefill_8k", dict(Lq=2048, q_pos0=6144)),
+    # the same chunk through dsa_forward_fused (top-k inside the indexer kernel)
+    "prefill_chunk_fused": ("prefill_8k", dict(Lq=2048, q_pos0=6144)),
     # 16 decode sequences against 131072 cached keys
     "decode_small": ("decode_128k", dict(B=16)),
     # the indexer KL target over the forward's top-k sets of the prefill chunk above
@@ -671,7 +673,7 @@ def profile_case(name: str) -> None:
                             dI)
     else:
         for _ in range(2):
-            dsa.forward(p, inp)
+            dsa.forward(p, inp, fused=name.endswith("_fused"))
     torch.cuda.synchronize()
     dsa.check_status()
     print(f"profile case {name}: {cfg}")

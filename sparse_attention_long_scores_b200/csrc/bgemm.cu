@@ -17,9 +17,9 @@
 // One CTA computes one 128 x BN tile: thread 0 streams 64-deep K tiles of A and
 // B with TMA (128-byte swizzle) through a ring of 2 to 4 stages, thread 32 issues
 // tcgen05.mma (M = 128, N = BN, K = 16) into a TMEM accumulator, and the four
-// warps then read their 32 TMEM lanes each and store the rows; two CTAs share
-// an SM, so one's stores overlap the other's main loop. Every wait is bounded
-// (site kSiteGemm).
+// warps then read their 32 TMEM lanes each and store the rows (transposed through
+// shared memory into full-row stores); two CTAs share an SM, so one's stores
+// overlap the other's main loop. Every wait is bounded (site kSiteGemm).
 #include <cuda_bf16.h>
 
 #include "dsa_kernels.h"
@@ -138,30 +138,38 @@ __global__ void __launch_bounds__(BG_THREADS, 2)
   // epilogue: warp w holds rows m0 + 32 w .. + 31 in TMEM lanes 32 w ..
   const bool have = mbar_wait(done, 0u, a.ctl, abort_flag, kSiteGemm, 3);
   tc_fence_after();
+  fence_proxy_async_smem();   // the stages' TMA data is consumed; their space is reused below
   if (have) {
-    const int m = m0 + warp * 32 + lane;
-    float* crow = a.C + (long long)z * a.sC + (long long)m * a.c_sm;
-    const bool vec = a.c_sn == 1 && (a.c_sm % 4) == 0 && (a.sC % 4) == 0 &&
-                     (reinterpret_cast<uintptr_t>(a.C) & 15u) == 0;
+    // Row-major C (c_sn == 1): each 32 x 32 block goes through shared memory (the
+    // drained pipeline stages), so that a store instruction writes 32 consecutive
+    // columns of one row instead of one column of 32 rows.
+    float* tile = reinterpret_cast<float*>(smem) + warp * (32 * 33);
+    const int m_lane = m0 + warp * 32 + lane;
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 32) {
       if (n0 + c0 >= a.N) break;   // uniform across the CTA
       uint32_t r[32];
       tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, r);
       tmem_wait_ld();
-      if (m < a.M) {
-        const int n = n0 + c0;
-        if (vec && n + 32 <= a.N) {
-          float4* d4 = reinterpret_cast<float4*>(crow + n);
+      const int n = n0 + c0;
+      if (a.c_sn == 1) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            d4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (n + j < a.N) crow[(long long)(n + j) * a.c_sn] = __uint_as_float(r[j]);
+        for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = __uint_as_float(r[j]);
+        __syncwarp();
+        const bool col_ok = n + lane < a.N;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; ++rr) {
+          const int m = m0 + warp * 32 + rr;
+          if (m < a.M && col_ok)
+            a.C[(long long)z * a.sC + (long long)m * a.c_sm + n + lane] = tile[rr * 33 + lane];
         }
+        __syncwarp();
+      } else if (m_lane < a.M) {
+        // column-strided C: consecutive lanes (rows) are consecutive when c_sm == 1
+        float* crow = a.C + (long long)z * a.sC + (long long)m_lane * a.c_sm;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (n + j < a.N) crow[(long long)(n + j) * a.c_sn] = __uint_as_float(r[j]);
       }
     }
   }
