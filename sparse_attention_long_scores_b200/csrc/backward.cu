@@ -6,10 +6,9 @@
 //
 // The contractions of both gradients run as batched tensor-core GEMMs
 // (bgemm.cu) over the selected rows gathered here into a dense per-token block;
-// these kernels do the gathers, the softmax / ReLU gradient in between and the
-// scatter-add of the per-token key gradients back into the shared rows. The
-// row kernels are grid-stride loops with one warp per row, so any grid size is
-// correct.
+// these kernels do the gathers and the softmax / ReLU gradient in between (the
+// GEMMs add the key gradients into the shared rows themselves). The row kernels
+// are grid-stride loops with one warp per row, so any grid size is correct.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -175,25 +174,6 @@ __global__ void mla_bwd_softmax_kernel(const float* __restrict__ SP,
       *reinterpret_cast<uint2*>(p_out + j) = make_uint2(pb[0] | (uint32_t(pb[1]) << 16), pb[2] | (uint32_t(pb[3]) << 16));
       *reinterpret_cast<uint2*>(z_out + j) = make_uint2(zb[0] | (uint32_t(zb[1]) << 16), zb[2] | (uint32_t(zb[3]) << 16));
     }
-  }
-}
-
-// dst[b][idx[tok][j]][:] += src[tt][j][:] over rows of V float4 vectors (atomic:
-// tokens of one sequence share keys).
-__global__ void scatter_add_rows_kernel(const float4* __restrict__ src,
-                                        const int32_t* __restrict__ idx, float4* __restrict__ dst,
-                                        long long tok0, int T, int Lq, int Lk, int k, int V) {
-  const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(T) * k;
-  for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
-    const long long tok = tok0 + r / k;
-    const int j = static_cast<int>(r % k);
-    const int s = selected_key(idx, tok, j, k, Lk);
-    if (s < 0) continue;
-    const long long b = tok / Lq;
-    float4* d = dst + (b * Lk + s) * V;
-    const float4* x = src + r * V;
-    for (int v = lane; v < V; v += 32) atomicAdd(d + v, x[v]);
   }
 }
 
@@ -443,16 +423,6 @@ cudaError_t launch_mla_bwd_softmax(const float* SP, const float* lse, const int3
   const long long rows = static_cast<long long>(T) * H;
   mla_bwd_softmax_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
       SP, lse, idx, PZ, tok0, T, H, k, Lk, sm_scale);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float* dst,
-                                    long long tok0, int T, int Lq, int Lk, int k, int D,
-                                    int num_sms, cudaStream_t stream) {
-  const long long rows = static_cast<long long>(T) * k;
-  scatter_add_rows_kernel<<<row_blocks(rows, num_sms), kRowThreads, 0, stream>>>(
-      reinterpret_cast<const float4*>(src), idx, reinterpret_cast<float4*>(dst), tok0, T, Lq, Lk,
-      k, D / 4);
   return cudaGetLastError();
 }
 

@@ -12,7 +12,9 @@
 // arrive as zeros. A K-period (in 64-element tiles) lets one operand repeat
 // along K, which the split-precision products use (A [a0|a1|a2] times B
 // [b|b|b]). C is written with arbitrary element strides for m and n, so a
-// transposed result needs no separate pass.
+// transposed result needs no separate pass, or added row by row with fp32
+// atomics into rows chosen by an index list (the key gradients of the selected
+// rows go straight into the shared key rows).
 //
 // One CTA computes one 128 x BN tile: thread 0 streams 64-deep K tiles of A and
 // B with TMA (128-byte swizzle) through a ring of 2 to 4 stages, thread 32 issues
@@ -157,11 +159,25 @@ __global__ void __launch_bounds__(BG_THREADS, 2)
         for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = __uint_as_float(r[j]);
         __syncwarp();
         const bool col_ok = n + lane < a.N;
+        if (a.sidx != nullptr) {
+          // scatter-add: each row goes to its key's row of the sequence
+          const long long tok = a.s_tok0 + z;
+          float* cseq = a.C + (tok / a.s_Lq) * (long long)a.s_Lk * a.c_sm;
+          const int32_t* srow = a.sidx + tok * a.s_k;
 #pragma unroll 4
-        for (int rr = 0; rr < 32; ++rr) {
-          const int m = m0 + warp * 32 + rr;
-          if (m < a.M && col_ok)
-            a.C[(long long)z * a.sC + (long long)m * a.c_sm + n + lane] = tile[rr * 33 + lane];
+          for (int rr = 0; rr < 32; ++rr) {
+            const int m = m0 + warp * 32 + rr;
+            const int key = m < a.M ? srow[m] : -1;
+            if (key >= 0 && key < a.s_Lk && col_ok)
+              atomicAdd(cseq + (long long)key * a.c_sm + n + lane, tile[rr * 33 + lane]);
+          }
+        } else {
+#pragma unroll 4
+          for (int rr = 0; rr < 32; ++rr) {
+            const int m = m0 + warp * 32 + rr;
+            if (m < a.M && col_ok)
+              a.C[(long long)z * a.sC + (long long)m * a.c_sm + n + lane] = tile[rr * 33 + lane];
+          }
         }
         __syncwarp();
       } else if (m_lane < a.M) {
@@ -215,6 +231,8 @@ int bgemm_tile_n(int N) {
 cudaError_t launch_bgemm(const CUtensorMap& ta, const CUtensorMap& tb, const BgemmArgs& a,
                          int batch, bool a_mn, bool b_mn, int bn, cudaStream_t stream) {
   if (batch < 1 || batch > 65535 || a.M < 1 || a.N < 1 || a.K < 1 || a.a_kt < 1 || a.b_kt < 1)
+    return cudaErrorInvalidValue;
+  if (a.sidx != nullptr && (a.c_sn != 1 || a.s_k < a.M || a.s_Lq < 1 || a.s_Lk < 1))
     return cudaErrorInvalidValue;
   if (a_mn) {
     return b_mn ? launch_bgemm_bn<true, true>(ta, tb, a, batch, bn, stream)

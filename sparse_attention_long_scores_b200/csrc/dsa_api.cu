@@ -1149,8 +1149,8 @@ int dsa_debug_wait_timeout(void* stream) {
 //
 // Per chunk of T tokens the selected rows are gathered into a dense [T, k, D]
 // block, the per-token contractions run as batched bf16 tensor-core GEMMs with
-// fp32 accumulation (bgemm.cu), and the per-token key gradients are
-// scatter-added into the shared rows. The indexer's code dots are exact up to
+// fp32 accumulation (bgemm.cu), and the key-gradient products add their rows
+// straight into the shared key rows with fp32 atomics. The indexer's code dots are exact up to
 // fp32 rounding and the ReLU mask is re-decided exactly in fp64 wherever that
 // rounding could change its sign; its real-valued gradient operands enter the
 // products as three bf16 terms (24 significant bits).
@@ -1169,10 +1169,19 @@ struct GemmOperand {
   int period;
 };
 
-// C[z] (fp32, element (z, m, n) at C + z sC + m c_sm + n c_sn) = A[z] B[z]^T.
+// Key-row scatter of a product's rows (see BgemmArgs): row m of batch z adds into
+// row idx[(tok0 + z) * k + m] of sequence (tok0 + z) / Lq.
+struct RowScatter {
+  const int32_t* idx;
+  long long tok0;
+  int k, Lq, Lk;
+};
+
+// C[z] (fp32, element (z, m, n) at C + z sC + m c_sm + n c_sn) = A[z] B[z]^T, or,
+// with a RowScatter, C's key rows += the rows of A[z] B[z]^T.
 int tc_gemm(const GemmOperand& A, const GemmOperand& B, int M, int N, int K, float* C,
             long long c_sm, long long c_sn, long long sC, int batch, const dsa::DevCtl& ctl,
-            cudaStream_t s, const char* what) {
+            cudaStream_t s, const char* what, const RowScatter* scatter = nullptr) {
   const int bn = dsa::bgemm_tile_n(N);
   CUtensorMap ta, tb;
   DSA_TRY(make_map_3d(&ta, A.base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A.inner, A.rows, A.depth,
@@ -1192,6 +1201,13 @@ int tc_gemm(const GemmOperand& A, const GemmOperand& B, int M, int N, int K, flo
   a.c_sm = c_sm;
   a.c_sn = c_sn;
   a.sC = sC;
+  if (scatter != nullptr) {
+    a.sidx = scatter->idx;
+    a.s_tok0 = scatter->tok0;
+    a.s_k = scatter->k;
+    a.s_Lq = scatter->Lq;
+    a.s_Lk = scatter->Lk;
+  }
   a.ctl = ctl;
   DSA_TRY_CUDA(dsa::launch_bgemm(ta, tb, a, batch, A.mn, B.mn, bn, s), what);
   return DSA_OK;
@@ -1204,7 +1220,7 @@ char* align256(void* p) {
 // Workspace of the attention backward for T tokens (offsets from a 256-byte
 // aligned base; total includes the alignment slack).
 struct MlaBwdLayout {
-  size_t cg, qo, sp, pz, dc, total;
+  size_t cg, qo, sp, pz, total;
 };
 MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
   MlaBwdLayout L{};
@@ -1219,7 +1235,6 @@ MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
   L.qo = take((size_t)T * 2 * H * Dqk * sizeof(uint16_t));  // [q; dout padded], bf16
   L.sp = take(t2hk * sizeof(float));                     // [q . c; dout . c[:Dv]]
   L.pz = take(t2hk * sizeof(uint16_t));                  // [dz; P], bf16
-  L.dc = take(tk * Dqk * sizeof(float));                 // per-token row gradients
   L.total = off + 256;
   return L;
 }
@@ -1227,7 +1242,7 @@ MlaBwdLayout mla_bwd_layout(int T, int H, int Dqk, int k) {
 // Workspace of the indexer backward for T tokens; kp = k rounded up to 64,
 // hp = H_I rounded up to 64 (the K tiles of the split products).
 struct IdxBwdLayout {
-  size_t kb, qb, xt, g1, g2, dk, total;
+  size_t kb, qb, xt, g1, g2, total;
   int kp, hp;
 };
 IdxBwdLayout idx_bwd_layout(int T, int H_I, int d_I, int k) {
@@ -1246,7 +1261,6 @@ IdxBwdLayout idx_bwd_layout(int T, int H_I, int d_I, int k) {
   L.xt = take(tk * H_I * sizeof(float));                           // code dots [T][k][H_I]
   L.g1 = take((size_t)T * H_I * 3 * L.kp * sizeof(uint16_t));      // G1 in three parts
   L.g2 = take((size_t)T * 3 * L.hp * k * sizeof(uint16_t));        // G2 in three parts
-  L.dk = take(tk * d_I * sizeof(float));                           // per-token key gradients
   L.total = off + 256;
   return L;
 }
@@ -1298,7 +1312,6 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
   uint16_t* QO = reinterpret_cast<uint16_t*>(base + L.qo);
   float* SP = reinterpret_cast<float*>(base + L.sp);
   uint16_t* PZ = reinterpret_cast<uint16_t*>(base + L.pz);
-  float* dC = reinterpret_cast<float*>(base + L.dc);
   int launched = 0;
   if (!accumulate_dkv)
     DSA_TRY_CUDA(cudaMemsetAsync(dkv, 0, (size_t)B * Lk * Dqk * sizeof(float), s), "dkv clear");
@@ -1327,11 +1340,11 @@ int dsa_sparse_mla_bwd(const uint16_t* q, const uint16_t* kv, const int32_t* idx
                  "softmax gradient launch");
     DSA_TRY(tc_gemm(dz_k, c_mn, H, Dqk, k, dq + tok0 * H * Dqk, Dqk, 1, (long long)H * Dqk, Tc,
                     ctl, s, "dq = dz C"));
-    DSA_TRY(tc_gemm(pz_mn, qo_mn, k, Dqk, 2 * H, dC, Dqk, 1, (long long)k * Dqk, Tc, ctl, s,
-                    "dC = [dz; P]^T QO"));
-    DSA_TRY_CUDA(dsa::launch_scatter_add_rows(dC, idx, dkv, tok0, Tc, Lq, Lk, k, Dqk, sms, s),
-                 "row gradient scatter launch");
-    launched += 7;
+    // dC = [dz; P]^T QO, added row by row into the selected latent rows of dkv
+    const RowScatter to_dkv{idx, tok0, k, Lq, Lk};
+    DSA_TRY(tc_gemm(pz_mn, qo_mn, k, Dqk, 2 * H, dkv, Dqk, 1, 0, Tc, ctl, s,
+                    "dkv += [dz; P]^T QO", &to_dkv));
+    launched += 6;
   }
   g_last_launches = launched;
   return DSA_OK;
@@ -1381,7 +1394,6 @@ int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
   float* XT = reinterpret_cast<float*>(base + L.xt);
   uint16_t* G1s = reinterpret_cast<uint16_t*>(base + L.g1);
   uint16_t* G2s = reinterpret_cast<uint16_t*>(base + L.g2);
-  float* dK = reinterpret_cast<float*>(base + L.dk);
   int launched = 0;
   if (!accumulate_dkI)
     DSA_TRY_CUDA(cudaMemsetAsync(dkI, 0, (size_t)B * Lk * d_I * sizeof(float), s), "dkI clear");
@@ -1411,12 +1423,11 @@ int dsa_indexer_bwd(const uint8_t* qI, const float* qI_scale, const uint8_t* kI,
     // dq^I [H_I x d_I], written transposed from (dq^I)^T = khat^T G1^T over K = 3 kp
     DSA_TRY(tc_gemm(kb_mn, g1_k, d_I, H_I, 3 * L.kp, dqI + tok0 * qs, 1, d_I, qs, Tc, ctl, s,
                     "dqI = G1 khat"));
-    // dK [k x d_I] = G2^T qhat over K = 3 hp
-    DSA_TRY(tc_gemm(g2_mn, qb_mn, k, d_I, 3 * L.hp, dK, d_I, 1, (long long)k * d_I, Tc, ctl, s,
-                    "dK = G2^T qhat"));
-    DSA_TRY_CUDA(dsa::launch_scatter_add_rows(dK, idx, dkI, tok0, Tc, Lq, Lk, k, d_I, sms, s),
-                 "key gradient scatter launch");
-    launched += 7;
+    // G2^T qhat over K = 3 hp [k x d_I], added row by row into the selected keys of dkI
+    const RowScatter to_dkI{idx, tok0, k, Lq, Lk};
+    DSA_TRY(tc_gemm(g2_mn, qb_mn, k, d_I, 3 * L.hp, dkI, d_I, 1, 0, Tc, ctl, s,
+                    "dkI += G2^T qhat", &to_dkI));
+    launched += 6;
   }
   g_last_launches = launched;
   return DSA_OK;

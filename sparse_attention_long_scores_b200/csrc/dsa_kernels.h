@@ -126,10 +126,6 @@ cudaError_t launch_pack_qo(const uint16_t* q, const uint16_t* dout, uint16_t* qo
 cudaError_t launch_mla_bwd_softmax(const float* SP, const float* lse, const int32_t* idx,
                                    uint16_t* PZ, long long tok0, int T, int H, int k, int Lk,
                                    float sm_scale, int num_sms, cudaStream_t stream);
-// dst [B, Lk, D] fp32 += src [T, k, D] fp32 row by row (atomic); D % 4 == 0.
-cudaError_t launch_scatter_add_rows(const float* src, const int32_t* idx, float* dst,
-                                    long long tok0, int T, int Lq, int Lk, int k, int D,
-                                    int num_sms, cudaStream_t stream);
 // out [T, k, d_I] bf16 = the selected e4m3 rows of kI [B, Lk, d_I] (codes, exact).
 cudaError_t launch_gather_e4m3_rows_bf16(const uint8_t* kI, const int32_t* idx, uint16_t* out,
                                          long long tok0, int T, int Lq, int Lk, int k, int d_I,
@@ -163,6 +159,13 @@ struct BgemmArgs {
   int a_kt, b_kt;
   float* C;                  // element (z, m, n) at C + z * sC + m * c_sm + n * c_sn
   long long c_sm, c_sn, sC;
+  // Scatter-add mode (sidx != null, c_sn == 1): row m of batch z is added with fp32
+  // atomics into row s = sidx[(s_tok0 + z) * s_k + m] of sequence (s_tok0 + z) / s_Lq,
+  // i.e. at C + (((s_tok0 + z) / s_Lq) * s_Lk + s) * c_sm; rows with s outside
+  // [0, s_Lk) are dropped (sC is unused).
+  const int32_t* sidx;
+  long long s_tok0;
+  int s_k, s_Lq, s_Lk;
   DevCtl ctl;
 };
 // Tile width (N) used for an N-column product: 64, 128, 192 or 256.
