@@ -160,14 +160,18 @@ __device__ __noinline__ bool mla_issue_tiles(int ntiles, uint32_t tbase, uint32_
   uint64_t* p_full = bars + Tr::BAR_P_FULL;
   uint64_t* pv_done = bars + Tr::BAR_PV_DONE;
   const uint32_t o_tmem = tbase, s_tmem = tbase + Tr::COL_S, qt_tmem = tbase + Tr::COL_Q;
-  // stage descriptors: K-major for S, and this slice's value blocks MN-major for PV
-  const uint64_t kd[2] = {make_sdesc(kv_base, 16, 1024, 2),
-                          make_sdesc(kv_base + NKB * Tr::KVBLK, 16, 1024, 2)};
+  // stage descriptors: K-major for S, and this slice's value blocks MN-major for PV.
+  // They are chosen per stage with selects, not indexed from an array: an array
+  // indexed at run time lives in local memory, and every MMA's memory clobber
+  // would then reload it, putting a local-memory round trip in front of each
+  // MMA issue.
+  const uint64_t kd0 = make_sdesc(kv_base, 16, 1024, 2);
+  const uint64_t kd1 = make_sdesc(kv_base + NKB * Tr::KVBLK, 16, 1024, 2);
   constexpr uint32_t v_off = (uint32_t)(DVCI * Tr::NB_B) * Tr::KVBLK;
-  const uint64_t bd[2] = {make_sdesc(kv_base + v_off, Tr::KVBLK, 1024, 2),
-                          make_sdesc(kv_base + NKB * Tr::KVBLK + v_off, Tr::KVBLK, 1024, 2)};
+  const uint64_t bd0 = make_sdesc(kv_base + v_off, Tr::KVBLK, 1024, 2);
+  const uint64_t bd1 = make_sdesc(kv_base + NKB * Tr::KVBLK + v_off, Tr::KVBLK, 1024, 2);
   auto pv = [&](int j) {
-    issue_pv<NKB, DVC>(o_tmem, s_tmem + (uint32_t)((j & 1) * KEYS), bd[j & 1], j == 0);
+    issue_pv<NKB, DVC>(o_tmem, s_tmem + (uint32_t)((j & 1) * KEYS), (j & 1) ? bd1 : bd0, j == 0);
     mma_commit(&kvB_empty[j & 1]);
     mma_commit(&pv_done[j & 1]);
   };
@@ -177,7 +181,8 @@ __device__ __noinline__ bool mla_issue_tiles(int ntiles, uint32_t tbase, uint32_
     const uint32_t sb = s_tmem + (uint32_t)(st * KEYS);
     if (!mbar_wait(&kvA_full[st], ph, ctl, abort_flag, kSiteMla, 3)) return false;
     tc_fence_after();
-    issue_s_part<NKB, DVC, DVCI, 0>(sb, qt_tmem, qd0, kd[st]);
+    const uint64_t kds = st ? kd1 : kd0;
+    issue_s_part<NKB, DVC, DVCI, 0>(sb, qt_tmem, qd0, kds);
     mma_commit(&kvA_empty[st]);
     bool pv_pending = i > 0;
     if (pv_pending && mbar_test_wait(smem_u32(&p_full[(i - 1) & 1]), (uint32_t)((i - 1) >> 1) & 1u)) {
@@ -187,7 +192,7 @@ __device__ __noinline__ bool mla_issue_tiles(int ntiles, uint32_t tbase, uint32_
     }
     if (!mbar_wait(&kvB_full[st], ph, ctl, abort_flag, kSiteMla, 4)) return false;
     tc_fence_after();
-    issue_s_part<NKB, DVC, DVCI, 1>(sb, qt_tmem, qd0, kd[st]);
+    issue_s_part<NKB, DVC, DVCI, 1>(sb, qt_tmem, qd0, kds);
     mma_commit(&s_full[st]);
     if (pv_pending) {
       if (!mbar_wait(&p_full[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, ctl, abort_flag, kSiteMla, 5))
