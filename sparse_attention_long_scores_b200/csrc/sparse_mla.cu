@@ -311,7 +311,15 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_map(&tmap_q);
+    // All of the token's Q rows are requested at once, before anything else of
+    // the prologue: the blocks read from shared memory to their place, and the
+    // blocks that go to TMEM into the second KV stage, which no tile uses before
+    // the softmax warps have moved them on (qt_full).
+    mbar_arrive_expect_tx(q_full, NKB * Tr::QBLK);
+    for (int kb = 0; kb < Tr::QS_KB; ++kb)
+      tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, (Tr::QT_KB + kb) * 64, (int)(token * a.H), q_full);
+    for (int kb = 0; kb < Tr::QT_KB; ++kb)
+      tma_load_2d(kv_smem + NKB * Tr::KVBLK + kb * Tr::QBLK, &tmap_q, kb * 64, (int)(token * a.H), q_full);
   }
   if (warp == 1) {
     // number of 32-key tiles this CTA covers: trailing invalid entries are trimmed
@@ -344,20 +352,15 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------ MMA issuer (and the Q load)
     if (lane == 0) {
-      bool ok = true;
-      if (ntiles > 0) {
-        mbar_arrive_expect_tx(q_full, Tr::QS_KB * Tr::QBLK);
-        for (int kb = 0; kb < Tr::QS_KB; ++kb)
-          tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, (Tr::QT_KB + kb) * 64, (int)(token * a.H),
-                      q_full);
-        ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 1);
-        if (!ok) {
-          DevCtl drain = a.ctl;
-          volatile int never = 0;
-          mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
-        }
-        ok = ok && mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 12);
+      // Q's copies land even when the CTA has no tile (they were issued before
+      // the tile count was known) and must not be in flight when it exits
+      bool ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 1);
+      if (!ok) {
+        DevCtl drain = a.ctl;
+        volatile int never = 0;
+        mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
       }
+      if (ntiles > 0) ok = ok && mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 12);
       // Descriptors are built once; per MMA only the start-address field moves
       // (byte offset / 16 added to the low bits, which never carry: smem < 256 KB).
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
@@ -416,6 +419,8 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
       const uint32_t ph = ((i / Tr::STAGES) & 1) ^ 1;
+      // the second stage first holds Q's TMEM blocks
+      if (i == 1 && !mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 18)) break;
       // this warp's rows: index, validity and source row (invalid keys read row 0
       // and are masked later; paged: the key's pool row, a page outside the pool
       // reads pool row 0)
@@ -456,30 +461,32 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     constexpr int OCOLS = DVC / 2;           // O columns this thread rescales and writes
     // this head's first QT_KB * 64 query columns go to TMEM (the MMA's A operand:
-    // lane = head, 32-bit column = two consecutive bf16 of the row); each half
+    // lane = head, 32-bit column = two consecutive bf16 of the row), read from the
+    // 128-byte-swizzled rows the TMA put into the second KV stage; each half
     // writes its share of the blocks
+    bool ok = true;
     if (ntiles > 0) {
-      const long long qrow = token * a.H + h;
-      const bool have = qrow < (long long)a.B * a.Lq * a.H;
-      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) + (have ? qrow : 0) * (long long)a.Dqk * 2;
+      ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 17);
+      if (ok) {
+        const uint32_t qrow = smem_u32(kv_smem + NKB * Tr::KVBLK) + (uint32_t)h * 128u;
 #pragma unroll 1
-      for (int kb = hf; kb < Tr::QT_KB; kb += 2) {
-        uint32_t qv[32];
+        for (int kb = hf; kb < Tr::QT_KB; kb += 2) {
+          uint32_t qv[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 u = have ? *reinterpret_cast<const uint4*>(qsrc + kb * 128 + c * 16) : make_uint4(0u, 0u, 0u, 0u);
-          qv[4 * c] = u.x; qv[4 * c + 1] = u.y; qv[4 * c + 2] = u.z; qv[4 * c + 3] = u.w;
+          for (int c = 0; c < 8; ++c) {
+            const uint4 u = ld_shared_v4(qrow + (uint32_t)(kb * Tr::QBLK) + ((uint32_t)(c ^ (h & 7)) << 4));
+            qv[4 * c] = u.x; qv[4 * c + 1] = u.y; qv[4 * c + 2] = u.z; qv[4 * c + 3] = u.w;
+          }
+          tmem_st32(qt_tmem + lane_off + kb * 32, qv);
         }
-        tmem_st32(qt_tmem + lane_off + kb * 32, qv);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(qt_full);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(qt_full);
     }
     float m_used = -INFINITY;  // running max (log2 domain) that P is relative to
     float l = 0.f;             // this thread's 32-key share of the row sum
-    bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
+    for (int i = 0; ok && i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
       if (!mbar_wait(&s_full[i & 1], (i >> 1) & 1, a.ctl, abort_flag, kSiteMla, 10)) { ok = false; break; }
       if (!mbar_wait(&kvB_full[st], (i / Tr::STAGES) & 1, a.ctl, abort_flag, kSiteMla, 11)) { ok = false; break; }
