@@ -336,6 +336,11 @@ DSA_DEVICE_INLINE uint4 ld_shared_v4(uint32_t addr) {
                : "memory");
   return v;
 }
+// 16-byte shared-memory store.
+DSA_DEVICE_INLINE void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
 DSA_DEVICE_INLINE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 DSA_DEVICE_INLINE void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }

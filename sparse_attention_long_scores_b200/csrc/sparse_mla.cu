@@ -562,17 +562,24 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       ok = mbar_wait(xl_bar, 0, a.ctl, abort_flag, kSiteMla, 16);
       if (ok) l += xl[(hf ^ 1) * 128 + h];
     }
+    ok = __all_sync(0xffffffffu, ok);   // the epilogue below synchronises the warp
     if (ok) {
       const bool row_ok = h < a.H;
       const bool empty = !(l > 0.f);
       if (a.splits == 1) {
         const float inv = empty ? 0.f : 1.f / l;
-        uint16_t* orow = a.out + (token * a.H + h) * (long long)a.Dv + dvc * DVC;
+        // The warp's 32 rows of OCOLS bf16 go through shared memory (the KV stages:
+        // every MMA is done) so that the global stores are row-contiguous: written
+        // one row per lane with the 16-byte chunks rotated by the row (no bank
+        // conflicts), read back NCH lanes per row.
+        constexpr int NCH = OCOLS * 2 / 16;            // 16-byte chunks per row
+        const uint32_t stg = smem_u32(kv_smem) + (uint32_t)(sw * 32 * OCOLS * 2);
+        const uint32_t my_row = stg + (uint32_t)(lane * OCOLS * 2);
 #pragma unroll 1
-        for (int c0 = hf * OCOLS; c0 < (hf + 1) * OCOLS; c0 += 32) {
+        for (int c0 = 0; c0 < OCOLS; c0 += 32) {
           uint32_t o[32];
           if (ntiles > 0) {
-            tmem_ld32(o_tmem + lane_off + c0, o);
+            tmem_ld32(o_tmem + lane_off + hf * OCOLS + c0, o);
             tmem_wait_ld();
           } else {
 #pragma unroll
@@ -582,11 +589,21 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
-          if (row_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) {
+            const int ch = c0 / 8 + c;
+            st_shared_v4(my_row + (uint32_t)(((ch + lane) % NCH) * 16),
+                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
           }
+        }
+        __syncwarp();
+        uint16_t* obase = a.out + token * a.H * (long long)a.Dv + dvc * DVC + hf * OCOLS;
+#pragma unroll 4
+        for (int e = lane; e < 32 * NCH; e += 32) {
+          const int r = e / NCH, ch = e % NCH;
+          const uint4 v = ld_shared_v4(stg + (uint32_t)(r * OCOLS * 2 + ((ch + r) % NCH) * 16));
+          const int hr = quad * 32 + r;
+          if (hr < a.H) *reinterpret_cast<uint4*>(obase + (long long)hr * a.Dv + ch * 8) = v;
         }
         if (row_ok && hf == 0 && dvc == 0 && a.lse != nullptr)
           a.lse[token * a.H + h] = empty ? -INFINITY : (m_used + __log2f(l)) * 0.69314718055994531f;
