@@ -293,7 +293,18 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     }
   }
   if (threadIdx.x == 0) {
+    // All of the token's Q rows are requested first, before anything else of the
+    // prologue (they are its longest wait): the blocks read from shared memory to
+    // their place, and the blocks that go to TMEM into the second KV stage, which
+    // no tile uses before the softmax warps have moved them on (qt_full).
+    tma_prefetch_map(&tmap_q);
     mbar_init(q_full, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(q_full, NKB * Tr::QBLK);
+    for (int kb = 0; kb < Tr::QS_KB; ++kb)
+      tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, (Tr::QT_KB + kb) * 64, (int)(token * a.H), q_full);
+    for (int kb = 0; kb < Tr::QT_KB; ++kb)
+      tma_load_2d(kv_smem + NKB * Tr::KVBLK + kb * Tr::QBLK, &tmap_q, kb * 64, (int)(token * a.H), q_full);
     mbar_init(qt_full, SMX_WARPS * 32);
     for (int i = 0; i < Tr::STAGES; ++i) {
       mbar_init(&kvA_full[i], Tr::NP);
@@ -311,15 +322,6 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    // All of the token's Q rows are requested at once, before anything else of
-    // the prologue: the blocks read from shared memory to their place, and the
-    // blocks that go to TMEM into the second KV stage, which no tile uses before
-    // the softmax warps have moved them on (qt_full).
-    mbar_arrive_expect_tx(q_full, NKB * Tr::QBLK);
-    for (int kb = 0; kb < Tr::QS_KB; ++kb)
-      tma_load_2d(q_smem + kb * Tr::QBLK, &tmap_q, (Tr::QT_KB + kb) * 64, (int)(token * a.H), q_full);
-    for (int kb = 0; kb < Tr::QT_KB; ++kb)
-      tma_load_2d(kv_smem + NKB * Tr::KVBLK + kb * Tr::QBLK, &tmap_q, kb * 64, (int)(token * a.H), q_full);
   }
   if (warp == 1) {
     // number of 32-key tiles this CTA covers: trailing invalid entries are trimmed
@@ -339,7 +341,8 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
       ntiles_slot[1] = t_lo;
     }
   }
-  if (warp == 0) tmem_alloc(tmem_slot, Tr::TMEM_COLS);
+  // TMEM comes from a warp that has nothing else to do before the barrier
+  if (warp == 2) tmem_alloc(tmem_slot, Tr::TMEM_COLS);
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
@@ -637,7 +640,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   }
 
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tbase, Tr::TMEM_COLS);
   }
