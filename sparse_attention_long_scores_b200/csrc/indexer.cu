@@ -475,13 +475,31 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N, SEL>::THREADS, IdxTrait
         if (!mbar_wait(&acc_full[ac], aph, a.ctl, abort_flag, kSiteIndexer, 8)) { ok = false; break; }
         tc_fence_after();
         if constexpr (H_I == 64) {
-          // one token (64 heads) per step: both TMEM loads in flight, one wait
-#pragma unroll 1
-          for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 64) {
-            uint32_t r[64];
-            tmem_ld32(t_lane + (uint32_t)(ac * N + c0), *reinterpret_cast<uint32_t(*)[32]>(r));
-            tmem_ld32(t_lane + (uint32_t)(ac * N + c0 + 32), *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-            tmem_wait_ld();
+          // all of this warp's columns (one token of 64 heads per 64 columns) are
+          // loaded with one wait, and the accumulator goes back to the MMA issuer
+          // before the head reduction runs from registers
+          // (with the fused selectors' threads the registers allow one token per wait)
+          constexpr int NTOK = COLS / 64;
+          constexpr int G = SEL ? 1 : NTOK;   // tokens per wait
+#pragma unroll
+          for (int tg = 0; tg < NTOK; tg += G) {
+          uint32_t rr[G][64];
+#pragma unroll
+          for (int tk = 0; tk < G; ++tk) {
+            tmem_ld32(t_lane + (uint32_t)(ac * N + c_begin + 64 * (tg + tk)),
+                      *reinterpret_cast<uint32_t(*)[32]>(rr[tk]));
+            tmem_ld32(t_lane + (uint32_t)(ac * N + c_begin + 64 * (tg + tk) + 32),
+                      *reinterpret_cast<uint32_t(*)[32]>(rr[tk] + 32));
+          }
+          tmem_wait_ld();
+          if (tg + G >= NTOK) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ac]);
+          }
+#pragma unroll
+          for (int tk = 0; tk < G; ++tk) {
+            const int c0 = c_begin + 64 * (tg + tk);
+            const uint32_t* r = rr[tk];
             // four independent packed partial sums: no serial FMA chain
             float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                               make_float2(0.f, 0.f)};
@@ -506,6 +524,7 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N, SEL>::THREADS, IdxTrait
             if (key_ok && t < un.t_b && s <= qp + t)
               a.scores[((long long)un.b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + s] = part * ks;
           }
+          }
         } else {
 #pragma unroll 1
           for (int c0 = c_begin; c0 < c_begin + COLS; c0 += 32) {
@@ -526,9 +545,9 @@ __global__ void __launch_bounds__(IdxTraits<D_I, H_I, N, SEL>::THREADS, IdxTrait
               }
             }
           }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ac]);
         }
-        tc_fence_before();
-        mbar_arrive(&acc_empty[ac]);
         if (++ac == Tr::ACC) { ac = 0; aph ^= 1; }
       }
       if constexpr (SEL) {
