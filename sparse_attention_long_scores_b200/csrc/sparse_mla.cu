@@ -10,11 +10,12 @@
 //     online softmax over the key tiles     (base 2, lazy rescale of O)
 //     O[h, chunk] += P[h,s] . c_s[chunk]    (tcgen05, M = 128, N = DVC, K = 64 keys)
 // Layout of the work:
-//   warp 0      tcgen05 issuer: Q's shared-memory part once (TMA tiles), then for
-//               each 64-key tile, in a fixed order, S_i = Q K_i^T into one of two
-//               TMEM buffers (part A of the columns, then part B) and, between the
-//               two parts as soon as P_{i-1} is ready, O += P_{i-1} V_{i-1} with P
-//               read from TMEM;
+//   warp 0      tcgen05 issuer: for each 64-key tile, in a fixed order, S_i =
+//               Q K_i^T into one of two TMEM buffers (part A of the columns, then
+//               part B) and, between the two parts as soon as P_{i-1} is ready,
+//               O += P_{i-1} V_{i-1} with P read from TMEM. One lane runs the loop
+//               when each sequence has one query row (decode); with several rows
+//               (prefill) the whole warp runs it and one elected lane issues;
 //   warps 1..8  softmax, two warps per TMEM lane quadrant: a thread owns one head
 //               (TMEM lane) and 32 of the tile's 64 keys. The two threads of a head
 //               exchange their maxima through shared memory, write P_i (bf16) over
@@ -210,6 +211,94 @@ __device__ __noinline__ bool mla_issue_tiles(int ntiles, uint32_t tbase, uint32_
   return true;
 }
 
+// elect.sync over the full warp: true in exactly one lane (the same one every time).
+__device__ __forceinline__ bool elect_one_lane() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
+// The same issue order run by the whole issuer warp: every lane computes the
+// descriptors (warp-uniform values), one elected lane issues the MMAs and the
+// commits, lane 0 waits on the barriers and passes the outcome on by shuffle.
+// Issuing is faster this way, the barrier hand-offs slower: it pays where the
+// tensor pipe is the limit (many query rows per sequence, gathers mostly from
+// L2), not where the gathers' latency is (one decode row per sequence).
+template <int NKB, int DVC, int DVCI>
+__device__ __noinline__ bool mla_issue_tiles_warp(int ntiles, uint32_t tbase, uint32_t kv_base, uint64_t qd0,
+                                             uint64_t* bars, const DevCtl& ctl, volatile int* abort_flag) {
+  using Tr = MlaTraits<NKB, DVC>;
+  const int lane = lane_id();
+  uint64_t* kvA_full = bars + Tr::BAR_KV_FULL;
+  uint64_t* kvB_full = bars + Tr::BAR_KV_FULL + Tr::STAGES;
+  uint64_t* kvA_empty = bars + Tr::BAR_KV_EMPTY;
+  uint64_t* kvB_empty = bars + Tr::BAR_KV_EMPTY + Tr::STAGES;
+  uint64_t* s_full = bars + Tr::BAR_S_FULL;
+  uint64_t* p_full = bars + Tr::BAR_P_FULL;
+  uint64_t* pv_done = bars + Tr::BAR_PV_DONE;
+  const uint32_t o_tmem = tbase, s_tmem = tbase + Tr::COL_S, qt_tmem = tbase + Tr::COL_Q;
+  const uint64_t kd0 = make_sdesc(kv_base, 16, 1024, 2);
+  const uint64_t kd1 = make_sdesc(kv_base + NKB * Tr::KVBLK, 16, 1024, 2);
+  constexpr uint32_t v_off = (uint32_t)(DVCI * Tr::NB_B) * Tr::KVBLK;
+  const uint64_t bd0 = make_sdesc(kv_base + v_off, Tr::KVBLK, 1024, 2);
+  const uint64_t bd1 = make_sdesc(kv_base + NKB * Tr::KVBLK + v_off, Tr::KVBLK, 1024, 2);
+  auto wait_w = [&](uint64_t* bar, uint32_t par, int id) -> bool {
+    int r = 1;
+    if (lane == 0) r = mbar_wait(bar, par, ctl, abort_flag, kSiteMla, id) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, r, 0) != 0;
+  };
+  auto pv = [&](int j) {
+    if (elect_one_lane()) {
+      issue_pv<NKB, DVC>(o_tmem, s_tmem + (uint32_t)((j & 1) * KEYS), (j & 1) ? bd1 : bd0, j == 0);
+      mma_commit(&kvB_empty[j & 1]);
+      mma_commit(&pv_done[j & 1]);
+    }
+    __syncwarp();
+  };
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i & 1;   // STAGES == 2
+    const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+    const uint32_t sb = s_tmem + (uint32_t)(st * KEYS);
+    const uint64_t kds = st ? kd1 : kd0;
+    if (!wait_w(&kvA_full[st], ph, 3)) return false;
+    tc_fence_after();
+    if (elect_one_lane()) {
+      issue_s_part<NKB, DVC, DVCI, 0>(sb, qt_tmem, qd0, kds);
+      mma_commit(&kvA_empty[st]);
+    }
+    __syncwarp();
+    bool pv_pending = i > 0;
+    if (pv_pending) {
+      int ready = 0;
+      if (lane == 0) ready = mbar_test_wait(smem_u32(&p_full[(i - 1) & 1]), (uint32_t)((i - 1) >> 1) & 1u) ? 1 : 0;
+      if (__shfl_sync(0xffffffffu, ready, 0)) {
+        tc_fence_after();
+        pv(i - 1);
+        pv_pending = false;
+      }
+    }
+    if (!wait_w(&kvB_full[st], ph, 4)) return false;
+    tc_fence_after();
+    if (elect_one_lane()) {
+      issue_s_part<NKB, DVC, DVCI, 1>(sb, qt_tmem, qd0, kds);
+      mma_commit(&s_full[st]);
+    }
+    __syncwarp();
+    if (pv_pending) {
+      if (!wait_w(&p_full[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, 5)) return false;
+      tc_fence_after();
+      pv(i - 1);
+    }
+  }
+  if (ntiles > 0) {
+    const int j = ntiles - 1;
+    if (!wait_w(&p_full[j & 1], (uint32_t)(j >> 1) & 1u, 6)) return false;
+    tc_fence_after();
+    pv(j);
+  }
+  return true;
+}
+
 // The smallest bf16 value >= x (x not NaN), as its bit pattern. Both softmax
 // halves of a head derive the running max from the same two such values, so they
 // agree on it exactly; an upper bound of the tile max serves the online softmax as
@@ -235,7 +324,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 // PAGED: latent rows are gathered through the block table (pool rows); the
 // unpaged instantiation reads sequence b's rows directly.
-template <int NKB, int DVC, bool PAGED>
+template <int NKB, int DVC, bool PAGED, bool WARP_ISSUE>
 __global__ void __launch_bounds__(MLA_THREADS, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ kv,
                       const MlaArgs a) {
@@ -353,31 +442,61 @@ __global__ void __launch_bounds__(MLA_THREADS, 1)
   const uint32_t qt_tmem = tbase + Tr::COL_Q;
 
   if (warp == 0) {
-    // ------------------------------------------------ MMA issuer (and the Q load)
-    if (lane == 0) {
-      // Q's copies land even when the CTA has no tile (they were issued before
-      // the tile count was known) and must not be in flight when it exits
-      bool ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 1);
-      if (!ok) {
-        DevCtl drain = a.ctl;
-        volatile int never = 0;
-        mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
+    // ------------------------------------------------ MMA issuer (Q was requested at CTA start)
+    if constexpr (WARP_ISSUE) {
+      int okl = 1;
+      if (lane == 0) {
+        bool ok0 = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 1);
+        if (!ok0) {
+          DevCtl drain = a.ctl;
+          volatile int never = 0;
+          mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
+        }
+        if (ntiles > 0) ok0 = ok0 && mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 12);
+        okl = ok0 ? 1 : 0;
       }
-      if (ntiles > 0) ok = ok && mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 12);
-      // Descriptors are built once; per MMA only the start-address field moves
-      // (byte offset / 16 added to the low bits, which never carry: smem < 256 KB).
+      bool ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
       const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
       if (ok && ntiles > 0) {
         if (Tr::NB_B * 2 <= NKB && dvc != 0)
-          ok = mla_issue_tiles<NKB, DVC, 1>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
+          ok = mla_issue_tiles_warp<NKB, DVC, 1>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
         else
-          ok = mla_issue_tiles<NKB, DVC, 0>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
+          ok = mla_issue_tiles_warp<NKB, DVC, 0>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
       }
-      if (!ok) *abort_flag = 1;
-      mma_commit(done_bar);
-      DevCtl drain = a.ctl;
-      volatile int never = 0;
-      mbar_wait(done_bar, 0, drain, &never, kSiteMla, 7);
+      if (elect_one_lane()) {
+        if (!ok) *abort_flag = 1;
+        mma_commit(done_bar);
+        DevCtl drain = a.ctl;
+        volatile int never = 0;
+        mbar_wait(done_bar, 0, drain, &never, kSiteMla, 7);
+      }
+      __syncwarp();
+    } else {
+      if (lane == 0) {
+        // Q's copies land even when the CTA has no tile (they were issued before
+        // the tile count was known) and must not be in flight when it exits
+        bool ok = mbar_wait(q_full, 0, a.ctl, abort_flag, kSiteMla, 1);
+        if (!ok) {
+          DevCtl drain = a.ctl;
+          volatile int never = 0;
+          mbar_wait(q_full, 0, drain, &never, kSiteMla, 2);
+        }
+        if (ntiles > 0) ok = ok && mbar_wait(qt_full, 0, a.ctl, abort_flag, kSiteMla, 12);
+        // Descriptors are built once; per MMA only the start-address field moves
+        // (byte offset / 16 added to the low bits, which never carry: smem < 256 KB).
+        const uint64_t qd0 = make_sdesc(smem_u32(q_smem), 16, 1024, 2);
+        if (ok && ntiles > 0) {
+          if (Tr::NB_B * 2 <= NKB && dvc != 0)
+            ok = mla_issue_tiles<NKB, DVC, 1>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
+          else
+            ok = mla_issue_tiles<NKB, DVC, 0>(ntiles, tbase, smem_u32(kv_smem), qd0, bars, a.ctl, abort_flag);
+        }
+        if (!ok) *abort_flag = 1;
+        mma_commit(done_bar);
+        DevCtl drain = a.ctl;
+        volatile int never = 0;
+        mbar_wait(done_bar, 0, drain, &never, kSiteMla, 7);
+      }
     }
   } else if (warp >= PROD_T0 / 32) {
     // ------------------------------------------------ gather producers
@@ -703,7 +822,11 @@ template <int NKB, int DVC>
 cudaError_t launch_mla_variant(const CUtensorMap& tq, const uint16_t* kv, const MlaArgs& a,
                                cudaStream_t stream) {
   using Tr = MlaTraits<NKB, DVC>;
-  auto kern = a.block_table != nullptr ? sparse_mla_kernel<NKB, DVC, true> : sparse_mla_kernel<NKB, DVC, false>;
+  // several query rows per sequence (prefill): the warp-wide issuer
+  const bool warp_issue = a.Lq > 1;
+  auto kern = a.block_table != nullptr
+                  ? (warp_issue ? sparse_mla_kernel<NKB, DVC, true, true> : sparse_mla_kernel<NKB, DVC, true, false>)
+                  : (warp_issue ? sparse_mla_kernel<NKB, DVC, false, true> : sparse_mla_kernel<NKB, DVC, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
