@@ -46,12 +46,12 @@ CSRC = os.path.join(ROOT, "sparse_attention_long_scores_b200", "csrc")
 # the source has changed since the capture the figure no longer describes the kernel,
 # and the traffic is reported as null.
 TRAFFIC = {
-    # --profile-case prefill_chunk: 329.7 MB read + 235.0 MB written, 2048 rows
-    ("sparse_mla", "prefill"): {"source": "sparse_mla.cu", "rows": 2048, "bytes": 564718080,
-                                "sha256": "27c881c4cc0d417d8884c2546abf4b4126db0bca5f3791782d83d4b88fbcb059"},
-    # --profile-case decode_small: 40.4 MB read + 0.2 MB written, 16 rows
-    ("sparse_mla", "decode"): {"source": "sparse_mla.cu", "rows": 16, "bytes": 40567040,
-                               "sha256": "27c881c4cc0d417d8884c2546abf4b4126db0bca5f3791782d83d4b88fbcb059"},
+    # --profile-case prefill_chunk: 329.3 MB read + 235.0 MB written, 2048 rows
+    ("sparse_mla", "prefill"): {"source": "sparse_mla.cu", "rows": 2048, "bytes": 564293888,
+                                "sha256": "a7dee1cf4177f8d389ff2b42f4a20e640f5c073749741b8ea1aa4d00aa048ac4"},
+    # --profile-case decode_small: 40.3 MB read + 0.4 MB written, 16 rows
+    ("sparse_mla", "decode"): {"source": "sparse_mla.cu", "rows": 16, "bytes": 40730880,
+                               "sha256": "a7dee1cf4177f8d389ff2b42f4a20e640f5c073749741b8ea1aa4d00aa048ac4"},
 }
 DTYPE = "fp8_e4m3+bf16"
 
