@@ -369,19 +369,30 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
 // ---------------------------------------------------------------------------
 constexpr int TKC = 8;
 
-// Sum the CTAs' histograms of one digit over the cluster and pick the digit.
+// Sum the CTAs' histograms of one digit over the cluster and pick the digit, as a
+// reduce-scatter: CTA r sums bins [r SL, (r + 1) SL) over the cluster into its own
+// `ghist` slice and publishes the slice total; then every CTA reads the TKC totals,
+// picks the slice that holds the need-th largest key, and finds the bin inside it
+// from that slice's sums (read from the CTA that holds them). Every CTA reaches the
+// same digit from the same sums. Each CTA reads 1/TKC of the bins from each peer
+// instead of all of them.
 template <int BITS>
 __device__ __forceinline__ void cluster_find(bool first, uint32_t& prefix, uint32_t& need,
                                              uint32_t* hist, uint32_t* ghist, uint32_t* tmp,
-                                             uint32_t* sel) {
+                                             uint32_t* sel, uint32_t* stot) {
   constexpr int NB = 1 << BITS;
+  constexpr int SL = NB / TKC;        // bins per slice
+  constexpr int G4 = SL / 4;          // threads summing a slice, four bins each
+  constexpr int PER = SL / 32;        // bins per lane when one warp searches a slice
+  static_assert(G4 % 32 == 0 && G4 <= TK_THREADS && PER >= 1, "slice shape");
+  const uint32_t rank = cluster_ctarank();
+  const int tid = threadIdx.x, lane = tid & 31;
   cluster_sync();   // every CTA's histogram is complete and visible
-  // cluster sum, four bins per load with all TKC loads of a thread in flight
-  const uint32_t h0 = smem_u32(hist);
-  for (int i = threadIdx.x; i < NB / 4; i += TK_THREADS) {
+  if (tid < G4) {
+    const uint32_t h0 = smem_u32(hist) + (uint32_t)(rank * SL + 4 * tid) * 4u;
     uint4 v[TKC];
 #pragma unroll
-    for (int p = 0; p < TKC; ++p) v[p] = ld_cluster_v4(mapa_shared(h0 + 16u * i, p));
+    for (int p = 0; p < TKC; ++p) v[p] = ld_cluster_v4(mapa_shared(h0, p));
     uint4 acc = v[0];
 #pragma unroll
     for (int p = 1; p < TKC; ++p) {
@@ -390,21 +401,73 @@ __device__ __forceinline__ void cluster_find(bool first, uint32_t& prefix, uint3
       acc.z += v[p].z;
       acc.w += v[p].w;
     }
-    reinterpret_cast<uint4*>(ghist)[i] = acc;
+    reinterpret_cast<uint4*>(ghist + rank * SL)[tid] = acc;
+    const uint32_t part = warp_sum_u32(acc.x + acc.y + acc.z + acc.w);
+    if (lane == 0) tmp[tid >> 5] = part;
   }
-  cluster_sync();   // peers are done reading `hist` before it is cleared again
-  find_bin<BITS>(ghist, first, prefix, need, tmp, sel);
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int w = 0; w < G4 / 32; ++w) t += tmp[w];
+    *stot = t;
+  }
+  cluster_sync();   // slices and totals are published; peers are done reading `hist`
+  if (tid < 32) {
+    // the slice: above(s) = keys in the slices above s (higher digits hold larger keys)
+    const uint32_t tot = lane < TKC ? ld_cluster_u32(mapa_shared(smem_u32(stot), (uint32_t)lane)) : 0u;
+    uint32_t above = 0;
+#pragma unroll
+    for (int q = TKC - 1; q > 0; --q) {
+      const uint32_t tq = __shfl_sync(0xffffffffu, tot, q);
+      if (q > lane) above += tq;
+    }
+    const bool hit = lane < TKC && above < need && need <= above + tot;
+    const uint32_t hits = __ballot_sync(0xffffffffu, hit);   // exactly one slice holds it
+    const int s_sel = hits != 0u ? __ffs(hits) - 1 : 0;
+    const uint32_t need_s = need - __shfl_sync(0xffffffffu, above, s_sel);
+    // the bin inside slice s_sel: lane l holds bins [l PER, (l + 1) PER) of it
+    const uint32_t g0 = mapa_shared(smem_u32(ghist) + (uint32_t)(s_sel * SL + lane * PER) * 4u, (uint32_t)s_sel);
+    uint32_t h[PER];
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      h[j] = ld_cluster_u32(g0 + 4u * (uint32_t)j);
+      mine += h[j];
+    }
+    // keys in the bins of higher lanes
+    uint32_t incl = mine;   // inclusive suffix sum over lanes >= this one
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += x;
+    }
+    uint32_t ab = incl - mine;
+#pragma unroll
+    for (int j = PER - 1; j >= 0; --j) {
+      if (ab < need_s && need_s <= ab + h[j]) {
+        sel[0] = (uint32_t)(s_sel * SL + lane * PER + j);
+        sel[1] = need_s - ab;
+      }
+      ab += h[j];
+    }
+  }
+  __syncthreads();
+  prefix = first ? sel[0] : ((prefix << BITS) | sel[0]);
+  need = sel[1];
+  __syncthreads();
 }
 
 template <int BITS>
 __device__ __forceinline__ void cluster_pass(const SmemKeys& keys, int m, int shift,
                                              uint32_t& prefix, uint32_t& need, uint32_t* hist,
-                                             uint32_t* ghist, uint32_t* tmp, uint32_t* sel) {
+                                             uint32_t* ghist, uint32_t* tmp, uint32_t* sel,
+                                             uint32_t* stot) {
   constexpr int NB = 1 << BITS;
   for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
   __syncthreads();
   histogram_digit<BITS>(keys, m, shift, false, prefix, hist);
-  cluster_find<BITS>(false, prefix, need, hist, ghist, tmp, sel);
+  cluster_find<BITS>(false, prefix, need, hist, ghist, tmp, sel, stot);
 }
 
 __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
@@ -415,6 +478,7 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   __shared__ uint32_t tmp[2 * TK_WARPS];
   __shared__ uint32_t sel[2];
   __shared__ uint32_t counts[2];
+  __shared__ uint32_t stot;   // this CTA's slice total of the current digit
   const uint32_t rank = cluster_ctarank();
   const int rows_per_b = a.t_hi - a.t_lo;
   const long long r = blockIdx.x / TKC;
@@ -442,9 +506,9 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   stage_keys(src, m, seg_keys, hist);   // with the first digit's histogram
   const SmemKeys keys{seg_keys};
   uint32_t prefix = 0, need = (uint32_t)a.k;
-  cluster_find<11>(true, prefix, need, hist, ghist, tmp, sel);   // its cluster barrier publishes the keys
-  cluster_pass<11>(keys, m, 10, prefix, need, hist, ghist, tmp, sel);
-  cluster_pass<10>(keys, m, 0, prefix, need, hist, ghist, tmp, sel);
+  cluster_find<11>(true, prefix, need, hist, ghist, tmp, sel, &stot);   // its cluster barrier publishes the keys
+  cluster_pass<11>(keys, m, 10, prefix, need, hist, ghist, tmp, sel, &stot);
+  cluster_pass<10>(keys, m, 0, prefix, need, hist, ghist, tmp, sel, &stot);
   const uint32_t T = prefix;
   const uint32_t need_eq = need;
 
