@@ -17,8 +17,9 @@
 //   warp 0      tcgen05 issuer: S_i = Q K_i^T of each 64-key tile into one of two
 //               TMEM buffers; Q lives entirely in TMEM (there is no output
 //               accumulator here), so shared memory holds three KV stages;
-//   warps 5..12 gather producers: the selected latent rows of each tile, 16 bytes
-//               per thread per cp.async, into the 128-byte-swizzled K-major layout;
+//   warps 5..12 gather producers: each warp owns 8 rows of every tile, loads their
+//               indices once and copies the rows 16 bytes per thread per cp.async
+//               into the 128-byte-swizzled K-major layout;
 //   warps 1..4  one head per thread (TMEM lane): a[h,s] for the tile's 64 keys,
 //               summed over the warp's 32 heads by a butterfly reduce-scatter (each
 //               lane ends with two keys), then over the four warps in shared
@@ -39,7 +40,6 @@ struct KlTraits {
   static constexpr int KVBLK = KEYS * 128;          // one 64-column block of a KV tile
   static constexpr int STAGES = 3;
   static constexpr int NP = PROD_WARPS * 32;
-  static constexpr int CPT = (KEYS * NKB * 8 + NP - 1) / NP;   // 16-byte chunks per thread
   static constexpr int OFF_KV = 0;
   static constexpr int OFF_RED = OFF_KV + STAGES * NKB * KVBLK;   // [2][4 warps][KEYS] fp32
   static constexpr int OFF_BAR = OFF_RED + 2 * 4 * KEYS * 4;
@@ -179,27 +179,35 @@ __global__ void __launch_bounds__(KL_THREADS, 1)
     // Chunk c of a tile is 16 bytes: row r = c / (8 NKB), 16-byte chunk q of that
     // row, stored at column block q / 8, row r, slot (q % 8) ^ (r % 8) of the
     // 128-byte-swizzled K-major layout. Chunks past the end of a row are zeros.
-    const int ptid = threadIdx.x - PROD_T0;
+    const int pw = warp - PROD_T0 / 32;   // this warp owns rows 8 pw .. 8 pw + 7 of every tile
     const int row_bytes = a.Dqk * 2;
     const uint8_t* kv_b = reinterpret_cast<const uint8_t*>(kv) + (size_t)b * a.Lk * row_bytes;
     const uint32_t kv_base = smem_u32(kv_smem);
+    constexpr int CHUNKS = 8 * NKB * 8;   // 16-byte chunks of the warp's 8 rows
+    static_assert(CHUNKS % 32 == 0 && PROD_WARPS * 8 == KEYS, "producer mapping");
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % Tr::STAGES;
+      // the rows' indices once per tile (lanes 0..7); invalid keys read row 0, masked later
+      const int pos = i * KEYS + pw * 8 + lane;
+      int v = -1;
+      if (lane < 8 && pos < a.k) v = __ldg(idx_row + pos);
+      const int row = (v >= 0 && v < a.Lk) ? v : 0;
+      const uint8_t* src_row = kv_b + (size_t)row * row_bytes;
       if (!mbar_wait(&kv_empty[st], ((i / Tr::STAGES) & 1) ^ 1, a.ctl, abort_flag, kSiteKl, 5)) break;
       const uint32_t stage = kv_base + st * NKB * Tr::KVBLK;
 #pragma unroll
-      for (int jj = 0; jj < Tr::CPT; ++jj) {
-        const int c = ptid + jj * Tr::NP;
-        if (c < KEYS * NKB * 8) {
-          const int r = c / (NKB * 8);
-          const int q = c - r * NKB * 8;
-          const int pos = i * KEYS + r;
-          const int v = pos < a.k ? __ldg(idx_row + pos) : -1;
-          const int row = (v >= 0 && v < a.Lk) ? v : 0;   // invalid keys read row 0, masked later
-          const bool in_row = q * 16 < row_bytes;
-          cp_async16(stage + (q >> 3) * Tr::KVBLK + r * 128 + (((q & 7) ^ (r & 7)) << 4),
-                     kv_b + (size_t)row * row_bytes + (in_row ? q * 16 : 0), in_row ? 16u : 0u);
-        }
+      for (int jj = 0; jj < CHUNKS / 32; ++jj) {
+        const int q = lane + jj * 32;
+        const int rr = q / (NKB * 8);
+        const int rem = q - rr * NKB * 8;
+        const int kb = rem >> 3, q8 = rem & 7;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(src_row), rr));
+        const int r = pw * 8 + rr;
+        const int qc = kb * 8 + q8;   // 16-byte chunk within the row
+        const bool in_row = qc * 16 < row_bytes;
+        cp_async16(stage + kb * Tr::KVBLK + r * 128 + ((q8 ^ (r & 7)) << 4), src + (in_row ? qc * 16 : 0),
+                   in_row ? 16u : 0u);
       }
       cp_async_commit();
       cp_async_wait<0>();
