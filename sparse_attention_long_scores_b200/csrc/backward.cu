@@ -185,14 +185,33 @@ __global__ void gather_e4m3_rows_bf16_kernel(const uint8_t* __restrict__ kI,
                                              int Lq, int Lk, int k, int d_I) {
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(T) * k;
+  // whole 4-code words when the rows allow it (the codes come from the caller)
+  const bool vec = (d_I & 3) == 0 && (reinterpret_cast<uintptr_t>(kI) & 3u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(out) & 7u) == 0;
   for (long long r = warp_id_global(); r < rows; r += warps_in_grid()) {
     const long long tok = tok0 + r / k;
     const int j = static_cast<int>(r % k);
     const int s = selected_key(idx, tok, j, k, Lk);
     const long long b = tok / Lq;
     uint16_t* dst = out + r * d_I;
-    for (int c = lane; c < d_I; c += 32)
-      dst[c] = s < 0 ? uint16_t(0) : float_to_bf16_bits(e4m3_to_float(kI[(b * Lk + s) * d_I + c]));
+    const uint8_t* src = kI + (b * Lk + (s < 0 ? 0 : s)) * d_I;
+    if (vec) {
+      // four codes per lane: one 4-byte load, one 8-byte store
+      for (int c = 4 * lane; c < d_I; c += 128) {
+        uint32_t w = s < 0 ? 0u : *reinterpret_cast<const uint32_t*>(src + c);
+        uint32_t lo = 0u, hi = 0u;
+        if (s >= 0) {
+          lo = (uint32_t)float_to_bf16_bits(e4m3_to_float((uint8_t)(w & 0xFFu))) |
+               ((uint32_t)float_to_bf16_bits(e4m3_to_float((uint8_t)((w >> 8) & 0xFFu))) << 16);
+          hi = (uint32_t)float_to_bf16_bits(e4m3_to_float((uint8_t)((w >> 16) & 0xFFu))) |
+               ((uint32_t)float_to_bf16_bits(e4m3_to_float((uint8_t)(w >> 24))) << 16);
+        }
+        *reinterpret_cast<uint2*>(dst + c) = make_uint2(lo, hi);
+      }
+    } else {
+      for (int c = lane; c < d_I; c += 32)
+        dst[c] = s < 0 ? uint16_t(0) : float_to_bf16_bits(e4m3_to_float(src[c]));
+    }
   }
 }
 
