@@ -13,7 +13,8 @@
 //     tokens x H_I heads (N = 256, or 64 for single-token decode blocks),
 //     K = d_I. One tcgen05.mma kind::f8f6f4 per 32 bytes of K.
 //   * Warp 0 streams key tiles with TMA into a STAGES-deep ring; warp 1 issues
-//     the MMAs into two TMEM accumulators; warps 2.. are the epilogue: each
+//     the MMAs into two TMEM accumulators; warps 2.. are the epilogue (four per
+//     TMEM lane quadrant at N = 256, one token each): each
 //     thread owns one key, reads its accumulator row with tcgen05.ld, applies
 //     ReLU and the folded weight w*s^q per column, reduces over heads in
 //     registers and writes one fp32 score per (token, key). The L x L score
@@ -220,7 +221,10 @@ struct IdxTraits {
   static constexpr int ACC = 2;
   static constexpr int TMEM_COLS = (ACC * N <= 32) ? 32 : (ACC * N <= 64) ? 64
                                    : (ACC * N <= 128) ? 128 : (ACC * N <= 256) ? 256 : 512;
-  static constexpr int EPI_WARPS = (T_BLK >= 2) ? 8 : 4;
+  // epilogue warps: four per TMEM lane quadrant with one token each at N = 256 (the
+  // epilogue is latency-bound; with the fused selectors' threads the registers
+  // allow two per quadrant)
+  static constexpr int EPI_WARPS = (T_BLK >= 4 && !SEL) ? 16 : (T_BLK >= 2) ? 8 : 4;
   static constexpr int MIN_CTAS = (N == 64) ? 2 : 1;        // CTAs per SM the registers must allow
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
   // selector warps of the fused top-k (two beside the single-token epilogue, so two
