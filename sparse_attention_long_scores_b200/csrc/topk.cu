@@ -27,8 +27,13 @@
 namespace dsa {
 namespace {
 
-constexpr int TK_THREADS = 512;
-constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_THREADS = 512;                   // a CTA of the cluster kernel (rows split over 8)
+constexpr int TK1_THREADS = 1024;                 // a CTA of the single-CTA kernel on long rows
+constexpr int TK_MAX_WARPS = TK1_THREADS / 32;
+// Rows staged in more shared memory than two CTAs of an SM can hold run with
+// TK1_THREADS threads per CTA (one row per SM: more warps hide the passes'
+// latency); shorter rows run with TK_THREADS, several CTAs per SM.
+constexpr int TK_WIDE_KEYS = 26 * 1024;
 constexpr int TK_SMEM_MAX = 48 * 1024;            // candidates staged in shared memory
 constexpr int TK_STEP = 128;                      // keys per warp step of the output pass
 
@@ -50,7 +55,9 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
 }
 
 // Exclusive block scan of one int per thread; also returns the block total.
+template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t& total) {
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint32_t incl = v;
 #pragma unroll
@@ -61,17 +68,17 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, u
   if (lane == 31) tmp[wid] = incl;
   __syncthreads();
   if (wid == 0) {
-    uint32_t x = lane < TK_WARPS ? tmp[lane] : 0u;
+    uint32_t x = lane < NW ? tmp[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       uint32_t n = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += n;
     }
-    if (lane < TK_WARPS) tmp[lane] = x;
+    if (lane < NW) tmp[lane] = x;
   }
   __syncthreads();
   uint32_t off = wid > 0 ? tmp[wid - 1] : 0u;
-  total = tmp[TK_WARPS - 1];
+  total = tmp[NW - 1];
   __syncthreads();
   return off + incl - v;
 }
@@ -79,16 +86,16 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, u
 // Given a histogram of the candidate digits, pick the digit holding the
 // `need`-th largest key; extend `prefix` by it and make `need` the rank within
 // that digit (uniform across the block).
-template <int BITS>
+template <int BITS, int NT>
 __device__ __forceinline__ void find_bin(const uint32_t* hist, bool first, uint32_t& prefix,
                                          uint32_t& need, uint32_t* tmp, uint32_t* sel) {
-  constexpr int BPT = (1 << BITS) / TK_THREADS;
+  constexpr int BPT = (1 << BITS) / NT;
   uint32_t local = 0;
   const int b0 = threadIdx.x * BPT;
 #pragma unroll
   for (int j = 0; j < BPT; ++j) local += hist[b0 + j];
   uint32_t total;
-  uint32_t before = block_excl_scan(local, tmp, total);
+  uint32_t before = block_excl_scan<NT>(local, tmp, total);
   uint32_t above = total - before - local;  // keys in bins of higher-numbered threads
 #pragma unroll
   for (int j = BPT - 1; j >= 0; --j) {
@@ -135,7 +142,7 @@ struct GlobalKeys {
 
 // Histogram (into `hist`, already cleared) the digit (key >> shift) of the keys
 // of [0, m) whose bits above `shift + BITS` equal `prefix`.
-template <int BITS, class Keys>
+template <int BITS, int NT, class Keys>
 __device__ __forceinline__ void histogram_digit(const Keys& keys, int m, int shift, bool first,
                                                 uint32_t prefix, uint32_t* hist) {
   constexpr uint32_t MASK = (1u << BITS) - 1u;
@@ -145,7 +152,7 @@ __device__ __forceinline__ void histogram_digit(const Keys& keys, int m, int shi
   };
   const int groups = (m + 3) >> 2;
 #pragma unroll 4
-  for (int g = threadIdx.x; g < groups; g += TK_THREADS) {
+  for (int g = threadIdx.x; g < groups; g += NT) {
     const int i = g << 2;
     const uint4 v = keys.load4(i, m);
     count(v.x, true);
@@ -157,17 +164,17 @@ __device__ __forceinline__ void histogram_digit(const Keys& keys, int m, int shi
 
 // One radix pass of the single-CTA kernel: histogram, then find the digit
 // holding the `need`-th largest key. Updates prefix/need in place.
-template <int BITS, class Keys>
+template <int BITS, int NT, class Keys>
 __device__ __forceinline__ void radix_pass(const Keys& keys, int n, int shift, bool first,
                                            uint32_t& prefix, uint32_t& need, uint32_t* hist,
                                            uint32_t* tmp, uint32_t* sel) {
   constexpr int NB = 1 << BITS;
-  static_assert(NB / TK_THREADS >= 1, "bins");
-  for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
+  static_assert(NB / NT >= 1, "bins");
+  for (int i = threadIdx.x; i < NB; i += NT) hist[i] = 0u;
   __syncthreads();
-  histogram_digit<BITS>(keys, n, shift, first, prefix, hist);
+  histogram_digit<BITS, NT>(keys, n, shift, first, prefix, hist);
   __syncthreads();
-  find_bin<BITS>(hist, first, prefix, need, tmp, sel);
+  find_bin<BITS, NT>(hist, first, prefix, need, tmp, sel);
 }
 
 // ---------------------------------------------------------------------------
@@ -177,9 +184,11 @@ struct Run {
   int s0, s1;
 };
 
+template <int NT>
 __device__ __forceinline__ Run warp_run(int m) {
+  constexpr int NW = NT / 32;
   const int steps = (m + TK_STEP - 1) / TK_STEP;
-  const int per = (steps + TK_WARPS - 1) / TK_WARPS;
+  const int per = (steps + NW - 1) / NW;
   const int s0 = min(steps, (int)(threadIdx.x >> 5) * per);
   return Run{s0, min(steps, s0 + per)};
 }
@@ -253,9 +262,9 @@ __device__ __forceinline__ void write_run(const Keys& keys, int m, uint32_t T, u
   }
 }
 
-// Per-warp counts of the run into tmp[wid] / tmp[TK_WARPS + wid], then this
+// Per-warp counts of the run into tmp[wid] / tmp[NT / 32 + wid], then this
 // warp's (G, E) offsets within the block and the block totals.
-template <class Keys>
+template <int NT, class Keys>
 __device__ __forceinline__ void block_run_offsets(const Keys& keys, int m, uint32_t T, Run run,
                                                   uint32_t* tmp, uint32_t& G, uint32_t& E,
                                                   uint32_t& g_tot, uint32_t& e_tot) {
@@ -264,7 +273,7 @@ __device__ __forceinline__ void block_run_offsets(const Keys& keys, int m, uint3
   run_counts(keys, m, T, run, g, e);
   if (lane == 0) {
     tmp[wid] = g;
-    tmp[TK_WARPS + wid] = e;
+    tmp[(NT / 32) + wid] = e;
   }
   __syncthreads();
   G = 0;
@@ -272,8 +281,8 @@ __device__ __forceinline__ void block_run_offsets(const Keys& keys, int m, uint3
   g_tot = 0;
   e_tot = 0;
 #pragma unroll
-  for (int w = 0; w < TK_WARPS; ++w) {
-    const uint32_t gw = tmp[w], ew = tmp[TK_WARPS + w];
+  for (int w = 0; w < (NT / 32); ++w) {
+    const uint32_t gw = tmp[w], ew = tmp[(NT / 32) + w];
     if (w < wid) {
       G += gw;
       E += ew;
@@ -285,6 +294,7 @@ __device__ __forceinline__ void block_run_offsets(const Keys& keys, int m, uint3
 
 // Stage scores [0, m) as keys in shared memory and histogram their top 11 bits
 // (hist already cleared). The caller synchronises.
+template <int NT>
 __device__ __forceinline__ void stage_keys(const float* src, int m, uint32_t* keys, uint32_t* hist) {
   auto put = [&](int i, uint32_t key) {
     keys[i] = key;
@@ -295,7 +305,7 @@ __device__ __forceinline__ void stage_keys(const float* src, int m, uint32_t* ke
     const float4* s4 = reinterpret_cast<const float4*>(src);
     uint4* k4 = reinterpret_cast<uint4*>(keys);
 #pragma unroll 4
-    for (int i = threadIdx.x; i < m4; i += TK_THREADS) {
+    for (int i = threadIdx.x; i < m4; i += NT) {
       const float4 v = __ldg(s4 + i);
       const uint4 kk = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
       k4[i] = kk;
@@ -304,17 +314,17 @@ __device__ __forceinline__ void stage_keys(const float* src, int m, uint32_t* ke
       atomicAdd(&hist[kk.z >> 21], 1u);
       atomicAdd(&hist[kk.w >> 21], 1u);
     }
-    for (int i = (m4 << 2) + threadIdx.x; i < m; i += TK_THREADS) put(i, score_key(__ldg(src + i)));
+    for (int i = (m4 << 2) + threadIdx.x; i < m; i += NT) put(i, score_key(__ldg(src + i)));
   } else {
-    for (int i = threadIdx.x; i < m; i += TK_THREADS) put(i, score_key(__ldg(src + i)));
+    for (int i = threadIdx.x; i < m; i += NT) put(i, score_key(__ldg(src + i)));
   }
 }
 
-template <bool SMEM_ROW>
-__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
+template <bool SMEM_ROW, int NT>
+__global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint32_t row_keys[];
   __shared__ uint32_t hist[2048];
-  __shared__ uint32_t tmp[2 * TK_WARPS];
+  __shared__ uint32_t tmp[2 * TK_MAX_WARPS];
   __shared__ uint32_t sel[2];
   using Keys = typename std::conditional<SMEM_ROW, SmemKeys, GlobalKeys>::type;
   const int rows_per_b = a.t_hi - a.t_lo;
@@ -327,7 +337,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
     float* dsc = a.sel != nullptr ? a.sel + ((long long)b * a.Lq + t) * a.k : nullptr;
     const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld;
     if (n <= a.k) {
-      for (int i = threadIdx.x; i < a.k; i += TK_THREADS) {
+      for (int i = threadIdx.x; i < a.k; i += NT) {
         dst[i] = i < n ? i : -1;
         if (dsc != nullptr) dsc[i] = i < n ? src[i] : 0.f;
       }
@@ -337,24 +347,24 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a) {
     uint32_t prefix = 0, need = (uint32_t)a.k;
     if constexpr (SMEM_ROW) {
       // staging builds the first digit's histogram on the way
-      for (int i = threadIdx.x; i < 2048; i += TK_THREADS) hist[i] = 0u;
+      for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
       __syncthreads();
-      stage_keys(src, n, row_keys, hist);
+      stage_keys<NT>(src, n, row_keys, hist);
       __syncthreads();
-      find_bin<11>(hist, true, prefix, need, tmp, sel);
+      find_bin<11, NT>(hist, true, prefix, need, tmp, sel);
       keys = SmemKeys{row_keys};
     } else {
       keys = GlobalKeys{src, a.vec4 != 0};
-      radix_pass<11>(keys, n, 21, true, prefix, need, hist, tmp, sel);
+      radix_pass<11, NT>(keys, n, 21, true, prefix, need, hist, tmp, sel);
     }
-    radix_pass<11>(keys, n, 10, false, prefix, need, hist, tmp, sel);
-    radix_pass<10>(keys, n, 0, false, prefix, need, hist, tmp, sel);
+    radix_pass<11, NT>(keys, n, 10, false, prefix, need, hist, tmp, sel);
+    radix_pass<10, NT>(keys, n, 0, false, prefix, need, hist, tmp, sel);
     const uint32_t T = prefix;
     const uint32_t need_eq = need;  // keys equal to T that are selected (lowest indices first)
 
-    const Run run = warp_run(n);
+    const Run run = warp_run<NT>(n);
     uint32_t G, E, g_tot, e_tot;
-    block_run_offsets(keys, n, T, run, tmp, G, E, g_tot, e_tot);
+    block_run_offsets<NT>(keys, n, T, run, tmp, G, E, g_tot, e_tot);
     write_run(keys, n, T, need_eq, G, E, 0, run, dst, dsc);
     __syncthreads();   // tmp, hist and the staged row are reused by the next row
   }
@@ -466,7 +476,7 @@ __device__ __forceinline__ void cluster_pass(const SmemKeys& keys, int m, int sh
   constexpr int NB = 1 << BITS;
   for (int i = threadIdx.x; i < NB; i += TK_THREADS) hist[i] = 0u;
   __syncthreads();
-  histogram_digit<BITS>(keys, m, shift, false, prefix, hist);
+  histogram_digit<BITS, TK_THREADS>(keys, m, shift, false, prefix, hist);
   cluster_find<BITS>(false, prefix, need, hist, ghist, tmp, sel, stot);
 }
 
@@ -475,7 +485,7 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   extern __shared__ __align__(16) uint32_t seg_keys[];
   __shared__ __align__(16) uint32_t hist[2048];
   __shared__ __align__(16) uint32_t ghist[2048];
-  __shared__ uint32_t tmp[2 * TK_WARPS];
+  __shared__ uint32_t tmp[2 * (TK_THREADS / 32)];
   __shared__ uint32_t sel[2];
   __shared__ uint32_t counts[2];
   __shared__ uint32_t stot;   // this CTA's slice total of the current digit
@@ -503,7 +513,7 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   const float* src = a.scores + ((long long)b * a.sc_bstride + (t - a.sc_t0)) * a.sc_ld + lo;
   for (int i = threadIdx.x; i < 2048; i += TK_THREADS) hist[i] = 0u;
   __syncthreads();
-  stage_keys(src, m, seg_keys, hist);   // with the first digit's histogram
+  stage_keys<TK_THREADS>(src, m, seg_keys, hist);   // with the first digit's histogram
   const SmemKeys keys{seg_keys};
   uint32_t prefix = 0, need = (uint32_t)a.k;
   cluster_find<11>(true, prefix, need, hist, ghist, tmp, sel, &stot);   // its cluster barrier publishes the keys
@@ -513,9 +523,9 @@ __global__ void __cluster_dims__(TKC, 1, 1) __launch_bounds__(TK_THREADS)
   const uint32_t need_eq = need;
 
   // this CTA's counts, then the counts of the segments before it
-  const Run run = warp_run(m);
+  const Run run = warp_run<TK_THREADS>(m);
   uint32_t G, E, g_tot, e_tot;
-  block_run_offsets(keys, m, T, run, tmp, G, E, g_tot, e_tot);
+  block_run_offsets<TK_THREADS>(keys, m, T, run, tmp, G, E, g_tot, e_tot);
   if (threadIdx.x == 0) {
     counts[0] = g_tot;
     counts[1] = e_tot;
@@ -548,12 +558,13 @@ cudaError_t launch_topk(const TopkArgs& a, int num_sms, cudaStream_t stream) {
     topk_cluster_kernel<<<(unsigned)(nrows * TKC), TK_THREADS, smem, stream>>>(a);
   } else if (n_max <= TK_SMEM_MAX) {
     size_t smem = (size_t)((n_max + 3) & ~3) * 4;
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool wide = n_max > TK_WIDE_KEYS;
+    auto kern = wide ? topk_kernel<true, TK1_THREADS> : topk_kernel<true, TK_THREADS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_kernel<true><<<grid, TK_THREADS, smem, stream>>>(a);
+    kern<<<grid, wide ? TK1_THREADS : TK_THREADS, smem, stream>>>(a);
   } else {
-    topk_kernel<false><<<grid, TK_THREADS, 0, stream>>>(a);
+    topk_kernel<false, TK1_THREADS><<<grid, TK1_THREADS, 0, stream>>>(a);
   }
   return cudaGetLastError();
 }
